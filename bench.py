@@ -1,0 +1,372 @@
+#!/usr/bin/env python
+"""KDA operator benchmark: prefill tokens/s on B=1, H=16, d=128, L=65536 (bf16
+inputs, fp32 state, chunk 64) plus decode steps/s on B=256, H=16, d=128.
+
+One JSON line on rank 0.  A step is one kda_forward over the whole prefill
+workload (gate, normalisation, chunk cumsum, intra-chunk products, UT
+inverse, WY blocks, state pass, final state).  The decode step (the remaining
+hot-path row) is measured in the same run and reported under "decode".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kda|reference]
+
+With N > 1 (torchrun, one rank per GPU) every rank runs its own copy of the
+workload (independent problems, no data-path collective: weak scaling); the
+time is the max over ranks.  ``--impl reference`` times the float64 CPU oracle
+on a bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+B, H, D, L_DEFAULT, CHUNK = 1, 16, 128, 65536, 64
+DEC_B = 256
+METRIC = "KDA prefill tokens/s (B=1,H=16,d=128,L=64k) & decode steps/s; % tensor/HBM roofline"
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def alg_flops(T, C=CHUNK, d=D, heads=H):
+    """Kimi Linear summary §6.3: 6 T d^2 + 3 T C d + T C^2 per head."""
+    return heads * (6 * T * d * d + 3 * T * C * d + T * C * C)
+
+
+def alg_bytes_prefill(T, N=1, heads=H, dk=D, dv=D, elt=2, s0=False, sfinal=True):
+    """q, k, z, v, beta read and o written per token-head, plus states."""
+    per_tok = elt * (3 * dk + dv + 1 + dv)
+    st = N * heads * dk * dv * 4
+    return T * heads * per_tok + (st if s0 else 0) + (st if sfinal else 0)
+
+
+def alg_bytes_decode(Bd=DEC_B, heads=H, dk=D, dv=D, elt=2):
+    """State read + written, q, k, z, v, beta read and o written per (b, h)."""
+    return Bd * heads * (2 * dk * dv * 4 + elt * (3 * dk + dv + 1 + dv))
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"], src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, src="fallback")
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gated_delta_rule_98_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        h.update(fn.encode())
+        h.update(open(os.path.join(csrc, fn), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kind):
+    """ncu DRAM bytes per launch recorded for the current kernel sources, or None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(kind)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 200 ms while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.f = None
+
+    def __enter__(self):
+        try:
+            self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        self.f.flush()
+        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except (ValueError, IndexError):
+                continue
+            for nm, val in zip(names, r[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def oracle_baseline(inp, n_tokens):
+    """Float64 oracle on the first n_tokens of the workload (all heads)."""
+    from oracle import ref
+    sl = slice(0, n_tokens)
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    ref.forward(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["beta"][sl], z=inp["z"][sl],
+                A=inp["A"], num_seqs=1, threads=threads)
+    dt = time.perf_counter() - t0
+    return dt, min(threads, H)
+
+
+def run_reference(args):
+    """The reference arm: the float64 CPU oracle, timed on a bounded sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from gated_delta_rule_98_b200 import synth
+    n_tok = 4096
+    inp = synth.draw(n_tok, H, D, D, seed=2, dtype="bf16")  # same generators, shorter draw
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt, cores = oracle_baseline(inp, n_tok)
+        if i >= args.warmup:
+            times.append(dt)
+    t = sum(times) / len(times)
+    val = n_tok / t
+    sample = f"{n_tok} tokens x {H} heads (B=1, d=128, bf16-rounded inputs widened to f64)"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "KDA fwd long (float64 CPU oracle, bounded sample)", "B": 1,
+                   "H": H, "L": L_DEFAULT, "dk": D, "dv": D, "sample_tokens": n_tok},
+        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
+    ap.add_argument("--L", type=int, default=L_DEFAULT, help="prefill length (sweep)")
+    ap.add_argument("--decode-steps", type=int, default=1000)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    from gated_delta_rule_98_b200 import kda, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    L = args.L
+    T = B * L
+    log(f"[rank {rank}] generating inputs L={L}")
+    inp = synth.workload("long", L=L)
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    Sf = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    ws = kda.workspace(B, T, L, H, D, D, torch.bfloat16, CHUNK, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches = kda.kda_forward_launches(B, T, L, H, D, D, kda.KDA_BF16, CHUNK)
+
+    def fwd():
+        kda.forward(d["q"], d["k"], d["v"], d["z"], d["A"], d["beta"], num_seqs=B, chunk=CHUNK,
+                    o=o, S_final=Sf, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        fwd()
+    torch.cuda.synchronize()
+    assert kda.check_device_error(ws) == kda.KDA_OK
+
+    # ---------------------------------------------------------- prefill ---
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fwd()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms_local = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms_local)
+    clocks = clk.summary()
+    value = world * T / (ms / 1e3)
+
+    pk = peaks()
+    fwd_bytes = alg_bytes_prefill(T)
+    fwd_flops = alg_flops(T)
+    achieved = fwd_bytes / (ms_local / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": achieved / pk["hbm"], "traffic": recorded_traffic("forward"),
+                "kernel": "kda_forward (all launches of one call)",
+                "peak_source": pk["src"],
+                "tensor_flops_frac": fwd_flops / (ms_local / 1e3) / 1e12 / pk["bf16"],
+                "roofline_time_us": max(fwd_bytes / pk["hbm"] / 1e3,
+                                        fwd_flops / pk["bf16"] / 1e6)}
+    roofline["frac_of_roofline_time"] = roofline["roofline_time_us"] / (ms_local * 1e3)
+
+    # -------------------------------------------------------------- e2e ---
+    # Same metric through the public API with pinned host buffers; the H2D copy
+    # of the step's inputs and the D2H read of o and S_final are inside.
+    host = {k: inp[k].pin_memory() for k in ("q", "k", "v", "z", "beta", "A")}
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    S_h = torch.empty(Sf.shape, dtype=Sf.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_h.numel() * o_h.element_size() + S_h.numel() * S_h.element_size()
+
+    def e2e_step():
+        for k_, t in host.items():
+            d[k_].copy_(t, non_blocking=True)
+        fwd()
+        o_h.copy_(o, non_blocking=True)
+        S_h.copy_(Sf, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    n_e2e = max(3, min(args.steps, 10))
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / n_e2e)
+    e2e = {"value": world * T / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h}
+
+    # ----------------------------------------------------------- decode ---
+    del ws
+    torch.cuda.empty_cache()
+    A_dec, S_dec0 = synth.decode_state(DEC_B, H, D, D)
+    S_dec = S_dec0.to(dev)
+    A_dec = A_dec.to(dev)
+    pool = [{k: t.to(dev) for k, t in synth.decode_token(s, DEC_B, H, D, D).items()}
+            for s in range(8)]
+    o_dec = torch.empty((DEC_B, H, D), dtype=torch.bfloat16, device=dev)
+
+    def dec(s):
+        tk = pool[s % len(pool)]
+        kda.decode_step(tk["q"], tk["k"], tk["v"], tk["z"], A_dec, tk["beta"], S_dec, o=o_dec,
+                        stream=stream)
+
+    for s in range(10):
+        dec(s)
+    torch.cuda.synchronize()
+    barrier()
+    e0.record(stream)
+    for s in range(args.decode_steps):
+        dec(s)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms_dec_local = e0.elapsed_time(e1) / args.decode_steps
+    ms_dec = max_over_ranks(ms_dec_local)
+    dec_bytes = alg_bytes_decode()
+    dec_ach = dec_bytes / (ms_dec_local / 1e3) / 1e9
+    decode = {"value": world * 1e3 / ms_dec, "unit": "steps/s", "ms_per_step": ms_dec,
+              "tokens_per_s": world * DEC_B * 1e3 / ms_dec, "steps": args.decode_steps,
+              "config": {"B": DEC_B, "H": H, "dk": D, "dv": D, "dtype": "bf16",
+                         "state": "fp32 in place (268 MB, exceeds L2)"},
+              "gpu_launches": args.decode_steps,
+              "roofline": {"bound": "hbm", "achieved": dec_ach, "peak": pk["hbm"],
+                           "unit": "GB/s", "frac": dec_ach / pk["hbm"],
+                           "traffic": recorded_traffic("decode"),
+                           "kernel": "decode_step_kernel", "peak_source": pk["src"]}}
+
+    # ------------------------------------------------------ CPU baseline ---
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_tok = min(T, 16384)
+        dt_cpu, cores = oracle_baseline(inp, n_tok)
+        cpu = {"value": n_tok / dt_cpu, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+               "sample": f"first {n_tok} tokens x {H} heads of the same workload (float64)"}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": f"KDA fwd long: B={B} H={H} L={L} dk=dv={D}, bf16 inputs, "
+                               f"fp32 state, chunk {CHUNK}, S0=0", "B": B, "H": H, "L": L,
+                   "dk": D, "dv": D, "chunk": CHUNK,
+                   "l2": "inputs exceed L2 (q,k,v,z,o = %.0f MB per step)" % (
+                       T * H * D * 2 * 5 / 1e6),
+                   "parallelism": f"weak x{world} (independent problems per rank)"},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches * args.steps, "clocks": clocks, "decode": decode,
+    }), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,161 @@
+// kda_api.cu -- the C ABI of include/kda.h: argument validation, workspace
+// sizing and kernel selection.  Every host-visible fault returns before any
+// work is enqueued.
+#include <cuda_runtime.h>
+
+#include "../../include/kda.h"
+#include "kda_common.cuh"
+#include "kda_launch.h"
+
+namespace {
+
+bool dim_ok(int32_t d) { return d == 32 || d == 64 || d == 128; }
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+bool opt_aligned16(const void* p) { return p == nullptr || aligned16(p); }
+
+// Host checks common to kda_forward and kda_forward_g.  Returns KDA_OK or the
+// error to report.
+kda_status check_forward(const void* q, const void* k, const void* v,
+                         const void* gate_src, const void* beta, const float* S0,
+                         const int32_t* cu, int32_t N, int32_t T, int32_t max_len,
+                         int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
+                         int32_t chunk, const void* o, const float* S_final,
+                         const void* ws, size_t ws_bytes) {
+  if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_UNSUPPORTED;
+  if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  if (chunk != 16 && chunk != 64) return KDA_ERR_UNSUPPORTED;
+  if (N < 0 || T < 0 || max_len < 0 || H < 1) return KDA_ERR_INVALID_ARG;
+  if (!cu) {
+    if ((int64_t)N * max_len != T) return KDA_ERR_INVALID_ARG;
+  } else {
+    if (!aligned16(cu) && ((uintptr_t)cu & 3u)) return KDA_ERR_INVALID_ARG;
+  }
+  if (N > 0 && (int64_t)N * ((max_len + chunk - 1) / chunk) > 0x7fffffffLL)
+    return KDA_ERR_UNSUPPORTED;
+  if (T > 0) {
+    if (!q || !k || !v || !gate_src || !beta || !o) return KDA_ERR_INVALID_ARG;
+  }
+  if (!opt_aligned16(q) || !opt_aligned16(k) || !opt_aligned16(v) ||
+      !opt_aligned16(gate_src) || !opt_aligned16(beta) || !opt_aligned16(o) ||
+      !opt_aligned16(S0) || !opt_aligned16(S_final) || !opt_aligned16(ws))
+    return KDA_ERR_INVALID_ARG;
+  const size_t need = kda_forward_workspace_size(N, T, max_len, H, dk, dv, dt, chunk);
+  if (need == 0 || !ws || ws_bytes < need) return KDA_ERR_INVALID_ARG;
+  return KDA_OK;
+}
+
+kda_status forward_common(kda::ForwardArgs& a) {
+  if (a.N == 0) {
+    // nothing to launch: still leave a clean error word for this call
+    return cudaMemsetAsync(a.ws, 0, sizeof(uint32_t), a.stream) == cudaSuccess ? KDA_OK
+                                                                               : KDA_ERR_CUDA;
+  }
+  cudaError_t err = kda::launch_forward_simt(a);
+  return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kda_status_string(kda_status s) {
+  switch (s) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+    case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+  }
+  return "KDA_ERR_UNKNOWN";
+}
+
+int32_t kda_version(void) { return 100; }
+
+size_t kda_forward_workspace_size(int32_t num_seqs, int32_t total_tokens,
+                                  int32_t max_seqlen, int32_t H, int32_t dk,
+                                  int32_t dv, kda_dtype dt, int32_t chunk) {
+  if (dt != KDA_F32 && dt != KDA_BF16) return 0;
+  if (!dim_ok(dk) || !dim_ok(dv) || (chunk != 16 && chunk != 64)) return 0;
+  if (num_seqs < 0 || total_tokens < 0 || max_seqlen < 0 || H < 1) return 0;
+  return kda::simt_workspace_bytes(num_seqs, total_tokens, H, dk, dv, chunk);
+}
+
+int32_t kda_forward_launches(int32_t num_seqs, int32_t total_tokens,
+                             int32_t max_seqlen, int32_t H, int32_t dk,
+                             int32_t dv, kda_dtype dt, int32_t chunk) {
+  if (kda_forward_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv, dt, chunk) == 0)
+    return 0;
+  if (num_seqs == 0) return 0;  // a memset only
+  return kda::simt_launches(num_seqs, max_seqlen, chunk);
+}
+
+kda_status kda_forward(const void* q, const void* k, const void* v,
+                       const void* z, const float* A, const void* beta,
+                       const float* S0, const int32_t* cu_seqlens,
+                       int32_t num_seqs, int32_t total_tokens,
+                       int32_t max_seqlen, int32_t H, int32_t dk, int32_t dv,
+                       kda_dtype dt, int32_t chunk, void* o, float* S_final,
+                       void* workspace, size_t workspace_bytes,
+                       kda_stream_t stream) {
+  kda_status st = check_forward(q, k, v, z, beta, S0, cu_seqlens, num_seqs,
+                                total_tokens, max_seqlen, H, dk, dv, dt, chunk,
+                                o, S_final, workspace, workspace_bytes);
+  if (st != KDA_OK) return st;
+  if (total_tokens > 0 && (!A || !aligned16(A))) return KDA_ERR_INVALID_ARG;
+  kda::ForwardArgs a{q, k, v, z, beta, A, nullptr, S0, cu_seqlens, o, S_final,
+                     num_seqs, total_tokens, max_seqlen, H, dk, dv, chunk,
+                     dt == KDA_BF16, workspace, workspace_bytes,
+                     (cudaStream_t)stream};
+  return forward_common(a);
+}
+
+kda_status kda_forward_g(const void* q, const void* k, const void* v,
+                         const float* g, const void* beta, const float* S0,
+                         const int32_t* cu_seqlens, int32_t num_seqs,
+                         int32_t total_tokens, int32_t max_seqlen, int32_t H,
+                         int32_t dk, int32_t dv, kda_dtype dt, int32_t chunk,
+                         void* o, float* S_final, void* workspace,
+                         size_t workspace_bytes, kda_stream_t stream) {
+  kda_status st = check_forward(q, k, v, g, beta, S0, cu_seqlens, num_seqs,
+                                total_tokens, max_seqlen, H, dk, dv, dt, chunk,
+                                o, S_final, workspace, workspace_bytes);
+  if (st != KDA_OK) return st;
+  kda::ForwardArgs a{q, k, v, nullptr, beta, nullptr, g, S0, cu_seqlens, o,
+                     S_final, num_seqs, total_tokens, max_seqlen, H, dk, dv,
+                     chunk, dt == KDA_BF16, workspace, workspace_bytes,
+                     (cudaStream_t)stream};
+  return forward_common(a);
+}
+
+kda_status kda_decode_step(const void* q, const void* k, const void* v,
+                           const void* z, const float* A, const void* beta,
+                           float* S_inout, int32_t B, int32_t H, int32_t dk,
+                           int32_t dv, kda_dtype dt, void* o,
+                           kda_stream_t stream) {
+  if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_UNSUPPORTED;
+  if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  if (B < 0 || H < 1) return KDA_ERR_INVALID_ARG;
+  if ((int64_t)B * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+  if (B == 0) return KDA_OK;
+  if (!q || !k || !v || !z || !A || !beta || !S_inout || !o) return KDA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(z) ||
+      !aligned16(A) || !aligned16(beta) || !aligned16(S_inout) || !aligned16(o))
+    return KDA_ERR_INVALID_ARG;
+  kda::DecodeArgs a{q, k, v, z, beta, A, S_inout, o, B, H, dk, dv,
+                    dt == KDA_BF16, (cudaStream_t)stream};
+  return kda::launch_decode(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_check_device_error(const void* workspace, kda_stream_t stream) {
+  if (!workspace || !aligned16(workspace)) return KDA_ERR_INVALID_ARG;
+  uint32_t err = 0;
+  if (cudaMemcpyAsync(&err, workspace, sizeof(err), cudaMemcpyDeviceToHost,
+                      (cudaStream_t)stream) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return KDA_ERR_CUDA;
+  if (err == kda::kErrNone) return KDA_OK;
+  if (err & kda::kErrTimeout) return KDA_ERR_TIMEOUT;
+  return KDA_ERR_INVALID_ARG;
+}
+
+}  // extern "C"

@@ -1,0 +1,145 @@
+// kda_decode.cu -- one recurrent KDA step per (sequence, head), in place.
+//
+// Kimi Linear summary, §6.3: token generation uses the recurrent update; §3:
+//   S' = Diag(alpha) S,  u = beta (v - S'^T k^),  S = S' + k^ u^T,  o = S^T q^.
+// The output is taken as o = S'^T q^ + (k^ . q^) u, which equals S^T q^ for the
+// updated S, so the state is read once and written once: the step is bound by
+// the 2 * dk * dv * 4 bytes of state traffic per (sequence, head).
+//
+// One CTA of 256 threads owns one (b, h) state.  Threads tile the state as
+// (row group, float4 column group) so every warp reads and writes whole
+// contiguous 512-byte rows; the state lives in registers between the load and
+// the store.  Column sums are reduced across row groups through shared memory
+// in a fixed order (deterministic, no atomics).
+#include "kda_common.cuh"
+#include "kda_launch.h"
+
+namespace kda {
+
+template <int DK, int DV, typename T>
+__global__ void __launch_bounds__(256)
+decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k,
+                   const T* __restrict__ v, const T* __restrict__ z,
+                   const float* __restrict__ A, const T* __restrict__ beta,
+                   float* __restrict__ S, int H, T* __restrict__ o) {
+  constexpr int NT = 256;
+  constexpr int CG = DV / 4;   // float4 column groups per state row
+  constexpr int RG = NT / CG;  // row groups
+  constexpr int RPT = DK / RG; // state rows held by one thread
+  static_assert(RG * CG == NT && RPT * RG == DK, "tiling");
+
+  __shared__ __align__(16) float s_k[DK], s_q[DK], s_a[DK], s_v[DV];
+  __shared__ __align__(16) float s_p[RG][DV + 4], s_r[RG][DV + 4];
+  __shared__ __align__(16) float s_u[DV];
+  __shared__ float s_scal[4];
+
+  const int bh = blockIdx.x;
+  const int h = bh % H;
+  const int tid = threadIdx.x;
+  const int cg = tid % CG, rg = tid / CG;
+
+  // Issue the state loads first: they are the whole cost of the step.
+  float4* Sp = reinterpret_cast<float4*>(S + (size_t)bh * DK * DV);
+  float4 s[RPT];
+#pragma unroll
+  for (int m = 0; m < RPT; ++m) s[m] = __ldcs(&Sp[(rg + m * RG) * CG + cg]);
+
+  const float expA = expf(A[h]);
+  for (int i = tid; i < DK; i += NT) {
+    s_k[i] = to_f(k[(size_t)bh * DK + i]);
+    s_q[i] = to_f(q[(size_t)bh * DK + i]);
+    s_a[i] = expf(gate_logdecay(to_f(z[(size_t)bh * DK + i]), expA));
+  }
+  for (int j = tid; j < DV; j += NT) s_v[j] = to_f(v[(size_t)bh * DV + j]);
+  __syncthreads();
+  if (tid < 32) {
+    float kk = 0.f, qq = 0.f, kq = 0.f;
+    for (int i = tid; i < DK; i += 32) {
+      kk += s_k[i] * s_k[i];
+      qq += s_q[i] * s_q[i];
+      kq += s_k[i] * s_q[i];
+    }
+    kk = warp_sum(kk);
+    qq = warp_sum(qq);
+    kq = warp_sum(kq);
+    if (tid == 0) {
+      const float ik = 1.0f / sqrtf(kk + kNormEps);
+      const float iq = 1.0f / sqrtf(qq + kNormEps);
+      s_scal[0] = ik;
+      s_scal[1] = iq;
+      s_scal[2] = kq * ik * iq;  // k^ . q^
+    }
+  }
+  __syncthreads();
+  const float ik = s_scal[0], iq = s_scal[1], kq = s_scal[2];
+
+  // Decay and the two column reductions over this thread's rows.
+  float4 p = make_float4(0.f, 0.f, 0.f, 0.f), r = p;
+#pragma unroll
+  for (int m = 0; m < RPT; ++m) {
+    const int i = rg + m * RG;
+    const float a = s_a[i], kh = s_k[i] * ik, qh = s_q[i] * iq;
+    s[m].x *= a; s[m].y *= a; s[m].z *= a; s[m].w *= a;
+    p.x += kh * s[m].x; p.y += kh * s[m].y; p.z += kh * s[m].z; p.w += kh * s[m].w;
+    r.x += qh * s[m].x; r.y += qh * s[m].y; r.z += qh * s[m].z; r.w += qh * s[m].w;
+  }
+  *reinterpret_cast<float4*>(&s_p[rg][4 * cg]) = p;
+  *reinterpret_cast<float4*>(&s_r[rg][4 * cg]) = r;
+  __syncthreads();
+  const float b = to_f(beta[bh]);
+  for (int j = tid; j < DV; j += NT) {
+    float pj = 0.f, rj = 0.f;
+#pragma unroll
+    for (int g2 = 0; g2 < RG; ++g2) {
+      pj += s_p[g2][j];
+      rj += s_r[g2][j];
+    }
+    const float u = b * (s_v[j] - pj);
+    s_u[j] = u;
+    o[(size_t)bh * DV + j] = from_f<T>(rj + kq * u);
+  }
+  __syncthreads();
+  const float4 u4 = *reinterpret_cast<const float4*>(&s_u[4 * cg]);
+#pragma unroll
+  for (int m = 0; m < RPT; ++m) {
+    const int i = rg + m * RG;
+    const float kh = s_k[i] * ik;
+    float4 w = s[m];
+    w.x += kh * u4.x; w.y += kh * u4.y; w.z += kh * u4.z; w.w += kh * u4.w;
+    __stcs(&Sp[i * CG + cg], w);
+  }
+}
+
+template <int DK, int DV, typename T>
+static cudaError_t launch_decode_t(const DecodeArgs& a) {
+  decode_step_kernel<DK, DV, T><<<a.B * a.H, 256, 0, a.stream>>>(
+      (const T*)a.q, (const T*)a.k, (const T*)a.v, (const T*)a.z, a.A,
+      (const T*)a.beta, a.S, a.H, (T*)a.o);
+  return cudaGetLastError();
+}
+
+template <int DK, int DV>
+static cudaError_t launch_decode_d(const DecodeArgs& a) {
+  return a.bf16 ? launch_decode_t<DK, DV, __nv_bfloat16>(a) : launch_decode_t<DK, DV, float>(a);
+}
+
+template <int DK>
+static cudaError_t launch_decode_k(const DecodeArgs& a) {
+  switch (a.dv) {
+    case 32: return launch_decode_d<DK, 32>(a);
+    case 64: return launch_decode_d<DK, 64>(a);
+    case 128: return launch_decode_d<DK, 128>(a);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode(const DecodeArgs& a) {
+  switch (a.dk) {
+    case 32: return launch_decode_k<32>(a);
+    case 64: return launch_decode_k<64>(a);
+    case 128: return launch_decode_k<128>(a);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace kda

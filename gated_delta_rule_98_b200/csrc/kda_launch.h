@@ -1,0 +1,43 @@
+// kda_launch.h -- host-side launch descriptors shared by the API layer and the
+// kernel translation units (internal; not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace kda {
+
+struct DecodeArgs {
+  const void *q, *k, *v, *z, *beta;
+  const float* A;
+  float* S;
+  void* o;
+  int B, H, dk, dv;
+  bool bf16;
+  cudaStream_t stream;
+};
+
+struct ForwardArgs {
+  const void *q, *k, *v, *z, *beta;
+  const float* A;        // with z
+  const float* g;        // log-decay input (instead of z, A) or nullptr
+  const float* S0;       // nullptr = zeros
+  const int32_t* cu;     // nullptr = equal lengths
+  void* o;
+  float* S_final;        // nullptr = skip
+  int N, T, max_len, H, dk, dv, chunk;
+  bool bf16;
+  void* ws;              // workspace base (header at offset 0)
+  size_t ws_bytes;
+  cudaStream_t stream;
+};
+
+cudaError_t launch_decode(const DecodeArgs& a);
+
+// SIMT (CUDA-core, fp32) chunkwise path: any supported size and dtype.
+size_t simt_workspace_bytes(int N, int T, int H, int dk, int dv, int chunk);
+cudaError_t launch_forward_simt(const ForwardArgs& a);
+int simt_launches(int N, int max_len, int chunk);
+
+}  // namespace kda

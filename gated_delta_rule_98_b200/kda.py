@@ -1,0 +1,215 @@
+"""ctypes binding of the KDA C ABI (include/kda.h, libkda.so).
+
+Argument marshalling only: every step of the operator runs in the library's
+CUDA kernels.  torch is used for device memory (outputs, workspace) and for
+the current CUDA stream.  There is no CPU path: if ``libkda.so`` is missing
+the first call raises, and CPU tensors are rejected.
+
+Low-level functions keep the C names (``kda_forward``, ``kda_forward_g``,
+``kda_decode_step``, ``kda_forward_workspace_size``, ``kda_check_device_error``,
+``kda_status_string``) and take raw pointers/ints.  ``forward``,
+``forward_g``, ``decode_step`` and ``workspace`` are tensor-level helpers.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = 0, -1, -2, -3, -4
+KDA_F32, KDA_BF16 = 0, 1
+
+# Every symbol include/kda.h declares.
+EXPORTS = ("kda_status_string", "kda_version", "kda_forward_workspace_size",
+           "kda_forward_launches", "kda_forward",
+           "kda_forward_g", "kda_decode_step", "kda_check_device_error")
+
+_lib = None
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status, what=""):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+def lib():
+    """Load libkda.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m gated_delta_rule_98_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    L.kda_status_string.argtypes = [ctypes.c_int]
+    L.kda_status_string.restype = ctypes.c_char_p
+    L.kda_version.argtypes = []
+    L.kda_version.restype = i32
+    L.kda_forward_workspace_size.argtypes = [i32] * 6 + [ctypes.c_int, i32]
+    L.kda_forward_workspace_size.restype = sz
+    L.kda_forward_launches.argtypes = [i32] * 6 + [ctypes.c_int, i32]
+    L.kda_forward_launches.restype = i32
+    L.kda_forward.argtypes = [vp] * 8 + [i32] * 6 + [ctypes.c_int, i32, vp, vp, vp, sz, vp]
+    L.kda_forward.restype = ctypes.c_int
+    L.kda_forward_g.argtypes = [vp] * 7 + [i32] * 6 + [ctypes.c_int, i32, vp, vp, vp, sz, vp]
+    L.kda_forward_g.restype = ctypes.c_int
+    L.kda_decode_step.argtypes = [vp] * 7 + [i32] * 4 + [ctypes.c_int, vp, vp]
+    L.kda_decode_step.restype = ctypes.c_int
+    L.kda_check_device_error.argtypes = [vp, vp]
+    L.kda_check_device_error.restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def status_string(s):
+    return lib().kda_status_string(int(s)).decode()
+
+
+# ------------------------------------------------------------ raw C names ---
+
+def kda_forward_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv, dt, chunk):
+    return lib().kda_forward_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv, dt,
+                                            chunk)
+
+
+def kda_forward_launches(num_seqs, total_tokens, max_seqlen, H, dk, dv, dt, chunk):
+    return lib().kda_forward_launches(num_seqs, total_tokens, max_seqlen, H, dk, dv, dt, chunk)
+
+
+def kda_forward(q, k, v, z, A, beta, S0, cu_seqlens, num_seqs, total_tokens, max_seqlen, H,
+                dk, dv, dt, chunk, o, S_final, workspace, workspace_bytes, stream):
+    return lib().kda_forward(q, k, v, z, A, beta, S0, cu_seqlens, num_seqs, total_tokens,
+                             max_seqlen, H, dk, dv, dt, chunk, o, S_final, workspace,
+                             workspace_bytes, stream)
+
+
+def kda_forward_g(q, k, v, g, beta, S0, cu_seqlens, num_seqs, total_tokens, max_seqlen, H,
+                  dk, dv, dt, chunk, o, S_final, workspace, workspace_bytes, stream):
+    return lib().kda_forward_g(q, k, v, g, beta, S0, cu_seqlens, num_seqs, total_tokens,
+                               max_seqlen, H, dk, dv, dt, chunk, o, S_final, workspace,
+                               workspace_bytes, stream)
+
+
+def kda_decode_step(q, k, v, z, A, beta, S_inout, B, H, dk, dv, dt, o, stream):
+    return lib().kda_decode_step(q, k, v, z, A, beta, S_inout, B, H, dk, dv, dt, o, stream)
+
+
+def kda_check_device_error(workspace, stream):
+    return lib().kda_check_device_error(workspace, stream)
+
+
+# ------------------------------------------------------- tensor helpers ---
+
+def _dt(t):
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    if t.dtype == torch.float32:
+        return KDA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("KDA runs on the GPU only: pass CUDA tensors")
+        if t is not None and not t.is_contiguous():
+            raise ValueError("KDA tensors must be contiguous")
+
+
+def _geometry(q, v, cu_seqlens, num_seqs, max_seqlen):
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is None:
+        N = 1 if num_seqs is None else int(num_seqs)
+        L = T // N if N else 0
+        max_len = L if max_seqlen is None else int(max_seqlen)
+    else:
+        N = cu_seqlens.numel() - 1
+        if max_seqlen is None:
+            raise ValueError("max_seqlen is required with cu_seqlens")
+        max_len = int(max_seqlen)
+    return T, H, dk, dv, N, max_len
+
+
+def workspace(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype, chunk, device=None):
+    """A uint8 device tensor of kda_forward_workspace_size() bytes."""
+    nbytes = kda_forward_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv,
+                                        _dt(torch.empty(0, dtype=dtype)), chunk)
+    if nbytes == 0:
+        raise KdaError(KDA_ERR_UNSUPPORTED, "kda_forward_workspace_size")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
+
+
+def _forward(entry, q, k, v, gate_a, gate_b, beta, S0, cu_seqlens, num_seqs, max_seqlen, chunk,
+             o, S_final, ws, stream, want_state):
+    _check_cuda(q, k, v, gate_a, gate_b, beta, S0, cu_seqlens, o, S_final, ws)
+    T, H, dk, dv, N, max_len = _geometry(q, v, cu_seqlens, num_seqs, max_seqlen)
+    dt = _dt(q)
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
+    if S_final is None and want_state:
+        S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(N, T, max_len, H, dk, dv, q.dtype, chunk, device=q.device)
+    args = [_p(q), _p(k), _p(v), _p(gate_a)]
+    if entry == "z":
+        args.append(_p(gate_b))
+    args += [_p(beta), _p(S0), _p(cu_seqlens), N, T, max_len, H, dk, dv, dt, chunk, _p(o),
+             _p(S_final), _p(ws), ws.numel(), _stream(stream)]
+    fn = kda_forward if entry == "z" else kda_forward_g
+    st = fn(*args)
+    if st != KDA_OK:
+        raise KdaError(st, fn.__name__)
+    return o, S_final
+
+
+def forward(q, k, v, z, A, beta, *, S0=None, cu_seqlens=None, num_seqs=None, max_seqlen=None,
+            chunk=64, o=None, S_final=None, workspace=None, stream=None, output_final_state=True):
+    """KDA prefill.  q,k,z [T,H,dk], v [T,H,dv], beta [T,H] (all one dtype),
+    A [H] fp32, S0 [N,H,dk,dv] fp32 or None, cu_seqlens int32 [N+1] or None
+    (then ``num_seqs`` equal sequences).  Returns (o, S_final)."""
+    return _forward("z", q, k, v, z, A, beta, S0, cu_seqlens, num_seqs, max_seqlen, chunk, o,
+                    S_final, workspace, stream, output_final_state)
+
+
+def forward_g(q, k, v, g, beta, *, S0=None, cu_seqlens=None, num_seqs=None, max_seqlen=None,
+              chunk=64, o=None, S_final=None, workspace=None, stream=None,
+              output_final_state=True):
+    """KDA prefill with the fp32 log-decay g [T,H,dk] given directly (g in [-5, 0])."""
+    return _forward("g", q, k, v, g, None, beta, S0, cu_seqlens, num_seqs, max_seqlen, chunk, o,
+                    S_final, workspace, stream, output_final_state)
+
+
+def decode_step(q, k, v, z, A, beta, S, *, o=None, stream=None):
+    """One recurrent step: q,k,z [B,H,dk], v [B,H,dv], beta [B,H]; S [B,H,dk,dv]
+    fp32 is updated in place.  Returns o [B,H,dv]."""
+    _check_cuda(q, k, v, z, A, beta, S, o)
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    st = kda_decode_step(_p(q), _p(k), _p(v), _p(z), _p(A), _p(beta), _p(S), B, H, dk, dv,
+                         _dt(q), _p(o), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_decode_step")
+    return o
+
+
+def check_device_error(ws, stream=None):
+    """Status recorded on the device by the last forward call on ``ws``."""
+    return kda_check_device_error(_p(ws), _stream(stream))

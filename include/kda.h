@@ -1,0 +1,176 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention (KDA) operator.
+ *
+ * The operator (Kimi Linear: An Expressive, Efficient Attention Architecture,
+ * summary, §3 "Kimi Delta Attention"):
+ *
+ *   S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *   o_t = S_t^T q_t
+ *
+ * with the lower-bounded channel-wise gate (Kimi K3 architecture summary,
+ * hybrid KDA / Gated MLA section)
+ *
+ *   g_t = -5 * sigmoid(exp(A_h) * z_t),   alpha_t = exp(g_t)   (per channel)
+ *
+ * and q, k normalised to unit length inside the operator as
+ * x / sqrt(sum x^2 + 1e-6) (Kimi Linear summary, §4).  No 1/sqrt(d) scale is
+ * applied to q.  The memory is decayed before the delta correction, and o_t
+ * reads the state after token t's update.
+ *
+ * Prefill uses the chunkwise form (Kimi Linear summary, §3.1 "Hardware-
+ * Efficient Chunkwise Algorithm"; §6.3 for the chunk size): per-chunk
+ * cumulative log-decay, a WY / UT-transform of the rank-1 updates whose
+ * lower-triangular inverse is formed by forward substitution on 16-token
+ * sub-tiles, a sequential inter-chunk state carry, and the intra-chunk causal
+ * output plus the incoming-state term.  Decode is the recurrent form, one
+ * token per sequence (§6.3).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every tensor pointer is a DEVICE pointer, 16-byte aligned, contiguous,
+ *   row-major.  T = total tokens, N = sequences, H = heads.
+ *     q, k, z : [T, H, dk]      v, o : [T, H, dv]      beta : [T, H]
+ *     A       : [H]    float32
+ *     states  : [N, H, dk, dv]  float32, S[key][value]
+ *   q, k, v, z, beta and o share the element type `dt`.
+ * - Supported sizes: dk, dv in {32, 64, 128}; chunk in {16, 64}; H >= 1.
+ * - The caller owns every buffer, including the workspace.  The library never
+ *   allocates on the call path and keeps no global state between calls; calls
+ *   on different workspaces are independent.
+ * - All calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL
+ *   is the legacy default stream).  Nothing is copied device-to-host.
+ * - Errors that the host can see return synchronously and enqueue nothing:
+ *   KDA_ERR_INVALID_ARG (null pointer, misalignment, inconsistent sizes,
+ *   workspace too small), KDA_ERR_UNSUPPORTED (dims, chunk or dtype outside
+ *   the supported set).  A failed launch returns KDA_ERR_CUDA.  Errors only
+ *   the device can see (a cu_seqlens that is not non-decreasing from 0 to
+ *   total_tokens, or has a length above max_seqlen) are recorded in the
+ *   workspace's error word; the kernels then skip all work (o and S_final
+ *   are left unwritten) and kda_check_device_error() reports
+ *   KDA_ERR_INVALID_ARG.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARG = -1,
+  KDA_ERR_UNSUPPORTED = -2,
+  KDA_ERR_CUDA = -3,
+  KDA_ERR_TIMEOUT = -4
+} kda_status;
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+
+/* Opaque stream handle; pass a cudaStream_t (or NULL). */
+typedef void* kda_stream_t;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char* kda_status_string(kda_status s);
+
+/* Library version as an integer (major*10000 + minor*100 + patch). */
+int32_t kda_version(void);
+
+/*
+ * Bytes of device workspace kda_forward / kda_forward_g need for this
+ * problem.  Returns 0 when the arguments are invalid or unsupported.
+ * max_seqlen bounds every sequence's length; with cu_seqlens == NULL the
+ * batch is num_seqs sequences of max_seqlen tokens each.
+ */
+size_t kda_forward_workspace_size(int32_t num_seqs, int32_t total_tokens,
+                                  int32_t max_seqlen, int32_t H, int32_t dk,
+                                  int32_t dv, kda_dtype dt, int32_t chunk);
+
+/*
+ * Number of kernel launches one kda_forward / kda_forward_g call with these
+ * arguments enqueues (0 when the arguments are invalid or unsupported).
+ */
+int32_t kda_forward_launches(int32_t num_seqs, int32_t total_tokens,
+                             int32_t max_seqlen, int32_t H, int32_t dk,
+                             int32_t dv, kda_dtype dt, int32_t chunk);
+
+/*
+ * Chunkwise KDA prefill over packed sequences.
+ *
+ *  q, k, v, z, beta : inputs in `dt`, layouts above.
+ *  A          : [H] float32, per-head gate scale (the gate uses exp(A_h)).
+ *  S0         : [N, H, dk, dv] float32 initial states; NULL means zeros.
+ *  cu_seqlens : device int32 [N+1] token offsets (0 = cu[0] <= cu[1] <= ...
+ *               <= cu[N] = total_tokens, every length <= max_seqlen), or NULL
+ *               for N equal sequences of max_seqlen tokens
+ *               (total_tokens must then equal num_seqs * max_seqlen).
+ *               The chunk grid restarts at every sequence; the last chunk of a
+ *               sequence may be partial; an empty sequence passes S0 through.
+ *  o          : [T, H, dv] in `dt`, output; must not overlap any input.
+ *  S_final    : [N, H, dk, dv] float32 final states, or NULL to skip.  It may
+ *               equal S0 (in-place state passing); any other overlap with an
+ *               input is undefined.
+ *  chunk      : 16 or 64 tokens (the result does not depend on it beyond
+ *               rounding).
+ *  workspace  : device buffer of at least kda_forward_workspace_size() bytes,
+ *               16-byte aligned; its contents need no initialisation and are
+ *               overwritten.  Do not share one workspace between calls that
+ *               may run concurrently.
+ */
+kda_status kda_forward(const void* q, const void* k, const void* v,
+                       const void* z, const float* A, const void* beta,
+                       const float* S0, const int32_t* cu_seqlens,
+                       int32_t num_seqs, int32_t total_tokens,
+                       int32_t max_seqlen, int32_t H, int32_t dk, int32_t dv,
+                       kda_dtype dt, int32_t chunk, void* o, float* S_final,
+                       void* workspace, size_t workspace_bytes,
+                       kda_stream_t stream);
+
+/*
+ * Same operator with the log-decay given directly instead of (z, A):
+ *  g : [T, H, dk] float32 log-decay, alpha = exp(g).
+ * Precondition g in [-5, 0] (the range the gate produces); outside it the
+ * 16-token sub-tile rescaling loses its overflow guarantee and results are
+ * undefined (not checked).  g = 0 gives DeltaNet (Kimi Linear summary §2.2);
+ * g equal across a head's channels gives Gated DeltaNet's scalar gate.
+ */
+kda_status kda_forward_g(const void* q, const void* k, const void* v,
+                         const float* g, const void* beta, const float* S0,
+                         const int32_t* cu_seqlens, int32_t num_seqs,
+                         int32_t total_tokens, int32_t max_seqlen, int32_t H,
+                         int32_t dk, int32_t dv, kda_dtype dt, int32_t chunk,
+                         void* o, float* S_final, void* workspace,
+                         size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * One recurrent KDA step for B independent sequences (one token each),
+ * updating the float32 states in place (Kimi Linear summary §6.3: token
+ * generation uses the recurrent update).
+ *
+ *  q, k, z : [B, H, dk] in `dt`;  v : [B, H, dv];  beta : [B, H];
+ *  A       : [H] float32;
+ *  S_inout : [B, H, dk, dv] float32, read and overwritten with the new state;
+ *  o       : [B, H, dv] in `dt`, must not overlap any input.
+ * No workspace is needed; the call has no device-side error paths.
+ */
+kda_status kda_decode_step(const void* q, const void* k, const void* v,
+                           const void* z, const float* A, const void* beta,
+                           float* S_inout, int32_t B, int32_t H, int32_t dk,
+                           int32_t dv, kda_dtype dt, void* o,
+                           kda_stream_t stream);
+
+/*
+ * Reads the workspace's error word of the most recent kda_forward /
+ * kda_forward_g call on that workspace (synchronises `stream`).  Returns
+ * KDA_OK, KDA_ERR_INVALID_ARG (bad cu_seqlens seen on the device),
+ * KDA_ERR_TIMEOUT (a bounded device wait gave up) or KDA_ERR_CUDA.
+ */
+kda_status kda_check_device_error(const void* workspace, kda_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,115 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/kda.h declares, sizes workspaces, and rejects bad
+arguments synchronously (before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_98_b200 import kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from gated_delta_rule_98_b200 import build
+    build.build()
+    return kda.lib()
+
+
+def declared_entry_points():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(kda_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+def test_exports_every_declared_symbol(L):
+    declared = declared_entry_points()
+    assert declared >= {"kda_forward", "kda_decode_step", "kda_forward_workspace_size"}
+    for name in declared:
+        assert hasattr(L, name), f"libkda.so does not export {name}"
+    assert set(kda.EXPORTS) == declared
+
+
+def test_status_strings(L):
+    for s, name in [(0, "KDA_OK"), (-1, "KDA_ERR_INVALID_ARG"), (-2, "KDA_ERR_UNSUPPORTED"),
+                    (-3, "KDA_ERR_CUDA"), (-4, "KDA_ERR_TIMEOUT")]:
+        assert kda.status_string(s) == name
+    assert L.kda_version() >= 100
+
+
+def test_workspace_size(L):
+    ws = kda.kda_forward_workspace_size
+    assert ws(1, 4096, 4096, 16, 128, 128, kda.KDA_BF16, 64) > 0
+    assert ws(1, 4096, 4096, 16, 128, 128, kda.KDA_BF16, 64) >= \
+        ws(1, 2048, 2048, 16, 128, 128, kda.KDA_BF16, 64)
+    assert ws(1, 64, 64, 2, 48, 32, kda.KDA_F32, 16) == 0       # unsupported dk
+    assert ws(1, 64, 64, 2, 32, 32, kda.KDA_F32, 32) == 0       # unsupported chunk
+    assert ws(1, 64, 64, 2, 32, 32, 7, 16) == 0                 # unsupported dtype
+    assert ws(-1, 64, 64, 2, 32, 32, kda.KDA_F32, 16) == 0
+    assert ws(0, 0, 0, 2, 32, 32, kda.KDA_F32, 16) > 0          # empty problem: header only
+
+
+FAKE = 0x10000  # aligned fake device address: never dereferenced by these calls
+
+
+def _fwd(**over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, z=FAKE, A=FAKE, beta=FAKE, S0=None, cu=None, N=1, T=64,
+             L=64, H=2, dk=32, dv=32, dt=kda.KDA_F32, chunk=16, o=FAKE, Sf=FAKE, ws=FAKE,
+             wsb=1 << 40, stream=None)
+    a.update(over)
+    return kda.kda_forward(a["q"], a["k"], a["v"], a["z"], a["A"], a["beta"], a["S0"], a["cu"],
+                           a["N"], a["T"], a["L"], a["H"], a["dk"], a["dv"], a["dt"], a["chunk"],
+                           a["o"], a["Sf"], a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("over,want", [
+    (dict(q=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(z=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(A=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(o=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(ws=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(wsb=16), kda.KDA_ERR_INVALID_ARG),
+    (dict(q=FAKE + 8), kda.KDA_ERR_INVALID_ARG),
+    (dict(beta=FAKE + 2), kda.KDA_ERR_INVALID_ARG),
+    (dict(ws=FAKE + 4), kda.KDA_ERR_INVALID_ARG),
+    (dict(T=65), kda.KDA_ERR_INVALID_ARG),          # T != N * max_seqlen without cu_seqlens
+    (dict(H=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(N=-1), kda.KDA_ERR_INVALID_ARG),
+    (dict(dk=48), kda.KDA_ERR_UNSUPPORTED),
+    (dict(dv=256), kda.KDA_ERR_UNSUPPORTED),
+    (dict(chunk=32), kda.KDA_ERR_UNSUPPORTED),
+    (dict(dt=5), kda.KDA_ERR_UNSUPPORTED),
+])
+def test_forward_rejects_bad_arguments(L, over, want):
+    assert _fwd(**over) == want
+
+
+def test_forward_g_and_decode_reject_bad_arguments(L):
+    st = kda.kda_forward_g(FAKE, FAKE, FAKE, None, FAKE, None, None, 1, 64, 64, 2, 32, 32,
+                           kda.KDA_F32, 16, FAKE, None, FAKE, 1 << 40, None)
+    assert st == kda.KDA_ERR_INVALID_ARG
+    dec = kda.kda_decode_step
+    assert dec(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 4, 2, 32, 32, kda.KDA_F32, FAKE,
+               None) == kda.KDA_ERR_INVALID_ARG
+    assert dec(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 96, 32, kda.KDA_F32, FAKE,
+               None) == kda.KDA_ERR_UNSUPPORTED
+    assert dec(FAKE + 4, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 2, 32, 32, kda.KDA_F32, FAKE,
+               None) == kda.KDA_ERR_INVALID_ARG
+    # B = 0 is a no-op that touches nothing
+    assert dec(None, None, None, None, None, None, None, 0, 2, 32, 32, kda.KDA_F32, None,
+               None) == kda.KDA_OK
+    assert kda.kda_check_device_error(None, None) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_binding_rejects_cpu_tensors(L):
+    import torch
+    q = torch.zeros(4, 1, 32)
+    with pytest.raises(ValueError):
+        kda.decode_step(q, q, q, q, torch.zeros(1), torch.zeros(4, 1), torch.zeros(4, 1, 32, 32))
