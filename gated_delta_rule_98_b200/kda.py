@@ -26,7 +26,10 @@ KDA_F32, KDA_BF16 = 0, 1
 # Every symbol include/kda.h declares.
 EXPORTS = ("kda_status_string", "kda_version", "kda_forward_workspace_size",
            "kda_forward_launches", "kda_forward",
-           "kda_forward_g", "kda_decode_step", "kda_check_device_error")
+           "kda_forward_g", "kda_decode_step", "kda_forward_noalloc", "kda_check_device_error")
+
+# Bytes of the library's fixed scratch array used by kda_forward_noalloc.
+KDA_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
 
@@ -61,6 +64,8 @@ def lib():
     L.kda_forward_g.restype = ctypes.c_int
     L.kda_decode_step.argtypes = [vp] * 7 + [i32] * 4 + [ctypes.c_int, vp, vp]
     L.kda_decode_step.restype = ctypes.c_int
+    L.kda_forward_noalloc.argtypes = [vp] * 8 + [i32] * 6 + [ctypes.c_int, i32, vp, vp, vp]
+    L.kda_forward_noalloc.restype = ctypes.c_int
     L.kda_check_device_error.argtypes = [vp, vp]
     L.kda_check_device_error.restype = ctypes.c_int
     _lib = L
@@ -98,6 +103,15 @@ def kda_forward_g(q, k, v, g, beta, S0, cu_seqlens, num_seqs, total_tokens, max_
 
 def kda_decode_step(q, k, v, z, A, beta, S_inout, B, H, dk, dv, dt, o, stream):
     return lib().kda_decode_step(q, k, v, z, A, beta, S_inout, B, H, dk, dv, dt, o, stream)
+
+
+def kda_forward_noalloc(q, k, v, z, A, beta, S0, cu_seqlens, num_seqs, total_tokens,
+                        max_seqlen, H, dk, dv, dt, chunk, o, S_final, stream):
+    """kda_forward on the library's fixed scratch array (no workspace argument).
+    For callers that cannot allocate device memory; see include/kda.h."""
+    return lib().kda_forward_noalloc(q, k, v, z, A, beta, S0, cu_seqlens, num_seqs,
+                                     total_tokens, max_seqlen, H, dk, dv, dt, chunk, o, S_final,
+                                     stream)
 
 
 def kda_check_device_error(workspace, stream):

@@ -162,6 +162,44 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v,
                            kda_stream_t stream);
 
 /*
+ * kda_forward without a caller-provided workspace, for callers that cannot
+ * allocate device memory.  No passage of the pages corresponds to this entry
+ * point; it exists for integration only.
+ *
+ * Who needs it: a host whose device memory is owned by another allocator (a
+ * framework pool that reserved the GPU's memory up front, so a new cudaMalloc
+ * fails or fragments it), and code that must not call the CUDA allocator at
+ * all, since cudaMalloc/cudaFree can synchronise the whole device.
+ *
+ * Arguments and results are those of kda_forward, minus the workspace.  The
+ * scratch comes from one fixed array of KDA_NOALLOC_SCRATCH_BYTES in device
+ * memory that the library defines at file scope; it is held on every GPU
+ * where the entry point is used, until the process exits.  The call itself
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *  - Problems needing more scratch than KDA_NOALLOC_SCRATCH_BYTES (see
+ *    kda_forward_workspace_size) are rejected with KDA_ERR_UNSUPPORTED before
+ *    anything is enqueued; use kda_forward with your own workspace instead.
+ *  - The first call on a device, made with that device current, looks up the
+ *    array's device address (cudaGetSymbolAddress) and caches it; make that
+ *    first call before any stream capture begins on that device.
+ *  - Every call on a device shares the one array, and it keeps the previous
+ *    call's contents (nothing in it needs to start at zero).  Calls whose GPU
+ *    work may overlap -- different streams, or different host threads without
+ *    ordering -- race on it: order them on one stream.
+ *  - A bad cu_seqlens seen on the device is recorded in the shared array,
+ *    where it cannot be queried: validate cu_seqlens beforehand.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+kda_status kda_forward_noalloc(const void* q, const void* k, const void* v,
+                               const void* z, const float* A, const void* beta,
+                               const float* S0, const int32_t* cu_seqlens,
+                               int32_t num_seqs, int32_t total_tokens,
+                               int32_t max_seqlen, int32_t H, int32_t dk,
+                               int32_t dv, kda_dtype dt, int32_t chunk,
+                               void* o, float* S_final, kda_stream_t stream);
+
+/*
  * Reads the workspace's error word of the most recent kda_forward /
  * kda_forward_g call on that workspace (synchronises `stream`).  Returns
  * KDA_OK, KDA_ERR_INVALID_ARG (bad cu_seqlens seen on the device),
