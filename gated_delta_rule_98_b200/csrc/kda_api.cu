@@ -10,6 +10,12 @@
 namespace {
 
 bool dim_ok(int32_t d) { return d == 32 || d == 64 || d == 128; }
+
+// The tensor-core path serves bf16 inputs with dk = dv = 128 and 64-token
+// chunks; every other supported case runs on the fp32 CUDA-core path.
+bool use_tc(kda_dtype dt, int32_t dk, int32_t dv, int32_t chunk) {
+  return dt == KDA_BF16 && dk == 128 && dv == 128 && chunk == 64;
+}
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 bool opt_aligned16(const void* p) { return p == nullptr || aligned16(p); }
 
@@ -50,7 +56,9 @@ kda_status forward_common(kda::ForwardArgs& a) {
     return cudaMemsetAsync(a.ws, 0, sizeof(uint32_t), a.stream) == cudaSuccess ? KDA_OK
                                                                                : KDA_ERR_CUDA;
   }
-  cudaError_t err = kda::launch_forward_simt(a);
+  cudaError_t err = use_tc(a.bf16 ? KDA_BF16 : KDA_F32, a.dk, a.dv, a.chunk)
+                        ? kda::launch_forward_tc(a)
+                        : kda::launch_forward_simt(a);
   return err == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -77,6 +85,8 @@ size_t kda_forward_workspace_size(int32_t num_seqs, int32_t total_tokens,
   if (dt != KDA_F32 && dt != KDA_BF16) return 0;
   if (!dim_ok(dk) || !dim_ok(dv) || (chunk != 16 && chunk != 64)) return 0;
   if (num_seqs < 0 || total_tokens < 0 || max_seqlen < 0 || H < 1) return 0;
+  if (use_tc(dt, dk, dv, chunk))
+    return kda::tc_workspace_bytes(num_seqs, total_tokens, H, max_seqlen);
   return kda::simt_workspace_bytes(num_seqs, total_tokens, H, dk, dv, chunk);
 }
 
@@ -86,6 +96,7 @@ int32_t kda_forward_launches(int32_t num_seqs, int32_t total_tokens,
   if (kda_forward_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv, dt, chunk) == 0)
     return 0;
   if (num_seqs == 0) return 0;  // a memset only
+  if (use_tc(dt, dk, dv, chunk)) return kda::tc_launches(num_seqs, H, max_seqlen);
   return kda::simt_launches(num_seqs, max_seqlen, chunk);
 }
 

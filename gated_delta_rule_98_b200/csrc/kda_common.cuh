@@ -48,6 +48,30 @@ struct ChunkInfo {
   int32_t first;  // 1 if this is the sequence's first chunk
 };
 
+// Token range [a, b) of sequence n: from cu_seqlens, or n * L for equal lengths.
+__device__ __forceinline__ void seq_bounds(const int32_t* cu, int n, int L, int& a, int& b) {
+  if (cu) {
+    a = cu[n];
+    b = cu[n + 1];
+  } else {
+    a = n * L;
+    b = a + L;
+  }
+}
+
+// Every CTA checks the whole cu_seqlens (0 = cu[0] <= ... <= cu[N] = T, every
+// length <= max_len), so all CTAs of a launch agree on skipping.  Block-wide.
+__device__ __forceinline__ bool seqlens_valid(const int32_t* cu, int N, int T, int max_len) {
+  if (!cu) return true;
+  int bad = 0;
+  for (int n = threadIdx.x; n < N; n += blockDim.x) {
+    const int a = cu[n], b = cu[n + 1];
+    if (b < a || b - a > max_len) bad = 1;
+  }
+  if (threadIdx.x == 0 && (cu[0] != 0 || cu[N] != T)) bad = 1;
+  return __syncthreads_or(bad) == 0;
+}
+
 // Workspace header (offset 0, 256 bytes).
 struct WsHeader {
   uint32_t err;

@@ -40,4 +40,11 @@ size_t simt_workspace_bytes(int N, int T, int H, int dk, int dv, int chunk);
 cudaError_t launch_forward_simt(const ForwardArgs& a);
 int simt_launches(int N, int max_len, int chunk);
 
+// Tensor-core (tcgen05) chunkwise path: bf16, dk = dv = 128, chunk = 64.
+bool tc_supported(const ForwardArgs& a);
+int tc_segments(int N, int H, int max_len);
+size_t tc_workspace_bytes(int N, int T, int H, int max_len);
+int tc_launches(int N, int H, int max_len);
+cudaError_t launch_forward_tc(const ForwardArgs& a);
+
 }  // namespace kda

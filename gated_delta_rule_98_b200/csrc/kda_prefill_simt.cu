@@ -60,28 +60,6 @@ struct SimtParams {
   WsHeader* hdr;
 };
 
-__device__ __forceinline__ void seq_bounds(const int32_t* cu, int n, int L, int& a, int& b) {
-  if (cu) {
-    a = cu[n];
-    b = cu[n + 1];
-  } else {
-    a = n * L;
-    b = a + L;
-  }
-}
-
-// Every CTA checks the whole cu_seqlens, so all CTAs agree on skipping.
-__device__ bool seqlens_valid(const int32_t* cu, int N, int T, int max_len) {
-  if (!cu) return true;
-  int bad = 0;
-  for (int n = threadIdx.x; n < N; n += blockDim.x) {
-    const int a = cu[n], b = cu[n + 1];
-    if (b < a || b - a > max_len) bad = 1;
-  }
-  if (threadIdx.x == 0 && (cu[0] != 0 || cu[N] != T)) bad = 1;
-  return __syncthreads_or(bad) == 0;
-}
-
 template <int DK, int DV, int C>
 constexpr size_t prep_smem_floats() {
   return 3 * C * (DK + 1) + C * (DV + 1) + 3 * C * (C + 1) + C + (C / kSubTile) * 256;

@@ -65,10 +65,11 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row():
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
+    # fp32 inputs take the CUDA-core path, whose scratch grows with the tokens
     T, H, D = 1 << 16, 16, 128
-    need = kda.kda_forward_workspace_size(1, T, T, H, D, D, kda.KDA_BF16, 64)
+    need = kda.kda_forward_workspace_size(1, T, T, H, D, D, kda.KDA_F32, 64)
     assert need > kda.KDA_NOALLOC_SCRATCH_BYTES
     fake = ctypes.c_void_p(0x10000)  # never dereferenced: the size check comes first
     st = kda.kda_forward_noalloc(fake, fake, fake, fake, fake, fake, None, None, 1, T, T, H, D, D,
-                                 kda.KDA_BF16, 64, fake, fake, None)
+                                 kda.KDA_F32, 64, fake, fake, None)
     assert st == kda.KDA_ERR_UNSUPPORTED
