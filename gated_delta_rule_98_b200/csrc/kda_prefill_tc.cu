@@ -1,29 +1,32 @@
 // kda_prefill_tc.cu -- chunkwise KDA prefill on the sm_100a tensor cores
 // (tcgen05.mma, TMEM accumulators), bf16 inputs, dk = dv = 128, chunk = 64.
 //
-// One CTA of 256 threads runs one (sequence, head) over its chunks in order
-// (Kimi Linear summary §3.1: chunkwise WY / UT form with an inter-chunk state
-// carry; §3.2: sub-chunking keeps the channel-wise decay factors in range;
-// Appendix C: per-chunk cumulative log-decay, forward-substitution inverse).
-// The fp32 state S [dk x dv] lives in Tensor Memory for the whole sequence.
-// Per 64-token chunk, with Gam = chunk-local inclusive cumsum of the gate g:
+// One CTA of 256 threads runs one (sequence, head, segment) over its chunks in
+// order (Kimi Linear summary §3.1: chunkwise WY / UT form with an inter-chunk
+// state carry; §3.2: sub-chunking keeps the channel-wise decay factors in
+// range; Appendix C: per-chunk cumulative log-decay, forward-substitution
+// inverse).  The fp32 state S [dk x dv] stays in Tensor Memory.  Per 64-token
+// chunk, with Gam = chunk-local inclusive cumsum of the gate g:
 //
 //   products  A_kk = StrictTril(Diag(beta) K K^T (decayed)), A_qk = Tril(Q K^T
 //             (decayed)), from four M=64 MMAs: for row sub-tile b (16 tokens,
 //             reference rho_b = Gam at its first token) the rows carry
 //             E = e^{Gam_r - rho_b} <= 1 and the column operand C_b carries
 //             e^{rho_b - Gam_i} (<= e^75 on the diagonal sub-tile, <= 1 before)
-//   inverse   T = (I + A_kk)^{-1} by forward substitution on 16x16 diagonal
-//             blocks plus block combination (fp32, CUDA cores)
+//   inverse   T = (I + A_kk)^{-1}: forward substitution in registers on the
+//             16x16 diagonal blocks, then the blocks below the diagonal by
+//             T_ba = -T_bb sum_{a<=c<b} A_bc T_ca (fp32, CUDA cores)
 //   WY        [W | U~] = T [Diag(beta)(K e^Gam) | Diag(beta) V]   (one MMA)
-//   chain     D1 = [W ; Q e^Gam] S      (rows 0-63: W S, rows 64-127: Q' S)
-//             U  = U~ - D1[0:64]
-//             S  = Diag(e^{Gam_last}) S + (K e^{Gam_last - Gam})^T U
-//             O  = D1[64:128] + A_qk U
+//   chain     D_W = W S, D_Q = (Q e^Gam) S, U = U~ - D_W,
+//             S = Diag(e^{Gam_last}) S + (K e^{Gam_last - Gam})^T U,
+//             O = D_Q + A_qk U
 //
-// MMA operands are bf16 in shared memory (no swizzle, 8x16-byte core
-// matrices); every accumulator is fp32 in TMEM.  Rows of a partial chunk past
-// the sequence end are zero, so they contribute nothing.
+// Inputs arrive by TMA (3-D tensor maps over [T, H, 128], one 64x128 box per
+// tensor and chunk), prefetched one chunk ahead.  MMA operands are bf16 in
+// shared memory (no swizzle, 8 x 16-byte core matrices); each operand's major
+// order is chosen so that the threads that produce it store 16-byte vectors of
+// 8 consecutive tokens.  Accumulators are fp32 in TMEM.  Rows of a partial
+// chunk past the sequence end are zero, so they contribute nothing.
 //
 // Segments: with P > 1 a sequence is cut into P runs of chunks.  The
 // transition pass (mode 1) runs each segment but the last from a zero state
@@ -33,6 +36,9 @@
 // incoming state and writes the outputs.  This is the single-GPU form of the
 // prefix scan over per-segment state updates (Kimi K3 architecture summary,
 // KDA context parallelism).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "kda_common.cuh"
 #include "kda_launch.h"
 #include "tc_sm100.cuh"
@@ -46,51 +52,48 @@ constexpr int kC = 64;    // chunk tokens
 constexpr int kD = 128;   // dk = dv
 constexpr int kNT = 256;  // threads
 
-// ---- shared memory map (bytes) ----
-// Region P is reused through a chunk: R + C (products) | A_kk, T (fp32) |
-// [X_K | X_V] (WY operand) | U (chain operand).
-constexpr int kOffR = 0;               // 128 rows x 128 (K-major): sub-tile b rows 32b..32b+15 = K, +16..31 = Q
-constexpr int kOffC = 32768;           // 160 rows x 128 (K-major): C_b at rows 0,16,48,96
-constexpr int kOffAkk = 0;             // fp32 [64][65]
-constexpr int kOffT = 16640;           // fp32 [64][65]
-constexpr int kOffX = 0;               // 256 (N) x 64 (K) MN-major bf16
-constexpr int kOffU = 0;               // 128 (N) x 64 (K) MN-major bf16 (transition pass: 256 x 64)
-constexpr int kSizeP = 73728;
-constexpr int kOffA3 = kSizeP;         // 128 x 64 K-major: rows 0-63 zero, 64-127 A_qk
-constexpr int kOffTp = kOffA3 + 16384; // 128 x 64 K-major: rows 0-63 T, 64-127 zero
-constexpr int kOffA1 = kOffTp + 16384; // 128 x 128 K-major: rows 0-63 W, 64-127 Q'
-constexpr int kOffKp = kOffA1 + 32768; // K': M=128 (dk) x K=64 (tok) MN-major
-constexpr int kOffSb = kOffKp + 16384; // S bf16: N=128 (dv) x K=128 (dk) MN-major (transition: N=256)
-constexpr int kSizeSb = 65536;
-constexpr int kOffVec = kOffSb + kSizeSb;
-// vectors (floats)
+// ---- shared memory map (bytes), per pass ----
+template <int MODE>
+struct Smem {
+  static constexpr int kSb = 0;                                 // S (| X) bf16, B operand, MN-major
+  static constexpr int kSizeSb = MODE == 0 ? 32768 : 65536;
+  static constexpr int kRaw = kSb + kSizeSb;                    // q | k | z | v, [64][128] bf16
+  static constexpr int kP = kRaw + 65536;                       // region P, reused through a chunk:
+  static constexpr int kR = kP;                                 //   R   B op (N=128, K=128) MN-major
+  static constexpr int kCc = kP + 32768;                        //   C   A op (M=160, K=128) MN-major
+  static constexpr int kAkk = kP;                               //   A_kk fp32 [64][65]
+  static constexpr int kTf = kP + 16640;                        //   T    fp32 [64][65]
+  static constexpr int kX = kP;                                 //   X   B op (N=256, K=64) K-major
+  static constexpr int kQp = kP + 32768;                        //   Q'  A op (M=64, K=128) MN-major
+  static constexpr int kKp = kP + 49152;                        //   K'  A op (M=128, K=64) K-major
+  static constexpr int kW = kP;                                 //   W   A op (M=64, K=128) K-major
+  static constexpr int kU = kP;                                 //   U   B op (N=128|256, K=64) MN-major
+  static constexpr int kTop = kP + 73728;                       // T   A op (M=64, K=64) K-major
+  static constexpr int kA3 = kTop + 8192;                       // A_qk A op (M=64, K=64) MN-major
+  static constexpr int kVec = kA3 + (MODE == 0 ? 8192 : 0);
+  static constexpr int kBytes = kVec + 2176 * 4 + 64;
+};
+// vectors (floats) at Smem::kVec
 constexpr int kVecIq = 0, kVecIk = 64, kVecBeta = 128, kVecGam = 192, kVecRho = 320,
-              kVecTot = 832, kVecGlast = 960, kVecX = 1088, kVecEnd = 1088 + 1024;
-constexpr int kSmemBytes = kOffVec + kVecEnd * 4 + 64;
+              kVecTot = 832, kVecGlast = 960, kVecY = 1088;  // Y: 2 x 16 x 33 or 32 x 33 floats
 
-// TMEM columns
-constexpr uint32_t kTmWU = 0;    // [W | U~] (256 columns, rows 0-63 valid)
-constexpr uint32_t kTmD1 = 256;  // chain product (128 columns); A products during prep
-constexpr uint32_t kTmS = 384;   // fp32 state (128 columns)
-// transition pass: the identity-propagated block X uses columns 384..511 as
-// the state's partner, and the state moves to 256..383; see tc_kernel.
+// TMEM columns.  M=64 accumulators put row r in lane 32 (r / 16) + r % 16.
+constexpr uint32_t kTmA = 0;     // A products, 4 x 32 columns (prep)
+constexpr uint32_t kTmWU = 0;    // [W | U~]: 256 columns (after the products are read)
+constexpr uint32_t kTmW = 0;     // D_W = W S (128, or 256 for W [S | X])
+constexpr uint32_t kTmQ = 128;   // D_Q = Q' S (+ A_qk U)
+constexpr uint32_t kTmS = 256;   // fp32 state; identity-started block X at 384 (transition)
 
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s: a wait this long is a fault
 
-__device__ __forceinline__ uint32_t km128(int row, int k) {
-  return (row >> 3) * 2048 + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2;
+// 16-byte-vector layouts of bf16 operands
+__device__ __forceinline__ uint32_t kmaj(int row, int k, int sbo) {
+  return (row >> 3) * sbo + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2;
 }
-__device__ __forceinline__ uint32_t km64(int row, int k) {
-  return (row >> 3) * 1024 + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2;
-}
-template <int E>
-__device__ __forceinline__ uint32_t mnm(int m, int k) {
-  return (m >> 3) * 128 + (k >> 3) * (E / 8 * 128) + (k & 7) * 16 + (m & 7) * 2;
+__device__ __forceinline__ uint32_t mnmaj(int mn, int k, int lbo) {
+  return (mn >> 3) * 128 + (k >> 3) * lbo + (k & 7) * 16 + (mn & 7) * 2;
 }
 
-__device__ __forceinline__ void st_bf16(unsigned char* base, uint32_t off, float x) {
-  *reinterpret_cast<__nv_bfloat16*>(base + off) = __float2bfloat16_rn(x);
-}
 __device__ __forceinline__ uint4 pack8(const float* v) {
   uint4 u;
   __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]),
@@ -101,16 +104,19 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
   u.w = *reinterpret_cast<uint32_t*>(&d);
   return u;
 }
+__device__ __forceinline__ void st16(unsigned char* base, uint32_t off, const float* v) {
+  *reinterpret_cast<uint4*>(base + off) = pack8(v);
+}
 
-struct TcParams {
-  const __nv_bfloat16 *q, *k, *v, *z, *beta;
+struct alignas(64) TcParams {
+  CUtensorMap tq, tk, tz, tv;  // [T, H, 128] bf16, box 64 x 1 x 128
+  const __nv_bfloat16* beta;
   const float *A, *g, *S0;
   const int32_t* cu;
   __nv_bfloat16* o;
   float* S_final;
   int N, T, max_len, H, P;
-  float* seg;  // per (n, h, p): transition M [dk][dk] and offset N [dk][dv] (mode 1 output),
-               // incoming state S_in [dk][dv] (composition output, mode 0 input)
+  float* seg;  // per (n, h): transitions (M, N) of segments 0..P-2, incoming states of 0..P-1
   WsHeader* hdr;
 };
 
@@ -121,9 +127,6 @@ __device__ __forceinline__ void segment_chunks(int nch, int P, int p, int& c0, i
   c1 = min(nch, c0 + G);
 }
 
-// Layout of the segment workspace (floats), per (n, h):
-//   trans[p] (p < P-1): M then N, 2 * dk * dv each
-//   sin[p]   (p >= 1) : dk * dv
 __device__ __forceinline__ float* seg_trans(float* seg, int n, int h, int H, int P, int p) {
   const size_t per = (size_t)(P - 1) * 2 * kD * kD + (size_t)P * kD * kD;
   return seg + ((size_t)n * H + h) * per + (size_t)p * 2 * kD * kD;
@@ -133,16 +136,62 @@ __device__ __forceinline__ float* seg_sin(float* seg, int n, int h, int H, int P
   return seg + ((size_t)n * H + h) * per + (size_t)(P - 1) * 2 * kD * kD + (size_t)p * kD * kD;
 }
 
+// One TMA box (64 tokens x 1 head x 128 channels) of a [T, H, 128] tensor.
+__device__ __forceinline__ void tma_box(void* dst, const CUtensorMap* map, int h, int tok0,
+                                        uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(h), "r"(tok0), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// q, k, z, v rows of the chunk starting at tok0 (single thread).
+__device__ __forceinline__ void stage_chunk(const TcParams& p, unsigned char* raw, uint64_t* bar,
+                                            int tok0, int h) {
+  mbar_arrive_expect_tx(bar, 4 * 16384);
+  tma_box(raw + 0 * 16384, &p.tq, h, tok0, bar);
+  tma_box(raw + 1 * 16384, &p.tk, h, tok0, bar);
+  tma_box(raw + 2 * 16384, &p.tz, h, tok0, bar);
+  tma_box(raw + 3 * 16384, &p.tv, h, tok0, bar);
+}
+
+__device__ __forceinline__ float raw_at(const unsigned char* raw, int t, int r, int c) {
+  return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(raw + t * 16384 + r * 256)[c]);
+}
+
+// Block-wide bounded wait on an mbarrier phase; false if it timed out (the
+// error word then carries kErrTimeout).
+__device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t& phase, WsHeader* hdr) {
+  const bool got = mbar_wait_cycles(bar, phase, kWaitCycles);
+  phase ^= 1;
+  if (__syncthreads_or(!got)) {
+    if (threadIdx.x == 0) atomicOr(&hdr->err, kErrTimeout);
+    return false;
+  }
+  fence_after_sync();
+  return true;
+}
+
+__device__ __forceinline__ void sync_for_mma() {
+  fence_async_smem();
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+}
+
 // ---------------------------------------------------------------------------
 // MODE 0: full pass from the true incoming state, writes o and S_final.
 // MODE 1: transition pass of segments 0..P-2: from S = 0 (N) and X = I (M).
 template <int MODE>
-__global__ void __launch_bounds__(kNT, 1) tc_kernel(TcParams p) {
+__global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcParams p) {
+  using L = Smem<MODE>;
   extern __shared__ __align__(1024) unsigned char sm[];
-  __shared__ uint64_t s_bar;
+  __shared__ uint64_t s_bar, s_bar_raw;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
-  float* vec = reinterpret_cast<float*>(sm + kOffVec);
+  float* vec = reinterpret_cast<float*>(sm + L::kVec);
+  unsigned char* raw = sm + L::kRaw;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = blockIdx.x, h = blockIdx.y, seg = blockIdx.z;
@@ -157,60 +206,63 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(TcParams p) {
   const int nch = (b - a + kC - 1) / kC;
   int c0, c1;
   segment_chunks(nch, p.P, seg, c0, c1);
-  // MODE 1: the last segment needs no transition; empty segments have M = I, N = 0
-  if (MODE == 1 && seg >= p.P - 1) return;
 
-  // ---- set-up: TMEM, barrier, constant zero blocks
+  // ---- set-up: TMEM, barriers, first chunk's rows
   if (warp == 0) {
     tmem_alloc(&s_tmem, 512);
     tmem_relinquish();
   }
   if (tid == 0) {
     mbar_init(&s_bar, 1);
+    mbar_init(&s_bar_raw, 1);
     fence_mbar_init();
     s_abort = 0;
-  }
-  for (int e = tid * 16; e < 16384; e += kNT * 16) {
-    *reinterpret_cast<uint4*>(sm + kOffA3 + e) = make_uint4(0, 0, 0, 0);
-    *reinterpret_cast<uint4*>(sm + kOffTp + e) = make_uint4(0, 0, 0, 0);
   }
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tm = s_tmem;
-  uint32_t phase = 0;
+  uint32_t phase = 0, phase_raw = 0;
+  bool raw_pending = c0 < c1;  // a TMA load into the staging area is in flight
+  if (tid == 0 && c0 < c1) stage_chunk(p, raw, &s_bar_raw, a + c0 * kC, h);
 
-  // MODE 0: S lives in TMEM columns [384, 512).  MODE 1: the zero-start state
-  // S in [256, 384) and the identity-start block X in [384, 512); the chain
-  // product then uses [0, 256) after W/U~ have been read out.
-  constexpr uint32_t tmS = MODE == 0 ? kTmS : 256;
-  constexpr uint32_t tmA = MODE == 0 ? kTmD1 : 0;  // A products (free columns during prep)
-  const int q4 = warp & 3, ch = warp >> 2;  // TMEM lane quarter, column half
-  const int srow = 32 * q4 + lane;          // dk row held by this thread
+  constexpr int SbN = MODE == 0 ? 128 : 256;  // N extent of the bf16 state operand
+  constexpr int SbL = SbN * 16;               // its K-group stride (LBO)
+  const int q4 = warp & 3, ch = warp >> 2;    // TMEM lane quarter, column half
+  const int srow = 32 * q4 + lane;            // dk row (M=128 accumulators)
+  const int r64 = 16 * q4 + lane;             // token row of M=64 accumulators (lane < 16)
+  const bool m64 = lane < 16;
 
-  // ---- initial state
+  // ---- initial state: S0 (or the composed incoming state), and X = I
   {
     const float* S0 = nullptr;
     if (MODE == 0)
       S0 = seg > 0 ? seg_sin(p.seg, n, h, H, p.P, seg)
                    : (p.S0 ? p.S0 + ((size_t)n * H + h) * kD * kD : nullptr);
+#pragma unroll
     for (int c16 = 0; c16 < 64; c16 += 16) {
       float v16[16];
       const int col = 64 * ch + c16;
+      if (S0) {
+        const float4* src = reinterpret_cast<const float4*>(S0 + (size_t)srow * kD + col);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) v16[i] = S0 ? S0[(size_t)srow * kD + col + i] : 0.f;
-      tmem_st16(tmem_addr(tm, 32 * q4, tmS + col), v16);
+        for (int i = 0; i < 4; ++i) {
+          const float4 f = src[i];
+          v16[4 * i] = f.x; v16[4 * i + 1] = f.y; v16[4 * i + 2] = f.z; v16[4 * i + 3] = f.w;
+        }
+      } else {
 #pragma unroll
-      for (int i = 0; i < 16; i += 8)
-        *reinterpret_cast<uint4*>(sm + kOffSb + mnm<(MODE == 0 ? 128 : 256)>(col + i, srow)) =
-            pack8(v16 + i);
+        for (int i = 0; i < 16; ++i) v16[i] = 0.f;
+      }
+      tmem_st16(tmem_addr(tm, 32 * q4, kTmS + col), v16);
+      st16(sm + L::kSb, mnmaj(col, srow, SbL), v16);
+      st16(sm + L::kSb, mnmaj(col + 8, srow, SbL), v16 + 8);
       if (MODE == 1) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) v16[i] = (col + i == srow) ? 1.f : 0.f;
-        tmem_st16(tmem_addr(tm, 32 * q4, 384 + col), v16);
-#pragma unroll
-        for (int i = 0; i < 16; i += 8)
-          *reinterpret_cast<uint4*>(sm + kOffSb + mnm<256>(128 + col + i, srow)) = pack8(v16 + i);
+        tmem_st16(tmem_addr(tm, 32 * q4, kTmS + 128 + col), v16);
+        st16(sm + L::kSb, mnmaj(128 + col, srow, SbL), v16);
+        st16(sm + L::kSb, mnmaj(128 + col + 8, srow, SbL), v16 + 8);
       }
     }
     tmem_st_wait();
@@ -218,60 +270,74 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(TcParams p) {
 
   const float expA = p.g ? 0.f : expf(p.A[h]);
   const int j = tid & 127, hf = tid >> 7;  // prep ownership: channel j, rows 32hf..32hf+31
+  const int cbase[4] = {0, 16, 48, 96};     // C_b windows (rows of C)
 
+  // beta of the chunk, loaded one chunk ahead (thread t < 64 holds token t)
+  auto load_beta = [&](int cc) -> float {
+    const int t0 = a + cc * kC;
+    return (tid < kC && cc < c1 && tid < b - t0) ? __bfloat162float(p.beta[(size_t)(t0 + tid) * H + h]) : 0.f;
+  };
+  float beta_next = load_beta(c0);
   for (int c = c0; c < c1; ++c) {
     const int tok0 = a + c * kC;
     const int len = min(kC, b - tok0);
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
+    sync_for_mma();
+    if (tid < kC) vec[kVecBeta + tid] = beta_next;
+    beta_next = load_beta(c + 1);
+    if (!block_wait(&s_bar_raw, phase_raw, p.hdr)) { s_abort = 1; break; }
+    raw_pending = false;
 
-    // ---- row norms, beta (one warp per 8 rows)
-    for (int r = warp; r < kC; r += 8) {
-      float sq = 0.f, sk = 0.f;
-      if (r < len) {
-        const size_t base = ((size_t)(tok0 + r) * H + h) * kD + 4 * lane;
-        const uint2 qq = *reinterpret_cast<const uint2*>(p.q + base);
-        const uint2 kk = *reinterpret_cast<const uint2*>(p.k + base);
-        const __nv_bfloat162* q2 = reinterpret_cast<const __nv_bfloat162*>(&qq);
-        const __nv_bfloat162* k2 = reinterpret_cast<const __nv_bfloat162*>(&kk);
+    // ---- row norms: warp w takes rows w, w+8, ..., w+56
+    {
+      float sq[8], sk[8];
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const float2 fq = __bfloat1622float2(q2[i]), fk = __bfloat1622float2(k2[i]);
-          sq += fq.x * fq.x + fq.y * fq.y;
-          sk += fk.x * fk.x + fk.y * fk.y;
-        }
+      for (int m = 0; m < 8; ++m) {
+        const int r = warp + 8 * m;
+        const uint2 uq = *reinterpret_cast<const uint2*>(raw + 0 * 16384 + r * 256 + 8 * lane);
+        const uint2 uk = *reinterpret_cast<const uint2*>(raw + 1 * 16384 + r * 256 + 8 * lane);
+        const float2 q0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uq.x));
+        const float2 q1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uq.y));
+        const float2 k0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uk.x));
+        const float2 k1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uk.y));
+        sq[m] = q0.x * q0.x + q0.y * q0.y + q1.x * q1.x + q1.y * q1.y;
+        sk[m] = k0.x * k0.x + k0.y * k0.y + k1.x * k1.x + k1.y * k1.y;
       }
-      sq = warp_sum(sq);
-      sk = warp_sum(sk);
-      if (lane == 0) {
-        vec[kVecIq + r] = r < len ? 1.0f / sqrtf(sq + kNormEps) : 0.f;
-        vec[kVecIk + r] = r < len ? 1.0f / sqrtf(sk + kNormEps) : 0.f;
-        vec[kVecBeta + r] = r < len ? __bfloat162float(p.beta[(size_t)(tok0 + r) * H + h]) : 0.f;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+          sq[m] += __shfl_xor_sync(0xffffffffu, sq[m], o);
+          sk[m] += __shfl_xor_sync(0xffffffffu, sk[m], o);
+        }
+      if (lane < 8) {
+        const int r = warp + 8 * lane;
+        float vq = sq[0], vk = sk[0];
+#pragma unroll
+        for (int m = 1; m < 8; ++m)
+          if (lane == m) { vq = sq[m]; vk = sk[m]; }
+        vec[kVecIq + r] = r < len ? rsqrtf(vq + kNormEps) : 0.f;
+        vec[kVecIk + r] = r < len ? rsqrtf(vk + kNormEps) : 0.f;
       }
     }
     // ---- gate and chunk-local cumsum for channel j, rows 32hf..32hf+31
-    float E[32], kh[32], qh[32];
+    float E[32];
     {
-      float acc = 0.f;
+      if (p.g) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int r = 32 * hf + i;
-        float gv = 0.f;
-        if (r < len) {
-          const size_t idx = ((size_t)(tok0 + r) * H + h) * kD + j;
-          gv = p.g ? p.g[idx] : gate_logdecay(__bfloat162float(p.z[idx]), expA);
-          kh[i] = __bfloat162float(p.k[idx]);
-          qh[i] = __bfloat162float(p.q[idx]);
-        } else {
-          kh[i] = 0.f;
-          qh[i] = 0.f;
+        for (int i = 0; i < 32; ++i) {
+          const int r = 32 * hf + i;
+          E[i] = r < len ? p.g[((size_t)(tok0 + r) * H + h) * kD + j] : 0.f;
         }
-        acc += gv;
-        E[i] = acc;  // Gam (local to this half for now)
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) E[i] = raw_at(raw, 2, 32 * hf + i, j);
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          E[i] = (32 * hf + i < len) ? __fdividef(kGateMin, 1.0f + __expf(-expA * E[i])) : 0.f;
       }
-      if (hf == 0) vec[kVecTot + j] = acc;
+#pragma unroll
+      for (int i = 1; i < 32; ++i) E[i] += E[i - 1];
+      if (hf == 0) vec[kVecTot + j] = E[31];
     }
     __syncthreads();
     {
@@ -281,194 +347,232 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(TcParams p) {
       vec[kVecRho + (2 * hf) * 128 + j] = E[0];
       vec[kVecRho + (2 * hf + 1) * 128 + j] = E[16];
       if (hf == 1) vec[kVecGlast + j] = E[31];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int r = 32 * hf + i;
-        kh[i] *= vec[kVecIk + r];
-        qh[i] *= vec[kVecIq + r];
-      }
     }
     __syncthreads();
-    // E = e^{Gam_r - rho_b(r)}; per-channel factors
     float rho[4];
 #pragma unroll
     for (int bb = 0; bb < 4; ++bb) rho[bb] = vec[kVecRho + bb * 128 + j];
     const float glast = vec[kVecGlast + j];
+    const float rho0 = hf ? rho[2] : rho[0], rho1 = hf ? rho[3] : rho[1];
+    float Ei[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) E[i] = expf(E[i] - (hf ? rho[2 + (i >> 4)] : rho[i >> 4]));
+    for (int i = 0; i < 32; ++i) {
+      E[i] = __expf(E[i] - (i < 16 ? rho0 : rho1));
+      Ei[i] = __fdividef(1.0f, E[i]);
+    }
 
-    // ---- product operands: R (rows) and C_b (columns per row sub-tile b)
+    // ---- product operands R (rows, MN-major) and C_b (columns, MN-major)
     {
-      unsigned char* R = sm + kOffR;
-      unsigned char* Cm = sm + kOffC;
-      const int cbase[4] = {0, 16, 48, 96};
-      // F[t2][bb] = e^{rho_bb - rho_bt} for this half's sub-tiles bt = 2hf + t2
-      float F[2][4];
+      float F0[4], F1[4];  // e^{rho_bb - rho_bt} for bt = this half's two sub-tiles
 #pragma unroll
-      for (int t2 = 0; t2 < 2; ++t2)
-#pragma unroll
-        for (int bb = 0; bb < 4; ++bb) {
-          const float rb = hf ? rho[2 + t2] : rho[t2];
-          F[t2][bb] = expf(rho[bb] - rb);
-        }
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int t2 = i >> 4, r = 32 * hf + i, bt = r >> 4, rr = r & 15;
-        st_bf16(R, km128(32 * bt + rr, j), kh[i] * E[i]);
-        st_bf16(R, km128(32 * bt + 16 + rr, j), qh[i] * E[i]);
-        const float kinv = kh[i] / E[i];
-#pragma unroll
-        for (int bb = 0; bb < 4; ++bb)
-          if (bb >= bt) st_bf16(Cm, km128(cbase[bb] + r, j), bb == bt ? kinv : kinv * F[t2][bb]);
-      }
-    }
-    fence_async_smem();
-    __syncthreads();
-    {
-      // ---- M1: four M=64 MMAs -> TMEM [256 + 32b, +32): cols 0-15 A_kk^T, 16-31 A_qk^T
-      if (tid == 0) {
-        fence_after_sync();
-        constexpr uint32_t id = instr_desc(kFmtBF16, 64, 32, false, false);
-        const int cbase[4] = {0, 16, 48, 96};
-        for (int bb = 0; bb < 4; ++bb) {
-          const uint32_t abase = smem_u32(sm + kOffC) + (cbase[bb] >> 3) * 2048;
-          const uint32_t bbase = smem_u32(sm + kOffR) + (32 * bb >> 3) * 2048;
-          for (int k = 0; k < 8; ++k)
-            mma_bf16(tm + tmA + 32 * bb, smem_desc(abase + 256 * k, 128, 2048),
-                     smem_desc(bbase + 256 * k, 128, 2048), id, k > 0);
-        }
-        mma_commit(&s_bar);
-      }
-      const bool got = mbar_wait_cycles(&s_bar, phase, kWaitCycles);
-      phase ^= 1;
-      if (__syncthreads_or(!got)) {
-        if (tid == 0) { s_abort = 1; atomicOr(&p.hdr->err, kErrTimeout); }
-        break;
-      }
-      fence_after_sync();
-    }
-    // ---- A_kk (fp32 smem, beta-scaled, strictly lower) and A_qk (bf16 into A3)
-    float* Akk = reinterpret_cast<float*>(sm + kOffAkk);
-    if (warp < 4) {
-      const int i = 16 * warp + lane;  // valid for lane < 16
-#pragma unroll 1
       for (int bb = 0; bb < 4; ++bb) {
+        F0[bb] = __expf(rho[bb] - rho0);
+        F1[bb] = __expf(rho[bb] - rho1);
+      }
+#pragma unroll
+      for (int g8 = 0; g8 < 4; ++g8) {
+        const int r0 = 32 * hf + 8 * g8, bt = r0 >> 4, rr0 = r0 & 15;
+        float kv[8], qv[8], cv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = r0 + i;
+          const float e = E[8 * g8 + i];
+          const float kh = r < len ? raw_at(raw, 1, r, j) * vec[kVecIk + r] : 0.f;
+          const float qh = r < len ? raw_at(raw, 0, r, j) * vec[kVecIq + r] : 0.f;
+          kv[i] = kh * e;
+          qv[i] = qh * e;
+          cv[i] = kh * Ei[8 * g8 + i];
+        }
+        st16(sm + L::kR, mnmaj(32 * bt + rr0, j, 2048), kv);
+        st16(sm + L::kR, mnmaj(32 * bt + 16 + rr0, j, 2048), qv);
+        const float* F = (g8 & 2) ? F1 : F0;
+#pragma unroll
+        for (int bb = 0; bb < 4; ++bb) {
+          if (bb < bt) continue;
+          float w8[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) w8[i] = bb == bt ? cv[i] : cv[i] * F[bb];
+          st16(sm + L::kCc, mnmaj(cbase[bb] + r0, j, 2560), w8);
+        }
+      }
+    }
+    sync_for_mma();
+    // ---- M1: four M=64 MMAs -> TMEM [32b, +32): cols 0-15 A_kk^T, 16-31 A_qk^T
+    if (tid == 0) {
+      constexpr uint32_t id = instr_desc(kFmtBF16, 64, 32, true, true);
+      for (int bb = 0; bb < 4; ++bb) {
+        const uint32_t abase = smem_u32(sm + L::kCc) + (cbase[bb] >> 3) * 128;
+        const uint32_t bbase = smem_u32(sm + L::kR) + (32 * bb >> 3) * 128;
+        for (int k = 0; k < 8; ++k)
+          mma_bf16(tm + kTmA + 32 * bb, smem_desc(abase + 2 * 2560 * k, 2560, 128),
+                   smem_desc(bbase + 2 * 2048 * k, 2048, 128), id, k > 0);
+      }
+      mma_commit(&s_bar);
+    }
+    if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
+    // ---- A_kk (fp32 smem, beta-scaled, strictly lower) and A_qk (bf16 A3, MN-major)
+    float* Akk = reinterpret_cast<float*>(sm + L::kAkk);
+    {
+      const int i = r64;  // column of A (row of the M=64 accumulator)
+#pragma unroll
+      for (int b2 = 0; b2 < 2; ++b2) {
+        const int bb = 2 * ch + b2;
         float va[16], vq[16];
-        tmem_ld16(tmem_addr(tm, 32 * warp, tmA + 32 * bb), va);
-        tmem_ld16(tmem_addr(tm, 32 * warp, tmA + 32 * bb + 16), vq);
+        tmem_ld16(tmem_addr(tm, 32 * q4, kTmA + 32 * bb), va);
+        tmem_ld16(tmem_addr(tm, 32 * q4, kTmA + 32 * bb + 16), vq);
         tmem_ld_wait();
-        if (lane < 16) {
+        if (m64) {
 #pragma unroll
           for (int cc = 0; cc < 16; ++cc) {
             const int r = 16 * bb + cc;
             Akk[r * 65 + i] = (i < r) ? vec[kVecBeta + r] * va[cc] : 0.f;
-            if (MODE == 0) st_bf16(sm + kOffA3, km64(64 + r, i), (i <= r) ? vq[cc] : 0.f);
+            vq[cc] = (i <= r) ? vq[cc] : 0.f;
+          }
+          if (MODE == 0) {
+            st16(sm + L::kA3, mnmaj(16 * bb, i, 1024), vq);
+            st16(sm + L::kA3, mnmaj(16 * bb + 8, i, 1024), vq + 8);
           }
         }
       }
     }
     fence_before_sync();
     __syncthreads();
-    // ---- T = (I + A_kk)^{-1}: forward substitution on 16x16 diagonal blocks
-    float* Tm = reinterpret_cast<float*>(sm + kOffT);
-    float* Xs = vec + kVecX;
-    for (int e = tid; e < kC * 65; e += kNT) Tm[e] = 0.f;
-    __syncthreads();
+    // ---- T = (I + A_kk)^{-1}
+    // diagonal 16x16 blocks by forward substitution (registers), then the
+    // blocks below them by merging: [[P,0],[B,Q]]^{-1} has lower-left block
+    // -Q^{-1} B P^{-1}; first 16 -> 32 (block pairs 0|1 and 2|3), then 32 -> 64.
+    float* Tf = reinterpret_cast<float*>(sm + L::kTf);
+    float* Y = vec + kVecY;  // scratch, up to 32 x 32 (stride 33)
     if (tid < kC) {
-      const int r0 = (tid >> 4) << 4, col = tid;
-      for (int r = r0; r < r0 + 16; ++r) {
-        float x = (r == col) ? 1.f : 0.f;
-        if (r > col)
-          for (int i = col; i < r; ++i) x -= Akk[r * 65 + i] * Tm[i * 65 + col];
-        Tm[r * 65 + col] = x;
+      const int bk = tid >> 4, cc = tid & 15, base = 16 * bk;
+      float x[16];
+#pragma unroll
+      for (int rr = 0; rr < 16; ++rr) {
+        float acc = (rr == cc) ? 1.f : 0.f;
+#pragma unroll
+        for (int i = 0; i < rr; ++i) acc -= Akk[(base + rr) * 65 + base + i] * x[i];
+        x[rr] = (rr < cc) ? 0.f : acc;
       }
+#pragma unroll
+      for (int rr = 0; rr < 16; ++rr) Tf[(base + rr) * 65 + base + cc] = x[rr];
     }
     __syncthreads();
-    // block rows below the diagonal: T_ba = -T_bb sum_{a<=c<b} A_bc T_ca
-    for (int dist = 1; dist < 4; ++dist) {
-      const int npairs = 4 - dist;
-      for (int e = tid; e < npairs * 256; e += kNT) {
-        const int pr = e >> 8, rr = (e >> 4) & 15, cc = e & 15, bb = pr + dist, aa = pr;
-        float x = 0.f;
-        for (int m = aa * 16; m < bb * 16; ++m) x += Akk[(bb * 16 + rr) * 65 + m] * Tm[m * 65 + aa * 16 + cc];
-        Xs[e] = x;
-      }
-      __syncthreads();
-      for (int e = tid; e < npairs * 256; e += kNT) {
-        const int pr = e >> 8, rr = (e >> 4) & 15, cc = e & 15, bb = pr + dist, aa = pr;
-        float y = 0.f;
-        for (int m = 0; m < 16; ++m) y -= Tm[(bb * 16 + rr) * 65 + bb * 16 + m] * Xs[pr * 256 + m * 16 + cc];
-        Tm[(bb * 16 + rr) * 65 + aa * 16 + cc] = y;
-      }
-      __syncthreads();
-    }
-    for (int e = tid; e < kC * kC; e += kNT) {
-      const int r = e >> 6, i = e & 63;
-      st_bf16(sm + kOffTp, km64(r, i), Tm[r * 65 + i]);
-    }
-    __syncthreads();  // T (fp32) is dead from here: region P holds [X_K | X_V] next
-
-    // ---- WY / chain operands from registers: X_K, X_V, Q', K', gamma
     {
-      float erho[2], elast[2];
+      // 16 -> 32: for pair pr (blocks 2pr, 2pr+1): Y = A[hi][lo] T[lo][lo]; T[hi][lo] = -T[hi][hi] Y
+      const int pr = tid >> 7, e = tid & 127, rr = e >> 3, c2 = (e & 7) * 2;  // 2 outputs
+      const int lo = 32 * pr, hi = lo + 16;
+      float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-      for (int t2 = 0; t2 < 2; ++t2) {
-        const float rb = hf ? rho[2 + t2] : rho[t2];
-        erho[t2] = expf(rb);
-        elast[t2] = expf(glast - rb);
+      for (int i = 0; i < 16; ++i) {
+        const float av = Akk[(hi + rr) * 65 + lo + i];
+        y0 += av * Tf[(lo + i) * 65 + lo + c2];
+        y1 += av * Tf[(lo + i) * 65 + lo + c2 + 1];
       }
-      if (hf == 0) vec[kVecGam + j] = expf(glast);
-      unsigned char* X = sm + kOffX;
+      Y[pr * 528 + rr * 33 + c2] = y0;
+      Y[pr * 528 + rr * 33 + c2 + 1] = y1;
+      __syncthreads();
+      float t0 = 0.f, t1 = 0.f;
 #pragma unroll
+      for (int m = 0; m < 16; ++m) {
+        const float tv = Tf[(hi + rr) * 65 + hi + m];
+        t0 += tv * Y[pr * 528 + m * 33 + c2];
+        t1 += tv * Y[pr * 528 + m * 33 + c2 + 1];
+      }
+      Tf[(hi + rr) * 65 + lo + c2] = -t0;
+      Tf[(hi + rr) * 65 + lo + c2 + 1] = -t1;
+    }
+    __syncthreads();
+    {
+      // 32 -> 64: Y = A[32:64][0:32] T[0:32][0:32]; T[32:64][0:32] = -T[32:64][32:64] Y
+      const int rr = tid >> 3, c4 = (tid & 7) * 4;  // 4 outputs
+      float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
       for (int i = 0; i < 32; ++i) {
-        const int r = 32 * hf + i, t2 = i >> 4;
-        const float bet = vec[kVecBeta + r];
-        const float eg = E[i] * erho[t2];
-        st_bf16(X, mnm<256>(j, r), bet * kh[i] * eg);
-        const float vv = r < len ? __bfloat162float(p.v[((size_t)(tok0 + r) * H + h) * kD + j]) : 0.f;
-        st_bf16(X, mnm<256>(128 + j, r), bet * vv);
-        if (MODE == 0) st_bf16(sm + kOffA1, km128(64 + r, j), qh[i] * eg);
-        st_bf16(sm + kOffKp, mnm<128>(j, r), (kh[i] / E[i]) * elast[t2]);
+        const float av = Akk[(32 + rr) * 65 + i];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) y[u] += av * (i >= c4 + u ? Tf[i * 65 + c4 + u] : 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) Y[rr * 33 + c4 + u] = y[u];
+      __syncthreads();
+      float t[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+      for (int m = 0; m < 32; ++m) {
+        const float tv = m <= rr ? Tf[(32 + rr) * 65 + 32 + m] : 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) t[u] += tv * Y[m * 33 + c4 + u];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) Tf[(32 + rr) * 65 + c4 + u] = -t[u];
+    }
+    __syncthreads();
+    // T -> bf16 A operand (K-major), upper triangle zero
+    for (int e = tid; e < kC * 8; e += kNT) {
+      const int r = e >> 3, i0 = (e & 7) * 8;
+      float t8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) t8[i] = (i0 + i <= r) ? Tf[r * 65 + i0 + i] : 0.f;
+      st16(sm + L::kTop, kmaj(r, i0, 1024), t8);
+    }
+    __syncthreads();  // A_kk / T (fp32) are dead from here: region P takes X, Q', K'
+
+    // ---- WY / chain operands: X_K, X_V (K-major), Q' (MN-major), K' (K-major), gamma
+    {
+      const float er0 = __expf(rho0), er1 = __expf(rho1);
+      const float el0 = __expf(glast - rho0), el1 = __expf(glast - rho1);
+      if (hf == 0) vec[kVecGam + j] = __expf(glast);
+#pragma unroll
+      for (int g8 = 0; g8 < 4; ++g8) {
+        const int r0 = 32 * hf + 8 * g8;
+        const float er = g8 < 2 ? er0 : er1, el = g8 < 2 ? el0 : el1;
+        float xk[8], xv[8], qp[8], kp[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = r0 + i;
+          const bool in = r < len;
+          const float e = E[8 * g8 + i];
+          const float kh = in ? raw_at(raw, 1, r, j) * vec[kVecIk + r] : 0.f;
+          const float bet = vec[kVecBeta + r];
+          xk[i] = bet * kh * e * er;
+          xv[i] = in ? bet * raw_at(raw, 3, r, j) : 0.f;
+          kp[i] = kh * Ei[8 * g8 + i] * el;
+          if (MODE == 0) qp[i] = in ? raw_at(raw, 0, r, j) * vec[kVecIq + r] * e * er : 0.f;
+        }
+        st16(sm + L::kX, kmaj(j, r0, 1024), xk);
+        st16(sm + L::kX, kmaj(128 + j, r0, 1024), xv);
+        st16(sm + L::kKp, kmaj(j, r0, 1024), kp);
+        if (MODE == 0) st16(sm + L::kQp, mnmaj(r0, j, 1024), qp);
       }
     }
-    fence_async_smem();
-    __syncthreads();
-    // ---- M2: [W | U~] = T_pad [X_K | X_V]  (M=128, N=256, K=64) -> TMEM [0, 256)
+    sync_for_mma();
+    // the staged rows are consumed: prefetch the next chunk
+    if (c + 1 < c1) {
+      raw_pending = true;
+      if (tid == 0) stage_chunk(p, raw, &s_bar_raw, a + (c + 1) * kC, h);
+    }
+    // ---- M2: [W | U~] = T [X_K | X_V]  (M=64, N=256, K=64)
     if (tid == 0) {
-      fence_after_sync();
-      constexpr uint32_t id = instr_desc(kFmtBF16, 128, 256, false, true);
-      const uint32_t abase = smem_u32(sm + kOffTp), bbase = smem_u32(sm + kOffX);
+      constexpr uint32_t id = instr_desc(kFmtBF16, 64, 256, false, false);
+      const uint32_t abase = smem_u32(sm + L::kTop), bbase = smem_u32(sm + L::kX);
       for (int k = 0; k < 4; ++k)
         mma_bf16(tm + kTmWU, smem_desc(abase + 256 * k, 128, 1024),
-                 smem_desc(bbase + 2 * 4096 * k, 4096, 128), id, k > 0);
+                 smem_desc(bbase + 256 * k, 128, 1024), id, k > 0);
       mma_commit(&s_bar);
     }
-    {
-      const bool got = mbar_wait_cycles(&s_bar, phase, kWaitCycles);
-      phase ^= 1;
-      if (__syncthreads_or(!got)) {
-        if (tid == 0) { s_abort = 1; atomicOr(&p.hdr->err, kErrTimeout); }
-        break;
-      }
-      fence_after_sync();
-    }
-    // ---- W -> bf16 A1 rows 0-63 (warps 0,1,4,5 hold TMEM lanes 0-63);
-    //      U~ stays in TMEM columns [128, 256)
+    if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
+    // ---- W -> bf16 A operand (K-major); U~ -> registers (M=64 rows, lane < 16)
     float ut[64];
-    if (q4 < 2) {
-      const int r = srow;
 #pragma unroll
-      for (int c16 = 0; c16 < 64; c16 += 16) {
-        float w16[16];
-        tmem_ld16(tmem_addr(tm, 32 * q4, kTmWU + 64 * ch + c16), w16);
-        float u16[16];
-        tmem_ld16(tmem_addr(tm, 32 * q4, kTmWU + 128 + 64 * ch + c16), u16);
-        tmem_ld_wait();
+    for (int c16 = 0; c16 < 64; c16 += 16) {
+      float w16[16], u16[16];
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmWU + 64 * ch + c16), w16);
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmWU + 128 + 64 * ch + c16), u16);
+      tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) ut[c16 + i] = u16[i];
-#pragma unroll
-        for (int i = 0; i < 16; i += 8)
-          *reinterpret_cast<uint4*>(sm + kOffA1 + km128(r, 64 * ch + c16 + i)) = pack8(w16 + i);
+      for (int i = 0; i < 16; ++i) ut[c16 + i] = u16[i];
+      if (m64) {
+        st16(sm + L::kW, kmaj(r64, 64 * ch + c16, 2048), w16);
+        st16(sm + L::kW, kmaj(r64, 64 * ch + c16 + 8, 2048), w16 + 8);
       }
     }
     // ---- decay the state(s) by gamma = e^{Gam_last} (rows = dk = TMEM lanes)
@@ -480,7 +584,7 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(TcParams p) {
 #pragma unroll
         for (int c16 = 0; c16 < 64; c16 += 16) {
           float s16[16];
-          const uint32_t col = tmS + 128 * blk + 64 * ch + c16;
+          const uint32_t col = kTmS + 128 * blk + 64 * ch + c16;
           tmem_ld16(tmem_addr(tm, 32 * q4, col), s16);
           tmem_ld_wait();
 #pragma unroll
@@ -489,92 +593,62 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(TcParams p) {
         }
       tmem_st_wait();
     }
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    // ---- C1: D1 = A1 S  (M=128 [W;Q'] or M=64 W, K=128)
-    //      MODE 0: N=128 -> TMEM [256, 384);  MODE 1: N=256 ([S|X]) -> TMEM [0, 256)
+    sync_for_mma();
+    // ---- C1: D_W = W S (M=64, N=128|256), D_Q = Q' S (M=64, N=128)
     if (tid == 0) {
-      fence_after_sync();
-      const uint32_t abase = smem_u32(sm + kOffA1), bbase = smem_u32(sm + kOffSb);
+      const uint32_t sb = smem_u32(sm + L::kSb);
+      const uint32_t wb = smem_u32(sm + L::kW);
+      constexpr uint32_t idw = instr_desc(kFmtBF16, 64, SbN, false, true);
+      for (int k = 0; k < 8; ++k)
+        mma_bf16(tm + kTmW, smem_desc(wb + 256 * k, 128, 2048),
+                 smem_desc(sb + 2 * SbL * k, SbL, 128), idw, k > 0);
       if (MODE == 0) {
-        constexpr uint32_t id = instr_desc(kFmtBF16, 128, 128, false, true);
+        constexpr uint32_t idq = instr_desc(kFmtBF16, 64, 128, true, true);
+        const uint32_t qb = smem_u32(sm + L::kQp);
         for (int k = 0; k < 8; ++k)
-          mma_bf16(tm + kTmD1, smem_desc(abase + 256 * k, 128, 2048),
-                   smem_desc(bbase + 2 * 2048 * k, 2048, 128), id, k > 0);
-      } else {
-        constexpr uint32_t id = instr_desc(kFmtBF16, 128, 256, false, true);
-        for (int k = 0; k < 8; ++k)
-          mma_bf16(tm + 0, smem_desc(abase + 256 * k, 128, 2048),
-                   smem_desc(bbase + 2 * 4096 * k, 4096, 128), id, k > 0);
+          mma_bf16(tm + kTmQ, smem_desc(qb + 2 * 1024 * k, 1024, 128),
+                   smem_desc(sb + 2 * SbL * k, SbL, 128), idq, k > 0);
       }
       mma_commit(&s_bar);
     }
+    if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
+    // ---- U = U~ - W S  (transition: [U_S | U_X] = [U~ | 0] - W [S | X]); B operand MN-major
     {
-      const bool got = mbar_wait_cycles(&s_bar, phase, kWaitCycles);
-      phase ^= 1;
-      if (__syncthreads_or(!got)) {
-        if (tid == 0) { s_abort = 1; atomicOr(&p.hdr->err, kErrTimeout); }
-        break;
-      }
-      fence_after_sync();
-    }
-    // ---- U = U~ - W S  (MODE 1: [U_S | U_X] = [U~ | 0] - W [S | X])
-    if (q4 < 2) {
-      const int r = srow;
       constexpr int NB = MODE == 0 ? 1 : 2;
 #pragma unroll
       for (int blk = 0; blk < NB; ++blk)
 #pragma unroll
         for (int c16 = 0; c16 < 64; c16 += 16) {
           float d16[16];
-          const uint32_t col = (MODE == 0 ? kTmD1 : 0) + 128 * blk + 64 * ch + c16;
-          tmem_ld16(tmem_addr(tm, 32 * q4, col), d16);
+          const int col = 128 * blk + 64 * ch + c16;
+          tmem_ld16(tmem_addr(tm, 32 * q4, kTmW + col), d16);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 16; ++i) d16[i] = (blk == 0 ? ut[c16 + i] : 0.f) - d16[i];
-#pragma unroll
-          for (int i = 0; i < 16; i += 8) {
-            const int n = 128 * blk + 64 * ch + c16 + i;
-            const uint32_t off = MODE == 0 ? mnm<128>(n, r) : mnm<256>(n, r);
-            *reinterpret_cast<uint4*>(sm + kOffU + off) = pack8(d16 + i);
+          if (m64) {
+            st16(sm + L::kU, mnmaj(col, r64, SbL), d16);
+            st16(sm + L::kU, mnmaj(col + 8, r64, SbL), d16 + 8);
           }
         }
     }
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    // ---- C2: S += K'^T U  (and O += A_qk U in MODE 0)
+    sync_for_mma();
+    // ---- C2: S += K'^T U (M=128); D_Q += A_qk U (M=64)
     if (tid == 0) {
-      fence_after_sync();
-      const uint32_t kb = smem_u32(sm + kOffKp), ub = smem_u32(sm + kOffU);
+      const uint32_t kb = smem_u32(sm + L::kKp), ub = smem_u32(sm + L::kU);
+      constexpr uint32_t ids = instr_desc(kFmtBF16, 128, SbN, false, true);
+      for (int k = 0; k < 4; ++k)
+        mma_bf16(tm + kTmS, smem_desc(kb + 256 * k, 128, 1024),
+                 smem_desc(ub + 2 * SbL * k, SbL, 128), ids, 1);
       if (MODE == 0) {
-        constexpr uint32_t id = instr_desc(kFmtBF16, 128, 128, true, true);
+        constexpr uint32_t ido = instr_desc(kFmtBF16, 64, 128, true, true);
+        const uint32_t a3 = smem_u32(sm + L::kA3);
         for (int k = 0; k < 4; ++k)
-          mma_bf16(tm + kTmS, smem_desc(kb + 2 * 2048 * k, 2048, 128),
-                   smem_desc(ub + 2 * 2048 * k, 2048, 128), id, 1);
-        constexpr uint32_t id2 = instr_desc(kFmtBF16, 128, 128, false, true);
-        const uint32_t a3 = smem_u32(sm + kOffA3);
-        for (int k = 0; k < 4; ++k)
-          mma_bf16(tm + kTmD1, smem_desc(a3 + 256 * k, 128, 1024),
-                   smem_desc(ub + 2 * 2048 * k, 2048, 128), id2, 1);
-      } else {
-        constexpr uint32_t id = instr_desc(kFmtBF16, 128, 256, true, true);
-        for (int k = 0; k < 4; ++k)
-          mma_bf16(tm + 256, smem_desc(kb + 2 * 2048 * k, 2048, 128),
-                   smem_desc(ub + 2 * 4096 * k, 4096, 128), id, 1);
+          mma_bf16(tm + kTmQ, smem_desc(a3 + 2 * 1024 * k, 1024, 128),
+                   smem_desc(ub + 2 * SbL * k, SbL, 128), ido, 1);
       }
       mma_commit(&s_bar);
     }
-    {
-      const bool got = mbar_wait_cycles(&s_bar, phase, kWaitCycles);
-      phase ^= 1;
-      if (__syncthreads_or(!got)) {
-        if (tid == 0) { s_abort = 1; atomicOr(&p.hdr->err, kErrTimeout); }
-        break;
-      }
-      fence_after_sync();
-    }
+    if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
     // ---- S (and X) -> bf16 operand for the next chunk; O -> global
     {
       constexpr int NB = MODE == 0 ? 1 : 2;
@@ -584,23 +658,19 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(TcParams p) {
         for (int c16 = 0; c16 < 64; c16 += 16) {
           float s16[16];
           const int col = 128 * blk + 64 * ch + c16;
-          tmem_ld16(tmem_addr(tm, 32 * q4, tmS + col), s16);
+          tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + col), s16);
           tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; i += 8) {
-            const uint32_t off = MODE == 0 ? mnm<128>(col + i, srow) : mnm<256>(col + i, srow);
-            *reinterpret_cast<uint4*>(sm + kOffSb + off) = pack8(s16 + i);
-          }
+          st16(sm + L::kSb, mnmaj(col, srow, SbL), s16);
+          st16(sm + L::kSb, mnmaj(col + 8, srow, SbL), s16 + 8);
         }
-      if (MODE == 0 && q4 >= 2) {
-        const int r = srow - 64;
+      if (MODE == 0) {
 #pragma unroll
         for (int c16 = 0; c16 < 64; c16 += 16) {
           float o16[16];
-          tmem_ld16(tmem_addr(tm, 32 * q4, kTmD1 + 64 * ch + c16), o16);
+          tmem_ld16(tmem_addr(tm, 32 * q4, kTmQ + 64 * ch + c16), o16);
           tmem_ld_wait();
-          if (r < len) {
-            uint4* dst = reinterpret_cast<uint4*>(p.o + ((size_t)(tok0 + r) * H + h) * kD + 64 * ch + c16);
+          if (m64 && r64 < len) {
+            uint4* dst = reinterpret_cast<uint4*>(p.o + ((size_t)(tok0 + r64) * H + h) * kD + 64 * ch + c16);
             dst[0] = pack8(o16);
             dst[1] = pack8(o16 + 8);
           }
@@ -620,7 +690,7 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(TcParams p) {
 #pragma unroll
         for (int c16 = 0; c16 < 64; c16 += 16) {
           float s16[16];
-          tmem_ld16(tmem_addr(tm, 32 * q4, tmS + 64 * ch + c16), s16);
+          tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + 64 * ch + c16), s16);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 16; i += 4)
@@ -628,7 +698,7 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(TcParams p) {
         }
       }
     } else {
-      // transition: M (from X, columns 384..511) and N (from S, columns 256..383)
+      // transition: N from S (columns 256..383), M from X (columns 384..511)
       float* Mt = seg_trans(p.seg, n, h, H, p.P, seg);
       float* Nt = Mt + kD * kD;
 #pragma unroll
@@ -636,7 +706,7 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(TcParams p) {
 #pragma unroll
         for (int c16 = 0; c16 < 64; c16 += 16) {
           float s16[16];
-          tmem_ld16(tmem_addr(tm, 32 * q4, 256 + 128 * blk + 64 * ch + c16), s16);
+          tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + 128 * blk + 64 * ch + c16), s16);
           tmem_ld_wait();
           float* dst = (blk == 0 ? Nt : Mt) + (size_t)srow * kD + 64 * ch + c16;
 #pragma unroll
@@ -644,6 +714,9 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(TcParams p) {
             *reinterpret_cast<float4*>(dst + i) = make_float4(s16[i], s16[i + 1], s16[i + 2], s16[i + 3]);
         }
     }
+  } else if (raw_pending) {
+    // a wait gave up: let the TMA load still in flight land before leaving
+    mbar_wait_cycles(&s_bar_raw, phase_raw, kWaitCycles);
   }
   fence_before_sync();
   __syncthreads();
@@ -651,39 +724,53 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(TcParams p) {
 }
 
 // Incoming state of every segment: S_in(0) = S0, S_in(p+1) = M_p S_in(p) + N_p.
-// One CTA per (n, h, 16-column block of the state); fp32 on CUDA cores.
-__global__ void __launch_bounds__(256) compose_kernel(TcParams p) {
+// One CTA per (n, h, 16-column block of the state); fp32 on CUDA cores, with
+// M staged 32 columns at a time by coalesced row loads, one tile ahead.
+__global__ void __launch_bounds__(256) compose_kernel(const __grid_constant__ TcParams p) {
   const int n = blockIdx.x, h = blockIdx.y, cb = blockIdx.z * 16;
   const int H = p.H;
   if (!seqlens_valid(p.cu, p.N, p.T, p.max_len)) return;
   __shared__ float Sc[kD][16];
-  __shared__ float Mrow[8][kD];
+  __shared__ float Ms[2][kD][33];
   const int tid = threadIdx.x;
   for (int e = tid; e < kD * 16; e += 256) {
-    const int r = e >> 4, c = e & 15;
-    Sc[r][c] = p.S0 ? p.S0[((size_t)n * H + h) * kD * kD + (size_t)r * kD + cb + c] : 0.f;
+    const int r = e >> 4, cc = e & 15;
+    Sc[r][cc] = p.S0 ? p.S0[((size_t)n * H + h) * kD * kD + (size_t)r * kD + cb + cc] : 0.f;
   }
-  __syncthreads();
+  const int c = tid & 15, r0 = tid >> 4;  // rows r0 + 16 m
   for (int sg = 0; sg + 1 < p.P; ++sg) {
     const float* Mt = seg_trans(p.seg, n, h, H, p.P, sg);
     const float* Nt = Mt + kD * kD;
-    // thread: column c = tid & 15, rows r = tid >> 4 + 16 m
     float acc[8];
-    const int c = tid & 15, r0 = tid >> 4;
 #pragma unroll
     for (int m = 0; m < 8; ++m) acc[m] = Nt[(size_t)(r0 + 16 * m) * kD + cb + c];
-    for (int k0 = 0; k0 < kD; k0 += 8) {
+    float pre[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int e = tid + 256 * u;
+      pre[u] = Mt[(size_t)(e >> 5) * kD + (e & 31)];
+    }
+    for (int k0 = 0; k0 < kD; k0 += 32) {
+      const int buf = (k0 >> 5) & 1;
       __syncthreads();
-      for (int e = tid; e < 8 * kD; e += 256) {
-        const int kk = e >> 7, r = e & 127;
-        Mrow[kk][r] = Mt[(size_t)r * kD + k0 + kk];  // column k0+kk of M
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int e = tid + 256 * u;
+        Ms[buf][e >> 5][e & 31] = pre[u];
+      }
+      if (k0 + 32 < kD) {
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int e = tid + 256 * u;
+          pre[u] = Mt[(size_t)(e >> 5) * kD + k0 + 32 + (e & 31)];
+        }
       }
       __syncthreads();
+#pragma unroll 8
+      for (int kk = 0; kk < 32; ++kk) {
+        const float sv = Sc[k0 + kk][c];
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const float s = Sc[k0 + kk][c];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) acc[m] += Mrow[kk][r0 + 16 * m] * s;
+        for (int m = 0; m < 8; ++m) acc[m] += Ms[buf][r0 + 16 * m][kk] * sv;
       }
     }
     __syncthreads();
@@ -696,6 +783,33 @@ __global__ void __launch_bounds__(256) compose_kernel(TcParams p) {
       Sin[(size_t)r * kD + cb + cc] = Sc[r][cc];
     }
   }
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once (no link to libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+// [T, H, 128] bf16 tensor, box 64 tokens x 1 head x 128 channels; rows past T
+// read as zero.
+bool make_map(CUtensorMap* map, const void* base, int T, int H) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)T};
+  const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)kD, 1, (cuuint32_t)kC};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -728,10 +842,12 @@ int tc_launches(int N, int H, int max_len) {
 
 cudaError_t launch_forward_tc(const ForwardArgs& a) {
   TcParams p;
-  p.q = (const __nv_bfloat16*)a.q;
-  p.k = (const __nv_bfloat16*)a.k;
-  p.v = (const __nv_bfloat16*)a.v;
-  p.z = (const __nv_bfloat16*)a.z;
+  memset(&p, 0, sizeof(p));
+  if (a.T > 0) {
+    if (!make_map(&p.tq, a.q, a.T, a.H) || !make_map(&p.tk, a.k, a.T, a.H) ||
+        !make_map(&p.tz, a.z ? a.z : a.k, a.T, a.H) || !make_map(&p.tv, a.v, a.T, a.H))
+      return cudaErrorInvalidValue;
+  }
   p.beta = (const __nv_bfloat16*)a.beta;
   p.A = a.A;
   p.g = a.g;
@@ -748,16 +864,18 @@ cudaError_t launch_forward_tc(const ForwardArgs& a) {
   p.seg = (float*)((char*)a.ws + sizeof(WsHeader));
   cudaError_t err;
   if (p.P > 1) {
-    err = cudaFuncSetAttribute(tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    err = cudaFuncSetAttribute(tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Smem<1>::kBytes);
     if (err != cudaSuccess) return err;
-    tc_kernel<1><<<dim3(a.N, a.H, p.P - 1), kNT, kSmemBytes, a.stream>>>(p);
+    tc_kernel<1><<<dim3(a.N, a.H, p.P - 1), kNT, Smem<1>::kBytes, a.stream>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     compose_kernel<<<dim3(a.N, a.H, kD / 16), 256, 0, a.stream>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
-  err = cudaFuncSetAttribute(tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  err = cudaFuncSetAttribute(tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Smem<0>::kBytes);
   if (err != cudaSuccess) return err;
-  tc_kernel<0><<<dim3(a.N, a.H, p.P), kNT, kSmemBytes, a.stream>>>(p);
+  tc_kernel<0><<<dim3(a.N, a.H, p.P), kNT, Smem<0>::kBytes, a.stream>>>(p);
   return cudaGetLastError();
 }
 
