@@ -1,7 +1,7 @@
 // kda_prefill_tc.cu -- chunkwise KDA prefill on the sm_100a tensor cores
 // (tcgen05.mma, TMEM accumulators), bf16 inputs, dk = dv = 128, chunk = 64.
 //
-// One CTA of 256 threads runs one (sequence, head, segment) over its chunks in
+// One CTA of 512 threads runs one (sequence, head, segment) over its chunks in
 // order (Kimi Linear summary §3.1: chunkwise WY / UT form with an inter-chunk
 // state carry; §3.2: sub-chunking keeps the channel-wise decay factors in
 // range; Appendix C: per-chunk cumulative log-decay, forward-substitution
@@ -50,7 +50,7 @@ using namespace tc;
 
 constexpr int kC = 64;    // chunk tokens
 constexpr int kD = 128;   // dk = dv
-constexpr int kNT = 256;  // threads
+constexpr int kNT = 512;  // threads (16 warps)
 
 // ---- shared memory map (bytes), per pass ----
 template <int MODE>
@@ -61,8 +61,8 @@ struct Smem {
   static constexpr int kP = kRaw + 65536;                       // region P, reused through a chunk:
   static constexpr int kR = kP;                                 //   R   B op (N=128, K=128) MN-major
   static constexpr int kCc = kP + 32768;                        //   C   A op (M=160, K=128) MN-major
-  static constexpr int kAkk = kP;                               //   A_kk fp32 [64][65]
-  static constexpr int kTf = kP + 16640;                        //   T    fp32 [64][65]
+  static constexpr int kAkk = kP;                               //   A_kk fp32 [64][68]
+  static constexpr int kTf = kP + 17408;                        //   T    fp32 [64][68]
   static constexpr int kX = kP;                                 //   X   B op (N=256, K=64) K-major
   static constexpr int kQp = kP + 32768;                        //   Q'  A op (M=64, K=128) MN-major
   static constexpr int kKp = kP + 49152;                        //   K'  A op (M=128, K=64) K-major
@@ -71,11 +71,11 @@ struct Smem {
   static constexpr int kTop = kP + 73728;                       // T   A op (M=64, K=64) K-major
   static constexpr int kA3 = kTop + 8192;                       // A_qk A op (M=64, K=64) MN-major
   static constexpr int kVec = kA3 + (MODE == 0 ? 8192 : 0);
-  static constexpr int kBytes = kVec + 2176 * 4 + 64;
+  static constexpr int kBytes = kVec + 2304 * 4 + 64;
 };
 // vectors (floats) at Smem::kVec
 constexpr int kVecIq = 0, kVecIk = 64, kVecBeta = 128, kVecGam = 192, kVecRho = 320,
-              kVecTot = 832, kVecGlast = 960, kVecY = 1088;  // Y: 2 x 16 x 33 or 32 x 33 floats
+              kVecTot = 832, kVecGlast = 960, kVecY = 1088;  // Y: up to 32 x 36 floats
 
 // TMEM columns.  M=64 accumulators put row r in lane 32 (r / 16) + r % 16.
 constexpr uint32_t kTmA = 0;     // A products, 4 x 32 columns (prep)
@@ -83,6 +83,8 @@ constexpr uint32_t kTmWU = 0;    // [W | U~]: 256 columns (after the products ar
 constexpr uint32_t kTmW = 0;     // D_W = W S (128, or 256 for W [S | X])
 constexpr uint32_t kTmQ = 128;   // D_Q = Q' S (+ A_qk U)
 constexpr uint32_t kTmS = 256;   // fp32 state; identity-started block X at 384 (transition)
+
+constexpr int kLd = 68;  // row stride (floats) of the fp32 A_kk / T tiles
 
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s: a wait this long is a fault
 
@@ -228,7 +230,7 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
 
   constexpr int SbN = MODE == 0 ? 128 : 256;  // N extent of the bf16 state operand
   constexpr int SbL = SbN * 16;               // its K-group stride (LBO)
-  const int q4 = warp & 3, ch = warp >> 2;    // TMEM lane quarter, column half
+  const int q4 = warp & 3, cq = warp >> 2;    // TMEM lane quarter, 32-column quarter
   const int srow = 32 * q4 + lane;            // dk row (M=128 accumulators)
   const int r64 = 16 * q4 + lane;             // token row of M=64 accumulators (lane < 16)
   const bool m64 = lane < 16;
@@ -240,9 +242,9 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
       S0 = seg > 0 ? seg_sin(p.seg, n, h, H, p.P, seg)
                    : (p.S0 ? p.S0 + ((size_t)n * H + h) * kD * kD : nullptr);
 #pragma unroll
-    for (int c16 = 0; c16 < 64; c16 += 16) {
+    for (int c16 = 0; c16 < 32; c16 += 16) {
       float v16[16];
-      const int col = 64 * ch + c16;
+      const int col = 32 * cq + c16;
       if (S0) {
         const float4* src = reinterpret_cast<const float4*>(S0 + (size_t)srow * kD + col);
 #pragma unroll
@@ -269,8 +271,9 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
   }
 
   const float expA = p.g ? 0.f : expf(p.A[h]);
-  const int j = tid & 127, hf = tid >> 7;  // prep ownership: channel j, rows 32hf..32hf+31
-  const int cbase[4] = {0, 16, 48, 96};     // C_b windows (rows of C)
+  // prep ownership: channel j, row sub-tile qq (rows 16qq .. 16qq+15)
+  const int j = tid & 127, qq = tid >> 7;
+  // C_b window of row sub-tile b starts at row 8 b (b + 1) of C: 0, 16, 48, 96
 
   // beta of the chunk, loaded one chunk ahead (thread t < 64 holds token t)
   auto load_beta = [&](int cc) -> float {
@@ -287,112 +290,98 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
     if (!block_wait(&s_bar_raw, phase_raw, p.hdr)) { s_abort = 1; break; }
     raw_pending = false;
 
-    // ---- row norms: warp w takes rows w, w+8, ..., w+56
+    // ---- query row norms (warp w: rows w, w+16, w+32, w+48).  Key norms come
+    //      from the diagonal of the K K^T product below, where the decay
+    //      factors cancel; the query norm scales the output row at the end.
     {
-      float sq[8], sk[8];
+      float sq[4];
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const int r = warp + 8 * m;
+      for (int m = 0; m < 4; ++m) {
+        const int r = warp + 16 * m;
         const uint2 uq = *reinterpret_cast<const uint2*>(raw + 0 * 16384 + r * 256 + 8 * lane);
-        const uint2 uk = *reinterpret_cast<const uint2*>(raw + 1 * 16384 + r * 256 + 8 * lane);
         const float2 q0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uq.x));
         const float2 q1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uq.y));
-        const float2 k0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uk.x));
-        const float2 k1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uk.y));
         sq[m] = q0.x * q0.x + q0.y * q0.y + q1.x * q1.x + q1.y * q1.y;
-        sk[m] = k0.x * k0.x + k0.y * k0.y + k1.x * k1.x + k1.y * k1.y;
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-          sq[m] += __shfl_xor_sync(0xffffffffu, sq[m], o);
-          sk[m] += __shfl_xor_sync(0xffffffffu, sk[m], o);
-        }
-      if (lane < 8) {
-        const int r = warp + 8 * lane;
-        float vq = sq[0], vk = sk[0];
+        for (int m = 0; m < 4; ++m) sq[m] += __shfl_xor_sync(0xffffffffu, sq[m], o);
+      if (lane < 4) {
+        const int r = warp + 16 * lane;
+        float vq = sq[0];
 #pragma unroll
-        for (int m = 1; m < 8; ++m)
-          if (lane == m) { vq = sq[m]; vk = sk[m]; }
+        for (int m = 1; m < 4; ++m)
+          if (lane == m) vq = sq[m];
         vec[kVecIq + r] = r < len ? rsqrtf(vq + kNormEps) : 0.f;
-        vec[kVecIk + r] = r < len ? rsqrtf(vk + kNormEps) : 0.f;
       }
     }
-    // ---- gate and chunk-local cumsum for channel j, rows 32hf..32hf+31
-    float E[32];
+    // ---- gate and cumsum of channel j over sub-tile qq; E = e^{Gam_r - rho_qq}
+    //      depends only on this sub-tile's own partial sums
+    float E[16], Ei[16];
     {
       if (p.g) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int r = 32 * hf + i;
+        for (int i = 0; i < 16; ++i) {
+          const int r = 16 * qq + i;
           E[i] = r < len ? p.g[((size_t)(tok0 + r) * H + h) * kD + j] : 0.f;
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) E[i] = raw_at(raw, 2, 32 * hf + i, j);
+        for (int i = 0; i < 16; ++i) E[i] = raw_at(raw, 2, 16 * qq + i, j);
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          E[i] = (32 * hf + i < len) ? __fdividef(kGateMin, 1.0f + __expf(-expA * E[i])) : 0.f;
+        for (int i = 0; i < 16; ++i)
+          E[i] = (16 * qq + i < len) ? __fdividef(kGateMin, 1.0f + __expf(-expA * E[i])) : 0.f;
       }
 #pragma unroll
-      for (int i = 1; i < 32; ++i) E[i] += E[i - 1];
-      if (hf == 0) vec[kVecTot + j] = E[31];
+      for (int i = 1; i < 16; ++i) E[i] += E[i - 1];
+      vec[kVecTot + qq * 128 + j] = E[15];
+      vec[kVecRho + qq * 128 + j] = E[0];  // sub-tile-local; the offsets are added below
+#pragma unroll
+      for (int i = 15; i >= 0; --i) {
+        E[i] = __expf(E[i] - E[0]);
+        Ei[i] = __fdividef(1.0f, E[i]);
+      }
     }
     __syncthreads();
+    // rho_b = Gam at the first token of sub-tile b; Gam_last = Gam at row 63
+    float rho[4], glast;
     {
-      const float off = hf ? vec[kVecTot + j] : 0.f;
+      float acc = 0.f;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) E[i] += off;
-      vec[kVecRho + (2 * hf) * 128 + j] = E[0];
-      vec[kVecRho + (2 * hf + 1) * 128 + j] = E[16];
-      if (hf == 1) vec[kVecGlast + j] = E[31];
+      for (int bb = 0; bb < 4; ++bb) {
+        rho[bb] = acc + vec[kVecRho + bb * 128 + j];
+        acc += vec[kVecTot + bb * 128 + j];
+      }
+      glast = acc;
     }
-    __syncthreads();
-    float rho[4];
-#pragma unroll
-    for (int bb = 0; bb < 4; ++bb) rho[bb] = vec[kVecRho + bb * 128 + j];
-    const float glast = vec[kVecGlast + j];
-    const float rho0 = hf ? rho[2] : rho[0], rho1 = hf ? rho[3] : rho[1];
-    float Ei[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      E[i] = __expf(E[i] - (i < 16 ? rho0 : rho1));
-      Ei[i] = __fdividef(1.0f, E[i]);
-    }
+    const float rq = qq == 0 ? rho[0] : qq == 1 ? rho[1] : qq == 2 ? rho[2] : rho[3];
 
     // ---- product operands R (rows, MN-major) and C_b (columns, MN-major)
     {
-      float F0[4], F1[4];  // e^{rho_bb - rho_bt} for bt = this half's two sub-tiles
 #pragma unroll
-      for (int bb = 0; bb < 4; ++bb) {
-        F0[bb] = __expf(rho[bb] - rho0);
-        F1[bb] = __expf(rho[bb] - rho1);
-      }
-#pragma unroll
-      for (int g8 = 0; g8 < 4; ++g8) {
-        const int r0 = 32 * hf + 8 * g8, bt = r0 >> 4, rr0 = r0 & 15;
+      for (int g8 = 0; g8 < 2; ++g8) {
+        const int r0 = 16 * qq + 8 * g8;
         float kv[8], qv[8], cv[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int r = r0 + i;
-          const float e = E[8 * g8 + i];
-          const float kh = r < len ? raw_at(raw, 1, r, j) * vec[kVecIk + r] : 0.f;
-          const float qh = r < len ? raw_at(raw, 0, r, j) * vec[kVecIq + r] : 0.f;
-          kv[i] = kh * e;
-          qv[i] = qh * e;
+          const float kh = r < len ? raw_at(raw, 1, r, j) : 0.f;
+          const float qh = r < len ? raw_at(raw, 0, r, j) : 0.f;
+          kv[i] = kh * E[8 * g8 + i];
+          qv[i] = qh * E[8 * g8 + i];
           cv[i] = kh * Ei[8 * g8 + i];
         }
-        st16(sm + L::kR, mnmaj(32 * bt + rr0, j, 2048), kv);
-        st16(sm + L::kR, mnmaj(32 * bt + 16 + rr0, j, 2048), qv);
-        const float* F = (g8 & 2) ? F1 : F0;
+        st16(sm + L::kR, mnmaj(32 * qq + 8 * g8, j, 2048), kv);
+        st16(sm + L::kR, mnmaj(32 * qq + 16 + 8 * g8, j, 2048), qv);
 #pragma unroll
         for (int bb = 0; bb < 4; ++bb) {
-          if (bb < bt) continue;
+          if (bb < qq) continue;
           float w8[8];
+          const float f = bb == qq ? 1.f : __expf(rho[bb] - rq);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) w8[i] = bb == bt ? cv[i] : cv[i] * F[bb];
-          st16(sm + L::kCc, mnmaj(cbase[bb] + r0, j, 2560), w8);
+          for (int i = 0; i < 8; ++i) w8[i] = cv[i] * f;
+          st16(sm + L::kCc, mnmaj(8 * bb * (bb + 1) + r0, j, 2560), w8);
         }
       }
     }
@@ -400,38 +389,45 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
     // ---- M1: four M=64 MMAs -> TMEM [32b, +32): cols 0-15 A_kk^T, 16-31 A_qk^T
     if (tid == 0) {
       constexpr uint32_t id = instr_desc(kFmtBF16, 64, 32, true, true);
-      for (int bb = 0; bb < 4; ++bb) {
-        const uint32_t abase = smem_u32(sm + L::kCc) + (cbase[bb] >> 3) * 128;
-        const uint32_t bbase = smem_u32(sm + L::kR) + (32 * bb >> 3) * 128;
-        for (int k = 0; k < 8; ++k)
-          mma_bf16(tm + kTmA + 32 * bb, smem_desc(abase + 2 * 2560 * k, 2560, 128),
-                   smem_desc(bbase + 2 * 2048 * k, 2048, 128), id, k > 0);
-      }
+      const uint64_t ad = smem_desc(smem_u32(sm + L::kCc), 2560, 128);
+      const uint64_t bd = smem_desc(smem_u32(sm + L::kR), 2048, 128);
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb)
+#pragma unroll
+        for (int k = 0; k < 8; ++k)  // descriptor addresses count 16-byte units
+          mma_bf16(tm + kTmA + 32 * bb, ad + ((bb * (bb + 1) * 128 + 2 * 2560 * k) >> 4),
+                   bd + ((32 * bb * 16 + 2 * 2048 * k) >> 4), id, k > 0);
       mma_commit(&s_bar);
     }
     if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
-    // ---- A_kk (fp32 smem, beta-scaled, strictly lower) and A_qk (bf16 A3, MN-major)
+    // ---- A products -> key norms (diagonal), A_kk (fp32 smem, beta- and
+    //      norm-scaled, strictly lower) and A_qk (bf16 A3, MN-major)
     float* Akk = reinterpret_cast<float*>(sm + L::kAkk);
     {
-      const int i = r64;  // column of A (row of the M=64 accumulator)
+      const int i = r64, bb = cq;  // warp: lane quarter q4, row block bb
+      float va[16], vq[16];
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmA + 32 * bb), va);
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmA + 32 * bb + 16), vq);
+      tmem_ld_wait();
+      if (m64 && bb == q4) {
+        float dk = va[0];
 #pragma unroll
-      for (int b2 = 0; b2 < 2; ++b2) {
-        const int bb = 2 * ch + b2;
-        float va[16], vq[16];
-        tmem_ld16(tmem_addr(tm, 32 * q4, kTmA + 32 * bb), va);
-        tmem_ld16(tmem_addr(tm, 32 * q4, kTmA + 32 * bb + 16), vq);
-        tmem_ld_wait();
-        if (m64) {
+        for (int cc = 1; cc < 16; ++cc)
+          if (cc == lane) dk = va[cc];
+        vec[kVecIk + i] = i < len ? rsqrtf(dk + kNormEps) : 0.f;
+      }
+      __syncthreads();
+      if (m64) {
+        const float ki = vec[kVecIk + i];
 #pragma unroll
-          for (int cc = 0; cc < 16; ++cc) {
-            const int r = 16 * bb + cc;
-            Akk[r * 65 + i] = (i < r) ? vec[kVecBeta + r] * va[cc] : 0.f;
-            vq[cc] = (i <= r) ? vq[cc] : 0.f;
-          }
-          if (MODE == 0) {
-            st16(sm + L::kA3, mnmaj(16 * bb, i, 1024), vq);
-            st16(sm + L::kA3, mnmaj(16 * bb + 8, i, 1024), vq + 8);
-          }
+        for (int cc = 0; cc < 16; ++cc) {
+          const int r = 16 * bb + cc;
+          Akk[r * kLd + i] = (i < r) ? vec[kVecBeta + r] * vec[kVecIk + r] * ki * va[cc] : 0.f;
+          vq[cc] = (i <= r) ? vq[cc] * ki : 0.f;
+        }
+        if (MODE == 0) {
+          st16(sm + L::kA3, mnmaj(16 * bb, i, 1024), vq);
+          st16(sm + L::kA3, mnmaj(16 * bb + 8, i, 1024), vq + 8);
         }
       }
     }
@@ -441,8 +437,10 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
     // diagonal 16x16 blocks by forward substitution (registers), then the
     // blocks below them by merging: [[P,0],[B,Q]]^{-1} has lower-left block
     // -Q^{-1} B P^{-1}; first 16 -> 32 (block pairs 0|1 and 2|3), then 32 -> 64.
+    // The merges use 2x2 register tiles; the two upper blocks they read are
+    // zeroed first.
     float* Tf = reinterpret_cast<float*>(sm + L::kTf);
-    float* Y = vec + kVecY;  // scratch, up to 32 x 32 (stride 33)
+    float* Y = vec + kVecY;  // scratch, 32 x 36
     if (tid < kC) {
       const int bk = tid >> 4, cc = tid & 15, base = 16 * bk;
       float x[16];
@@ -450,93 +448,103 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
       for (int rr = 0; rr < 16; ++rr) {
         float acc = (rr == cc) ? 1.f : 0.f;
 #pragma unroll
-        for (int i = 0; i < rr; ++i) acc -= Akk[(base + rr) * 65 + base + i] * x[i];
+        for (int i = 0; i < rr; ++i) acc -= Akk[(base + rr) * kLd + base + i] * x[i];
         x[rr] = (rr < cc) ? 0.f : acc;
       }
 #pragma unroll
-      for (int rr = 0; rr < 16; ++rr) Tf[(base + rr) * 65 + base + cc] = x[rr];
+      for (int rr = 0; rr < 16; ++rr) Tf[(base + rr) * kLd + base + cc] = x[rr];
+    } else {
+      // zero T[0:16][16:32] and T[32:48][48:64]
+      const int e = tid - kC;  // 0..447
+      if (e < 512 - kC) {
+        for (int f = e; f < 512; f += 512 - kC) {
+          const int blk = f >> 8, rr = (f >> 4) & 15, cc = f & 15;
+          Tf[(32 * blk + rr) * kLd + 32 * blk + 16 + cc] = 0.f;
+        }
+      }
     }
     __syncthreads();
-    {
-      // 16 -> 32: for pair pr (blocks 2pr, 2pr+1): Y = A[hi][lo] T[lo][lo]; T[hi][lo] = -T[hi][hi] Y
-      const int pr = tid >> 7, e = tid & 127, rr = e >> 3, c2 = (e & 7) * 2;  // 2 outputs
+    if (tid < 128) {
+      // 16 -> 32, pair pr: Y = A[hi][lo] T[lo][lo]; T[hi][lo] = -T[hi][hi] Y (2x2 tiles)
+      const int pr = tid >> 6, r2 = ((tid >> 3) & 7) * 2, c2 = (tid & 7) * 2;
       const int lo = 32 * pr, hi = lo + 16;
-      float y0 = 0.f, y1 = 0.f;
+      float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const float av = Akk[(hi + rr) * 65 + lo + i];
-        y0 += av * Tf[(lo + i) * 65 + lo + c2];
-        y1 += av * Tf[(lo + i) * 65 + lo + c2 + 1];
+        const float a0 = Akk[(hi + r2) * kLd + lo + i], a1 = Akk[(hi + r2 + 1) * kLd + lo + i];
+        const float2 t = *reinterpret_cast<const float2*>(Tf + (lo + i) * kLd + lo + c2);
+        y00 += a0 * t.x; y01 += a0 * t.y; y10 += a1 * t.x; y11 += a1 * t.y;
       }
-      Y[pr * 528 + rr * 33 + c2] = y0;
-      Y[pr * 528 + rr * 33 + c2 + 1] = y1;
-      __syncthreads();
-      float t0 = 0.f, t1 = 0.f;
+      float* Yp = Y + pr * 16 * 34;
+      *reinterpret_cast<float2*>(Yp + r2 * 34 + c2) = make_float2(y00, y01);
+      *reinterpret_cast<float2*>(Yp + (r2 + 1) * 34 + c2) = make_float2(y10, y11);
+      __syncwarp();
+      // all of this pair's Y rows come from the same two warps: sync those
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + pr), "r"(64) : "memory");
+      float t00 = 0.f, t01 = 0.f, t10 = 0.f, t11 = 0.f;
 #pragma unroll
       for (int m = 0; m < 16; ++m) {
-        const float tv = Tf[(hi + rr) * 65 + hi + m];
-        t0 += tv * Y[pr * 528 + m * 33 + c2];
-        t1 += tv * Y[pr * 528 + m * 33 + c2 + 1];
+        const float a0 = Tf[(hi + r2) * kLd + hi + m], a1 = Tf[(hi + r2 + 1) * kLd + hi + m];
+        const float2 y = *reinterpret_cast<const float2*>(Yp + m * 34 + c2);
+        t00 += a0 * y.x; t01 += a0 * y.y; t10 += a1 * y.x; t11 += a1 * y.y;
       }
-      Tf[(hi + rr) * 65 + lo + c2] = -t0;
-      Tf[(hi + rr) * 65 + lo + c2 + 1] = -t1;
+      *reinterpret_cast<float2*>(Tf + (hi + r2) * kLd + lo + c2) = make_float2(-t00, -t01);
+      *reinterpret_cast<float2*>(Tf + (hi + r2 + 1) * kLd + lo + c2) = make_float2(-t10, -t11);
     }
     __syncthreads();
-    {
+    if (tid < 256) {
       // 32 -> 64: Y = A[32:64][0:32] T[0:32][0:32]; T[32:64][0:32] = -T[32:64][32:64] Y
-      const int rr = tid >> 3, c4 = (tid & 7) * 4;  // 4 outputs
-      float y[4] = {0.f, 0.f, 0.f, 0.f};
+      const int r2 = (tid >> 4) * 2, c2 = (tid & 15) * 2;
+      float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
 #pragma unroll 8
       for (int i = 0; i < 32; ++i) {
-        const float av = Akk[(32 + rr) * 65 + i];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) y[u] += av * (i >= c4 + u ? Tf[i * 65 + c4 + u] : 0.f);
+        const float a0 = Akk[(32 + r2) * kLd + i], a1 = Akk[(33 + r2) * kLd + i];
+        const float2 t = *reinterpret_cast<const float2*>(Tf + i * kLd + c2);
+        y00 += a0 * t.x; y01 += a0 * t.y; y10 += a1 * t.x; y11 += a1 * t.y;
       }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) Y[rr * 33 + c4 + u] = y[u];
-      __syncthreads();
-      float t[4] = {0.f, 0.f, 0.f, 0.f};
+      *reinterpret_cast<float2*>(Y + r2 * 34 + c2) = make_float2(y00, y01);
+      *reinterpret_cast<float2*>(Y + (r2 + 1) * 34 + c2) = make_float2(y10, y11);
+      asm volatile("bar.sync %0, %1;" ::"r"(3), "r"(256) : "memory");
+      float t00 = 0.f, t01 = 0.f, t10 = 0.f, t11 = 0.f;
 #pragma unroll 8
       for (int m = 0; m < 32; ++m) {
-        const float tv = m <= rr ? Tf[(32 + rr) * 65 + 32 + m] : 0.f;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) t[u] += tv * Y[m * 33 + c4 + u];
+        const float a0 = Tf[(32 + r2) * kLd + 32 + m], a1 = Tf[(33 + r2) * kLd + 32 + m];
+        const float2 y = *reinterpret_cast<const float2*>(Y + m * 34 + c2);
+        t00 += a0 * y.x; t01 += a0 * y.y; t10 += a1 * y.x; t11 += a1 * y.y;
       }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) Tf[(32 + rr) * 65 + c4 + u] = -t[u];
+      *reinterpret_cast<float2*>(Tf + (32 + r2) * kLd + c2) = make_float2(-t00, -t01);
+      *reinterpret_cast<float2*>(Tf + (33 + r2) * kLd + c2) = make_float2(-t10, -t11);
     }
     __syncthreads();
-    // T -> bf16 A operand (K-major), upper triangle zero
-    for (int e = tid; e < kC * 8; e += kNT) {
-      const int r = e >> 3, i0 = (e & 7) * 8;
+    // T -> bf16 A operand (K-major), upper triangle zero; 8 consecutive threads
+    // take 8 consecutive rows so each 16-byte store phase is conflict-free
+    {
+      const int r = (tid >> 6) * 8 + (tid & 7), i0 = ((tid >> 3) & 7) * 8;
       float t8[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) t8[i] = (i0 + i <= r) ? Tf[r * 65 + i0 + i] : 0.f;
+      for (int i = 0; i < 8; ++i) t8[i] = (i0 + i <= r) ? Tf[r * kLd + i0 + i] : 0.f;
       st16(sm + L::kTop, kmaj(r, i0, 1024), t8);
     }
     __syncthreads();  // A_kk / T (fp32) are dead from here: region P takes X, Q', K'
 
     // ---- WY / chain operands: X_K, X_V (K-major), Q' (MN-major), K' (K-major), gamma
     {
-      const float er0 = __expf(rho0), er1 = __expf(rho1);
-      const float el0 = __expf(glast - rho0), el1 = __expf(glast - rho1);
-      if (hf == 0) vec[kVecGam + j] = __expf(glast);
+      const float er = __expf(rq), el = __expf(glast - rq);
+      if (qq == 0) vec[kVecGam + j] = __expf(glast);
 #pragma unroll
-      for (int g8 = 0; g8 < 4; ++g8) {
-        const int r0 = 32 * hf + 8 * g8;
-        const float er = g8 < 2 ? er0 : er1, el = g8 < 2 ? el0 : el1;
+      for (int g8 = 0; g8 < 2; ++g8) {
+        const int r0 = 16 * qq + 8 * g8;
         float xk[8], xv[8], qp[8], kp[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int r = r0 + i;
           const bool in = r < len;
-          const float e = E[8 * g8 + i];
           const float kh = in ? raw_at(raw, 1, r, j) * vec[kVecIk + r] : 0.f;
           const float bet = vec[kVecBeta + r];
-          xk[i] = bet * kh * e * er;
+          xk[i] = bet * kh * E[8 * g8 + i] * er;
           xv[i] = in ? bet * raw_at(raw, 3, r, j) : 0.f;
           kp[i] = kh * Ei[8 * g8 + i] * el;
-          if (MODE == 0) qp[i] = in ? raw_at(raw, 0, r, j) * vec[kVecIq + r] * e * er : 0.f;
+          if (MODE == 0) qp[i] = in ? raw_at(raw, 0, r, j) * E[8 * g8 + i] * er : 0.f;
         }
         st16(sm + L::kX, kmaj(j, r0, 1024), xk);
         st16(sm + L::kX, kmaj(128 + j, r0, 1024), xv);
@@ -553,26 +561,26 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
     // ---- M2: [W | U~] = T [X_K | X_V]  (M=64, N=256, K=64)
     if (tid == 0) {
       constexpr uint32_t id = instr_desc(kFmtBF16, 64, 256, false, false);
-      const uint32_t abase = smem_u32(sm + L::kTop), bbase = smem_u32(sm + L::kX);
-      for (int k = 0; k < 4; ++k)
-        mma_bf16(tm + kTmWU, smem_desc(abase + 256 * k, 128, 1024),
-                 smem_desc(bbase + 256 * k, 128, 1024), id, k > 0);
+      const uint64_t ad = smem_desc(smem_u32(sm + L::kTop), 128, 1024);
+      const uint64_t bd = smem_desc(smem_u32(sm + L::kX), 128, 1024);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mma_bf16(tm + kTmWU, ad + 16 * k, bd + 16 * k, id, k > 0);
       mma_commit(&s_bar);
     }
     if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
     // ---- W -> bf16 A operand (K-major); U~ -> registers (M=64 rows, lane < 16)
-    float ut[64];
+    float ut[32];
 #pragma unroll
-    for (int c16 = 0; c16 < 64; c16 += 16) {
+    for (int c16 = 0; c16 < 32; c16 += 16) {
       float w16[16], u16[16];
-      tmem_ld16(tmem_addr(tm, 32 * q4, kTmWU + 64 * ch + c16), w16);
-      tmem_ld16(tmem_addr(tm, 32 * q4, kTmWU + 128 + 64 * ch + c16), u16);
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmWU + 32 * cq + c16), w16);
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmWU + 128 + 32 * cq + c16), u16);
       tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 16; ++i) ut[c16 + i] = u16[i];
       if (m64) {
-        st16(sm + L::kW, kmaj(r64, 64 * ch + c16, 2048), w16);
-        st16(sm + L::kW, kmaj(r64, 64 * ch + c16 + 8, 2048), w16 + 8);
+        st16(sm + L::kW, kmaj(r64, 32 * cq + c16, 2048), w16);
+        st16(sm + L::kW, kmaj(r64, 32 * cq + c16 + 8, 2048), w16 + 8);
       }
     }
     // ---- decay the state(s) by gamma = e^{Gam_last} (rows = dk = TMEM lanes)
@@ -581,33 +589,32 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
       constexpr int NB = MODE == 0 ? 1 : 2;
 #pragma unroll
       for (int blk = 0; blk < NB; ++blk)
+      {
+        float s0[16], s1[16];
+        const uint32_t col = kTmS + 128 * blk + 32 * cq;
+        tmem_ld16(tmem_addr(tm, 32 * q4, col), s0);
+        tmem_ld16(tmem_addr(tm, 32 * q4, col + 16), s1);
+        tmem_ld_wait();
 #pragma unroll
-        for (int c16 = 0; c16 < 64; c16 += 16) {
-          float s16[16];
-          const uint32_t col = kTmS + 128 * blk + 64 * ch + c16;
-          tmem_ld16(tmem_addr(tm, 32 * q4, col), s16);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) s16[i] *= gm;
-          tmem_st16(tmem_addr(tm, 32 * q4, col), s16);
-        }
+        for (int i = 0; i < 16; ++i) { s0[i] *= gm; s1[i] *= gm; }
+        tmem_st16(tmem_addr(tm, 32 * q4, col), s0);
+        tmem_st16(tmem_addr(tm, 32 * q4, col + 16), s1);
+      }
       tmem_st_wait();
     }
     sync_for_mma();
     // ---- C1: D_W = W S (M=64, N=128|256), D_Q = Q' S (M=64, N=128)
     if (tid == 0) {
-      const uint32_t sb = smem_u32(sm + L::kSb);
-      const uint32_t wb = smem_u32(sm + L::kW);
+      const uint64_t sd = smem_desc(smem_u32(sm + L::kSb), SbL, 128);
+      const uint64_t wd = smem_desc(smem_u32(sm + L::kW), 128, 2048);
       constexpr uint32_t idw = instr_desc(kFmtBF16, 64, SbN, false, true);
-      for (int k = 0; k < 8; ++k)
-        mma_bf16(tm + kTmW, smem_desc(wb + 256 * k, 128, 2048),
-                 smem_desc(sb + 2 * SbL * k, SbL, 128), idw, k > 0);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mma_bf16(tm + kTmW, wd + 16 * k, sd + (2 * SbL >> 4) * k, idw, k > 0);
       if (MODE == 0) {
         constexpr uint32_t idq = instr_desc(kFmtBF16, 64, 128, true, true);
-        const uint32_t qb = smem_u32(sm + L::kQp);
-        for (int k = 0; k < 8; ++k)
-          mma_bf16(tm + kTmQ, smem_desc(qb + 2 * 1024 * k, 1024, 128),
-                   smem_desc(sb + 2 * SbL * k, SbL, 128), idq, k > 0);
+        const uint64_t qd = smem_desc(smem_u32(sm + L::kQp), 1024, 128);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mma_bf16(tm + kTmQ, qd + 128 * k, sd + (2 * SbL >> 4) * k, idq, k > 0);
       }
       mma_commit(&s_bar);
     }
@@ -617,34 +624,38 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
       constexpr int NB = MODE == 0 ? 1 : 2;
 #pragma unroll
       for (int blk = 0; blk < NB; ++blk)
+      {
+        float d0[16], d1[16];
+        const int col = 128 * blk + 32 * cq;
+        tmem_ld16(tmem_addr(tm, 32 * q4, kTmW + col), d0);
+        tmem_ld16(tmem_addr(tm, 32 * q4, kTmW + col + 16), d1);
+        tmem_ld_wait();
+        if (m64) {
 #pragma unroll
-        for (int c16 = 0; c16 < 64; c16 += 16) {
-          float d16[16];
-          const int col = 128 * blk + 64 * ch + c16;
-          tmem_ld16(tmem_addr(tm, 32 * q4, kTmW + col), d16);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) d16[i] = (blk == 0 ? ut[c16 + i] : 0.f) - d16[i];
-          if (m64) {
-            st16(sm + L::kU, mnmaj(col, r64, SbL), d16);
-            st16(sm + L::kU, mnmaj(col + 8, r64, SbL), d16 + 8);
+          for (int i = 0; i < 16; ++i) {
+            d0[i] = (blk == 0 ? ut[i] : 0.f) - d0[i];
+            d1[i] = (blk == 0 ? ut[16 + i] : 0.f) - d1[i];
           }
+          st16(sm + L::kU, mnmaj(col, r64, SbL), d0);
+          st16(sm + L::kU, mnmaj(col + 8, r64, SbL), d0 + 8);
+          st16(sm + L::kU, mnmaj(col + 16, r64, SbL), d1);
+          st16(sm + L::kU, mnmaj(col + 24, r64, SbL), d1 + 8);
         }
+      }
     }
     sync_for_mma();
     // ---- C2: S += K'^T U (M=128); D_Q += A_qk U (M=64)
     if (tid == 0) {
-      const uint32_t kb = smem_u32(sm + L::kKp), ub = smem_u32(sm + L::kU);
+      const uint64_t kd = smem_desc(smem_u32(sm + L::kKp), 128, 1024);
+      const uint64_t ud = smem_desc(smem_u32(sm + L::kU), SbL, 128);
       constexpr uint32_t ids = instr_desc(kFmtBF16, 128, SbN, false, true);
-      for (int k = 0; k < 4; ++k)
-        mma_bf16(tm + kTmS, smem_desc(kb + 256 * k, 128, 1024),
-                 smem_desc(ub + 2 * SbL * k, SbL, 128), ids, 1);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mma_bf16(tm + kTmS, kd + 16 * k, ud + (2 * SbL >> 4) * k, ids, 1);
       if (MODE == 0) {
         constexpr uint32_t ido = instr_desc(kFmtBF16, 64, 128, true, true);
-        const uint32_t a3 = smem_u32(sm + L::kA3);
-        for (int k = 0; k < 4; ++k)
-          mma_bf16(tm + kTmQ, smem_desc(a3 + 2 * 1024 * k, 1024, 128),
-                   smem_desc(ub + 2 * SbL * k, SbL, 128), ido, 1);
+        const uint64_t a3 = smem_desc(smem_u32(sm + L::kA3), 1024, 128);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) mma_bf16(tm + kTmQ, a3 + 128 * k, ud + (2 * SbL >> 4) * k, ido, 1);
       }
       mma_commit(&s_bar);
     }
@@ -654,26 +665,31 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
       constexpr int NB = MODE == 0 ? 1 : 2;
 #pragma unroll
       for (int blk = 0; blk < NB; ++blk)
-#pragma unroll
-        for (int c16 = 0; c16 < 64; c16 += 16) {
-          float s16[16];
-          const int col = 128 * blk + 64 * ch + c16;
-          tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + col), s16);
-          tmem_ld_wait();
-          st16(sm + L::kSb, mnmaj(col, srow, SbL), s16);
-          st16(sm + L::kSb, mnmaj(col + 8, srow, SbL), s16 + 8);
-        }
+      {
+        float s0[16], s1[16];
+        const int col = 128 * blk + 32 * cq;
+        tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + col), s0);
+        tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + col + 16), s1);
+        tmem_ld_wait();
+        st16(sm + L::kSb, mnmaj(col, srow, SbL), s0);
+        st16(sm + L::kSb, mnmaj(col + 8, srow, SbL), s0 + 8);
+        st16(sm + L::kSb, mnmaj(col + 16, srow, SbL), s1);
+        st16(sm + L::kSb, mnmaj(col + 24, srow, SbL), s1 + 8);
+      }
       if (MODE == 0) {
+        float o0[16], o1[16];
+        tmem_ld16(tmem_addr(tm, 32 * q4, kTmQ + 32 * cq), o0);
+        tmem_ld16(tmem_addr(tm, 32 * q4, kTmQ + 32 * cq + 16), o1);
+        tmem_ld_wait();
+        if (m64 && r64 < len) {
+          const float iq = vec[kVecIq + r64];
 #pragma unroll
-        for (int c16 = 0; c16 < 64; c16 += 16) {
-          float o16[16];
-          tmem_ld16(tmem_addr(tm, 32 * q4, kTmQ + 64 * ch + c16), o16);
-          tmem_ld_wait();
-          if (m64 && r64 < len) {
-            uint4* dst = reinterpret_cast<uint4*>(p.o + ((size_t)(tok0 + r64) * H + h) * kD + 64 * ch + c16);
-            dst[0] = pack8(o16);
-            dst[1] = pack8(o16 + 8);
-          }
+          for (int i = 0; i < 16; ++i) { o0[i] *= iq; o1[i] *= iq; }
+          uint4* dst = reinterpret_cast<uint4*>(p.o + ((size_t)(tok0 + r64) * H + h) * kD + 32 * cq);
+          dst[0] = pack8(o0);
+          dst[1] = pack8(o0 + 8);
+          dst[2] = pack8(o1);
+          dst[3] = pack8(o1 + 8);
         }
       }
     }
@@ -688,13 +704,13 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
       if (p.S_final && seg == p.P - 1) {
         float* dst = p.S_final + ((size_t)n * H + h) * kD * kD + (size_t)srow * kD;
 #pragma unroll
-        for (int c16 = 0; c16 < 64; c16 += 16) {
+        for (int c16 = 0; c16 < 32; c16 += 16) {
           float s16[16];
-          tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + 64 * ch + c16), s16);
+          tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + 32 * cq + c16), s16);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4*>(dst + 64 * ch + c16 + i) = make_float4(s16[i], s16[i + 1], s16[i + 2], s16[i + 3]);
+            *reinterpret_cast<float4*>(dst + 32 * cq + c16 + i) = make_float4(s16[i], s16[i + 1], s16[i + 2], s16[i + 3]);
         }
       }
     } else {
@@ -704,11 +720,11 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
 #pragma unroll
       for (int blk = 0; blk < 2; ++blk)
 #pragma unroll
-        for (int c16 = 0; c16 < 64; c16 += 16) {
+        for (int c16 = 0; c16 < 32; c16 += 16) {
           float s16[16];
-          tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + 128 * blk + 64 * ch + c16), s16);
+          tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + 128 * blk + 32 * cq + c16), s16);
           tmem_ld_wait();
-          float* dst = (blk == 0 ? Nt : Mt) + (size_t)srow * kD + 64 * ch + c16;
+          float* dst = (blk == 0 ? Nt : Mt) + (size_t)srow * kD + 32 * cq + c16;
 #pragma unroll
           for (int i = 0; i < 16; i += 4)
             *reinterpret_cast<float4*>(dst + i) = make_float4(s16[i], s16[i + 1], s16[i + 2], s16[i + 3]);
