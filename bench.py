@@ -85,7 +85,7 @@ def recorded_traffic(kind):
 
 
 class ClockSampler:
-    """nvidia-smi clocks/throttle reasons sampled every 200 ms while running."""
+    """nvidia-smi clocks/throttle reasons sampled every 20 ms while running."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -100,7 +100,7 @@ class ClockSampler:
             self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -136,6 +136,22 @@ class ClockSampler:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def max_over_ranks(x, world, device=None):
+    """Max of a per-rank scalar over all ranks (identity for one rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(units_per_rank, world, ms_max):
+    """Whole-job throughput: every rank processed units_per_rank in ms_max."""
+    return world * units_per_rank / (ms_max / 1e3)
 
 
 def oracle_baseline(inp, n_tokens):
@@ -183,7 +199,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--L", type=int, default=L_DEFAULT, help="prefill length (sweep)")
@@ -214,12 +230,8 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def rank_max(x):
+        return max_over_ranks(x, world, dev)
 
     L = args.L
     T = B * L
@@ -254,9 +266,9 @@ def main():
         torch.cuda.synchronize()
         barrier()
         ms_local = e0.elapsed_time(e1) / args.steps
-    ms = max_over_ranks(ms_local)
+    ms = rank_max(ms_local)
     clocks = clk.summary()
-    value = world * T / (ms / 1e3)
+    value = weak_scaling_value(T, world, ms)
 
     pk = peaks()
     fwd_bytes = alg_bytes_prefill(T)
@@ -297,8 +309,8 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / n_e2e)
-    e2e = {"value": world * T / (ms_e2e / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+    ms_e2e = rank_max(e0.elapsed_time(e1) / n_e2e)
+    e2e = {"value": weak_scaling_value(T, world, ms_e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h}
 
     # ----------------------------------------------------------- decode ---
@@ -326,7 +338,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     ms_dec_local = e0.elapsed_time(e1) / args.decode_steps
-    ms_dec = max_over_ranks(ms_dec_local)
+    ms_dec = rank_max(ms_dec_local)
     dec_bytes = alg_bytes_decode()
     dec_ach = dec_bytes / (ms_dec_local / 1e3) / 1e9
     decode = {"value": world * 1e3 / ms_dec, "unit": "steps/s", "ms_per_step": ms_dec,
