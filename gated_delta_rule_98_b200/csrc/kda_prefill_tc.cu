@@ -75,7 +75,7 @@ struct Smem {
 };
 // vectors (floats) at Smem::kVec
 constexpr int kVecIq = 0, kVecIk = 64, kVecBeta = 128, kVecGam = 192, kVecRho = 320,
-              kVecTot = 832, kVecGlast = 960, kVecY = 1088;  // Y: up to 32 x 36 floats
+              kVecTot = 832, kVecY = 1088;  // Y: up to 32 x 36 floats
 
 // TMEM columns.  M=64 accumulators put row r in lane 32 (r / 16) + r % 16.
 constexpr uint32_t kTmA = 0;     // A products, 4 x 32 columns (prep)
@@ -85,6 +85,27 @@ constexpr uint32_t kTmQ = 128;   // D_Q = Q' S (+ A_qk U)
 constexpr uint32_t kTmS = 256;   // fp32 state; identity-started block X at 384 (transition)
 
 constexpr int kLd = 68;  // row stride (floats) of the fp32 A_kk / T tiles
+
+// Chain operands of one (chunk, head), written by the transition pass and read
+// by the chain pass with one bulk copy.  The bf16 images have exactly the
+// shared-memory layouts the MMAs read: W (A, K-major, M=64 K=128), K' (A,
+// K-major, M=128 K=64), Q' (A, MN-major, M=64 K=128), A_qk (A, MN-major, M=64
+// K=64); U~ is fp32 in the order the chain threads read it (see ut_index);
+// then gamma (128 fp32) and the query row scales (64 fp32).
+constexpr int kSlotW = 0, kSlotK = 16384, kSlotQ = 32768, kSlotA3 = 49152, kSlotU = 57344,
+              kSlotGam = 90112, kSlotIq = 90624, kSlotBytes = 90880;
+// Chunk c of sequence n (first token a) has slot a / C + n + c: distinct for
+// every chunk of every sequence and below T / C + N.
+__device__ __forceinline__ unsigned char* chunk_slot(const unsigned char* prep_base, int a, int n,
+                                                     int c, int h, int H) {
+  return const_cast<unsigned char*>(prep_base) +
+         ((size_t)(a / 64 + n + c) * H + h) * (size_t)kSlotBytes;
+}
+// float index of U~ (row r = 16 q4 + l, l < 16; column 32 cq + 4 pc + e) in a
+// slot: each warp's 16 active lanes read 256 consecutive bytes per float4.
+__device__ __forceinline__ int ut_index(int q4, int cq, int pc, int l) {
+  return (((cq * 4 + q4) * 8 + pc) * 16 + l) * 4;
+}
 
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s: a wait this long is a fault
 
@@ -119,6 +140,7 @@ struct alignas(64) TcParams {
   float* S_final;
   int N, T, max_len, H, P;
   float* seg;  // per (n, h): transitions (M, N) of segments 0..P-2, incoming states of 0..P-1
+  unsigned char* prep;  // per (chunk slot, h): chain operands left by the transition pass
   WsHeader* hdr;
 };
 
@@ -183,8 +205,10 @@ __device__ __forceinline__ void sync_for_mma() {
 }
 
 // ---------------------------------------------------------------------------
-// MODE 0: full pass from the true incoming state, writes o and S_final.
-// MODE 1: transition pass of segments 0..P-2: from S = 0 (N) and X = I (M).
+// MODE 0: full pass from the true incoming state, writes o and S_final (used
+//         when the sequences are not split into segments).
+// MODE 1: transition pass: for segments 0..P-2, the chain from S = 0 (N) and
+//         X = I (M); for every segment, each chunk's chain operands to its slot.
 template <int MODE>
 __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcParams p) {
   using L = Smem<MODE>;
@@ -200,7 +224,7 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
   const int H = p.H;
 
   const bool ok = seqlens_valid(p.cu, p.N, p.T, p.max_len);
-  if (MODE == 0 && n == 0 && h == 0 && seg == 0 && tid == 0)
+  if (n == 0 && h == 0 && seg == 0 && tid == 0)
     p.hdr->err = ok ? kErrNone : kErrBadSeqlens;
   if (!ok) return;
   int a, b;
@@ -208,6 +232,8 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
   const int nch = (b - a + kC - 1) / kC;
   int c0, c1;
   segment_chunks(nch, p.P, seg, c0, c1);
+  // the last segment's transition is never used: its pass only fills slots
+  const bool chain = MODE == 0 || seg < p.P - 1;
 
   // ---- set-up: TMEM, barriers, first chunk's rows
   if (warp == 0) {
@@ -284,6 +310,7 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
   for (int c = c0; c < c1; ++c) {
     const int tok0 = a + c * kC;
     const int len = min(kC, b - tok0);
+    unsigned char* slot = MODE == 1 ? chunk_slot(p.prep, a, n, c, h, H) : nullptr;
     sync_for_mma();
     if (tid < kC) vec[kVecBeta + tid] = beta_next;
     beta_next = load_beta(c + 1);
@@ -425,10 +452,9 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
           Akk[r * kLd + i] = (i < r) ? vec[kVecBeta + r] * vec[kVecIk + r] * ki * va[cc] : 0.f;
           vq[cc] = (i <= r) ? vq[cc] * ki : 0.f;
         }
-        if (MODE == 0) {
-          st16(sm + L::kA3, mnmaj(16 * bb, i, 1024), vq);
-          st16(sm + L::kA3, mnmaj(16 * bb + 8, i, 1024), vq + 8);
-        }
+        unsigned char* a3 = MODE == 0 ? sm + L::kA3 : slot + kSlotA3;
+        st16(a3, mnmaj(16 * bb, i, 1024), vq);
+        st16(a3, mnmaj(16 * bb + 8, i, 1024), vq + 8);
       }
     }
     fence_before_sync();
@@ -530,7 +556,12 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
     // ---- WY / chain operands: X_K, X_V (K-major), Q' (MN-major), K' (K-major), gamma
     {
       const float er = __expf(rq), el = __expf(glast - rq);
-      if (qq == 0) vec[kVecGam + j] = __expf(glast);
+      if (qq == 0) {
+        const float gam = __expf(glast);
+        vec[kVecGam + j] = gam;
+        if (MODE == 1) reinterpret_cast<float*>(slot + kSlotGam)[j] = gam;
+      }
+      if (MODE == 1 && tid < kC) reinterpret_cast<float*>(slot + kSlotIq)[tid] = vec[kVecIq + tid];
 #pragma unroll
       for (int g8 = 0; g8 < 2; ++g8) {
         const int r0 = 16 * qq + 8 * g8;
@@ -544,12 +575,13 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
           xk[i] = bet * kh * E[8 * g8 + i] * er;
           xv[i] = in ? bet * raw_at(raw, 3, r, j) : 0.f;
           kp[i] = kh * Ei[8 * g8 + i] * el;
-          if (MODE == 0) qp[i] = in ? raw_at(raw, 0, r, j) * E[8 * g8 + i] * er : 0.f;
+          qp[i] = in ? raw_at(raw, 0, r, j) * E[8 * g8 + i] * er : 0.f;
         }
         st16(sm + L::kX, kmaj(j, r0, 1024), xk);
         st16(sm + L::kX, kmaj(128 + j, r0, 1024), xv);
-        st16(sm + L::kKp, kmaj(j, r0, 1024), kp);
-        if (MODE == 0) st16(sm + L::kQp, mnmaj(r0, j, 1024), qp);
+        if (chain) st16(sm + L::kKp, kmaj(j, r0, 1024), kp);
+        if (MODE == 1) st16(slot + kSlotK, kmaj(j, r0, 1024), kp);
+        st16(MODE == 0 ? sm + L::kQp : slot + kSlotQ, mnmaj(r0, j, 1024), qp);
       }
     }
     sync_for_mma();
@@ -578,11 +610,21 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
       tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 16; ++i) ut[c16 + i] = u16[i];
-      if (m64) {
+      if (m64 && chain) {
         st16(sm + L::kW, kmaj(r64, 32 * cq + c16, 2048), w16);
         st16(sm + L::kW, kmaj(r64, 32 * cq + c16 + 8, 2048), w16 + 8);
       }
+      if (MODE == 1 && m64) {
+        st16(slot + kSlotW, kmaj(r64, 32 * cq + c16, 2048), w16);
+        st16(slot + kSlotW, kmaj(r64, 32 * cq + c16 + 8, 2048), w16 + 8);
+        float4* ug = reinterpret_cast<float4*>(slot + kSlotU);
+#pragma unroll
+        for (int pc = 0; pc < 4; ++pc)
+          ug[ut_index(q4, cq, (c16 >> 2) + pc, lane) >> 2] =
+              make_float4(u16[4 * pc], u16[4 * pc + 1], u16[4 * pc + 2], u16[4 * pc + 3]);
+      }
     }
+    if (!chain) continue;
     // ---- decay the state(s) by gamma = e^{Gam_last} (rows = dk = TMEM lanes)
     {
       const float gm = vec[kVecGam + srow];
@@ -713,7 +755,7 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
             *reinterpret_cast<float4*>(dst + 32 * cq + c16 + i) = make_float4(s16[i], s16[i + 1], s16[i + 2], s16[i + 3]);
         }
       }
-    } else {
+    } else if (chain) {
       // transition: N from S (columns 256..383), M from X (columns 384..511)
       float* Mt = seg_trans(p.seg, n, h, H, p.P, seg);
       float* Nt = Mt + kD * kD;
@@ -733,6 +775,241 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
   } else if (raw_pending) {
     // a wait gave up: let the TMA load still in flight land before leaving
     mbar_wait_cycles(&s_bar_raw, phase_raw, kWaitCycles);
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tm, 512);
+}
+
+// Chain pass of a segmented sequence: only the state-dependent half of each
+// chunk, from the operands the transition pass stored in the chunk's slot.
+// Per chunk: D_W = W S and D_Q = Q' S (C1); S <- gamma S meanwhile; U = U~ - D_W;
+// S += K'^T U and D_Q += A_qk U (C2); o = D_Q scaled by the query row norms.
+// Slots are bulk-copied two chunks ahead into two stages.
+struct ChainSmem {
+  static constexpr int kSb = 0;         // S bf16, B operand (N=128, K=128), MN-major
+  static constexpr int kU = 32768;      // U bf16, B operand (N=128, K=64), MN-major
+  static constexpr int kStage = 49152;  // two slots
+  static constexpr int kBytes = kStage + 2 * kSlotBytes;
+};
+
+__global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ TcParams p) {
+  using L = ChainSmem;
+  extern __shared__ __align__(1024) unsigned char sm[];
+  __shared__ uint64_t s_bar, s_ld[2];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x, h = blockIdx.y, seg = blockIdx.z;
+  const int H = p.H;
+  if (!seqlens_valid(p.cu, p.N, p.T, p.max_len)) return;  // the error word is already set
+  int a, b;
+  seq_bounds(p.cu, n, p.max_len, a, b);
+  const int nch = (b - a + kC - 1) / kC;
+  int c0, c1;
+  segment_chunks(nch, p.P, seg, c0, c1);
+
+  if (warp == 0) {
+    tmem_alloc(&s_tmem, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&s_bar, 1);
+    mbar_init(&s_ld[0], 1);
+    mbar_init(&s_ld[1], 1);
+    fence_mbar_init();
+    s_abort = 0;
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tm = s_tmem;
+  auto load_slot = [&](int c) {  // single thread
+    const int s = (c - c0) & 1;
+    mbar_arrive_expect_tx(&s_ld[s], kSlotBytes);
+    bulk_g2s(sm + L::kStage + s * kSlotBytes, chunk_slot(p.prep, a, n, c, h, H), kSlotBytes,
+             &s_ld[s]);
+  };
+  if (tid == 0) {
+    if (c0 < c1) load_slot(c0);
+    if (c0 + 1 < c1) load_slot(c0 + 1);
+  }
+  uint32_t phase = 0, ph_ld = 0;  // ph_ld bit s: parity of stage s's next completion
+  uint32_t inflight = (c0 < c1 ? 1u : 0u) | (c0 + 1 < c1 ? 2u : 0u);  // stages being filled
+
+  const int q4 = warp & 3, cq = warp >> 2;  // TMEM lane quarter, 32-column quarter
+  const int srow = 32 * q4 + lane;          // dk row (M=128 accumulators)
+  const int r64 = 16 * q4 + lane;           // token row of M=64 accumulators (lane < 16)
+  const bool m64 = lane < 16;
+  constexpr int SbL = 2048;                 // K-group stride of the N=128 B operands
+
+  // ---- incoming state -> TMEM (fp32) and the bf16 operand
+  {
+    const float* S0 = seg > 0 ? seg_sin(p.seg, n, h, H, p.P, seg)
+                              : (p.S0 ? p.S0 + ((size_t)n * H + h) * kD * kD : nullptr);
+#pragma unroll
+    for (int c16 = 0; c16 < 32; c16 += 16) {
+      float v16[16];
+      const int col = 32 * cq + c16;
+      if (S0) {
+        const float4* src = reinterpret_cast<const float4*>(S0 + (size_t)srow * kD + col);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 f = src[i];
+          v16[4 * i] = f.x; v16[4 * i + 1] = f.y; v16[4 * i + 2] = f.z; v16[4 * i + 3] = f.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v16[i] = 0.f;
+      }
+      tmem_st16(tmem_addr(tm, 32 * q4, kTmS + col), v16);
+      st16(sm + L::kSb, mnmaj(col, srow, SbL), v16);
+      st16(sm + L::kSb, mnmaj(col + 8, srow, SbL), v16 + 8);
+    }
+    tmem_st_wait();
+  }
+
+  for (int c = c0; c < c1; ++c) {
+    const int tok0 = a + c * kC;
+    const int len = min(kC, b - tok0);
+    const int s = (c - c0) & 1;
+    unsigned char* st = sm + L::kStage + s * kSlotBytes;
+    sync_for_mma();
+    {
+      const bool got = mbar_wait_cycles(&s_ld[s], (ph_ld >> s) & 1, kWaitCycles);
+      if (__syncthreads_or(!got)) {
+        if (tid == 0) atomicOr(&p.hdr->err, kErrTimeout);
+        s_abort = 1;
+        break;
+      }
+      ph_ld ^= 1u << s;
+      inflight &= ~(1u << s);
+    }
+    // ---- C1: D_W = W S, D_Q = Q' S  (M=64, N=128, K=128)
+    if (tid == 0) {
+      const uint64_t sd = smem_desc(smem_u32(sm + L::kSb), SbL, 128);
+      const uint64_t wd = smem_desc(smem_u32(st + kSlotW), 128, 2048);
+      const uint64_t qd = smem_desc(smem_u32(st + kSlotQ), 1024, 128);
+      constexpr uint32_t idw = instr_desc(kFmtBF16, 64, 128, false, true);
+      constexpr uint32_t idq = instr_desc(kFmtBF16, 64, 128, true, true);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mma_bf16(tm + kTmW, wd + 16 * k, sd + (2 * SbL >> 4) * k, idw, k > 0);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mma_bf16(tm + kTmQ, qd + 128 * k, sd + (2 * SbL >> 4) * k, idq, k > 0);
+      mma_commit(&s_bar);
+    }
+    // ---- meanwhile decay the fp32 state by gamma (C1 reads the bf16 copy)
+    {
+      const float gm = reinterpret_cast<const float*>(st + kSlotGam)[srow];
+      float s0[16], s1[16];
+      const uint32_t col = kTmS + 32 * cq;
+      tmem_ld16(tmem_addr(tm, 32 * q4, col), s0);
+      tmem_ld16(tmem_addr(tm, 32 * q4, col + 16), s1);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) { s0[i] *= gm; s1[i] *= gm; }
+      tmem_st16(tmem_addr(tm, 32 * q4, col), s0);
+      tmem_st16(tmem_addr(tm, 32 * q4, col + 16), s1);
+      tmem_st_wait();
+    }
+    if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
+    // ---- U = U~ - D_W -> B operand (MN-major)
+    {
+      float d0[16], d1[16];
+      const int col = 32 * cq;
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmW + col), d0);
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmW + col + 16), d1);
+      tmem_ld_wait();
+      if (m64) {
+        const float4* ug = reinterpret_cast<const float4*>(st + kSlotU);
+#pragma unroll
+        for (int pc = 0; pc < 4; ++pc) {
+          const float4 u0 = ug[ut_index(q4, cq, pc, lane) >> 2];
+          const float4 u1 = ug[ut_index(q4, cq, pc + 4, lane) >> 2];
+          d0[4 * pc] = u0.x - d0[4 * pc];
+          d0[4 * pc + 1] = u0.y - d0[4 * pc + 1];
+          d0[4 * pc + 2] = u0.z - d0[4 * pc + 2];
+          d0[4 * pc + 3] = u0.w - d0[4 * pc + 3];
+          d1[4 * pc] = u1.x - d1[4 * pc];
+          d1[4 * pc + 1] = u1.y - d1[4 * pc + 1];
+          d1[4 * pc + 2] = u1.z - d1[4 * pc + 2];
+          d1[4 * pc + 3] = u1.w - d1[4 * pc + 3];
+        }
+        st16(sm + L::kU, mnmaj(col, r64, SbL), d0);
+        st16(sm + L::kU, mnmaj(col + 8, r64, SbL), d0 + 8);
+        st16(sm + L::kU, mnmaj(col + 16, r64, SbL), d1);
+        st16(sm + L::kU, mnmaj(col + 24, r64, SbL), d1 + 8);
+      }
+    }
+    sync_for_mma();
+    // ---- C2: S += K'^T U (M=128, K=64); D_Q += A_qk U (M=64, K=64)
+    if (tid == 0) {
+      const uint64_t kd = smem_desc(smem_u32(st + kSlotK), 128, 1024);
+      const uint64_t ud = smem_desc(smem_u32(sm + L::kU), SbL, 128);
+      const uint64_t a3 = smem_desc(smem_u32(st + kSlotA3), 1024, 128);
+      constexpr uint32_t ids = instr_desc(kFmtBF16, 128, 128, false, true);
+      constexpr uint32_t ido = instr_desc(kFmtBF16, 64, 128, true, true);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mma_bf16(tm + kTmS, kd + 16 * k, ud + (2 * SbL >> 4) * k, ids, 1);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mma_bf16(tm + kTmQ, a3 + 128 * k, ud + (2 * SbL >> 4) * k, ido, 1);
+      mma_commit(&s_bar);
+    }
+    if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
+    // the stage is consumed (its reads ended before the barrier above): refill it
+    if (c + 2 < c1) {
+      inflight |= 1u << s;
+      if (tid == 0) load_slot(c + 2);
+    }
+    // ---- S -> bf16 operand of the next chunk; o = D_Q * |q|^-1 -> global
+    {
+      float s0[16], s1[16];
+      const int col = 32 * cq;
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + col), s0);
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + col + 16), s1);
+      tmem_ld_wait();
+      st16(sm + L::kSb, mnmaj(col, srow, SbL), s0);
+      st16(sm + L::kSb, mnmaj(col + 8, srow, SbL), s0 + 8);
+      st16(sm + L::kSb, mnmaj(col + 16, srow, SbL), s1);
+      st16(sm + L::kSb, mnmaj(col + 24, srow, SbL), s1 + 8);
+      float o0[16], o1[16];
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmQ + col), o0);
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmQ + col + 16), o1);
+      tmem_ld_wait();
+      if (m64 && r64 < len) {
+        const float iq = reinterpret_cast<const float*>(st + kSlotIq)[r64];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) { o0[i] *= iq; o1[i] *= iq; }
+        uint4* dst = reinterpret_cast<uint4*>(p.o + ((size_t)(tok0 + r64) * H + h) * kD + col);
+        dst[0] = pack8(o0);
+        dst[1] = pack8(o0 + 8);
+        dst[2] = pack8(o1);
+        dst[3] = pack8(o1 + 8);
+      }
+    }
+  }
+
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  if (!s_abort) {
+    if (p.S_final && seg == p.P - 1) {
+      float* dst = p.S_final + ((size_t)n * H + h) * kD * kD + (size_t)srow * kD;
+#pragma unroll
+      for (int c16 = 0; c16 < 32; c16 += 16) {
+        float s16[16];
+        tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + 32 * cq + c16), s16);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; i += 4)
+          *reinterpret_cast<float4*>(dst + 32 * cq + c16 + i) = make_float4(s16[i], s16[i + 1], s16[i + 2], s16[i + 3]);
+      }
+    }
+  } else if (tid == 0) {
+    // a wait gave up: let the slot copies still in flight land before leaving
+    for (int s = 0; s < 2; ++s)
+      if (inflight & (1u << s)) (void)mbar_wait_cycles(&s_ld[s], (ph_ld >> s) & 1, kWaitCycles);
   }
   fence_before_sync();
   __syncthreads();
@@ -845,10 +1122,19 @@ int tc_segments(int N, int H, int max_len) {
   return P;
 }
 
+// Workspace: header | per (n, h) segment transitions and incoming states |
+// (segmented only) one chain-operand slot per (chunk, head), 1 KB aligned.
+static size_t seg_bytes(int N, int H, int P) {
+  const size_t per = (size_t)(P - 1) * 2 * kD * kD + (size_t)P * kD * kD;
+  return sizeof(WsHeader) + (size_t)N * H * per * sizeof(float);
+}
+static size_t prep_offset(int N, int H, int P) { return (seg_bytes(N, H, P) + 1023) & ~(size_t)1023; }
+
 size_t tc_workspace_bytes(int N, int T, int H, int max_len) {
   const int P = tc_segments(N, H, max_len);
-  size_t per = (size_t)(P - 1) * 2 * kD * kD + (size_t)P * kD * kD;
-  return sizeof(WsHeader) + (size_t)N * H * per * sizeof(float);
+  if (P == 1) return seg_bytes(N, H, P);
+  const size_t slots = (size_t)T / kC + (size_t)N;
+  return prep_offset(N, H, P) + slots * H * kSlotBytes;
 }
 
 int tc_launches(int N, int H, int max_len) {
@@ -880,13 +1166,20 @@ cudaError_t launch_forward_tc(const ForwardArgs& a) {
   p.seg = (float*)((char*)a.ws + sizeof(WsHeader));
   cudaError_t err;
   if (p.P > 1) {
+    // transition pass (+ chain operands) -> incoming states -> chain pass
+    p.prep = (unsigned char*)a.ws + prep_offset(a.N, a.H, p.P);
     err = cudaFuncSetAttribute(tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                Smem<1>::kBytes);
     if (err != cudaSuccess) return err;
-    tc_kernel<1><<<dim3(a.N, a.H, p.P - 1), kNT, Smem<1>::kBytes, a.stream>>>(p);
+    tc_kernel<1><<<dim3(a.N, a.H, p.P), kNT, Smem<1>::kBytes, a.stream>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     compose_kernel<<<dim3(a.N, a.H, kD / 16), 256, 0, a.stream>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    err = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               ChainSmem::kBytes);
+    if (err != cudaSuccess) return err;
+    chain_kernel<<<dim3(a.N, a.H, p.P), kNT, ChainSmem::kBytes, a.stream>>>(p);
+    return cudaGetLastError();
   }
   err = cudaFuncSetAttribute(tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Smem<0>::kBytes);
