@@ -68,6 +68,7 @@ struct Smem {
   static constexpr int kKp = kP + 49152;                        //   K'  A op (M=128, K=64) K-major
   static constexpr int kW = kP;                                 //   W   A op (M=64, K=128) K-major
   static constexpr int kU = kP;                                 //   U   B op (N=128|256, K=64) MN-major
+  static constexpr int kUt = kP + 16384;                        //   U~  fp32 slot image (transition)
   static constexpr int kTop = kP + 73728;                       // T   A op (M=64, K=64) K-major
   static constexpr int kA3 = kTop + 8192;                       // A_qk A op (M=64, K=64) MN-major
   static constexpr int kVec = kA3 + (MODE == 0 ? 8192 : 0);
@@ -131,9 +132,31 @@ __device__ __forceinline__ void st16(unsigned char* base, uint32_t off, const fl
   *reinterpret_cast<uint4*>(base + off) = pack8(v);
 }
 
+// c += A B for a 2 x 2 tile: A rows a0, a1 (16-byte aligned, read as float4),
+// B rows ldb floats apart (float2 at the tile's column); NK a multiple of 4.
+template <int NK>
+__device__ __forceinline__ void mm2x2(const float* a0, const float* a1, const float* b, int ldb,
+                                      float (&c)[4]) {
+#pragma unroll
+  for (int i = 0; i < NK; i += 4) {
+    const float4 x = *reinterpret_cast<const float4*>(a0 + i);
+    const float4 y = *reinterpret_cast<const float4*>(a1 + i);
+    const float xa[4] = {x.x, x.y, x.z, x.w}, ya[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 t = *reinterpret_cast<const float2*>(b + (i + u) * ldb);
+      c[0] += xa[u] * t.x;
+      c[1] += xa[u] * t.y;
+      c[2] += ya[u] * t.x;
+      c[3] += ya[u] * t.y;
+    }
+  }
+}
+
 struct alignas(64) TcParams {
-  CUtensorMap tq, tk, tz, tv;  // [T, H, 128] bf16, box 64 x 1 x 128
-  const __nv_bfloat16* beta;
+  CUtensorMap tq, tk, tz, tv;  // [T, H, 128] bf16, box 64 tokens x 1 x 128 channels
+  CUtensorMap sq, sk, sz, sv;  // the same, box 64 tokens x 1 x 64 channels, 128-byte swizzle
+  const __nv_bfloat16 *q, *k, *beta, *z, *v;
   const float *A, *g, *S0;
   const int32_t* cu;
   __nv_bfloat16* o;
@@ -167,6 +190,16 @@ __device__ __forceinline__ void tma_box(void* dst, const CUtensorMap* map, int h
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes "
       "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(h), "r"(tok0), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// One TMA box at channel offset x (a multiple of 64) of a [T, H, 128] tensor.
+__device__ __forceinline__ void tma_box_x(void* dst, const CUtensorMap* map, int x, int h, int tok0,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(h), "r"(tok0), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -317,15 +350,14 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
     if (!block_wait(&s_bar_raw, phase_raw, p.hdr)) { s_abort = 1; break; }
     raw_pending = false;
 
-    // ---- query row norms (warp w: rows w, w+16, w+32, w+48).  Key norms come
-    //      from the diagonal of the K K^T product below, where the decay
-    //      factors cancel; the query norm scales the output row at the end.
+    // ---- inverse row norms of q and k (warp w: rows w, w+16, w+32, w+48); the
+    //      query norm scales the output row at the end
     {
-      float sq[4];
+      float sq[8];  // q rows, then k rows
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int r = warp + 16 * m;
-        const uint2 uq = *reinterpret_cast<const uint2*>(raw + 0 * 16384 + r * 256 + 8 * lane);
+      for (int m = 0; m < 8; ++m) {
+        const int r = warp + 16 * (m & 3);
+        const uint2 uq = *reinterpret_cast<const uint2*>(raw + (m >> 2) * 16384 + r * 256 + 8 * lane);
         const float2 q0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uq.x));
         const float2 q1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&uq.y));
         sq[m] = q0.x * q0.x + q0.y * q0.y + q1.x * q1.x + q1.y * q1.y;
@@ -333,14 +365,14 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
-        for (int m = 0; m < 4; ++m) sq[m] += __shfl_xor_sync(0xffffffffu, sq[m], o);
-      if (lane < 4) {
-        const int r = warp + 16 * lane;
-        float vq = sq[0];
+        for (int m = 0; m < 8; ++m) sq[m] += __shfl_xor_sync(0xffffffffu, sq[m], o);
+      if (lane < 8) {
+        const int r = warp + 16 * (lane & 3);
+        float v = sq[0];
 #pragma unroll
-        for (int m = 1; m < 4; ++m)
-          if (lane == m) vq = sq[m];
-        vec[kVecIq + r] = r < len ? rsqrtf(vq + kNormEps) : 0.f;
+        for (int m = 1; m < 8; ++m)
+          if (lane == m) v = sq[m];
+        vec[(lane < 4 ? kVecIq : kVecIk) + r] = r < len ? rsqrtf(v + kNormEps) : 0.f;
       }
     }
     // ---- gate and cumsum of channel j over sub-tile qq; E = e^{Gam_r - rho_qq}
@@ -370,6 +402,8 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
         Ei[i] = __fdividef(1.0f, E[i]);
       }
     }
+    // region P is rewritten from here on: the previous chunk's bulk stores must have read it
+    if (MODE == 1 && tid == 0) bulk_wait_read();
     __syncthreads();
     // rho_b = Gam at the first token of sub-tile b; Gam_last = Gam at row 63
     float rho[4], glast;
@@ -427,8 +461,8 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
       mma_commit(&s_bar);
     }
     if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
-    // ---- A products -> key norms (diagonal), A_kk (fp32 smem, beta- and
-    //      norm-scaled, strictly lower) and A_qk (bf16 A3, MN-major)
+    // ---- A products -> A_kk (fp32 smem, beta- and norm-scaled, strictly
+    //      lower) and A_qk (bf16 A3, MN-major)
     float* Akk = reinterpret_cast<float*>(sm + L::kAkk);
     {
       const int i = r64, bb = cq;  // warp: lane quarter q4, row block bb
@@ -436,14 +470,6 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
       tmem_ld16(tmem_addr(tm, 32 * q4, kTmA + 32 * bb), va);
       tmem_ld16(tmem_addr(tm, 32 * q4, kTmA + 32 * bb + 16), vq);
       tmem_ld_wait();
-      if (m64 && bb == q4) {
-        float dk = va[0];
-#pragma unroll
-        for (int cc = 1; cc < 16; ++cc)
-          if (cc == lane) dk = va[cc];
-        vec[kVecIk + i] = i < len ? rsqrtf(dk + kNormEps) : 0.f;
-      }
-      __syncthreads();
       if (m64) {
         const float ki = vec[kVecIk + i];
 #pragma unroll
@@ -494,52 +520,33 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
       // 16 -> 32, pair pr: Y = A[hi][lo] T[lo][lo]; T[hi][lo] = -T[hi][hi] Y (2x2 tiles)
       const int pr = tid >> 6, r2 = ((tid >> 3) & 7) * 2, c2 = (tid & 7) * 2;
       const int lo = 32 * pr, hi = lo + 16;
-      float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float a0 = Akk[(hi + r2) * kLd + lo + i], a1 = Akk[(hi + r2 + 1) * kLd + lo + i];
-        const float2 t = *reinterpret_cast<const float2*>(Tf + (lo + i) * kLd + lo + c2);
-        y00 += a0 * t.x; y01 += a0 * t.y; y10 += a1 * t.x; y11 += a1 * t.y;
-      }
+      float y[4] = {0.f, 0.f, 0.f, 0.f};
+      mm2x2<16>(Akk + (hi + r2) * kLd + lo, Akk + (hi + r2 + 1) * kLd + lo, Tf + lo * kLd + lo + c2,
+                kLd, y);
       float* Yp = Y + pr * 16 * 34;
-      *reinterpret_cast<float2*>(Yp + r2 * 34 + c2) = make_float2(y00, y01);
-      *reinterpret_cast<float2*>(Yp + (r2 + 1) * 34 + c2) = make_float2(y10, y11);
+      *reinterpret_cast<float2*>(Yp + r2 * 34 + c2) = make_float2(y[0], y[1]);
+      *reinterpret_cast<float2*>(Yp + (r2 + 1) * 34 + c2) = make_float2(y[2], y[3]);
       __syncwarp();
       // all of this pair's Y rows come from the same two warps: sync those
       asm volatile("bar.sync %0, %1;" ::"r"(1 + pr), "r"(64) : "memory");
-      float t00 = 0.f, t01 = 0.f, t10 = 0.f, t11 = 0.f;
-#pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        const float a0 = Tf[(hi + r2) * kLd + hi + m], a1 = Tf[(hi + r2 + 1) * kLd + hi + m];
-        const float2 y = *reinterpret_cast<const float2*>(Yp + m * 34 + c2);
-        t00 += a0 * y.x; t01 += a0 * y.y; t10 += a1 * y.x; t11 += a1 * y.y;
-      }
-      *reinterpret_cast<float2*>(Tf + (hi + r2) * kLd + lo + c2) = make_float2(-t00, -t01);
-      *reinterpret_cast<float2*>(Tf + (hi + r2 + 1) * kLd + lo + c2) = make_float2(-t10, -t11);
+      float t[4] = {0.f, 0.f, 0.f, 0.f};
+      mm2x2<16>(Tf + (hi + r2) * kLd + hi, Tf + (hi + r2 + 1) * kLd + hi, Yp + c2, 34, t);
+      *reinterpret_cast<float2*>(Tf + (hi + r2) * kLd + lo + c2) = make_float2(-t[0], -t[1]);
+      *reinterpret_cast<float2*>(Tf + (hi + r2 + 1) * kLd + lo + c2) = make_float2(-t[2], -t[3]);
     }
     __syncthreads();
     if (tid < 256) {
       // 32 -> 64: Y = A[32:64][0:32] T[0:32][0:32]; T[32:64][0:32] = -T[32:64][32:64] Y
       const int r2 = (tid >> 4) * 2, c2 = (tid & 15) * 2;
-      float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-#pragma unroll 8
-      for (int i = 0; i < 32; ++i) {
-        const float a0 = Akk[(32 + r2) * kLd + i], a1 = Akk[(33 + r2) * kLd + i];
-        const float2 t = *reinterpret_cast<const float2*>(Tf + i * kLd + c2);
-        y00 += a0 * t.x; y01 += a0 * t.y; y10 += a1 * t.x; y11 += a1 * t.y;
-      }
-      *reinterpret_cast<float2*>(Y + r2 * 34 + c2) = make_float2(y00, y01);
-      *reinterpret_cast<float2*>(Y + (r2 + 1) * 34 + c2) = make_float2(y10, y11);
+      float y[4] = {0.f, 0.f, 0.f, 0.f};
+      mm2x2<32>(Akk + (32 + r2) * kLd, Akk + (33 + r2) * kLd, Tf + c2, kLd, y);
+      *reinterpret_cast<float2*>(Y + r2 * 34 + c2) = make_float2(y[0], y[1]);
+      *reinterpret_cast<float2*>(Y + (r2 + 1) * 34 + c2) = make_float2(y[2], y[3]);
       asm volatile("bar.sync %0, %1;" ::"r"(3), "r"(256) : "memory");
-      float t00 = 0.f, t01 = 0.f, t10 = 0.f, t11 = 0.f;
-#pragma unroll 8
-      for (int m = 0; m < 32; ++m) {
-        const float a0 = Tf[(32 + r2) * kLd + 32 + m], a1 = Tf[(33 + r2) * kLd + 32 + m];
-        const float2 y = *reinterpret_cast<const float2*>(Y + m * 34 + c2);
-        t00 += a0 * y.x; t01 += a0 * y.y; t10 += a1 * y.x; t11 += a1 * y.y;
-      }
-      *reinterpret_cast<float2*>(Tf + (32 + r2) * kLd + c2) = make_float2(-t00, -t01);
-      *reinterpret_cast<float2*>(Tf + (33 + r2) * kLd + c2) = make_float2(-t10, -t11);
+      float t[4] = {0.f, 0.f, 0.f, 0.f};
+      mm2x2<32>(Tf + (32 + r2) * kLd + 32, Tf + (33 + r2) * kLd + 32, Y + c2, 34, t);
+      *reinterpret_cast<float2*>(Tf + (32 + r2) * kLd + c2) = make_float2(-t[0], -t[1]);
+      *reinterpret_cast<float2*>(Tf + (33 + r2) * kLd + c2) = make_float2(-t[2], -t[3]);
     }
     __syncthreads();
     // T -> bf16 A operand (K-major), upper triangle zero; 8 consecutive threads
@@ -579,12 +586,16 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
         }
         st16(sm + L::kX, kmaj(j, r0, 1024), xk);
         st16(sm + L::kX, kmaj(128 + j, r0, 1024), xv);
-        if (chain) st16(sm + L::kKp, kmaj(j, r0, 1024), kp);
-        if (MODE == 1) st16(slot + kSlotK, kmaj(j, r0, 1024), kp);
-        st16(MODE == 0 ? sm + L::kQp : slot + kSlotQ, mnmaj(r0, j, 1024), qp);
+        st16(sm + L::kKp, kmaj(j, r0, 1024), kp);
+        st16(sm + L::kQp, mnmaj(r0, j, 1024), qp);
       }
     }
     sync_for_mma();
+    if (MODE == 1 && tid == 0) {
+      bulk_s2g(slot + kSlotQ, sm + L::kQp, 16384);
+      bulk_s2g(slot + kSlotK, sm + L::kKp, 16384);
+      bulk_commit();
+    }
     // the staged rows are consumed: prefetch the next chunk
     if (c + 1 < c1) {
       raw_pending = true;
@@ -598,6 +609,7 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
 #pragma unroll
       for (int k = 0; k < 4; ++k) mma_bf16(tm + kTmWU, ad + 16 * k, bd + 16 * k, id, k > 0);
       mma_commit(&s_bar);
+      if (MODE == 1) bulk_wait_read();  // Q' is overwritten by the U~ image below
     }
     if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
     // ---- W -> bf16 A operand (K-major); U~ -> registers (M=64 rows, lane < 16)
@@ -610,22 +622,42 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
       tmem_ld_wait();
 #pragma unroll
       for (int i = 0; i < 16; ++i) ut[c16 + i] = u16[i];
-      if (m64 && chain) {
+      if (m64) {
         st16(sm + L::kW, kmaj(r64, 32 * cq + c16, 2048), w16);
         st16(sm + L::kW, kmaj(r64, 32 * cq + c16 + 8, 2048), w16 + 8);
       }
       if (MODE == 1 && m64) {
-        st16(slot + kSlotW, kmaj(r64, 32 * cq + c16, 2048), w16);
-        st16(slot + kSlotW, kmaj(r64, 32 * cq + c16 + 8, 2048), w16 + 8);
-        float4* ug = reinterpret_cast<float4*>(slot + kSlotU);
+        float4* ug = reinterpret_cast<float4*>(sm + L::kUt);
 #pragma unroll
         for (int pc = 0; pc < 4; ++pc)
           ug[ut_index(q4, cq, (c16 >> 2) + pc, lane) >> 2] =
               make_float4(u16[4 * pc], u16[4 * pc + 1], u16[4 * pc + 2], u16[4 * pc + 3]);
       }
     }
+    sync_for_mma();
+    if (MODE == 1 && tid == 0) {
+      bulk_s2g(slot + kSlotW, sm + L::kW, 16384);
+      bulk_s2g(slot + kSlotU, sm + L::kUt, 32768);
+      bulk_commit();
+    }
     if (!chain) continue;
-    // ---- decay the state(s) by gamma = e^{Gam_last} (rows = dk = TMEM lanes)
+    // ---- C1: D_W = W S (M=64, N=128|256), D_Q = Q' S (M=64, N=128)
+    if (tid == 0) {
+      const uint64_t sd = smem_desc(smem_u32(sm + L::kSb), SbL, 128);
+      const uint64_t wd = smem_desc(smem_u32(sm + L::kW), 128, 2048);
+      constexpr uint32_t idw = instr_desc(kFmtBF16, 64, SbN, false, true);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mma_bf16(tm + kTmW, wd + 16 * k, sd + (2 * SbL >> 4) * k, idw, k > 0);
+      if (MODE == 0) {
+        constexpr uint32_t idq = instr_desc(kFmtBF16, 64, 128, true, true);
+        const uint64_t qd = smem_desc(smem_u32(sm + L::kQp), 1024, 128);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mma_bf16(tm + kTmQ, qd + 128 * k, sd + (2 * SbL >> 4) * k, idq, k > 0);
+      }
+      mma_commit(&s_bar);
+    }
+    // ---- meanwhile decay the fp32 state(s) by gamma = e^{Gam_last} (rows = dk =
+    //      TMEM lanes); C1 reads the bf16 copy
     {
       const float gm = vec[kVecGam + srow];
       constexpr int NB = MODE == 0 ? 1 : 2;
@@ -644,22 +676,7 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
       }
       tmem_st_wait();
     }
-    sync_for_mma();
-    // ---- C1: D_W = W S (M=64, N=128|256), D_Q = Q' S (M=64, N=128)
-    if (tid == 0) {
-      const uint64_t sd = smem_desc(smem_u32(sm + L::kSb), SbL, 128);
-      const uint64_t wd = smem_desc(smem_u32(sm + L::kW), 128, 2048);
-      constexpr uint32_t idw = instr_desc(kFmtBF16, 64, SbN, false, true);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mma_bf16(tm + kTmW, wd + 16 * k, sd + (2 * SbL >> 4) * k, idw, k > 0);
-      if (MODE == 0) {
-        constexpr uint32_t idq = instr_desc(kFmtBF16, 64, 128, true, true);
-        const uint64_t qd = smem_desc(smem_u32(sm + L::kQp), 1024, 128);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mma_bf16(tm + kTmQ, qd + 128 * k, sd + (2 * SbL >> 4) * k, idq, k > 0);
-      }
-      mma_commit(&s_bar);
-    }
+    if (MODE == 1 && tid == 0) bulk_wait_read();  // U overwrites the W and U~ images
     if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
     // ---- U = U~ - W S  (transition: [U_S | U_X] = [U~ | 0] - W [S | X]); B operand MN-major
     {
@@ -776,25 +793,593 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
     // a wait gave up: let the TMA load still in flight land before leaving
     mbar_wait_cycles(&s_bar_raw, phase_raw, kWaitCycles);
   }
+  if (MODE == 1 && tid == 0) bulk_wait_all();
   fence_before_sync();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tm, 512);
 }
 
-// Chain pass of a segmented sequence: only the state-dependent half of each
-// chunk, from the operands the transition pass stored in the chunk's slot.
-// Per chunk: D_W = W S and D_Q = Q' S (C1); S <- gamma S meanwhile; U = U~ - D_W;
-// S += K'^T U and D_Q += A_qk U (C2); o = D_Q scaled by the query row norms.
-// Slots are bulk-copied two chunks ahead into two stages.
+// ---------------------------------------------------------------------------
+// Chunk preparation: everything of one (chunk, head) that does not depend on
+// the state, left in the chunk's slot for the chain passes.  Persistent: each
+// CTA (one per SM; a kernel that uses Tensor Memory gets one CTA per SM) walks
+// its share of the (chunk, sequence, head) items, loading the next item's q,
+// k, z, v rows by TMA while it finishes the current one.  The 512 threads form
+// one group with its own named barriers (the layout allows more groups per CTA
+// when registers and shared memory permit).  Warp w covers sub-tile w / 4 and
+// 32 channels; each lane owns 8 channels of a token pair, so every row access
+// is one 16-byte vector and every operand image is K-major or MN-major such
+// that each such vector is one 16-byte row of a core matrix.
+// Per (chunk, head): gate and cumulative log-decay (scans within 16-token
+// sub-tiles); q/k row norms; sub-tile decay factors; product operands R, C
+// and Q', K'; M1 (A products); X_K, X_V; A_kk and A_qk; T = (I + A_kk)^{-1};
+// M2 ([W | U~] = T [X_K | X_V]); bulk stores.
+constexpr int kPrepGroups = 1;  // 512-thread groups per CTA (each with its own smem part)
+constexpr int kPrepThreads = kNT * kPrepGroups;
+struct PrepSmem {  // one group's part
+  static constexpr int kP = 0;               // region P, reused through the chunk:
+  static constexpr int kR = kP;              //   R   B op (N=128 rows, K=128) K-major
+  static constexpr int kCc = kP + 32768;     //   C   A op (M=160 rows, K=128) K-major
+  static constexpr int kAkk = kP;            //   A_kk fp32 [64][68]  (after M1)
+  static constexpr int kTf = kP + 17408;     //   T    fp32 [64][68]
+  static constexpr int kY = kP + 34816;      //   merge scratch fp32 [32][34]
+  static constexpr int kX = kP + 40960;      //   X   B op (N=256, K=64 tokens) MN-major
+  static constexpr int kW = kP;              //   W   slot image   (after M2)
+  static constexpr int kUt = kP + 16384;     //   U~  slot image
+  static constexpr int kTop = kP + 73728;    // sub-tile sums and first gates, then T (A op, K-major)
+  static constexpr int kFac = kTop + 8192;   // decay factors [4 sub-tiles][5][128] fp32
+  static constexpr int kNrm = kFac + 10240;  // squared-norm partials [16 channel groups][64][2]
+  static constexpr int kVec = kNrm + 8192;   // 1/|q|, 1/|k|, beta (64 floats each)
+  static constexpr int kRaw = 101376;        // q | k | z | v, [64 tokens][2 x 64 channels] bf16,
+                                             //   128-byte swizzled (TMA), 16 KB each
+  static constexpr int kGroup = kRaw + 65536;  // bytes per group
+  static constexpr int kBar = kPrepGroups * kGroup;  // per group: two mbarriers; then the TMEM base
+  static constexpr int kBytes = kBar + 48;
+};
+// decay factor rows of sub-tile b (128 channels each): e^{rho_b}, e^{Gam_last - rho_b},
+// then e^{rho_c - rho_b} for the later sub-tiles c = b+1 .. 3
+constexpr int kFacEr = 0, kFacEl = 1, kFacWin = 2;
+
+// Barrier of one 512-thread group (ids 1 + 4 g .. 4 + 4 g are the group's).
+__device__ __forceinline__ void group_sync(int id) {
+  asm volatile("bar.sync %0, 512;" ::"r"(id) : "memory");
+}
+__device__ __forceinline__ bool group_sync_or(int id, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, 512, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void group_sync_for_mma(int id) {
+  fence_async_smem();
+  fence_before_sync();
+  group_sync(id);
+  fence_after_sync();
+}
+// Group-wide bounded wait on an mbarrier phase; false if it timed out.
+__device__ __forceinline__ bool group_wait(uint64_t* bar, uint32_t& phase, WsHeader* hdr, int id,
+                                           int gtid) {
+  const bool got = mbar_wait_cycles(bar, phase, kWaitCycles);
+  phase ^= 1;
+  if (group_sync_or(id, !got)) {
+    if (gtid == 0) atomicOr(&hdr->err, kErrTimeout);
+    return false;
+  }
+  fence_after_sync();
+  return true;
+}
+
+// 8 bf16 (one 16-byte vector) -> fp32, exactly
+__device__ __forceinline__ void unpack8(const uint4 u, float* f) {
+  f[0] = __uint_as_float(u.x << 16); f[1] = __uint_as_float(u.x & 0xffff0000u);
+  f[2] = __uint_as_float(u.y << 16); f[3] = __uint_as_float(u.y & 0xffff0000u);
+  f[4] = __uint_as_float(u.z << 16); f[5] = __uint_as_float(u.z & 0xffff0000u);
+  f[6] = __uint_as_float(u.w << 16); f[7] = __uint_as_float(u.w & 0xffff0000u);
+}
+__device__ __forceinline__ void ld8f(const float* p, float* f) {  // 8 fp32, 16-byte aligned
+  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+__device__ __forceinline__ void st8f(float* p, const float* f) {
+  *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
+  *reinterpret_cast<float4*>(p + 4) = make_float4(f[4], f[5], f[6], f[7]);
+}
+
+__global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_constant__ TcParams p) {
+  using L = PrepSmem;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const int tid = threadIdx.x;
+  const int grp = tid >> 9, gtid = tid & 511;  // group, thread within it
+  const int warp = gtid >> 5, lane = tid & 31;
+  unsigned char* sm = smem + grp * L::kGroup;
+  float* vec = reinterpret_cast<float*>(sm + L::kVec);
+  float* fac = reinterpret_cast<float*>(sm + L::kFac);
+  uint64_t* bar_mma = reinterpret_cast<uint64_t*>(smem + L::kBar) + 2 * grp;
+  uint64_t* bar_raw = bar_mma + 1;
+  const unsigned char* raw = sm + L::kRaw;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::kBar + 32);
+  const int bid = 1 + 4 * grp;  // the group's barrier: bid; merges: bid + 1, bid + 2, bid + 3
+  const int H = p.H;
+
+  if (!seqlens_valid(p.cu, p.N, p.T, p.max_len)) {
+    if (blockIdx.x == 0 && tid == 0) p.hdr->err = kErrBadSeqlens;
+    return;
+  }
+  if (blockIdx.x == 0 && tid == 0) p.hdr->err = kErrNone;
+  // the 128-byte swizzle needs 1024-byte aligned destinations
+  if (smem_u32(smem) & 1023u) {
+    if (tid == 0) atomicOr(&p.hdr->err, kErrTimeout);
+    return;
+  }
+  if (tid < 32) {
+    tmem_alloc(s_tmem, 256 * kPrepGroups);
+    tmem_relinquish();
+  }
+  if (gtid == 0) {
+    mbar_init(bar_mma, 1);
+    mbar_init(bar_raw, 1);
+    fence_mbar_init();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tm = *s_tmem + 256 * grp;  // this group's 256 columns
+  uint32_t ph_mma = 0, ph_raw = 0;          // next parity of each barrier
+  bool ok = true, raw_pending = false;
+
+  // warp: sub-tile qq (tokens 16 qq ..) and 32 channels; lane: 8 of those
+  // channels (group cg) and a token pair of the sub-tile (lanes 8 m .. 8 m + 7
+  // share a channel group and scan its 16 tokens)
+  const int qq = warp >> 2, pr = lane & 7;
+  const int cg = 4 * (warp & 3) + (lane >> 3), c0 = 8 * cg;
+  const int t0 = 16 * qq + 2 * pr;          // tokens t0, t0 + 1
+  const int sw = pr >> 2;                   // row-store order: conflict-free 16-byte stores
+  const int q4 = warp & 3, cq = warp >> 2;  // TMEM lane quarter, 32-column quarter
+  const int r64 = 16 * q4 + lane;           // token row of M=64 accumulators (lane < 16)
+  const bool m64 = lane < 16;
+
+  // items (chunk c, sequence n, head h), heads fastest; each group takes every
+  // (2 * gridDim.x)-th one, stepping the mixed-radix index without divisions
+  const int maxch = (p.max_len + kC - 1) / kC;
+  const long long it0 = (long long)kPrepGroups * blockIdx.x + grp;
+  const long long stride = (long long)kPrepGroups * gridDim.x;
+  int h = (int)(it0 % H), n = (int)((it0 / H) % p.N), c = (int)(it0 / ((long long)H * p.N));
+  const int sh = (int)(stride % H), sn = (int)((stride / H) % p.N);
+  const int sc = (int)(stride / ((long long)H * p.N));
+  int a = 0, b = 0;
+  // the group's next item that holds tokens, from (c, n, h) on
+  auto next_item = [&]() -> bool {
+    for (; c < maxch;) {
+      seq_bounds(p.cu, n, p.max_len, a, b);
+      if (a + c * kC < b) return true;
+      h += sh;
+      if (h >= H) { h -= H; ++n; }
+      n += sn;
+      if (n >= p.N) { n -= p.N; ++c; }
+      c += sc;
+    }
+    return false;
+  };
+  // q, k, z, v rows of an item -> the staging tile (two 64-channel boxes each)
+  auto stage = [&](int tok, int hh) {
+    mbar_arrive_expect_tx(bar_raw, 4 * 16384);
+    tma_box_x(sm + L::kRaw, &p.sq, 0, hh, tok, bar_raw);
+    tma_box_x(sm + L::kRaw + 8192, &p.sq, 64, hh, tok, bar_raw);
+    tma_box_x(sm + L::kRaw + 16384, &p.sk, 0, hh, tok, bar_raw);
+    tma_box_x(sm + L::kRaw + 24576, &p.sk, 64, hh, tok, bar_raw);
+    tma_box_x(sm + L::kRaw + 32768, &p.sz, 0, hh, tok, bar_raw);
+    tma_box_x(sm + L::kRaw + 40960, &p.sz, 64, hh, tok, bar_raw);
+    tma_box_x(sm + L::kRaw + 49152, &p.sv, 0, hh, tok, bar_raw);
+    tma_box_x(sm + L::kRaw + 57344, &p.sv, 64, hh, tok, bar_raw);
+  };
+  // 16-byte row vector (token t, channels c0 .. c0+7) of staged tensor ti
+  auto rawv = [&](int ti, int t) -> uint4 {
+    return *reinterpret_cast<const uint4*>(raw + ti * 16384 + (cg >> 3) * 8192 + t * 128 +
+                                           (((cg & 7) ^ (t & 7)) << 4));
+  };
+  bool have = next_item();
+  if (have) {
+    if (gtid == 0) stage(a + c * kC, h);
+    raw_pending = true;
+  }
+  while (ok && have) {
+    const int hc = h, nc = n, cc0 = c, ac = a, bc = b;
+    h += sh;
+    if (h >= H) { h -= H; ++n; }
+    n += sn;
+    if (n >= p.N) { n -= p.N; ++c; }
+    c += sc;
+    have = next_item();  // the item after this one (its rows are loaded during this one)
+    const int tok0 = ac + cc0 * kC;
+    const int len = min(kC, bc - tok0);
+    unsigned char* slot = chunk_slot(p.prep, ac, nc, cc0, hc, H);
+    const bool in0 = t0 < len, in1 = t0 + 1 < len;
+    const size_t row0 = ((size_t)(tok0 + t0) * H + hc) * kD + c0;  // element offset of (t0, c0)
+    const size_t rstep = (size_t)H * kD;                          // next token
+    const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
+
+    if (gtid < kC)
+      vec[kVecBeta + gtid] = gtid < len ? __bfloat162float(p.beta[(size_t)(tok0 + gtid) * H + hc]) : 0.f;
+    if (!group_wait(bar_raw, ph_raw, p.hdr, bid, gtid)) {
+      ph_raw ^= 1;  // the load is still pending in this phase
+      ok = false;
+      break;
+    }
+    raw_pending = false;
+    // ---- rows of q and k (16-byte vectors; the token order of the two reads
+    //      keeps each 8-lane phase on distinct banks)
+    uint4 qa, qb, ka, kb;
+    {
+      const int ta = t0 + sw, tb = t0 + 1 - sw;
+      const uint4 q1 = rawv(0, ta), q2 = rawv(0, tb), k1 = rawv(1, ta), k2 = rawv(1, tb);
+      qa = sw ? q2 : q1; qb = sw ? q1 : q2;
+      ka = sw ? k2 : k1; kb = sw ? k1 : k2;
+      if (!in0) { qa = zero4; ka = zero4; }
+      if (!in1) { qb = zero4; kb = zero4; }
+    }
+
+    // ---- log-decay gate g of the 16 elements; E[8 s + i]: token t0 + s, channel c0 + i
+    float E[16];
+    if (p.g) {
+      const float* g0 = p.g + row0;
+      if (in0) { ld8f(g0, E); } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) E[i] = 0.f;
+      }
+      if (in1) { ld8f(g0 + rstep, E + 8); } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) E[8 + i] = 0.f;
+      }
+    } else {
+      const float expA = expf(p.A[hc]);
+      const uint4 z1 = rawv(2, t0 + sw), z2 = rawv(2, t0 + 1 - sw);
+      unpack8(sw ? z2 : z1, E);
+      unpack8(sw ? z1 : z2, E + 8);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const bool in = i < 8 ? in0 : in1;
+        E[i] = in ? __fdividef(kGateMin, 1.0f + __expf(-expA * E[i])) : 0.f;
+      }
+    }
+    // ---- cumulative log-decay within the sub-tile: scan over its 8 lanes
+    float gf[8];  // g of the sub-tile's first token (lane 8 qq, token t0)
+    {
+      float x[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = E[i] + E[8 + i];  // pair sums
+#pragma unroll
+      for (int off = 1; off < 8; off <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float y = __shfl_up_sync(0xffffffffu, x[i], off);
+          if ((lane & 7) >= off) x[i] += y;
+        }
+      }
+      // x = inclusive sum of the sub-tile through token t0 + 1
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        gf[i] = __shfl_sync(0xffffffffu, E[i], lane & ~7);
+        const float g1 = E[8 + i];
+        E[8 + i] = x[i];       // through t0 + 1
+        E[i] = x[i] - g1;      // through t0
+      }
+      float* tot = reinterpret_cast<float*>(sm + L::kTop);  // [4][128] sub-tile sums
+      float* fst = tot + 512;                               // [4][128] first gates
+      if ((lane & 7) == 7) st8f(tot + qq * 128 + c0, x);
+      if ((lane & 7) == 0) st8f(fst + qq * 128 + c0, gf);
+    }
+    // E = e^{Gam_r - rho_qq}, rho_qq = Gam at the sub-tile's first token
+#pragma unroll
+    for (int i = 0; i < 16; ++i) E[i] = __expf(E[i] - gf[i & 7]);
+    // ---- squared row norms of q and k: partial sums over this channel group
+    {
+      float qf[8], kf[8];
+      float4 part;
+      unpack8(qa, qf); unpack8(ka, kf);
+      part.x = 0.f; part.y = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { part.x += qf[i] * qf[i]; part.y += kf[i] * kf[i]; }
+      unpack8(qb, qf); unpack8(kb, kf);
+      part.z = 0.f; part.w = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { part.z += qf[i] * qf[i]; part.w += kf[i] * kf[i]; }
+      *reinterpret_cast<float4*>(sm + L::kNrm + (cg * 64 + t0) * 8) = part;
+    }
+    // region P is rewritten from here on: the previous item's bulk stores must have read it
+    if (gtid == 0) bulk_wait_read();
+    group_sync(bid);
+    // ---- decay factors of (sub-tile b, channel ch); 1/|q|, 1/|k|; gamma
+    {
+      const float* tot = reinterpret_cast<const float*>(sm + L::kTop);
+      const float* fst = tot + 512;
+      const int ch = gtid & 127, bq = gtid >> 7;
+      float rho[4], acc = 0.f;
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb) {
+        rho[bb] = acc + fst[bb * 128 + ch];
+        acc += tot[bb * 128 + ch];
+      }
+      const float rb = bq == 0 ? rho[0] : bq == 1 ? rho[1] : bq == 2 ? rho[2] : rho[3];
+      fac[(bq * 5 + kFacEr) * 128 + ch] = __expf(rb);
+      fac[(bq * 5 + kFacEl) * 128 + ch] = __expf(acc - rb);
+#pragma unroll
+      for (int bb = 1; bb < 4; ++bb)
+        if (bb > bq) fac[(bq * 5 + kFacWin + bb - bq - 1) * 128 + ch] = __expf(rho[bb] - rb);
+      if (bq == 0) reinterpret_cast<float*>(slot + kSlotGam)[ch] = __expf(acc);
+      if (gtid < 128) {
+        const int t = gtid & 63, w = gtid >> 6;  // token, q (0) or k (1)
+        const float* np = reinterpret_cast<const float*>(sm + L::kNrm) + 2 * t + w;
+        float ss = 0.f;
+#pragma unroll
+        for (int g = 0; g < 16; ++g) ss += np[g * 128];
+        const float inv = t < len ? rsqrtf(ss + kNormEps) : 0.f;
+        vec[(w == 0 ? kVecIq : kVecIk) + t] = inv;
+        if (w == 0) reinterpret_cast<float*>(slot + kSlotIq)[t] = inv;
+      }
+    }
+    group_sync(bid);
+    // ---- R rows (k e, q e; K-major), Q' = q e^{Gam_r} (norm applied to o), C_b
+    //      windows (k e^{rho_b - Gam_r}; K-major)
+    {
+      const float* fq = fac + qq * 5 * 128 + c0;
+      float er[8];
+      ld8f(fq + kFacEr * 128, er);
+#pragma unroll
+      for (int s2 = 0; s2 < 2; ++s2) {
+        const int s = s2 ^ sw, t = t0 + s;
+        float qf[8], kf[8], w8[8];
+        unpack8(s ? qb : qa, qf);
+        unpack8(s ? kb : ka, kf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { qf[i] *= (sw ? E[8 * (s2 ^ 1) + i] : E[8 * s2 + i]); w8[i] = kf[i] * (sw ? E[8 * (s2 ^ 1) + i] : E[8 * s2 + i]); }
+        const int rr = 32 * qq + (t & 15);  // R row: k rows then q rows of the sub-tile
+        st16(sm + L::kR, kmaj(rr, c0, 2048), w8);
+        st16(sm + L::kR, kmaj(rr + 16, c0, 2048), qf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qf[i] *= er[i];
+        st16(slot + kSlotQ, kmaj(t, c0, 2048), qf);
+      }
+      // k e^{rho_qq - Gam_r}: window qq as is, later windows times e^{rho_b - rho_qq};
+      // K' = k / |k| e^{Gam_last - Gam_r} -> slot (MN-major)
+      float el[8];
+      ld8f(fq + kFacEl * 128, el);
+#pragma unroll
+      for (int s2 = 0; s2 < 2; ++s2) {
+        const int s = s2 ^ sw, t = t0 + s;
+        const float ik = vec[kVecIk + t];
+        float kf[8], w8[8];
+        unpack8(s ? kb : ka, kf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) kf[i] = __fdividef(kf[i], (sw ? E[8 * (s2 ^ 1) + i] : E[8 * s2 + i]));
+        st16(sm + L::kCc, kmaj(8 * qq * (qq + 1) + t, c0, 2048), kf);
+        for (int bb = qq + 1; bb < 4; ++bb) {  // warp-uniform
+          float f[8];
+          ld8f(fq + (kFacWin + bb - qq - 1) * 128, f);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) w8[i] = kf[i] * f[i];
+          st16(sm + L::kCc, kmaj(8 * bb * (bb + 1) + t, c0, 2048), w8);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) kf[i] *= ik * el[i];
+        st16(slot + kSlotK, mnmaj(c0, t, 2048), kf);
+      }
+    }
+    group_sync_for_mma(bid);
+    // ---- M1: four M=64 MMAs (K-major operands) -> TMEM [32b, +32): cols 0-15 A_kk^T,
+    //      16-31 A_qk^T; C window b starts at row 8 b (b + 1), R sub-tile b at row 32 b
+    if (gtid == 0) {
+      constexpr uint32_t id = instr_desc(kFmtBF16, 64, 32, false, false);
+      const uint64_t ad = smem_desc(smem_u32(sm + L::kCc), 128, 2048);
+      const uint64_t bd = smem_desc(smem_u32(sm + L::kR), 128, 2048);
+#pragma unroll
+      for (int bb = 0; bb < 4; ++bb)
+#pragma unroll
+        for (int k = 0; k < 8; ++k)  // descriptor addresses count 16-byte units
+          mma_bf16(tm + kTmA + 32 * bb, ad + bb * (bb + 1) * 128 + 16 * k, bd + 512 * bb + 16 * k,
+                   id, k > 0);
+      mma_commit(bar_mma);
+    }
+    if (!group_wait(bar_mma, ph_mma, p.hdr, bid, gtid)) { ok = false; break; }
+    // ---- X_K = beta k / |k| e^{Gam_r}, X_V = beta v (MN-major; C is dead)
+    {
+      const float* fq = fac + qq * 5 * 128 + c0;
+      const uint4 v1 = rawv(3, t0 + sw), v2 = rawv(3, t0 + 1 - sw);
+      const uint4 va = in0 ? (sw ? v2 : v1) : zero4, vb = in1 ? (sw ? v1 : v2) : zero4;
+      float er[8];
+      ld8f(fq + kFacEr * 128, er);
+#pragma unroll
+      for (int s2 = 0; s2 < 2; ++s2) {
+        const int s = s2 ^ sw, t = t0 + s;
+        const float bet = vec[kVecBeta + t], bik = bet * vec[kVecIk + t];
+        float kf[8], vf[8];
+        unpack8(s ? kb : ka, kf);
+        unpack8(s ? vb : va, vf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          kf[i] *= bik * (sw ? E[8 * (s2 ^ 1) + i] : E[8 * s2 + i]) * er[i];
+          vf[i] *= bet;
+        }
+        st16(sm + L::kX, mnmaj(c0, t, 4096), kf);
+        st16(sm + L::kX, mnmaj(128 + c0, t, 4096), vf);
+      }
+    }
+    // ---- A products -> A_kk (fp32, beta- and norm-scaled, strictly lower) and
+    //      A_qk (bf16 slot image, MN-major)
+    float* Akk = reinterpret_cast<float*>(sm + L::kAkk);
+    {
+      const int i = r64, bb = cq;  // warp: lane quarter q4, row block bb
+      float va[16], vq[16];
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmA + 32 * bb), va);
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmA + 32 * bb + 16), vq);
+      tmem_ld_wait();
+      if (m64) {
+        const float ki = vec[kVecIk + i];
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) {
+          const int r = 16 * bb + cc;
+          Akk[r * kLd + i] = (i < r) ? vec[kVecBeta + r] * vec[kVecIk + r] * ki * va[cc] : 0.f;
+          vq[cc] = (i <= r) ? vq[cc] * ki : 0.f;
+        }
+        st16(slot + kSlotA3, mnmaj(16 * bb, i, 1024), vq);
+        st16(slot + kSlotA3, mnmaj(16 * bb + 8, i, 1024), vq + 8);
+      }
+    }
+    fence_before_sync();
+    group_sync(bid);
+    // the staged rows are consumed: load the next item's
+    if (have) {
+      if (gtid == 0) stage(a + c * kC, h);
+      raw_pending = true;
+    }
+    // ---- T = (I + A_kk)^{-1}: 16x16 diagonal blocks by forward substitution,
+    //      then merges 16 -> 32 -> 64 ([[P,0],[B,Q]]^{-1} has lower-left block
+    //      -Q^{-1} B P^{-1}) on 2x2 register tiles; upper blocks zeroed first.
+    float* Tf = reinterpret_cast<float*>(sm + L::kTf);
+    float* Y = reinterpret_cast<float*>(sm + L::kY);
+    if (gtid < kC) {
+      const int bk = gtid >> 4, cc = gtid & 15, base = 16 * bk;
+      float x[16];
+#pragma unroll
+      for (int rr = 0; rr < 16; ++rr) {
+        float acc = (rr == cc) ? 1.f : 0.f;
+#pragma unroll
+        for (int i = 0; i < rr; ++i) acc -= Akk[(base + rr) * kLd + base + i] * x[i];
+        x[rr] = (rr < cc) ? 0.f : acc;
+      }
+#pragma unroll
+      for (int rr = 0; rr < 16; ++rr) Tf[(base + rr) * kLd + base + cc] = x[rr];
+    } else {
+      // zero T[0:16][16:32] and T[32:48][48:64]
+      for (int e = gtid - kC; e < 512; e += kNT - kC) {
+        const int blk = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
+        Tf[(32 * blk + rr) * kLd + 32 * blk + 16 + cc] = 0.f;
+      }
+    }
+    group_sync(bid);
+    if (gtid < 128) {
+      const int pr = gtid >> 6, r2 = ((gtid >> 3) & 7) * 2, c2 = (gtid & 7) * 2;
+      const int lo = 32 * pr, hi = lo + 16;
+      float y[4] = {0.f, 0.f, 0.f, 0.f};
+      mm2x2<16>(Akk + (hi + r2) * kLd + lo, Akk + (hi + r2 + 1) * kLd + lo, Tf + lo * kLd + lo + c2,
+                kLd, y);
+      float* Yp = Y + pr * 16 * 34;
+      *reinterpret_cast<float2*>(Yp + r2 * 34 + c2) = make_float2(y[0], y[1]);
+      *reinterpret_cast<float2*>(Yp + (r2 + 1) * 34 + c2) = make_float2(y[2], y[3]);
+      __syncwarp();
+      // this pair's Y rows come from the same two warps: sync those
+      asm volatile("bar.sync %0, 64;" ::"r"(bid + 1 + pr) : "memory");
+      float t[4] = {0.f, 0.f, 0.f, 0.f};
+      mm2x2<16>(Tf + (hi + r2) * kLd + hi, Tf + (hi + r2 + 1) * kLd + hi, Yp + c2, 34, t);
+      *reinterpret_cast<float2*>(Tf + (hi + r2) * kLd + lo + c2) = make_float2(-t[0], -t[1]);
+      *reinterpret_cast<float2*>(Tf + (hi + r2 + 1) * kLd + lo + c2) = make_float2(-t[2], -t[3]);
+    }
+    group_sync(bid);
+    if (gtid < 256) {
+      const int r2 = (gtid >> 4) * 2, c2 = (gtid & 15) * 2;
+      float y[4] = {0.f, 0.f, 0.f, 0.f};
+      mm2x2<32>(Akk + (32 + r2) * kLd, Akk + (33 + r2) * kLd, Tf + c2, kLd, y);
+      *reinterpret_cast<float2*>(Y + r2 * 34 + c2) = make_float2(y[0], y[1]);
+      *reinterpret_cast<float2*>(Y + (r2 + 1) * 34 + c2) = make_float2(y[2], y[3]);
+      asm volatile("bar.sync %0, 256;" ::"r"(bid + 3) : "memory");
+      float t[4] = {0.f, 0.f, 0.f, 0.f};
+      mm2x2<32>(Tf + (32 + r2) * kLd + 32, Tf + (33 + r2) * kLd + 32, Y + c2, 34, t);
+      *reinterpret_cast<float2*>(Tf + (32 + r2) * kLd + c2) = make_float2(-t[0], -t[1]);
+      *reinterpret_cast<float2*>(Tf + (33 + r2) * kLd + c2) = make_float2(-t[2], -t[3]);
+    }
+    group_sync(bid);
+    // T -> bf16 A operand (K-major), upper triangle zero
+    {
+      const int r = (gtid >> 6) * 8 + (gtid & 7), i0 = ((gtid >> 3) & 7) * 8;
+      float t8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) t8[i] = (i0 + i <= r) ? Tf[r * kLd + i0 + i] : 0.f;
+      st16(sm + L::kTop, kmaj(r, i0, 1024), t8);
+    }
+    group_sync_for_mma(bid);
+    // ---- M2: [W | U~] = T [X_K | X_V]  (M=64, N=256, K=64; X MN-major)
+    if (gtid == 0) {
+      constexpr uint32_t id = instr_desc(kFmtBF16, 64, 256, false, true);
+      const uint64_t ad = smem_desc(smem_u32(sm + L::kTop), 128, 1024);
+      const uint64_t bd = smem_desc(smem_u32(sm + L::kX), 4096, 128);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mma_bf16(tm + kTmWU, ad + 16 * k, bd + 512 * k, id, k > 0);
+      mma_commit(bar_mma);
+    }
+    if (!group_wait(bar_mma, ph_mma, p.hdr, bid, gtid)) { ok = false; break; }
+    // ---- W (bf16 image) and U~ (fp32) -> shared memory -> slot
+#pragma unroll
+    for (int c16 = 0; c16 < 32; c16 += 16) {
+      float w16[16];
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmWU + 32 * cq + c16), w16);
+      tmem_ld_wait();
+      if (m64) {
+        st16(sm + L::kW, kmaj(r64, 32 * cq + c16, 2048), w16);
+        st16(sm + L::kW, kmaj(r64, 32 * cq + c16 + 8, 2048), w16 + 8);
+      }
+    }
+#pragma unroll
+    for (int c16 = 0; c16 < 32; c16 += 16) {
+      float u16[16];
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmWU + 128 + 32 * cq + c16), u16);
+      tmem_ld_wait();
+      if (m64) {
+        float4* ug = reinterpret_cast<float4*>(sm + L::kUt);
+#pragma unroll
+        for (int pc = 0; pc < 4; ++pc)
+          ug[ut_index(q4, cq, (c16 >> 2) + pc, lane) >> 2] =
+              make_float4(u16[4 * pc], u16[4 * pc + 1], u16[4 * pc + 2], u16[4 * pc + 3]);
+      }
+    }
+    group_sync_for_mma(bid);
+    if (gtid == 0) {
+      bulk_s2g(slot + kSlotW, sm + L::kW, 16384);
+      bulk_s2g(slot + kSlotU, sm + L::kUt, 32768);
+      bulk_commit();
+    }
+  }
+  if (gtid == 0) {
+    bulk_wait_all();
+    // a wait gave up: let the row load still in flight land before leaving
+    if (raw_pending) (void)mbar_wait_cycles(bar_raw, ph_raw, kWaitCycles);
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (tid < 32) tmem_dealloc(*s_tmem, 256 * kPrepGroups);
+}
+
+// ---------------------------------------------------------------------------
+// Chain passes of a segmented sequence: the state-dependent half of each chunk,
+// from the operands in its slot.  Per chunk: D_W = W S (and D_Q = Q' S) (C1),
+// S <- gamma S meanwhile, U = U~ - D_W, S += K'^T U (and D_Q += A_qk U) (C2),
+// o = D_Q scaled by the query row norms.
+//   TRANS = false: full pass of segment p from its true incoming state; o, S_final.
+//   TRANS = true : transition of segments 0..P-2 on [S | X], from S = 0 (-> N_p)
+//                  and X = I (-> M_p), 256 columns wide; no output.
+// Slot parts are bulk-copied two chunks ahead into two stages.
+template <bool TRANS>
 struct ChainSmem {
-  static constexpr int kSb = 0;         // S bf16, B operand (N=128, K=128), MN-major
-  static constexpr int kU = 32768;      // U bf16, B operand (N=128, K=64), MN-major
-  static constexpr int kStage = 49152;  // two slots
-  static constexpr int kBytes = kStage + 2 * kSlotBytes;
+  static constexpr int kSbN = TRANS ? 256 : 128;    // state columns
+  static constexpr int kSb = 0;                     // [S | X] bf16, B operand (K=128), MN-major
+  static constexpr int kU = kSbN * 256;             // U bf16, B operand (K=64), MN-major
+  static constexpr int kStage = kU + kSbN * 128;    // two stages
+  // stage layout: the slot (full pass), or W | K' | U~ | gamma (transition)
+  static constexpr int kW = kSlotW, kK = kSlotK, kQ = kSlotQ, kA3 = kSlotA3;
+  static constexpr int kUt = TRANS ? 32768 : kSlotU;
+  static constexpr int kGam = TRANS ? 65536 : kSlotGam;
+  static constexpr int kIq = kSlotIq;               // full pass only
+  static constexpr int kStageBytes = TRANS ? 65536 + 512 : kSlotBytes;
+  static constexpr int kBytes = kStage + 2 * kStageBytes;
 };
 
+template <bool TRANS>
 __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ TcParams p) {
-  using L = ChainSmem;
+  using L = ChainSmem<TRANS>;
+  constexpr int SbN = L::kSbN, SbL = SbN * 16;  // N extent of the state operands, their LBO
+  constexpr int NB = SbN / 128;                 // 128-column blocks
   extern __shared__ __align__(1024) unsigned char sm[];
   __shared__ uint64_t s_bar, s_ld[2];
   __shared__ uint32_t s_tmem;
@@ -827,9 +1412,15 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
   const uint32_t tm = s_tmem;
   auto load_slot = [&](int c) {  // single thread
     const int s = (c - c0) & 1;
-    mbar_arrive_expect_tx(&s_ld[s], kSlotBytes);
-    bulk_g2s(sm + L::kStage + s * kSlotBytes, chunk_slot(p.prep, a, n, c, h, H), kSlotBytes,
-             &s_ld[s]);
+    unsigned char* dst = sm + L::kStage + s * L::kStageBytes;
+    const unsigned char* src = chunk_slot(p.prep, a, n, c, h, H);
+    mbar_arrive_expect_tx(&s_ld[s], L::kStageBytes);
+    if (TRANS) {
+      bulk_g2s(dst, src, 32768, &s_ld[s]);                           // W | K'
+      bulk_g2s(dst + L::kUt, src + kSlotU, 32768 + 512, &s_ld[s]);   // U~ | gamma
+    } else {
+      bulk_g2s(dst, src, kSlotBytes, &s_ld[s]);
+    }
   };
   if (tid == 0) {
     if (c0 < c1) load_slot(c0);
@@ -842,31 +1433,35 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
   const int srow = 32 * q4 + lane;          // dk row (M=128 accumulators)
   const int r64 = 16 * q4 + lane;           // token row of M=64 accumulators (lane < 16)
   const bool m64 = lane < 16;
-  constexpr int SbL = 2048;                 // K-group stride of the N=128 B operands
 
-  // ---- incoming state -> TMEM (fp32) and the bf16 operand
+  // ---- initial state -> TMEM (fp32) and the bf16 operand: S_in (full pass),
+  //      or S = 0 and X = I (transition)
   {
-    const float* S0 = seg > 0 ? seg_sin(p.seg, n, h, H, p.P, seg)
-                              : (p.S0 ? p.S0 + ((size_t)n * H + h) * kD * kD : nullptr);
+    const float* S0 = nullptr;
+    if (!TRANS)
+      S0 = seg > 0 ? seg_sin(p.seg, n, h, H, p.P, seg)
+                   : (p.S0 ? p.S0 + ((size_t)n * H + h) * kD * kD : nullptr);
 #pragma unroll
-    for (int c16 = 0; c16 < 32; c16 += 16) {
-      float v16[16];
-      const int col = 32 * cq + c16;
-      if (S0) {
-        const float4* src = reinterpret_cast<const float4*>(S0 + (size_t)srow * kD + col);
+    for (int blk = 0; blk < NB; ++blk)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 f = src[i];
-          v16[4 * i] = f.x; v16[4 * i + 1] = f.y; v16[4 * i + 2] = f.z; v16[4 * i + 3] = f.w;
+      for (int c16 = 0; c16 < 32; c16 += 16) {
+        float v16[16];
+        const int col = 32 * cq + c16;
+        if (S0) {
+          const float4* src = reinterpret_cast<const float4*>(S0 + (size_t)srow * kD + col);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 f = src[i];
+            v16[4 * i] = f.x; v16[4 * i + 1] = f.y; v16[4 * i + 2] = f.z; v16[4 * i + 3] = f.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v16[i] = (blk == 1 && col + i == srow) ? 1.f : 0.f;
         }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v16[i] = 0.f;
+        tmem_st16(tmem_addr(tm, 32 * q4, kTmS + 128 * blk + col), v16);
+        st16(sm + L::kSb, mnmaj(128 * blk + col, srow, SbL), v16);
+        st16(sm + L::kSb, mnmaj(128 * blk + col + 8, srow, SbL), v16 + 8);
       }
-      tmem_st16(tmem_addr(tm, 32 * q4, kTmS + col), v16);
-      st16(sm + L::kSb, mnmaj(col, srow, SbL), v16);
-      st16(sm + L::kSb, mnmaj(col + 8, srow, SbL), v16 + 8);
-    }
     tmem_st_wait();
   }
 
@@ -874,7 +1469,7 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
     const int tok0 = a + c * kC;
     const int len = min(kC, b - tok0);
     const int s = (c - c0) & 1;
-    unsigned char* st = sm + L::kStage + s * kSlotBytes;
+    unsigned char* st = sm + L::kStage + s * L::kStageBytes;
     sync_for_mma();
     {
       const bool got = mbar_wait_cycles(&s_ld[s], (ph_ld >> s) & 1, kWaitCycles);
@@ -886,55 +1481,66 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       ph_ld ^= 1u << s;
       inflight &= ~(1u << s);
     }
-    // ---- C1: D_W = W S, D_Q = Q' S  (M=64, N=128, K=128)
+    // ---- C1: D_W = W [S | X] (M=64, N=SbN, K=128); D_Q = Q' S (full pass)
     if (tid == 0) {
       const uint64_t sd = smem_desc(smem_u32(sm + L::kSb), SbL, 128);
-      const uint64_t wd = smem_desc(smem_u32(st + kSlotW), 128, 2048);
-      const uint64_t qd = smem_desc(smem_u32(st + kSlotQ), 1024, 128);
-      constexpr uint32_t idw = instr_desc(kFmtBF16, 64, 128, false, true);
-      constexpr uint32_t idq = instr_desc(kFmtBF16, 64, 128, true, true);
+      const uint64_t wd = smem_desc(smem_u32(st + L::kW), 128, 2048);
+      constexpr uint32_t idw = instr_desc(kFmtBF16, 64, SbN, false, true);
 #pragma unroll
       for (int k = 0; k < 8; ++k) mma_bf16(tm + kTmW, wd + 16 * k, sd + (2 * SbL >> 4) * k, idw, k > 0);
+      if (!TRANS) {
+        const uint64_t qd = smem_desc(smem_u32(st + L::kQ), 128, 2048);  // Q' K-major
+        constexpr uint32_t idq = instr_desc(kFmtBF16, 64, 128, false, true);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mma_bf16(tm + kTmQ, qd + 128 * k, sd + (2 * SbL >> 4) * k, idq, k > 0);
+        for (int k = 0; k < 8; ++k) mma_bf16(tm + kTmQ, qd + 16 * k, sd + (2 * SbL >> 4) * k, idq, k > 0);
+      }
       mma_commit(&s_bar);
     }
     // ---- meanwhile decay the fp32 state by gamma (C1 reads the bf16 copy)
     {
-      const float gm = reinterpret_cast<const float*>(st + kSlotGam)[srow];
-      float s0[16], s1[16];
-      const uint32_t col = kTmS + 32 * cq;
-      tmem_ld16(tmem_addr(tm, 32 * q4, col), s0);
-      tmem_ld16(tmem_addr(tm, 32 * q4, col + 16), s1);
-      tmem_ld_wait();
+      const float gm = reinterpret_cast<const float*>(st + L::kGam)[srow];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) { s0[i] *= gm; s1[i] *= gm; }
-      tmem_st16(tmem_addr(tm, 32 * q4, col), s0);
-      tmem_st16(tmem_addr(tm, 32 * q4, col + 16), s1);
+      for (int blk = 0; blk < NB; ++blk) {
+        float s0[16], s1[16];
+        const uint32_t col = kTmS + 128 * blk + 32 * cq;
+        tmem_ld16(tmem_addr(tm, 32 * q4, col), s0);
+        tmem_ld16(tmem_addr(tm, 32 * q4, col + 16), s1);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) { s0[i] *= gm; s1[i] *= gm; }
+        tmem_st16(tmem_addr(tm, 32 * q4, col), s0);
+        tmem_st16(tmem_addr(tm, 32 * q4, col + 16), s1);
+      }
       tmem_st_wait();
     }
     if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
-    // ---- U = U~ - D_W -> B operand (MN-major)
-    {
+    // ---- U = U~ - D_W (transition: [U~ | 0] - W [S | X]) -> B operand (MN-major)
+#pragma unroll
+    for (int blk = 0; blk < NB; ++blk) {
       float d0[16], d1[16];
-      const int col = 32 * cq;
+      const int col = 128 * blk + 32 * cq;
       tmem_ld16(tmem_addr(tm, 32 * q4, kTmW + col), d0);
       tmem_ld16(tmem_addr(tm, 32 * q4, kTmW + col + 16), d1);
       tmem_ld_wait();
       if (m64) {
-        const float4* ug = reinterpret_cast<const float4*>(st + kSlotU);
+        if (blk == 0) {
+          const float4* ug = reinterpret_cast<const float4*>(st + L::kUt);
 #pragma unroll
-        for (int pc = 0; pc < 4; ++pc) {
-          const float4 u0 = ug[ut_index(q4, cq, pc, lane) >> 2];
-          const float4 u1 = ug[ut_index(q4, cq, pc + 4, lane) >> 2];
-          d0[4 * pc] = u0.x - d0[4 * pc];
-          d0[4 * pc + 1] = u0.y - d0[4 * pc + 1];
-          d0[4 * pc + 2] = u0.z - d0[4 * pc + 2];
-          d0[4 * pc + 3] = u0.w - d0[4 * pc + 3];
-          d1[4 * pc] = u1.x - d1[4 * pc];
-          d1[4 * pc + 1] = u1.y - d1[4 * pc + 1];
-          d1[4 * pc + 2] = u1.z - d1[4 * pc + 2];
-          d1[4 * pc + 3] = u1.w - d1[4 * pc + 3];
+          for (int pc = 0; pc < 4; ++pc) {
+            const float4 u0 = ug[ut_index(q4, cq, pc, lane) >> 2];
+            const float4 u1 = ug[ut_index(q4, cq, pc + 4, lane) >> 2];
+            d0[4 * pc] = u0.x - d0[4 * pc];
+            d0[4 * pc + 1] = u0.y - d0[4 * pc + 1];
+            d0[4 * pc + 2] = u0.z - d0[4 * pc + 2];
+            d0[4 * pc + 3] = u0.w - d0[4 * pc + 3];
+            d1[4 * pc] = u1.x - d1[4 * pc];
+            d1[4 * pc + 1] = u1.y - d1[4 * pc + 1];
+            d1[4 * pc + 2] = u1.z - d1[4 * pc + 2];
+            d1[4 * pc + 3] = u1.w - d1[4 * pc + 3];
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) { d0[i] = -d0[i]; d1[i] = -d1[i]; }
         }
         st16(sm + L::kU, mnmaj(col, r64, SbL), d0);
         st16(sm + L::kU, mnmaj(col + 8, r64, SbL), d0 + 8);
@@ -943,17 +1549,19 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       }
     }
     sync_for_mma();
-    // ---- C2: S += K'^T U (M=128, K=64); D_Q += A_qk U (M=64, K=64)
+    // ---- C2: [S | X] += K'^T U (M=128, K=64); D_Q += A_qk U (full pass)
     if (tid == 0) {
-      const uint64_t kd = smem_desc(smem_u32(st + kSlotK), 128, 1024);
+      const uint64_t kd = smem_desc(smem_u32(st + L::kK), 2048, 128);  // K' MN-major
       const uint64_t ud = smem_desc(smem_u32(sm + L::kU), SbL, 128);
-      const uint64_t a3 = smem_desc(smem_u32(st + kSlotA3), 1024, 128);
-      constexpr uint32_t ids = instr_desc(kFmtBF16, 128, 128, false, true);
-      constexpr uint32_t ido = instr_desc(kFmtBF16, 64, 128, true, true);
+      constexpr uint32_t ids = instr_desc(kFmtBF16, 128, SbN, true, true);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) mma_bf16(tm + kTmS, kd + 16 * k, ud + (2 * SbL >> 4) * k, ids, 1);
+      for (int k = 0; k < 4; ++k) mma_bf16(tm + kTmS, kd + 256 * k, ud + (2 * SbL >> 4) * k, ids, 1);
+      if (!TRANS) {
+        const uint64_t a3 = smem_desc(smem_u32(st + L::kA3), 1024, 128);
+        constexpr uint32_t ido = instr_desc(kFmtBF16, 64, 128, true, true);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) mma_bf16(tm + kTmQ, a3 + 128 * k, ud + (2 * SbL >> 4) * k, ido, 1);
+        for (int k = 0; k < 4; ++k) mma_bf16(tm + kTmQ, a3 + 128 * k, ud + (2 * SbL >> 4) * k, ido, 1);
+      }
       mma_commit(&s_bar);
     }
     if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
@@ -962,10 +1570,11 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       inflight |= 1u << s;
       if (tid == 0) load_slot(c + 2);
     }
-    // ---- S -> bf16 operand of the next chunk; o = D_Q * |q|^-1 -> global
-    {
+    // ---- [S | X] -> bf16 operand of the next chunk; o = D_Q / |q| -> global
+#pragma unroll
+    for (int blk = 0; blk < NB; ++blk) {
       float s0[16], s1[16];
-      const int col = 32 * cq;
+      const int col = 128 * blk + 32 * cq;
       tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + col), s0);
       tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + col + 16), s1);
       tmem_ld_wait();
@@ -973,12 +1582,15 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       st16(sm + L::kSb, mnmaj(col + 8, srow, SbL), s0 + 8);
       st16(sm + L::kSb, mnmaj(col + 16, srow, SbL), s1);
       st16(sm + L::kSb, mnmaj(col + 24, srow, SbL), s1 + 8);
+    }
+    if (!TRANS) {
+      const int col = 32 * cq;
       float o0[16], o1[16];
       tmem_ld16(tmem_addr(tm, 32 * q4, kTmQ + col), o0);
       tmem_ld16(tmem_addr(tm, 32 * q4, kTmQ + col + 16), o1);
       tmem_ld_wait();
       if (m64 && r64 < len) {
-        const float iq = reinterpret_cast<const float*>(st + kSlotIq)[r64];
+        const float iq = reinterpret_cast<const float*>(st + L::kIq)[r64];
 #pragma unroll
         for (int i = 0; i < 16; ++i) { o0[i] *= iq; o1[i] *= iq; }
         uint4* dst = reinterpret_cast<uint4*>(p.o + ((size_t)(tok0 + r64) * H + h) * kD + col);
@@ -994,17 +1606,25 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
   __syncthreads();
   fence_after_sync();
   if (!s_abort) {
-    if (p.S_final && seg == p.P - 1) {
-      float* dst = p.S_final + ((size_t)n * H + h) * kD * kD + (size_t)srow * kD;
+    float* dst0 = nullptr;
+    if (TRANS)
+      dst0 = seg_trans(p.seg, n, h, H, p.P, seg);  // M_p, then N_p
+    else if (p.S_final && seg == p.P - 1)
+      dst0 = p.S_final + ((size_t)n * H + h) * kD * kD;
+    if (dst0) {
 #pragma unroll
-      for (int c16 = 0; c16 < 32; c16 += 16) {
-        float s16[16];
-        tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + 32 * cq + c16), s16);
-        tmem_ld_wait();
+      for (int blk = 0; blk < NB; ++blk)
 #pragma unroll
-        for (int i = 0; i < 16; i += 4)
-          *reinterpret_cast<float4*>(dst + 32 * cq + c16 + i) = make_float4(s16[i], s16[i + 1], s16[i + 2], s16[i + 3]);
-      }
+        for (int c16 = 0; c16 < 32; c16 += 16) {
+          float s16[16];
+          tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + 128 * blk + 32 * cq + c16), s16);
+          tmem_ld_wait();
+          // transition: S (block 0) is N_p, X (block 1) is M_p
+          float* dst = (TRANS ? dst0 + (blk == 0 ? kD * kD : 0) : dst0) + (size_t)srow * kD + 32 * cq + c16;
+#pragma unroll
+          for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4*>(dst + i) = make_float4(s16[i], s16[i + 1], s16[i + 2], s16[i + 3]);
+        }
     }
   } else if (tid == 0) {
     // a wait gave up: let the slot copies still in flight land before leaving
@@ -1093,15 +1713,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // [T, H, 128] bf16 tensor, box 64 tokens x 1 head x 128 channels; rows past T
 // read as zero.
-bool make_map(CUtensorMap* map, const void* base, int T, int H) {
+// [T, H, 128] bf16 tensor; box 64 tokens x 1 head x 128 channels, or (swizzled)
+// x 64 channels with the 128-byte swizzle
+bool make_map(CUtensorMap* map, const void* base, int T, int H, bool swizzled = false) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)T};
   const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2};
-  const cuuint32_t box[3] = {(cuuint32_t)kD, 1, (cuuint32_t)kC};
+  const cuuint32_t box[3] = {(cuuint32_t)(swizzled ? kD / 2 : kD), 1, (cuuint32_t)kC};
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swizzled ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1139,18 +1762,25 @@ size_t tc_workspace_bytes(int N, int T, int H, int max_len) {
 
 int tc_launches(int N, int H, int max_len) {
   if (N <= 0) return 0;
-  return tc_segments(N, H, max_len) > 1 ? 3 : 1;
+  return tc_segments(N, H, max_len) > 1 ? 4 : 1;
 }
 
 cudaError_t launch_forward_tc(const ForwardArgs& a) {
   TcParams p;
   memset(&p, 0, sizeof(p));
   if (a.T > 0) {
+    const void* zz = a.z ? a.z : a.k;
     if (!make_map(&p.tq, a.q, a.T, a.H) || !make_map(&p.tk, a.k, a.T, a.H) ||
-        !make_map(&p.tz, a.z ? a.z : a.k, a.T, a.H) || !make_map(&p.tv, a.v, a.T, a.H))
+        !make_map(&p.tz, zz, a.T, a.H) || !make_map(&p.tv, a.v, a.T, a.H) ||
+        !make_map(&p.sq, a.q, a.T, a.H, true) || !make_map(&p.sk, a.k, a.T, a.H, true) ||
+        !make_map(&p.sz, zz, a.T, a.H, true) || !make_map(&p.sv, a.v, a.T, a.H, true))
       return cudaErrorInvalidValue;
   }
   p.beta = (const __nv_bfloat16*)a.beta;
+  p.q = (const __nv_bfloat16*)a.q;
+  p.k = (const __nv_bfloat16*)a.k;
+  p.z = (const __nv_bfloat16*)a.z;
+  p.v = (const __nv_bfloat16*)a.v;
   p.A = a.A;
   p.g = a.g;
   p.S0 = a.S0;
@@ -1166,19 +1796,28 @@ cudaError_t launch_forward_tc(const ForwardArgs& a) {
   p.seg = (float*)((char*)a.ws + sizeof(WsHeader));
   cudaError_t err;
   if (p.P > 1) {
-    // transition pass (+ chain operands) -> incoming states -> chain pass
+    // chunk preparation -> segment transitions -> incoming states -> chain pass
     p.prep = (unsigned char*)a.ws + prep_offset(a.N, a.H, p.P);
-    err = cudaFuncSetAttribute(tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               Smem<1>::kBytes);
+    err = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               PrepSmem::kBytes);
     if (err != cudaSuccess) return err;
-    tc_kernel<1><<<dim3(a.N, a.H, p.P), kNT, Smem<1>::kBytes, a.stream>>>(p);
+    int sms = 0, dev = 0;
+    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+    if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return err;
+    prep_kernel<<<sms, kPrepThreads, PrepSmem::kBytes, a.stream>>>(p);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    err = cudaFuncSetAttribute(chain_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               ChainSmem<true>::kBytes);
+    if (err != cudaSuccess) return err;
+    chain_kernel<true><<<dim3(a.N, a.H, p.P - 1), kNT, ChainSmem<true>::kBytes, a.stream>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     compose_kernel<<<dim3(a.N, a.H, kD / 16), 256, 0, a.stream>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    err = cudaFuncSetAttribute(chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               ChainSmem::kBytes);
+    err = cudaFuncSetAttribute(chain_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               ChainSmem<false>::kBytes);
     if (err != cudaSuccess) return err;
-    chain_kernel<<<dim3(a.N, a.H, p.P), kNT, ChainSmem::kBytes, a.stream>>>(p);
+    chain_kernel<false><<<dim3(a.N, a.H, p.P), kNT, ChainSmem<false>::kBytes, a.stream>>>(p);
     return cudaGetLastError();
   }
   err = cudaFuncSetAttribute(tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
