@@ -53,11 +53,9 @@ constexpr int kD = 128;   // dk = dv
 constexpr int kNT = 512;  // threads (16 warps)
 
 // ---- shared memory map (bytes), per pass ----
-template <int MODE>
-struct Smem {
-  static constexpr int kSb = 0;                                 // S (| X) bf16, B operand, MN-major
-  static constexpr int kSizeSb = MODE == 0 ? 32768 : 65536;
-  static constexpr int kRaw = kSb + kSizeSb;                    // q | k | z | v, [64][128] bf16
+struct FusedSmem {
+  static constexpr int kSb = 0;                                 // S bf16, B operand, MN-major
+  static constexpr int kRaw = kSb + 32768;                      // q | k | z | v, [64][128] bf16
   static constexpr int kP = kRaw + 65536;                       // region P, reused through a chunk:
   static constexpr int kR = kP;                                 //   R   B op (N=128, K=128) MN-major
   static constexpr int kCc = kP + 32768;                        //   C   A op (M=160, K=128) MN-major
@@ -67,11 +65,10 @@ struct Smem {
   static constexpr int kQp = kP + 32768;                        //   Q'  A op (M=64, K=128) MN-major
   static constexpr int kKp = kP + 49152;                        //   K'  A op (M=128, K=64) K-major
   static constexpr int kW = kP;                                 //   W   A op (M=64, K=128) K-major
-  static constexpr int kU = kP;                                 //   U   B op (N=128|256, K=64) MN-major
-  static constexpr int kUt = kP + 16384;                        //   U~  fp32 slot image (transition)
+  static constexpr int kU = kP;                                 //   U   B op (N=128, K=64) MN-major
   static constexpr int kTop = kP + 73728;                       // T   A op (M=64, K=64) K-major
   static constexpr int kA3 = kTop + 8192;                       // A_qk A op (M=64, K=64) MN-major
-  static constexpr int kVec = kA3 + (MODE == 0 ? 8192 : 0);
+  static constexpr int kVec = kA3 + 8192;
   static constexpr int kBytes = kVec + 2304 * 4 + 64;
 };
 // vectors (floats) at Smem::kVec
@@ -91,10 +88,10 @@ constexpr int kLd = 68;  // row stride (floats) of the fp32 A_kk / T tiles
 // by the chain pass with one bulk copy.  The bf16 images have exactly the
 // shared-memory layouts the MMAs read: W (A, K-major, M=64 K=128), K' (A,
 // K-major, M=128 K=64), Q' (A, MN-major, M=64 K=128), A_qk (A, MN-major, M=64
-// K=64); U~ is fp32 in the order the chain threads read it (see ut_index);
+// K=64); U~ is bf16 in the order the chain threads read it (see ut_index);
 // then gamma (128 fp32) and the query row scales (64 fp32).
 constexpr int kSlotW = 0, kSlotK = 16384, kSlotQ = 32768, kSlotA3 = 49152, kSlotU = 57344,
-              kSlotGam = 90112, kSlotIq = 90624, kSlotBytes = 90880;
+              kSlotGam = 73728, kSlotIq = 74240, kSlotBytes = 74496;
 // Chunk c of sequence n (first token a) has slot a / C + n + c: distinct for
 // every chunk of every sequence and below T / C + N.
 __device__ __forceinline__ unsigned char* chunk_slot(const unsigned char* prep_base, int a, int n,
@@ -102,10 +99,10 @@ __device__ __forceinline__ unsigned char* chunk_slot(const unsigned char* prep_b
   return const_cast<unsigned char*>(prep_base) +
          ((size_t)(a / 64 + n + c) * H + h) * (size_t)kSlotBytes;
 }
-// float index of U~ (row r = 16 q4 + l, l < 16; column 32 cq + 4 pc + e) in a
-// slot: each warp's 16 active lanes read 256 consecutive bytes per float4.
+// 16-byte unit of U~ (row r = 16 q4 + l, l < 16; columns 32 cq + 8 pc .. +7, bf16)
+// in a slot: each warp's 16 active lanes read 256 consecutive bytes per vector.
 __device__ __forceinline__ int ut_index(int q4, int cq, int pc, int l) {
-  return (((cq * 4 + q4) * 8 + pc) * 16 + l) * 4;
+  return ((cq * 4 + q4) * 4 + pc) * 16 + l;
 }
 
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s: a wait this long is a fault
@@ -238,13 +235,11 @@ __device__ __forceinline__ void sync_for_mma() {
 }
 
 // ---------------------------------------------------------------------------
-// MODE 0: full pass from the true incoming state, writes o and S_final (used
-//         when the sequences are not split into segments).
-// MODE 1: transition pass: for segments 0..P-2, the chain from S = 0 (N) and
-//         X = I (M); for every segment, each chunk's chain operands to its slot.
-template <int MODE>
-__global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcParams p) {
-  using L = Smem<MODE>;
+// Fused pass for sequences that are not split into segments: one CTA per
+// (sequence, head) prepares each chunk and advances the state through it,
+// chunk after chunk (incoming state S0 or S_in of its segment); o, S_final.
+__global__ void __launch_bounds__(kNT, 1) fused_kernel(const __grid_constant__ TcParams p) {
+  using L = FusedSmem;
   extern __shared__ __align__(1024) unsigned char sm[];
   __shared__ uint64_t s_bar, s_bar_raw;
   __shared__ uint32_t s_tmem;
@@ -265,8 +260,6 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
   const int nch = (b - a + kC - 1) / kC;
   int c0, c1;
   segment_chunks(nch, p.P, seg, c0, c1);
-  // the last segment's transition is never used: its pass only fills slots
-  const bool chain = MODE == 0 || seg < p.P - 1;
 
   // ---- set-up: TMEM, barriers, first chunk's rows
   if (warp == 0) {
@@ -287,19 +280,17 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
   bool raw_pending = c0 < c1;  // a TMA load into the staging area is in flight
   if (tid == 0 && c0 < c1) stage_chunk(p, raw, &s_bar_raw, a + c0 * kC, h);
 
-  constexpr int SbN = MODE == 0 ? 128 : 256;  // N extent of the bf16 state operand
+  constexpr int SbN = 128;                    // N extent of the bf16 state operand
   constexpr int SbL = SbN * 16;               // its K-group stride (LBO)
   const int q4 = warp & 3, cq = warp >> 2;    // TMEM lane quarter, 32-column quarter
   const int srow = 32 * q4 + lane;            // dk row (M=128 accumulators)
   const int r64 = 16 * q4 + lane;             // token row of M=64 accumulators (lane < 16)
   const bool m64 = lane < 16;
 
-  // ---- initial state: S0 (or the composed incoming state), and X = I
+  // ---- initial state: S0 (or the composed incoming state)
   {
-    const float* S0 = nullptr;
-    if (MODE == 0)
-      S0 = seg > 0 ? seg_sin(p.seg, n, h, H, p.P, seg)
-                   : (p.S0 ? p.S0 + ((size_t)n * H + h) * kD * kD : nullptr);
+    const float* S0 = seg > 0 ? seg_sin(p.seg, n, h, H, p.P, seg)
+                              : (p.S0 ? p.S0 + ((size_t)n * H + h) * kD * kD : nullptr);
 #pragma unroll
     for (int c16 = 0; c16 < 32; c16 += 16) {
       float v16[16];
@@ -318,13 +309,6 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
       tmem_st16(tmem_addr(tm, 32 * q4, kTmS + col), v16);
       st16(sm + L::kSb, mnmaj(col, srow, SbL), v16);
       st16(sm + L::kSb, mnmaj(col + 8, srow, SbL), v16 + 8);
-      if (MODE == 1) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v16[i] = (col + i == srow) ? 1.f : 0.f;
-        tmem_st16(tmem_addr(tm, 32 * q4, kTmS + 128 + col), v16);
-        st16(sm + L::kSb, mnmaj(128 + col, srow, SbL), v16);
-        st16(sm + L::kSb, mnmaj(128 + col + 8, srow, SbL), v16 + 8);
-      }
     }
     tmem_st_wait();
   }
@@ -343,7 +327,6 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
   for (int c = c0; c < c1; ++c) {
     const int tok0 = a + c * kC;
     const int len = min(kC, b - tok0);
-    unsigned char* slot = MODE == 1 ? chunk_slot(p.prep, a, n, c, h, H) : nullptr;
     sync_for_mma();
     if (tid < kC) vec[kVecBeta + tid] = beta_next;
     beta_next = load_beta(c + 1);
@@ -402,8 +385,6 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
         Ei[i] = __fdividef(1.0f, E[i]);
       }
     }
-    // region P is rewritten from here on: the previous chunk's bulk stores must have read it
-    if (MODE == 1 && tid == 0) bulk_wait_read();
     __syncthreads();
     // rho_b = Gam at the first token of sub-tile b; Gam_last = Gam at row 63
     float rho[4], glast;
@@ -478,9 +459,8 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
           Akk[r * kLd + i] = (i < r) ? vec[kVecBeta + r] * vec[kVecIk + r] * ki * va[cc] : 0.f;
           vq[cc] = (i <= r) ? vq[cc] * ki : 0.f;
         }
-        unsigned char* a3 = MODE == 0 ? sm + L::kA3 : slot + kSlotA3;
-        st16(a3, mnmaj(16 * bb, i, 1024), vq);
-        st16(a3, mnmaj(16 * bb + 8, i, 1024), vq + 8);
+        st16(sm + L::kA3, mnmaj(16 * bb, i, 1024), vq);
+        st16(sm + L::kA3, mnmaj(16 * bb + 8, i, 1024), vq + 8);
       }
     }
     fence_before_sync();
@@ -563,12 +543,7 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
     // ---- WY / chain operands: X_K, X_V (K-major), Q' (MN-major), K' (K-major), gamma
     {
       const float er = __expf(rq), el = __expf(glast - rq);
-      if (qq == 0) {
-        const float gam = __expf(glast);
-        vec[kVecGam + j] = gam;
-        if (MODE == 1) reinterpret_cast<float*>(slot + kSlotGam)[j] = gam;
-      }
-      if (MODE == 1 && tid < kC) reinterpret_cast<float*>(slot + kSlotIq)[tid] = vec[kVecIq + tid];
+      if (qq == 0) vec[kVecGam + j] = __expf(glast);
 #pragma unroll
       for (int g8 = 0; g8 < 2; ++g8) {
         const int r0 = 16 * qq + 8 * g8;
@@ -591,11 +566,6 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
       }
     }
     sync_for_mma();
-    if (MODE == 1 && tid == 0) {
-      bulk_s2g(slot + kSlotQ, sm + L::kQp, 16384);
-      bulk_s2g(slot + kSlotK, sm + L::kKp, 16384);
-      bulk_commit();
-    }
     // the staged rows are consumed: prefetch the next chunk
     if (c + 1 < c1) {
       raw_pending = true;
@@ -609,7 +579,6 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
 #pragma unroll
       for (int k = 0; k < 4; ++k) mma_bf16(tm + kTmWU, ad + 16 * k, bd + 16 * k, id, k > 0);
       mma_commit(&s_bar);
-      if (MODE == 1) bulk_wait_read();  // Q' is overwritten by the U~ image below
     }
     if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
     // ---- W -> bf16 A operand (K-major); U~ -> registers (M=64 rows, lane < 16)
@@ -626,80 +595,54 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
         st16(sm + L::kW, kmaj(r64, 32 * cq + c16, 2048), w16);
         st16(sm + L::kW, kmaj(r64, 32 * cq + c16 + 8, 2048), w16 + 8);
       }
-      if (MODE == 1 && m64) {
-        float4* ug = reinterpret_cast<float4*>(sm + L::kUt);
-#pragma unroll
-        for (int pc = 0; pc < 4; ++pc)
-          ug[ut_index(q4, cq, (c16 >> 2) + pc, lane) >> 2] =
-              make_float4(u16[4 * pc], u16[4 * pc + 1], u16[4 * pc + 2], u16[4 * pc + 3]);
-      }
     }
     sync_for_mma();
-    if (MODE == 1 && tid == 0) {
-      bulk_s2g(slot + kSlotW, sm + L::kW, 16384);
-      bulk_s2g(slot + kSlotU, sm + L::kUt, 32768);
-      bulk_commit();
-    }
-    if (!chain) continue;
-    // ---- C1: D_W = W S (M=64, N=128|256), D_Q = Q' S (M=64, N=128)
+    // ---- C1: D_W = W S, D_Q = Q' S (M=64, N=128, K=128)
     if (tid == 0) {
       const uint64_t sd = smem_desc(smem_u32(sm + L::kSb), SbL, 128);
       const uint64_t wd = smem_desc(smem_u32(sm + L::kW), 128, 2048);
+      const uint64_t qd = smem_desc(smem_u32(sm + L::kQp), 1024, 128);
       constexpr uint32_t idw = instr_desc(kFmtBF16, 64, SbN, false, true);
+      constexpr uint32_t idq = instr_desc(kFmtBF16, 64, 128, true, true);
 #pragma unroll
       for (int k = 0; k < 8; ++k) mma_bf16(tm + kTmW, wd + 16 * k, sd + (2 * SbL >> 4) * k, idw, k > 0);
-      if (MODE == 0) {
-        constexpr uint32_t idq = instr_desc(kFmtBF16, 64, 128, true, true);
-        const uint64_t qd = smem_desc(smem_u32(sm + L::kQp), 1024, 128);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mma_bf16(tm + kTmQ, qd + 128 * k, sd + (2 * SbL >> 4) * k, idq, k > 0);
-      }
+      for (int k = 0; k < 8; ++k) mma_bf16(tm + kTmQ, qd + 128 * k, sd + (2 * SbL >> 4) * k, idq, k > 0);
       mma_commit(&s_bar);
     }
-    // ---- meanwhile decay the fp32 state(s) by gamma = e^{Gam_last} (rows = dk =
+    // ---- meanwhile decay the fp32 state by gamma = e^{Gam_last} (rows = dk =
     //      TMEM lanes); C1 reads the bf16 copy
     {
       const float gm = vec[kVecGam + srow];
-      constexpr int NB = MODE == 0 ? 1 : 2;
+      float s0[16], s1[16];
+      const uint32_t col = kTmS + 32 * cq;
+      tmem_ld16(tmem_addr(tm, 32 * q4, col), s0);
+      tmem_ld16(tmem_addr(tm, 32 * q4, col + 16), s1);
+      tmem_ld_wait();
 #pragma unroll
-      for (int blk = 0; blk < NB; ++blk)
-      {
-        float s0[16], s1[16];
-        const uint32_t col = kTmS + 128 * blk + 32 * cq;
-        tmem_ld16(tmem_addr(tm, 32 * q4, col), s0);
-        tmem_ld16(tmem_addr(tm, 32 * q4, col + 16), s1);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) { s0[i] *= gm; s1[i] *= gm; }
-        tmem_st16(tmem_addr(tm, 32 * q4, col), s0);
-        tmem_st16(tmem_addr(tm, 32 * q4, col + 16), s1);
-      }
+      for (int i = 0; i < 16; ++i) { s0[i] *= gm; s1[i] *= gm; }
+      tmem_st16(tmem_addr(tm, 32 * q4, col), s0);
+      tmem_st16(tmem_addr(tm, 32 * q4, col + 16), s1);
       tmem_st_wait();
     }
-    if (MODE == 1 && tid == 0) bulk_wait_read();  // U overwrites the W and U~ images
     if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
-    // ---- U = U~ - W S  (transition: [U_S | U_X] = [U~ | 0] - W [S | X]); B operand MN-major
+    // ---- U = U~ - W S -> B operand (MN-major)
     {
-      constexpr int NB = MODE == 0 ? 1 : 2;
+      float d0[16], d1[16];
+      const int col = 32 * cq;
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmW + col), d0);
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmW + col + 16), d1);
+      tmem_ld_wait();
+      if (m64) {
 #pragma unroll
-      for (int blk = 0; blk < NB; ++blk)
-      {
-        float d0[16], d1[16];
-        const int col = 128 * blk + 32 * cq;
-        tmem_ld16(tmem_addr(tm, 32 * q4, kTmW + col), d0);
-        tmem_ld16(tmem_addr(tm, 32 * q4, kTmW + col + 16), d1);
-        tmem_ld_wait();
-        if (m64) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            d0[i] = (blk == 0 ? ut[i] : 0.f) - d0[i];
-            d1[i] = (blk == 0 ? ut[16 + i] : 0.f) - d1[i];
-          }
-          st16(sm + L::kU, mnmaj(col, r64, SbL), d0);
-          st16(sm + L::kU, mnmaj(col + 8, r64, SbL), d0 + 8);
-          st16(sm + L::kU, mnmaj(col + 16, r64, SbL), d1);
-          st16(sm + L::kU, mnmaj(col + 24, r64, SbL), d1 + 8);
+        for (int i = 0; i < 16; ++i) {
+          d0[i] = ut[i] - d0[i];
+          d1[i] = ut[16 + i] - d1[i];
         }
+        st16(sm + L::kU, mnmaj(col, r64, SbL), d0);
+        st16(sm + L::kU, mnmaj(col + 8, r64, SbL), d0 + 8);
+        st16(sm + L::kU, mnmaj(col + 16, r64, SbL), d1);
+        st16(sm + L::kU, mnmaj(col + 24, r64, SbL), d1 + 8);
       }
     }
     sync_for_mma();
@@ -707,49 +650,40 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
     if (tid == 0) {
       const uint64_t kd = smem_desc(smem_u32(sm + L::kKp), 128, 1024);
       const uint64_t ud = smem_desc(smem_u32(sm + L::kU), SbL, 128);
+      const uint64_t a3 = smem_desc(smem_u32(sm + L::kA3), 1024, 128);
       constexpr uint32_t ids = instr_desc(kFmtBF16, 128, SbN, false, true);
+      constexpr uint32_t ido = instr_desc(kFmtBF16, 64, 128, true, true);
 #pragma unroll
       for (int k = 0; k < 4; ++k) mma_bf16(tm + kTmS, kd + 16 * k, ud + (2 * SbL >> 4) * k, ids, 1);
-      if (MODE == 0) {
-        constexpr uint32_t ido = instr_desc(kFmtBF16, 64, 128, true, true);
-        const uint64_t a3 = smem_desc(smem_u32(sm + L::kA3), 1024, 128);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) mma_bf16(tm + kTmQ, a3 + 128 * k, ud + (2 * SbL >> 4) * k, ido, 1);
-      }
+      for (int k = 0; k < 4; ++k) mma_bf16(tm + kTmQ, a3 + 128 * k, ud + (2 * SbL >> 4) * k, ido, 1);
       mma_commit(&s_bar);
     }
     if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
-    // ---- S (and X) -> bf16 operand for the next chunk; O -> global
+    // ---- S -> bf16 operand for the next chunk; O -> global
     {
-      constexpr int NB = MODE == 0 ? 1 : 2;
+      float s0[16], s1[16];
+      const int col = 32 * cq;
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + col), s0);
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + col + 16), s1);
+      tmem_ld_wait();
+      st16(sm + L::kSb, mnmaj(col, srow, SbL), s0);
+      st16(sm + L::kSb, mnmaj(col + 8, srow, SbL), s0 + 8);
+      st16(sm + L::kSb, mnmaj(col + 16, srow, SbL), s1);
+      st16(sm + L::kSb, mnmaj(col + 24, srow, SbL), s1 + 8);
+      float o0[16], o1[16];
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmQ + col), o0);
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmQ + col + 16), o1);
+      tmem_ld_wait();
+      if (m64 && r64 < len) {
+        const float iq = vec[kVecIq + r64];
 #pragma unroll
-      for (int blk = 0; blk < NB; ++blk)
-      {
-        float s0[16], s1[16];
-        const int col = 128 * blk + 32 * cq;
-        tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + col), s0);
-        tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + col + 16), s1);
-        tmem_ld_wait();
-        st16(sm + L::kSb, mnmaj(col, srow, SbL), s0);
-        st16(sm + L::kSb, mnmaj(col + 8, srow, SbL), s0 + 8);
-        st16(sm + L::kSb, mnmaj(col + 16, srow, SbL), s1);
-        st16(sm + L::kSb, mnmaj(col + 24, srow, SbL), s1 + 8);
-      }
-      if (MODE == 0) {
-        float o0[16], o1[16];
-        tmem_ld16(tmem_addr(tm, 32 * q4, kTmQ + 32 * cq), o0);
-        tmem_ld16(tmem_addr(tm, 32 * q4, kTmQ + 32 * cq + 16), o1);
-        tmem_ld_wait();
-        if (m64 && r64 < len) {
-          const float iq = vec[kVecIq + r64];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) { o0[i] *= iq; o1[i] *= iq; }
-          uint4* dst = reinterpret_cast<uint4*>(p.o + ((size_t)(tok0 + r64) * H + h) * kD + 32 * cq);
-          dst[0] = pack8(o0);
-          dst[1] = pack8(o0 + 8);
-          dst[2] = pack8(o1);
-          dst[3] = pack8(o1 + 8);
-        }
+        for (int i = 0; i < 16; ++i) { o0[i] *= iq; o1[i] *= iq; }
+        uint4* dst = reinterpret_cast<uint4*>(p.o + ((size_t)(tok0 + r64) * H + h) * kD + col);
+        dst[0] = pack8(o0);
+        dst[1] = pack8(o0 + 8);
+        dst[2] = pack8(o1);
+        dst[3] = pack8(o1 + 8);
       }
     }
   }
@@ -759,41 +693,22 @@ __global__ void __launch_bounds__(kNT, 1) tc_kernel(const __grid_constant__ TcPa
   __syncthreads();
   fence_after_sync();
   if (!s_abort) {
-    if (MODE == 0) {
-      if (p.S_final && seg == p.P - 1) {
-        float* dst = p.S_final + ((size_t)n * H + h) * kD * kD + (size_t)srow * kD;
+    if (p.S_final && seg == p.P - 1) {
+      float* dst = p.S_final + ((size_t)n * H + h) * kD * kD + (size_t)srow * kD;
 #pragma unroll
-        for (int c16 = 0; c16 < 32; c16 += 16) {
-          float s16[16];
-          tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + 32 * cq + c16), s16);
-          tmem_ld_wait();
+      for (int c16 = 0; c16 < 32; c16 += 16) {
+        float s16[16];
+        tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + 32 * cq + c16), s16);
+        tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4*>(dst + 32 * cq + c16 + i) = make_float4(s16[i], s16[i + 1], s16[i + 2], s16[i + 3]);
-        }
+        for (int i = 0; i < 16; i += 4)
+          *reinterpret_cast<float4*>(dst + 32 * cq + c16 + i) = make_float4(s16[i], s16[i + 1], s16[i + 2], s16[i + 3]);
       }
-    } else if (chain) {
-      // transition: N from S (columns 256..383), M from X (columns 384..511)
-      float* Mt = seg_trans(p.seg, n, h, H, p.P, seg);
-      float* Nt = Mt + kD * kD;
-#pragma unroll
-      for (int blk = 0; blk < 2; ++blk)
-#pragma unroll
-        for (int c16 = 0; c16 < 32; c16 += 16) {
-          float s16[16];
-          tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + 128 * blk + 32 * cq + c16), s16);
-          tmem_ld_wait();
-          float* dst = (blk == 0 ? Nt : Mt) + (size_t)srow * kD + 32 * cq + c16;
-#pragma unroll
-          for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4*>(dst + i) = make_float4(s16[i], s16[i + 1], s16[i + 2], s16[i + 3]);
-        }
     }
   } else if (raw_pending) {
     // a wait gave up: let the TMA load still in flight land before leaving
     mbar_wait_cycles(&s_bar_raw, phase_raw, kWaitCycles);
   }
-  if (MODE == 1 && tid == 0) bulk_wait_all();
   fence_before_sync();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tm, 512);
@@ -1327,17 +1242,15 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
       tmem_ld16(tmem_addr(tm, 32 * q4, kTmWU + 128 + 32 * cq + c16), u16);
       tmem_ld_wait();
       if (m64) {
-        float4* ug = reinterpret_cast<float4*>(sm + L::kUt);
-#pragma unroll
-        for (int pc = 0; pc < 4; ++pc)
-          ug[ut_index(q4, cq, (c16 >> 2) + pc, lane) >> 2] =
-              make_float4(u16[4 * pc], u16[4 * pc + 1], u16[4 * pc + 2], u16[4 * pc + 3]);
+        uint4* ug = reinterpret_cast<uint4*>(sm + L::kUt);
+        ug[ut_index(q4, cq, (c16 >> 3), lane)] = pack8(u16);
+        ug[ut_index(q4, cq, (c16 >> 3) + 1, lane)] = pack8(u16 + 8);
       }
     }
     group_sync_for_mma(bid);
     if (gtid == 0) {
       bulk_s2g(slot + kSlotW, sm + L::kW, 16384);
-      bulk_s2g(slot + kSlotU, sm + L::kUt, 32768);
+      bulk_s2g(slot + kSlotU, sm + L::kUt, 16384);
       bulk_commit();
     }
   }
@@ -1369,9 +1282,9 @@ struct ChainSmem {
   // stage layout: the slot (full pass), or W | K' | U~ | gamma (transition)
   static constexpr int kW = kSlotW, kK = kSlotK, kQ = kSlotQ, kA3 = kSlotA3;
   static constexpr int kUt = TRANS ? 32768 : kSlotU;
-  static constexpr int kGam = TRANS ? 65536 : kSlotGam;
+  static constexpr int kGam = TRANS ? 32768 + 16384 : kSlotGam;
   static constexpr int kIq = kSlotIq;               // full pass only
-  static constexpr int kStageBytes = TRANS ? 65536 + 512 : kSlotBytes;
+  static constexpr int kStageBytes = TRANS ? 32768 + 16384 + 512 : kSlotBytes;
   static constexpr int kBytes = kStage + 2 * kStageBytes;
 };
 
@@ -1417,7 +1330,7 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
     mbar_arrive_expect_tx(&s_ld[s], L::kStageBytes);
     if (TRANS) {
       bulk_g2s(dst, src, 32768, &s_ld[s]);                           // W | K'
-      bulk_g2s(dst + L::kUt, src + kSlotU, 32768 + 512, &s_ld[s]);   // U~ | gamma
+      bulk_g2s(dst + L::kUt, src + kSlotU, 16384 + 512, &s_ld[s]);   // U~ | gamma
     } else {
       bulk_g2s(dst, src, kSlotBytes, &s_ld[s]);
     }
@@ -1524,19 +1437,17 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       tmem_ld_wait();
       if (m64) {
         if (blk == 0) {
-          const float4* ug = reinterpret_cast<const float4*>(st + L::kUt);
+          const uint4* ug = reinterpret_cast<const uint4*>(st + L::kUt);
 #pragma unroll
-          for (int pc = 0; pc < 4; ++pc) {
-            const float4 u0 = ug[ut_index(q4, cq, pc, lane) >> 2];
-            const float4 u1 = ug[ut_index(q4, cq, pc + 4, lane) >> 2];
-            d0[4 * pc] = u0.x - d0[4 * pc];
-            d0[4 * pc + 1] = u0.y - d0[4 * pc + 1];
-            d0[4 * pc + 2] = u0.z - d0[4 * pc + 2];
-            d0[4 * pc + 3] = u0.w - d0[4 * pc + 3];
-            d1[4 * pc] = u1.x - d1[4 * pc];
-            d1[4 * pc + 1] = u1.y - d1[4 * pc + 1];
-            d1[4 * pc + 2] = u1.z - d1[4 * pc + 2];
-            d1[4 * pc + 3] = u1.w - d1[4 * pc + 3];
+          for (int pc = 0; pc < 2; ++pc) {
+            float u0[8], u1[8];
+            unpack8(ug[ut_index(q4, cq, pc, lane)], u0);
+            unpack8(ug[ut_index(q4, cq, pc + 2, lane)], u1);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              d0[8 * pc + e] = u0[e] - d0[8 * pc + e];
+              d1[8 * pc + e] = u1[e] - d1[8 * pc + e];
+            }
           }
         } else {
 #pragma unroll
@@ -1820,10 +1731,10 @@ cudaError_t launch_forward_tc(const ForwardArgs& a) {
     chain_kernel<false><<<dim3(a.N, a.H, p.P), kNT, ChainSmem<false>::kBytes, a.stream>>>(p);
     return cudaGetLastError();
   }
-  err = cudaFuncSetAttribute(tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Smem<0>::kBytes);
+  err = cudaFuncSetAttribute(fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             FusedSmem::kBytes);
   if (err != cudaSuccess) return err;
-  tc_kernel<0><<<dim3(a.N, a.H, p.P), kNT, Smem<0>::kBytes, a.stream>>>(p);
+  fused_kernel<<<dim3(a.N, a.H, p.P), kNT, FusedSmem::kBytes, a.stream>>>(p);
   return cudaGetLastError();
 }
 
