@@ -81,6 +81,7 @@ constexpr uint32_t kTmWU = 0;    // [W | U~]: 256 columns (after the products ar
 constexpr uint32_t kTmW = 0;     // D_W = W S (128, or 256 for W [S | X])
 constexpr uint32_t kTmQ = 128;   // D_Q = Q' S (+ A_qk U)
 constexpr uint32_t kTmS = 256;   // fp32 state; identity-started block X at 384 (transition)
+constexpr uint32_t kTmQ2 = 384;  // second D_Q of the chain pass (alternate chunks)
 
 constexpr int kLd = 68;  // row stride (floats) of the fp32 A_kk / T tiles
 
@@ -896,10 +897,17 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
     return *reinterpret_cast<const uint4*>(raw + ti * 16384 + (cg >> 3) * 8192 + t * 128 +
                                            (((cg & 7) ^ (t & 7)) << 4));
   };
+  // beta of an item (thread t < 64: token t), loaded one item ahead
+  auto load_beta = [&](int tok, int end, int hh) -> float {
+    return (gtid < kC && tok + gtid < end) ? __bfloat162float(p.beta[(size_t)(tok + gtid) * H + hh])
+                                           : 0.f;
+  };
   bool have = next_item();
+  float beta_nx = 0.f;
   if (have) {
     if (gtid == 0) stage(a + c * kC, h);
     raw_pending = true;
+    beta_nx = load_beta(a + c * kC, b, h);
   }
   while (ok && have) {
     const int hc = h, nc = n, cc0 = c, ac = a, bc = b;
@@ -911,14 +919,14 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
     have = next_item();  // the item after this one (its rows are loaded during this one)
     const int tok0 = ac + cc0 * kC;
     const int len = min(kC, bc - tok0);
+    if (gtid < kC) vec[kVecBeta + gtid] = beta_nx;
+    if (have) beta_nx = load_beta(a + c * kC, b, h);
     unsigned char* slot = chunk_slot(p.prep, ac, nc, cc0, hc, H);
     const bool in0 = t0 < len, in1 = t0 + 1 < len;
     const size_t row0 = ((size_t)(tok0 + t0) * H + hc) * kD + c0;  // element offset of (t0, c0)
     const size_t rstep = (size_t)H * kD;                          // next token
     const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
 
-    if (gtid < kC)
-      vec[kVecBeta + gtid] = gtid < len ? __bfloat162float(p.beta[(size_t)(tok0 + gtid) * H + hc]) : 0.f;
     if (!group_wait(bar_raw, ph_raw, p.hdr, bid, gtid)) {
       ph_raw ^= 1;  // the load is still pending in this phase
       ok = false;
@@ -1091,9 +1099,9 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
       const uint64_t ad = smem_desc(smem_u32(sm + L::kCc), 128, 2048);
       const uint64_t bd = smem_desc(smem_u32(sm + L::kR), 128, 2048);
 #pragma unroll
-      for (int bb = 0; bb < 4; ++bb)
+      for (int k = 0; k < 8; ++k)  // descriptor addresses count 16-byte units
 #pragma unroll
-        for (int k = 0; k < 8; ++k)  // descriptor addresses count 16-byte units
+        for (int bb = 0; bb < 4; ++bb)  // four independent accumulators back to back
           mma_bf16(tm + kTmA + 32 * bb, ad + bb * (bb + 1) * 128 + 16 * k, bd + 512 * bb + 16 * k,
                    id, k > 0);
       mma_commit(bar_mma);
@@ -1156,15 +1164,15 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
     float* Tf = reinterpret_cast<float*>(sm + L::kTf);
     float* Y = reinterpret_cast<float*>(sm + L::kY);
     if (gtid < kC) {
+      // column cc of block bk: x = e_cc, then x_r -= A[r][m] x_m for m < r (right-looking)
       const int bk = gtid >> 4, cc = gtid & 15, base = 16 * bk;
       float x[16];
 #pragma unroll
-      for (int rr = 0; rr < 16; ++rr) {
-        float acc = (rr == cc) ? 1.f : 0.f;
+      for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == cc) ? 1.f : 0.f;
 #pragma unroll
-        for (int i = 0; i < rr; ++i) acc -= Akk[(base + rr) * kLd + base + i] * x[i];
-        x[rr] = (rr < cc) ? 0.f : acc;
-      }
+      for (int m = 0; m < 15; ++m)
+#pragma unroll
+        for (int rr = m + 1; rr < 16; ++rr) x[rr] -= Akk[(base + rr) * kLd + base + m] * x[m];
 #pragma unroll
       for (int rr = 0; rr < 16; ++rr) Tf[(base + rr) * kLd + base + cc] = x[rr];
     } else {
@@ -1176,6 +1184,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
     }
     group_sync(bid);
     if (gtid < 128) {
+      // 16 -> 32, pair pr: Y = A[hi][lo] T[lo][lo]; T[hi][lo] = -T[hi][hi] Y (2x2 tiles;
+      // the merges are bound by shared-memory loads, which larger tiles reuse)
       const int pr = gtid >> 6, r2 = ((gtid >> 3) & 7) * 2, c2 = (gtid & 7) * 2;
       const int lo = 32 * pr, hi = lo + 16;
       float y[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1194,6 +1204,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
     }
     group_sync(bid);
     if (gtid < 256) {
+      // 32 -> 64: Y = A[32:64][0:32] T[0:32][0:32]; T[32:64][0:32] = -T[32:64][32:64] Y
       const int r2 = (gtid >> 4) * 2, c2 = (gtid & 15) * 2;
       float y[4] = {0.f, 0.f, 0.f, 0.f};
       mm2x2<32>(Akk + (32 + r2) * kLd, Akk + (33 + r2) * kLd, Tf + c2, kLd, y);
@@ -1378,10 +1389,29 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
     tmem_st_wait();
   }
 
+  // o of a chunk = its D_Q (two alternating TMEM buffers) / |q|, written while
+  // the next chunk's C1 runs
+  float iq_prev = 0.f;  // 1/|q| of the previous chunk's row r64
+  auto write_o = [&](int cc, uint32_t dq, float iq) {
+    const int t0c = a + cc * kC, lenc = min(kC, b - t0c);
+    const int col = 32 * cq;
+    float o0[16], o1[16];
+    tmem_ld16(tmem_addr(tm, 32 * q4, dq + col), o0);
+    tmem_ld16(tmem_addr(tm, 32 * q4, dq + col + 16), o1);
+    tmem_ld_wait();
+    if (m64 && r64 < lenc) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) { o0[i] *= iq; o1[i] *= iq; }
+      uint4* dst = reinterpret_cast<uint4*>(p.o + ((size_t)(t0c + r64) * H + h) * kD + col);
+      dst[0] = pack8(o0);
+      dst[1] = pack8(o0 + 8);
+      dst[2] = pack8(o1);
+      dst[3] = pack8(o1 + 8);
+    }
+  };
   for (int c = c0; c < c1; ++c) {
-    const int tok0 = a + c * kC;
-    const int len = min(kC, b - tok0);
     const int s = (c - c0) & 1;
+    const uint32_t tmq = s ? kTmQ2 : kTmQ;  // this chunk's D_Q
     unsigned char* st = sm + L::kStage + s * L::kStageBytes;
     sync_for_mma();
     {
@@ -1399,13 +1429,12 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       const uint64_t sd = smem_desc(smem_u32(sm + L::kSb), SbL, 128);
       const uint64_t wd = smem_desc(smem_u32(st + L::kW), 128, 2048);
       constexpr uint32_t idw = instr_desc(kFmtBF16, 64, SbN, false, true);
+      const uint64_t qd = smem_desc(smem_u32(st + L::kQ), 128, 2048);  // Q' K-major
+      constexpr uint32_t idq = instr_desc(kFmtBF16, 64, 128, false, true);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mma_bf16(tm + kTmW, wd + 16 * k, sd + (2 * SbL >> 4) * k, idw, k > 0);
-      if (!TRANS) {
-        const uint64_t qd = smem_desc(smem_u32(st + L::kQ), 128, 2048);  // Q' K-major
-        constexpr uint32_t idq = instr_desc(kFmtBF16, 64, 128, false, true);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mma_bf16(tm + kTmQ, qd + 16 * k, sd + (2 * SbL >> 4) * k, idq, k > 0);
+      for (int k = 0; k < 8; ++k) {  // the two accumulators interleaved
+        mma_bf16(tm + kTmW, wd + 16 * k, sd + (2 * SbL >> 4) * k, idw, k > 0);
+        if (!TRANS) mma_bf16(tm + tmq, qd + 16 * k, sd + (2 * SbL >> 4) * k, idq, k > 0);
       }
       mma_commit(&s_bar);
     }
@@ -1426,6 +1455,7 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       }
       tmem_st_wait();
     }
+    if (!TRANS && c > c0) write_o(c - 1, s ? kTmQ : kTmQ2, iq_prev);
     if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
     // ---- U = U~ - D_W (transition: [U~ | 0] - W [S | X]) -> B operand (MN-major)
 #pragma unroll
@@ -1465,23 +1495,24 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       const uint64_t kd = smem_desc(smem_u32(st + L::kK), 2048, 128);  // K' MN-major
       const uint64_t ud = smem_desc(smem_u32(sm + L::kU), SbL, 128);
       constexpr uint32_t ids = instr_desc(kFmtBF16, 128, SbN, true, true);
+      const uint64_t a3 = smem_desc(smem_u32(st + L::kA3), 1024, 128);
+      constexpr uint32_t ido = instr_desc(kFmtBF16, 64, 128, true, true);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) mma_bf16(tm + kTmS, kd + 256 * k, ud + (2 * SbL >> 4) * k, ids, 1);
-      if (!TRANS) {
-        const uint64_t a3 = smem_desc(smem_u32(st + L::kA3), 1024, 128);
-        constexpr uint32_t ido = instr_desc(kFmtBF16, 64, 128, true, true);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) mma_bf16(tm + kTmQ, a3 + 128 * k, ud + (2 * SbL >> 4) * k, ido, 1);
+      for (int k = 0; k < 4; ++k) {
+        mma_bf16(tm + kTmS, kd + 256 * k, ud + (2 * SbL >> 4) * k, ids, 1);
+        if (!TRANS) mma_bf16(tm + tmq, a3 + 128 * k, ud + (2 * SbL >> 4) * k, ido, 1);
       }
       mma_commit(&s_bar);
     }
+    // (read before the barrier below, which orders it before the stage's refill)
+    if (!TRANS && m64) iq_prev = reinterpret_cast<const float*>(st + L::kIq)[r64];
     if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
     // the stage is consumed (its reads ended before the barrier above): refill it
     if (c + 2 < c1) {
       inflight |= 1u << s;
       if (tid == 0) load_slot(c + 2);
     }
-    // ---- [S | X] -> bf16 operand of the next chunk; o = D_Q / |q| -> global
+    // ---- [S | X] -> bf16 operand of the next chunk
 #pragma unroll
     for (int blk = 0; blk < NB; ++blk) {
       float s0[16], s1[16];
@@ -1494,23 +1525,11 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       st16(sm + L::kSb, mnmaj(col + 16, srow, SbL), s1);
       st16(sm + L::kSb, mnmaj(col + 24, srow, SbL), s1 + 8);
     }
-    if (!TRANS) {
-      const int col = 32 * cq;
-      float o0[16], o1[16];
-      tmem_ld16(tmem_addr(tm, 32 * q4, kTmQ + col), o0);
-      tmem_ld16(tmem_addr(tm, 32 * q4, kTmQ + col + 16), o1);
-      tmem_ld_wait();
-      if (m64 && r64 < len) {
-        const float iq = reinterpret_cast<const float*>(st + L::kIq)[r64];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) { o0[i] *= iq; o1[i] *= iq; }
-        uint4* dst = reinterpret_cast<uint4*>(p.o + ((size_t)(tok0 + r64) * H + h) * kD + col);
-        dst[0] = pack8(o0);
-        dst[1] = pack8(o0 + 8);
-        dst[2] = pack8(o1);
-        dst[3] = pack8(o1 + 8);
-      }
-    }
+  }
+  // o of the last chunk
+  if (!TRANS && !s_abort && c1 > c0) {
+    fence_after_sync();
+    write_o(c1 - 1, ((c1 - 1 - c0) & 1) ? kTmQ2 : kTmQ, iq_prev);
   }
 
   fence_before_sync();
