@@ -205,6 +205,8 @@ def main():
     ap.add_argument("--L", type=int, default=L_DEFAULT, help="prefill length (sweep)")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="run one part (profiling captures); the other part is reported as null")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -237,119 +239,128 @@ def main():
     T = B * L
     log(f"[rank {rank}] generating inputs L={L}")
     inp = synth.workload("long", L=L)
-    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
-    o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
-    Sf = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
-    ws = kda.workspace(B, T, L, H, D, D, torch.bfloat16, CHUNK, device=dev)
     stream = torch.cuda.current_stream(dev)
-    launches = kda.kda_forward_launches(B, T, L, H, D, D, kda.KDA_BF16, CHUNK)
-
-    def fwd():
-        kda.forward(d["q"], d["k"], d["v"], d["z"], d["A"], d["beta"], num_seqs=B, chunk=CHUNK,
-                    o=o, S_final=Sf, workspace=ws, stream=stream)
-
-    for _ in range(args.warmup):
-        fwd()
-    torch.cuda.synchronize()
-    assert kda.check_device_error(ws) == kda.KDA_OK
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    pk = peaks()
+    out = {"ms": None, "value": None, "roofline": None, "e2e": None, "clocks": None,
+           "launches": 0, "decode": None}
 
     # ---------------------------------------------------------- prefill ---
-    with ClockSampler(local) as clk:
-        barrier()
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
+    if args.only != "decode":
+        d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+        o = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+        Sf = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+        ws = kda.workspace(B, T, L, H, D, D, torch.bfloat16, CHUNK, device=dev)
+        launches = kda.kda_forward_launches(B, T, L, H, D, D, kda.KDA_BF16, CHUNK)
+
+        def fwd():
+            kda.forward(d["q"], d["k"], d["v"], d["z"], d["A"], d["beta"], num_seqs=B,
+                        chunk=CHUNK, o=o, S_final=Sf, workspace=ws, stream=stream)
+
+        for _ in range(args.warmup):
             fwd()
+        torch.cuda.synchronize()
+        assert kda.check_device_error(ws) == kda.KDA_OK
+
+        with ClockSampler(local) as clk:
+            barrier()
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for _ in range(args.steps):
+                fwd()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            ms_local = e0.elapsed_time(e1) / args.steps
+        ms = rank_max(ms_local)
+        out["clocks"] = clk.summary()
+        out["ms"] = ms
+        out["value"] = weak_scaling_value(T, world, ms)
+        out["launches"] = launches * args.steps
+
+        fwd_bytes = alg_bytes_prefill(T)
+        fwd_flops = alg_flops(T)
+        achieved = fwd_bytes / (ms_local / 1e3) / 1e9
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                    "frac": achieved / pk["hbm"], "traffic": recorded_traffic("forward"),
+                    "kernel": "kda_forward (one call: all %d launches)" % launches,
+                    "peak_source": pk["src"],
+                    "tensor_flops_frac": fwd_flops / (ms_local / 1e3) / 1e12 / pk["bf16"],
+                    "roofline_time_us": max(fwd_bytes / pk["hbm"] / 1e3,
+                                            fwd_flops / pk["bf16"] / 1e6)}
+        roofline["frac_of_roofline_time"] = roofline["roofline_time_us"] / (ms_local * 1e3)
+        out["roofline"] = roofline
+
+        # ---------------------------------------------------------- e2e ---
+        # Same metric through the public API with pinned host buffers; the H2D
+        # copy of the step's inputs and the D2H read of o and S_final are inside.
+        host = {k: inp[k].pin_memory() for k in ("q", "k", "v", "z", "beta", "A")}
+        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        S_h = torch.empty(Sf.shape, dtype=Sf.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = o_h.numel() * o_h.element_size() + S_h.numel() * S_h.element_size()
+
+        def e2e_step():
+            for k_, t in host.items():
+                d[k_].copy_(t, non_blocking=True)
+            fwd()
+            o_h.copy_(o, non_blocking=True)
+            S_h.copy_(Sf, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        n_e2e = max(3, min(args.steps, 10))
+        for _ in range(n_e2e):
+            e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        barrier()
-        ms_local = e0.elapsed_time(e1) / args.steps
-    ms = rank_max(ms_local)
-    clocks = clk.summary()
-    value = weak_scaling_value(T, world, ms)
-
-    pk = peaks()
-    fwd_bytes = alg_bytes_prefill(T)
-    fwd_flops = alg_flops(T)
-    achieved = fwd_bytes / (ms_local / 1e3) / 1e9
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
-                "frac": achieved / pk["hbm"], "traffic": recorded_traffic("forward"),
-                "kernel": "kda_forward (all launches of one call)",
-                "peak_source": pk["src"],
-                "tensor_flops_frac": fwd_flops / (ms_local / 1e3) / 1e12 / pk["bf16"],
-                "roofline_time_us": max(fwd_bytes / pk["hbm"] / 1e3,
-                                        fwd_flops / pk["bf16"] / 1e6)}
-    roofline["frac_of_roofline_time"] = roofline["roofline_time_us"] / (ms_local * 1e3)
-
-    # -------------------------------------------------------------- e2e ---
-    # Same metric through the public API with pinned host buffers; the H2D copy
-    # of the step's inputs and the D2H read of o and S_final are inside.
-    host = {k: inp[k].pin_memory() for k in ("q", "k", "v", "z", "beta", "A")}
-    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    S_h = torch.empty(Sf.shape, dtype=Sf.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = o_h.numel() * o_h.element_size() + S_h.numel() * S_h.element_size()
-
-    def e2e_step():
-        for k_, t in host.items():
-            d[k_].copy_(t, non_blocking=True)
-        fwd()
-        o_h.copy_(o, non_blocking=True)
-        S_h.copy_(Sf, non_blocking=True)
-
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier()
-    e0.record(stream)
-    n_e2e = max(3, min(args.steps, 10))
-    for _ in range(n_e2e):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms_e2e = rank_max(e0.elapsed_time(e1) / n_e2e)
-    e2e = {"value": weak_scaling_value(T, world, ms_e2e), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h}
+        ms_e2e = rank_max(e0.elapsed_time(e1) / n_e2e)
+        out["e2e"] = {"value": weak_scaling_value(T, world, ms_e2e), "unit": "tokens/s",
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        del ws
+        torch.cuda.empty_cache()
 
     # ----------------------------------------------------------- decode ---
-    del ws
-    torch.cuda.empty_cache()
-    A_dec, S_dec0 = synth.decode_state(DEC_B, H, D, D)
-    S_dec = S_dec0.to(dev)
-    A_dec = A_dec.to(dev)
-    pool = [{k: t.to(dev) for k, t in synth.decode_token(s, DEC_B, H, D, D).items()}
-            for s in range(8)]
-    o_dec = torch.empty((DEC_B, H, D), dtype=torch.bfloat16, device=dev)
+    if args.only != "prefill":
+        A_dec, S_dec0 = synth.decode_state(DEC_B, H, D, D)
+        S_dec = S_dec0.to(dev)
+        A_dec = A_dec.to(dev)
+        pool = [{k: t.to(dev) for k, t in synth.decode_token(s, DEC_B, H, D, D).items()}
+                for s in range(8)]
+        o_dec = torch.empty((DEC_B, H, D), dtype=torch.bfloat16, device=dev)
 
-    def dec(s):
-        tk = pool[s % len(pool)]
-        kda.decode_step(tk["q"], tk["k"], tk["v"], tk["z"], A_dec, tk["beta"], S_dec, o=o_dec,
-                        stream=stream)
+        def dec(s):
+            tk = pool[s % len(pool)]
+            kda.decode_step(tk["q"], tk["k"], tk["v"], tk["z"], A_dec, tk["beta"], S_dec,
+                            o=o_dec, stream=stream)
 
-    for s in range(10):
-        dec(s)
-    torch.cuda.synchronize()
-    barrier()
-    e0.record(stream)
-    for s in range(args.decode_steps):
-        dec(s)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms_dec_local = e0.elapsed_time(e1) / args.decode_steps
-    ms_dec = rank_max(ms_dec_local)
-    dec_bytes = alg_bytes_decode()
-    dec_ach = dec_bytes / (ms_dec_local / 1e3) / 1e9
-    decode = {"value": world * 1e3 / ms_dec, "unit": "steps/s", "ms_per_step": ms_dec,
-              "tokens_per_s": world * DEC_B * 1e3 / ms_dec, "steps": args.decode_steps,
-              "config": {"B": DEC_B, "H": H, "dk": D, "dv": D, "dtype": "bf16",
-                         "state": "fp32 in place (268 MB, exceeds L2)"},
-              "gpu_launches": args.decode_steps,
-              "roofline": {"bound": "hbm", "achieved": dec_ach, "peak": pk["hbm"],
-                           "unit": "GB/s", "frac": dec_ach / pk["hbm"],
-                           "traffic": recorded_traffic("decode"),
-                           "kernel": "decode_step_kernel", "peak_source": pk["src"]}}
+        for s in range(10):
+            dec(s)
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        for s in range(args.decode_steps):
+            dec(s)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms_dec_local = e0.elapsed_time(e1) / args.decode_steps
+        ms_dec = rank_max(ms_dec_local)
+        dec_bytes = alg_bytes_decode()
+        dec_ach = dec_bytes / (ms_dec_local / 1e3) / 1e9
+        out["decode"] = {
+            "value": world * 1e3 / ms_dec, "unit": "steps/s", "ms_per_step": ms_dec,
+            "tokens_per_s": world * DEC_B * 1e3 / ms_dec, "steps": args.decode_steps,
+            "config": {"B": DEC_B, "H": H, "dk": D, "dv": D, "dtype": "bf16",
+                       "state": "fp32 in place (268 MB, exceeds L2)"},
+            "gpu_launches": args.decode_steps,
+            "roofline": {"bound": "hbm", "achieved": dec_ach, "peak": pk["hbm"],
+                         "unit": "GB/s", "frac": dec_ach / pk["hbm"],
+                         "traffic": recorded_traffic("decode"),
+                         "kernel": "decode_step_kernel", "peak_source": pk["src"]}}
 
     # ------------------------------------------------------ CPU baseline ---
     cpu = None
@@ -365,8 +376,8 @@ def main():
     if rank != 0:
         return
     print(json.dumps({
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "metric": METRIC, "value": out["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": out["ms"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
         "config": {"workload": f"KDA fwd long: B={B} H={H} L={L} dk=dv={D}, bf16 inputs, "
@@ -375,8 +386,8 @@ def main():
                    "l2": "inputs exceed L2 (q,k,v,z,o = %.0f MB per step)" % (
                        T * H * D * 2 * 5 / 1e6),
                    "parallelism": f"weak x{world} (independent problems per rank)"},
-        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": launches * args.steps, "clocks": clocks, "decode": decode,
+        "roofline": out["roofline"], "cpu_baseline": cpu, "e2e": out["e2e"],
+        "gpu_launches": out["launches"], "clocks": out["clocks"], "decode": out["decode"],
     }), flush=True)
 
 
