@@ -1567,64 +1567,98 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
 }
 
 // Incoming state of every segment: S_in(0) = S0, S_in(p+1) = M_p S_in(p) + N_p.
-// One CTA per (n, h, 16-column block of the state); fp32 on CUDA cores, with
-// M staged 32 columns at a time by coalesced row loads, one tile ahead.
-__global__ void __launch_bounds__(256) compose_kernel(const __grid_constant__ TcParams p) {
+// One CTA per (n, h, 16-column block of the state); fp32 on CUDA cores.  Each
+// M_p (64 KB) is bulk-copied into shared memory one step ahead; the state
+// columns are kept transposed so both operands are read as float4.
+constexpr int kComposeThreads = 256;
+constexpr int kSct = kD + 4;  // row stride (floats) of the transposed state columns
+struct ComposeSmem {
+  static constexpr int kM = 0;                        // two M_p buffers, [128][128] fp32
+  static constexpr int kS = 2 * kD * kD * 4;          // state columns, [16][kSct] fp32
+  static constexpr int kBar = kS + 16 * kSct * 4;     // two mbarriers
+  static constexpr int kBytes = kBar + 16;
+};
+
+__global__ void __launch_bounds__(kComposeThreads) compose_kernel(const __grid_constant__ TcParams p) {
+  using L = ComposeSmem;
+  extern __shared__ __align__(1024) unsigned char sm[];
   const int n = blockIdx.x, h = blockIdx.y, cb = blockIdx.z * 16;
-  const int H = p.H;
+  const int H = p.H, tid = threadIdx.x;
   if (!seqlens_valid(p.cu, p.N, p.T, p.max_len)) return;
-  __shared__ float Sc[kD][16];
-  __shared__ float Ms[2][kD][33];
-  const int tid = threadIdx.x;
-  for (int e = tid; e < kD * 16; e += 256) {
-    const int r = e >> 4, cc = e & 15;
-    Sc[r][cc] = p.S0 ? p.S0[((size_t)n * H + h) * kD * kD + (size_t)r * kD + cb + cc] : 0.f;
+  float* Sct = reinterpret_cast<float*>(sm + L::kS);  // Sct[cc][r] = S[r][cb + cc]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kBar);
+  const int steps = p.P - 1;
+  auto load_m = [&](int sg) {  // single thread
+    mbar_arrive_expect_tx(&bar[sg & 1], kD * kD * 4);
+    bulk_g2s(sm + L::kM + (sg & 1) * kD * kD * 4, seg_trans(p.seg, n, h, H, p.P, sg), kD * kD * 4,
+             &bar[sg & 1]);
+  };
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    fence_mbar_init();
   }
-  const int c = tid & 15, r0 = tid >> 4;  // rows r0 + 16 m
-  for (int sg = 0; sg + 1 < p.P; ++sg) {
-    const float* Mt = seg_trans(p.seg, n, h, H, p.P, sg);
-    const float* Nt = Mt + kD * kD;
+  __syncthreads();
+  if (tid == 0 && steps > 0) load_m(0);
+  for (int e = tid; e < kD * 16; e += kComposeThreads) {
+    const int r = e >> 4, cc = e & 15;
+    Sct[cc * kSct + r] = p.S0 ? p.S0[((size_t)n * H + h) * kD * kD + (size_t)r * kD + cb + cc] : 0.f;
+  }
+  const int c = tid & 15, r0 = tid >> 4;  // column c, rows r0 + 16 m
+  uint32_t inflight = steps > 0 ? 1u : 0u;  // buffers being filled
+  uint32_t ph = 0;                            // bit b: parity of buffer b's next completion
+  bool ok = true;
+  // N_p columns, loaded one step ahead
+  auto load_n = [&](int sg, float (&v)[8]) {
+    const float* Nt = seg_trans(p.seg, n, h, H, p.P, sg) + kD * kD;
+#pragma unroll
+    for (int m = 0; m < 8; ++m) v[m] = Nt[(size_t)(r0 + 16 * m) * kD + cb + c];
+  };
+  float nxt[8];
+  if (steps > 0) load_n(0, nxt);
+  for (int sg = 0; sg < steps; ++sg) {
+    const int buf = sg & 1;
+    // M_{sg+1} into the other buffer (its readers finished before the last barrier)
+    if (sg + 1 < steps) {
+      if (tid == 0) load_m(sg + 1);
+      inflight |= 1u << (buf ^ 1);
+    }
     float acc[8];
 #pragma unroll
-    for (int m = 0; m < 8; ++m) acc[m] = Nt[(size_t)(r0 + 16 * m) * kD + cb + c];
-    float pre[16];
-#pragma unroll
-    for (int u = 0; u < 16; ++u) {
-      const int e = tid + 256 * u;
-      pre[u] = Mt[(size_t)(e >> 5) * kD + (e & 31)];
+    for (int m = 0; m < 8; ++m) acc[m] = nxt[m];
+    if (sg + 1 < steps) load_n(sg + 1, nxt);
+    const bool got = mbar_wait_cycles(&bar[buf], (ph >> buf) & 1, kWaitCycles);
+    if (__syncthreads_or(!got)) {
+      if (tid == 0) atomicOr(&p.hdr->err, kErrTimeout);
+      ok = false;
+      break;
     }
-    for (int k0 = 0; k0 < kD; k0 += 32) {
-      const int buf = (k0 >> 5) & 1;
-      __syncthreads();
+    ph ^= 1u << buf;
+    inflight &= ~(1u << buf);
+    const float* Ms = reinterpret_cast<const float*>(sm + L::kM + buf * kD * kD * 4);
+#pragma unroll 4
+    for (int k = 0; k < kD; k += 4) {
+      const float4 sv = *reinterpret_cast<const float4*>(Sct + c * kSct + k);
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int e = tid + 256 * u;
-        Ms[buf][e >> 5][e & 31] = pre[u];
-      }
-      if (k0 + 32 < kD) {
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int e = tid + 256 * u;
-          pre[u] = Mt[(size_t)(e >> 5) * kD + k0 + 32 + (e & 31)];
-        }
-      }
-      __syncthreads();
-#pragma unroll 8
-      for (int kk = 0; kk < 32; ++kk) {
-        const float sv = Sc[k0 + kk][c];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) acc[m] += Ms[buf][r0 + 16 * m][kk] * sv;
+      for (int m = 0; m < 8; ++m) {
+        const float4 mv = *reinterpret_cast<const float4*>(Ms + (r0 + 16 * m) * kD + k);
+        acc[m] += mv.x * sv.x + mv.y * sv.y + mv.z * sv.z + mv.w * sv.w;
       }
     }
     __syncthreads();
 #pragma unroll
-    for (int m = 0; m < 8; ++m) Sc[r0 + 16 * m][c] = acc[m];
+    for (int m = 0; m < 8; ++m) Sct[c * kSct + r0 + 16 * m] = acc[m];
     __syncthreads();
     float* Sin = seg_sin(p.seg, n, h, H, p.P, sg + 1);
-    for (int e = tid; e < kD * 16; e += 256) {
+    for (int e = tid; e < kD * 16; e += kComposeThreads) {
       const int r = e >> 4, cc = e & 15;
-      Sin[(size_t)r * kD + cb + cc] = Sc[r][cc];
+      Sin[(size_t)r * kD + cb + cc] = Sct[cc * kSct + r];
     }
+  }
+  if (!ok && tid == 0) {
+    // a wait gave up: let the copies still in flight land before leaving
+    for (int b2 = 0; b2 < 2; ++b2)
+      if (inflight & (1u << b2)) (void)mbar_wait_cycles(&bar[b2], (ph >> b2) & 1, kWaitCycles);
   }
 }
 
@@ -1742,7 +1776,10 @@ cudaError_t launch_forward_tc(const ForwardArgs& a) {
     if (err != cudaSuccess) return err;
     chain_kernel<true><<<dim3(a.N, a.H, p.P - 1), kNT, ChainSmem<true>::kBytes, a.stream>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    compose_kernel<<<dim3(a.N, a.H, kD / 16), 256, 0, a.stream>>>(p);
+    err = cudaFuncSetAttribute(compose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               ComposeSmem::kBytes);
+    if (err != cudaSuccess) return err;
+    compose_kernel<<<dim3(a.N, a.H, kD / 16), kComposeThreads, ComposeSmem::kBytes, a.stream>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     err = cudaFuncSetAttribute(chain_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                ChainSmem<false>::kBytes);
