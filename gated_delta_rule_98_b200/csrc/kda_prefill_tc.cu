@@ -735,20 +735,21 @@ constexpr int kPrepThreads = kNT * kPrepGroups;
 struct PrepSmem {  // one group's part
   static constexpr int kP = 0;               // region P, reused through the chunk:
   static constexpr int kR = kP;              //   R   B op (N=128 rows, K=128) K-major
-  static constexpr int kCc = kP + 32768;     //   C   A op (M=160 rows, K=128) K-major
+  static constexpr int kCc = kP + 32768;     //   C   A op, window b at rows 64 b (K=128) K-major
   static constexpr int kAkk = kP;            //   A_kk fp32 [64][68]  (after M1)
   static constexpr int kTf = kP + 17408;     //   T    fp32 [64][68]
   static constexpr int kY = kP + 34816;      //   merge scratch fp32 [32][34]
-  static constexpr int kX = kP + 40960;      //   X   B op (N=256, K=64 tokens) MN-major
   static constexpr int kW = kP;              //   W   slot image   (after M2)
   static constexpr int kUt = kP + 16384;     //   U~  slot image
-  static constexpr int kTop = kP + 73728;    // sub-tile sums and first gates, then T (A op, K-major)
+  static constexpr int kTop = kP + 98304;    // sub-tile sums and first gates, then T (A op, K-major)
   static constexpr int kFac = kTop + 8192;   // decay factors [4 sub-tiles][5][128] fp32
   static constexpr int kNrm = kFac + 10240;  // squared-norm partials [16 channel groups][64][2]
   static constexpr int kVec = kNrm + 8192;   // 1/|q|, 1/|k|, beta (64 floats each)
-  static constexpr int kRaw = 101376;        // q | k | z | v, [64 tokens][2 x 64 channels] bf16,
+  static constexpr int kRaw = 125952;        // q | k | z | v, [64 tokens][2 x 64 channels] bf16,
                                              //   128-byte swizzled (TMA), 16 KB each
-  static constexpr int kGroup = kRaw + 65536;  // bytes per group
+  static constexpr int kX = kRaw + 65536;    // X B op (N=256, K=64 tokens) MN-major: written
+                                             //   while M1 runs
+  static constexpr int kGroup = kX + 32768;  // bytes per group
   static constexpr int kBar = kPrepGroups * kGroup;  // per group: two mbarriers; then the TMEM base
   static constexpr int kBytes = kBar + 48;
 };
@@ -1078,13 +1079,13 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
         unpack8(s ? kb : ka, kf);
 #pragma unroll
         for (int i = 0; i < 8; ++i) kf[i] = __fdividef(kf[i], (sw ? E[8 * (s2 ^ 1) + i] : E[8 * s2 + i]));
-        st16(sm + L::kCc, kmaj(8 * qq * (qq + 1) + t, c0, 2048), kf);
+        st16(sm + L::kCc, kmaj(64 * qq + t, c0, 2048), kf);
         for (int bb = qq + 1; bb < 4; ++bb) {  // warp-uniform
           float f[8];
           ld8f(fq + (kFacWin + bb - qq - 1) * 128, f);
 #pragma unroll
           for (int i = 0; i < 8; ++i) w8[i] = kf[i] * f[i];
-          st16(sm + L::kCc, kmaj(8 * bb * (bb + 1) + t, c0, 2048), w8);
+          st16(sm + L::kCc, kmaj(64 * bb + t, c0, 2048), w8);
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) kf[i] *= ik * el[i];
@@ -1092,22 +1093,23 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
       }
     }
     group_sync_for_mma(bid);
-    // ---- M1: four M=64 MMAs (K-major operands) -> TMEM [32b, +32): cols 0-15 A_kk^T,
-    //      16-31 A_qk^T; C window b starts at row 8 b (b + 1), R sub-tile b at row 32 b
+    // ---- M1: per K step two M=128, N=64 MMAs (K-major operands): windows (0, 1)
+    //      against R sub-tiles (0, 1) -> TMEM columns 0-63, windows (2, 3) against
+    //      sub-tiles (2, 3) -> 64-127.  Lanes 0-63 hold window 2 P's rows, 64-127
+    //      window 2 P + 1's; of each sub-tile's 32 columns 0-15 are A_kk^T, 16-31
+    //      A_qk^T.  Window b is needed against sub-tile b only.
     if (gtid == 0) {
-      constexpr uint32_t id = instr_desc(kFmtBF16, 64, 32, false, false);
+      constexpr uint32_t id = instr_desc(kFmtBF16, 128, 64, false, false);
       const uint64_t ad = smem_desc(smem_u32(sm + L::kCc), 128, 2048);
       const uint64_t bd = smem_desc(smem_u32(sm + L::kR), 128, 2048);
 #pragma unroll
       for (int k = 0; k < 8; ++k)  // descriptor addresses count 16-byte units
 #pragma unroll
-        for (int bb = 0; bb < 4; ++bb)  // four independent accumulators back to back
-          mma_bf16(tm + kTmA + 32 * bb, ad + bb * (bb + 1) * 128 + 16 * k, bd + 512 * bb + 16 * k,
-                   id, k > 0);
+        for (int pr = 0; pr < 2; ++pr)  // two independent accumulators back to back
+          mma_bf16(tm + kTmA + 64 * pr, ad + 2048 * pr + 16 * k, bd + 1024 * pr + 16 * k, id, k > 0);
       mma_commit(bar_mma);
     }
-    if (!group_wait(bar_mma, ph_mma, p.hdr, bid, gtid)) { ok = false; break; }
-    // ---- X_K = beta k / |k| e^{Gam_r}, X_V = beta v (MN-major; C is dead)
+    // ---- while M1 runs: X_K = beta k / |k| e^{Gam_r}, X_V = beta v (MN-major)
     {
       const float* fq = fac + qq * 5 * 128 + c0;
       const uint4 v1 = rawv(3, t0 + sw), v2 = rawv(3, t0 + 1 - sw);
@@ -1130,25 +1132,28 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
         st16(sm + L::kX, mnmaj(128 + c0, t, 4096), vf);
       }
     }
+    if (!group_wait(bar_mma, ph_mma, p.hdr, bid, gtid)) { ok = false; break; }
     // ---- A products -> A_kk (fp32, beta- and norm-scaled, strictly lower) and
-    //      A_qk (bf16 slot image, MN-major)
+    //      A_qk (bf16 slot image, MN-major).  Warp (q4, cq): window bb = 2 (cq / 2) +
+    //      q4 / 2, key row i = 32 (q4 % 2) + lane; cq % 2 selects A_kk or A_qk.
     float* Akk = reinterpret_cast<float*>(sm + L::kAkk);
     {
-      const int i = r64, bb = cq;  // warp: lane quarter q4, row block bb
-      float va[16], vq[16];
-      tmem_ld16(tmem_addr(tm, 32 * q4, kTmA + 32 * bb), va);
-      tmem_ld16(tmem_addr(tm, 32 * q4, kTmA + 32 * bb + 16), vq);
+      const int pr = cq >> 1, part = cq & 1, bb = 2 * pr + (q4 >> 1), i = 32 * (q4 & 1) + lane;
+      float va[16];
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmA + 64 * pr + 32 * (q4 >> 1) + 16 * part), va);
       tmem_ld_wait();
-      if (m64) {
-        const float ki = vec[kVecIk + i];
+      const float ki = vec[kVecIk + i];
+      if (part == 0) {
 #pragma unroll
         for (int cc = 0; cc < 16; ++cc) {
           const int r = 16 * bb + cc;
           Akk[r * kLd + i] = (i < r) ? vec[kVecBeta + r] * vec[kVecIk + r] * ki * va[cc] : 0.f;
-          vq[cc] = (i <= r) ? vq[cc] * ki : 0.f;
         }
-        st16(slot + kSlotA3, mnmaj(16 * bb, i, 1024), vq);
-        st16(slot + kSlotA3, mnmaj(16 * bb + 8, i, 1024), vq + 8);
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) va[cc] = (i <= 16 * bb + cc) ? va[cc] * ki : 0.f;
+        st16(slot + kSlotA3, mnmaj(16 * bb, i, 1024), va);
+        st16(slot + kSlotA3, mnmaj(16 * bb + 8, i, 1024), va + 8);
       }
     }
     fence_before_sync();
@@ -1215,14 +1220,26 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
       mm2x2<32>(Tf + (32 + r2) * kLd + 32, Tf + (33 + r2) * kLd + 32, Y + c2, 34, t);
       *reinterpret_cast<float2*>(Tf + (32 + r2) * kLd + c2) = make_float2(-t[0], -t[1]);
       *reinterpret_cast<float2*>(Tf + (33 + r2) * kLd + c2) = make_float2(-t[2], -t[3]);
+    } else {
+      // meanwhile: the final diagonal halves T[0:32][0:32], T[32:64][32:64] and the
+      // zero block T[0:32][32:64] -> bf16 A operand (K-major), 8 columns per vector
+      for (int u = gtid - 256; u < 384; u += 256) {
+        const int blk = u >> 7, r = (u >> 2) & 31, i0 = (u & 3) * 8;  // blk 0: T11, 1: T22, 2: T12
+        const int row = blk == 1 ? 32 + r : r, col = blk == 0 ? i0 : 32 + i0;
+        float t8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          t8[i] = (blk < 2 && col + i <= row) ? Tf[row * kLd + col + i] : 0.f;
+        st16(sm + L::kTop, kmaj(row, col, 1024), t8);
+      }
     }
     group_sync(bid);
-    // T -> bf16 A operand (K-major), upper triangle zero
-    {
-      const int r = (gtid >> 6) * 8 + (gtid & 7), i0 = ((gtid >> 3) & 7) * 8;
+    // the merged block T[32:64][0:32] -> bf16 A operand
+    if (gtid < 128) {
+      const int r = 32 + (gtid >> 2), i0 = (gtid & 3) * 8;
       float t8[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) t8[i] = (i0 + i <= r) ? Tf[r * kLd + i0 + i] : 0.f;
+      for (int i = 0; i < 8; ++i) t8[i] = Tf[r * kLd + i0 + i];
       st16(sm + L::kTop, kmaj(r, i0, 1024), t8);
     }
     group_sync_for_mma(bid);
