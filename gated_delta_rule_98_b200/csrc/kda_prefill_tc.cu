@@ -81,17 +81,17 @@ constexpr uint32_t kTmWU = 0;    // [W | U~]: 256 columns (after the products ar
 constexpr uint32_t kTmW = 0;     // D_W = W S (128, or 256 for W [S | X])
 constexpr uint32_t kTmQ = 128;   // D_Q = Q' S (+ A_qk U)
 constexpr uint32_t kTmS = 256;   // fp32 state; identity-started block X at 384 (transition)
-constexpr uint32_t kTmQ2 = 384;  // second D_Q of the chain pass (alternate chunks)
 
 constexpr int kLd = 68;  // row stride (floats) of the fp32 A_kk / T tiles
 
-// Chain operands of one (chunk, head), written by the transition pass and read
-// by the chain pass with one bulk copy.  The bf16 images have exactly the
-// shared-memory layouts the MMAs read: W (A, K-major, M=64 K=128), K' (A,
-// K-major, M=128 K=64), Q' (A, MN-major, M=64 K=128), A_qk (A, MN-major, M=64
-// K=64); U~ is bf16 in the order the chain threads read it (see ut_index);
-// then gamma (128 fp32) and the query row scales (64 fp32).
-constexpr int kSlotW = 0, kSlotK = 16384, kSlotQ = 32768, kSlotA3 = 49152, kSlotU = 57344,
+// Chain operands of one (chunk, head), written by the preparation kernel and
+// read by the chain passes with bulk copies.  The bf16 images have exactly the
+// shared-memory layouts the MMAs read: W and Q' (K-major [token][dk], adjacent
+// so that [W ; Q'] is one N=128 operand), K' (MN-major [token][dk]), A_qk
+// (MN-major, N = query row, K = key row); U~^T is bf16 [dv][token] in the
+// order the chain threads read it (see ut_index); then gamma (128 fp32) and the
+// query row scales (64 fp32).
+constexpr int kSlotW = 0, kSlotQ = 16384, kSlotK = 32768, kSlotA3 = 49152, kSlotU = 57344,
               kSlotGam = 73728, kSlotIq = 74240, kSlotBytes = 74496;
 // Chunk c of sequence n (first token a) has slot a / C + n + c: distinct for
 // every chunk of every sequence and below T / C + N.
@@ -100,10 +100,10 @@ __device__ __forceinline__ unsigned char* chunk_slot(const unsigned char* prep_b
   return const_cast<unsigned char*>(prep_base) +
          ((size_t)(a / 64 + n + c) * H + h) * (size_t)kSlotBytes;
 }
-// 16-byte unit of U~ (row r = 16 q4 + l, l < 16; columns 32 cq + 8 pc .. +7, bf16)
-// in a slot: each warp's 16 active lanes read 256 consecutive bytes per vector.
-__device__ __forceinline__ int ut_index(int q4, int cq, int pc, int l) {
-  return ((cq * 4 + q4) * 4 + pc) * 16 + l;
+// 16-byte unit of U~^T (value column 32 q4 + l; tokens 16 cq + 8 half .. +7, bf16)
+// in a slot: each warp reads 512 consecutive bytes per vector.
+__device__ __forceinline__ int ut_index(int q4, int cq, int half, int l) {
+  return ((cq * 4 + q4) * 2 + half) * 32 + l;
 }
 
 constexpr long long kWaitCycles = 4000000000LL;  // ~2 s: a wait this long is a fault
@@ -1243,17 +1243,23 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
       st16(sm + L::kTop, kmaj(r, i0, 1024), t8);
     }
     group_sync_for_mma(bid);
-    // ---- M2: [W | U~] = T [X_K | X_V]  (M=64, N=256, K=64; X MN-major)
+    // ---- M2: W = T X_K (M=64, N=128, K=64; X MN-major) -> columns 0-127, and
+    //      U~^T = X_V^T T^T (M=128 value columns, N=64 tokens) -> columns 128-191
     if (gtid == 0) {
-      constexpr uint32_t id = instr_desc(kFmtBF16, 64, 256, false, true);
+      constexpr uint32_t id = instr_desc(kFmtBF16, 64, 128, false, true);
+      constexpr uint32_t idu = instr_desc(kFmtBF16, 128, 64, true, false);
       const uint64_t ad = smem_desc(smem_u32(sm + L::kTop), 128, 1024);
       const uint64_t bd = smem_desc(smem_u32(sm + L::kX), 4096, 128);
+      const uint64_t xv = smem_desc(smem_u32(sm + L::kX + 2048), 4096, 128);  // X_V, M = value column
 #pragma unroll
-      for (int k = 0; k < 4; ++k) mma_bf16(tm + kTmWU, ad + 16 * k, bd + 512 * k, id, k > 0);
+      for (int k = 0; k < 4; ++k) {
+        mma_bf16(tm + kTmWU, ad + 16 * k, bd + 512 * k, id, k > 0);
+        mma_bf16(tm + kTmWU + 128, xv + 512 * k, ad + 16 * k, idu, k > 0);
+      }
       mma_commit(bar_mma);
     }
     if (!group_wait(bar_mma, ph_mma, p.hdr, bid, gtid)) { ok = false; break; }
-    // ---- W (bf16 image) and U~ (fp32) -> shared memory -> slot
+    // ---- W and U~^T (bf16 images) -> shared memory -> slot
 #pragma unroll
     for (int c16 = 0; c16 < 32; c16 += 16) {
       float w16[16];
@@ -1264,16 +1270,13 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
         st16(sm + L::kW, kmaj(r64, 32 * cq + c16 + 8, 2048), w16 + 8);
       }
     }
-#pragma unroll
-    for (int c16 = 0; c16 < 32; c16 += 16) {
-      float u16[16];
-      tmem_ld16(tmem_addr(tm, 32 * q4, kTmWU + 128 + 32 * cq + c16), u16);
+    {
+      float u16[16];  // U~^T: value column 32 q4 + lane, tokens 16 cq .. 16 cq + 15
+      tmem_ld16(tmem_addr(tm, 32 * q4, kTmWU + 128 + 16 * cq), u16);
       tmem_ld_wait();
-      if (m64) {
-        uint4* ug = reinterpret_cast<uint4*>(sm + L::kUt);
-        ug[ut_index(q4, cq, (c16 >> 3), lane)] = pack8(u16);
-        ug[ut_index(q4, cq, (c16 >> 3) + 1, lane)] = pack8(u16 + 8);
-      }
+      uint4* ug = reinterpret_cast<uint4*>(sm + L::kUt);
+      ug[ut_index(q4, cq, 0, lane)] = pack8(u16);
+      ug[ut_index(q4, cq, 1, lane)] = pack8(u16 + 8);
     }
     group_sync_for_mma(bid);
     if (gtid == 0) {
@@ -1294,24 +1297,31 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
 
 // ---------------------------------------------------------------------------
 // Chain passes of a segmented sequence: the state-dependent half of each chunk,
-// from the operands in its slot.  Per chunk: D_W = W S (and D_Q = Q' S) (C1),
-// S <- gamma S meanwhile, U = U~ - D_W, S += K'^T U (and D_Q += A_qk U) (C2),
-// o = D_Q scaled by the query row norms.
+// from the operands in its slot, in transposed form so that the state's value
+// columns are the M=128 dimension of the MMAs.  Per chunk:
+//   C1: [D_W^T | D_Q^T] = S^T [W ; Q']^T   (M=128 value columns, N=128 tokens),
+//       while S <- gamma S (fp32, TMEM) and the previous chunk's o is staged;
+//   U^T = U~^T - D_W^T  (bf16, K-major [value column][token]);
+//   C2: S += K'^T U  (M=128, N=128);  D_Q^T += U^T A_qk^T  (N=64);
+//   o = (D_Q^T)^T / |q|, staged through shared memory during the next C1.
 //   TRANS = false: full pass of segment p from its true incoming state; o, S_final.
-//   TRANS = true : transition of segments 0..P-2 on [S | X], from S = 0 (-> N_p)
-//                  and X = I (-> M_p), 256 columns wide; no output.
+//   TRANS = true : transition of segments 0..P-2 on [S | X] (256 columns) from
+//                  S = 0 (-> N_p) and X = I (-> M_p); C1 is two M=128, N=64 MMAs
+//                  per K step (S and X against W); no Q', no output.
 // Slot parts are bulk-copied two chunks ahead into two stages.
 template <bool TRANS>
 struct ChainSmem {
-  static constexpr int kSbN = TRANS ? 256 : 128;    // state columns
-  static constexpr int kSb = 0;                     // [S | X] bf16, B operand (K=128), MN-major
-  static constexpr int kU = kSbN * 256;             // U bf16, B operand (K=64), MN-major
-  static constexpr int kStage = kU + kSbN * 128;    // two stages
-  // stage layout: the slot (full pass), or W | K' | U~ | gamma (transition)
-  static constexpr int kW = kSlotW, kK = kSlotK, kQ = kSlotQ, kA3 = kSlotA3;
+  static constexpr int kSbN = TRANS ? 256 : 128;   // state columns
+  static constexpr int kSb = 0;                    // [S | X] bf16, MN-major (M = column, K = dk)
+  static constexpr int kU = kSbN * 256;            // U^T bf16, K-major [column][token]
+  static constexpr int kO = kU + kSbN * 128;       // o staging [64 tokens][128] bf16 (full pass)
+  static constexpr int kIqs = kO + (TRANS ? 0 : 16384);     // 1/|q| of the staged chunk
+  static constexpr int kStage = kIqs + (TRANS ? 0 : 256);   // two stages
+  // stage layout: the slot (full pass), or W | K' | U~^T | gamma (transition)
+  static constexpr int kW = 0, kQ = kSlotQ, kA3 = kSlotA3, kIq = kSlotIq;
+  static constexpr int kK = TRANS ? 16384 : kSlotK;
   static constexpr int kUt = TRANS ? 32768 : kSlotU;
   static constexpr int kGam = TRANS ? 32768 + 16384 : kSlotGam;
-  static constexpr int kIq = kSlotIq;               // full pass only
   static constexpr int kStageBytes = TRANS ? 32768 + 16384 + 512 : kSlotBytes;
   static constexpr int kBytes = kStage + 2 * kStageBytes;
 };
@@ -1319,7 +1329,7 @@ struct ChainSmem {
 template <bool TRANS>
 __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ TcParams p) {
   using L = ChainSmem<TRANS>;
-  constexpr int SbN = L::kSbN, SbL = SbN * 16;  // N extent of the state operands, their LBO
+  constexpr int SbN = L::kSbN, SbL = SbN * 16;  // state columns, K-group stride of their copy
   constexpr int NB = SbN / 128;                 // 128-column blocks
   extern __shared__ __align__(1024) unsigned char sm[];
   __shared__ uint64_t s_bar, s_ld[2];
@@ -1357,8 +1367,9 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
     const unsigned char* src = chunk_slot(p.prep, a, n, c, h, H);
     mbar_arrive_expect_tx(&s_ld[s], L::kStageBytes);
     if (TRANS) {
-      bulk_g2s(dst, src, 32768, &s_ld[s]);                           // W | K'
-      bulk_g2s(dst + L::kUt, src + kSlotU, 16384 + 512, &s_ld[s]);   // U~ | gamma
+      bulk_g2s(dst, src + kSlotW, 16384, &s_ld[s]);                     // W
+      bulk_g2s(dst + L::kK, src + kSlotK, 16384, &s_ld[s]);             // K'
+      bulk_g2s(dst + L::kUt, src + kSlotU, 16384 + 512, &s_ld[s]);      // U~^T | gamma
     } else {
       bulk_g2s(dst, src, kSlotBytes, &s_ld[s]);
     }
@@ -1370,12 +1381,10 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
   uint32_t phase = 0, ph_ld = 0;  // ph_ld bit s: parity of stage s's next completion
   uint32_t inflight = (c0 < c1 ? 1u : 0u) | (c0 + 1 < c1 ? 2u : 0u);  // stages being filled
 
-  const int q4 = warp & 3, cq = warp >> 2;  // TMEM lane quarter, 32-column quarter
-  const int srow = 32 * q4 + lane;          // dk row (M=128 accumulators)
-  const int r64 = 16 * q4 + lane;           // token row of M=64 accumulators (lane < 16)
-  const bool m64 = lane < 16;
+  const int q4 = warp & 3, cq = warp >> 2;  // TMEM lane quarter, column quarter
+  const int srow = 32 * q4 + lane;          // TMEM lane: dk row of S, value column of D^T
 
-  // ---- initial state -> TMEM (fp32) and the bf16 operand: S_in (full pass),
+  // ---- initial state -> TMEM (fp32) and the bf16 copy: S_in (full pass),
   //      or S = 0 and X = I (transition)
   {
     const float* S0 = nullptr;
@@ -1406,29 +1415,32 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
     tmem_st_wait();
   }
 
-  // o of a chunk = its D_Q (two alternating TMEM buffers) / |q|, written while
-  // the next chunk's C1 runs
-  float iq_prev = 0.f;  // 1/|q| of the previous chunk's row r64
-  auto write_o = [&](int cc, uint32_t dq, float iq) {
-    const int t0c = a + cc * kC, lenc = min(kC, b - t0c);
-    const int col = 32 * cq;
-    float o0[16], o1[16];
-    tmem_ld16(tmem_addr(tm, 32 * q4, dq + col), o0);
-    tmem_ld16(tmem_addr(tm, 32 * q4, dq + col + 16), o1);
+  // o of a chunk: D_Q^T (columns dcol + 64 .. dcol + 127) / |q| -> staging [token][value]
+  float* iqs = reinterpret_cast<float*>(sm + L::kIqs);
+  __nv_bfloat16* ost = reinterpret_cast<__nv_bfloat16*>(sm + L::kO);
+  auto stage_o = [&](uint32_t dcol) {
+    float v[16];
+    tmem_ld16(tmem_addr(tm, 32 * q4, dcol + 64 + 16 * cq), v);
     tmem_ld_wait();
-    if (m64 && r64 < lenc) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) { o0[i] *= iq; o1[i] *= iq; }
-      uint4* dst = reinterpret_cast<uint4*>(p.o + ((size_t)(t0c + r64) * H + h) * kD + col);
-      dst[0] = pack8(o0);
-      dst[1] = pack8(o0 + 8);
-      dst[2] = pack8(o1);
-      dst[3] = pack8(o1 + 8);
+    for (int i = 0; i < 16; ++i) {
+      const int t = 16 * cq + i;
+      ost[t * kD + srow] = __float2bfloat16_rn(v[i] * iqs[t]);
     }
   };
+  auto write_o = [&](int cc) {  // staging -> o rows of chunk cc (after a barrier)
+    const int t0c = a + cc * kC, lenc = min(kC, b - t0c);
+    for (int u = tid; u < kC * kD / 8; u += kNT) {
+      const int t = u >> 4, d8 = (u & 15) * 8;
+      if (t < lenc)
+        *reinterpret_cast<uint4*>(p.o + ((size_t)(t0c + t) * H + h) * kD + d8) =
+            *reinterpret_cast<const uint4*>(ost + t * kD + d8);
+    }
+  };
+
   for (int c = c0; c < c1; ++c) {
     const int s = (c - c0) & 1;
-    const uint32_t tmq = s ? kTmQ2 : kTmQ;  // this chunk's D_Q
+    const uint32_t dcol = (!TRANS && s) ? 128u : 0u;  // this chunk's products (two buffers)
     unsigned char* st = sm + L::kStage + s * L::kStageBytes;
     sync_for_mma();
     {
@@ -1441,21 +1453,26 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       ph_ld ^= 1u << s;
       inflight &= ~(1u << s);
     }
-    // ---- C1: D_W = W [S | X] (M=64, N=SbN, K=128); D_Q = Q' S (full pass)
+    // ---- C1 (copy of S as the MN-major A operand; W, Q' as the K-major B operand)
     if (tid == 0) {
+      const uint64_t bd = smem_desc(smem_u32(st + L::kW), 128, 2048);
       const uint64_t sd = smem_desc(smem_u32(sm + L::kSb), SbL, 128);
-      const uint64_t wd = smem_desc(smem_u32(st + L::kW), 128, 2048);
-      constexpr uint32_t idw = instr_desc(kFmtBF16, 64, SbN, false, true);
-      const uint64_t qd = smem_desc(smem_u32(st + L::kQ), 128, 2048);  // Q' K-major
-      constexpr uint32_t idq = instr_desc(kFmtBF16, 64, 128, false, true);
+      if (!TRANS) {
+        constexpr uint32_t id = instr_desc(kFmtBF16, 128, 128, true, false);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {  // the two accumulators interleaved
-        mma_bf16(tm + kTmW, wd + 16 * k, sd + (2 * SbL >> 4) * k, idw, k > 0);
-        if (!TRANS) mma_bf16(tm + tmq, qd + 16 * k, sd + (2 * SbL >> 4) * k, idq, k > 0);
+        for (int k = 0; k < 8; ++k) mma_bf16(tm + dcol, sd + (2 * SbL >> 4) * k, bd + 16 * k, id, k > 0);
+      } else {
+        constexpr uint32_t id = instr_desc(kFmtBF16, 128, 64, true, false);
+        const uint64_t xd = smem_desc(smem_u32(sm + L::kSb + 2048), SbL, 128);  // X columns
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          mma_bf16(tm, sd + (2 * SbL >> 4) * k, bd + 16 * k, id, k > 0);
+          mma_bf16(tm + 64, xd + (2 * SbL >> 4) * k, bd + 16 * k, id, k > 0);
+        }
       }
       mma_commit(&s_bar);
     }
-    // ---- meanwhile decay the fp32 state by gamma (C1 reads the bf16 copy)
+    // ---- meanwhile: decay the fp32 state by gamma; stage the previous chunk's o
     {
       const float gm = reinterpret_cast<const float*>(st + L::kGam)[srow];
 #pragma unroll
@@ -1472,64 +1489,57 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       }
       tmem_st_wait();
     }
-    if (!TRANS && c > c0) write_o(c - 1, s ? kTmQ : kTmQ2, iq_prev);
+    if (!TRANS && c > c0) stage_o(dcol ^ 128u);
     if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
-    // ---- U = U~ - D_W (transition: [U~ | 0] - W [S | X]) -> B operand (MN-major)
+    if (!TRANS && c > c0) write_o(c - 1);
+    // ---- U^T = U~^T - D_W^T (transition: [U~^T - D_S^T ; -D_X^T]) -> K-major
 #pragma unroll
     for (int blk = 0; blk < NB; ++blk) {
-      float d0[16], d1[16];
-      const int col = 128 * blk + 32 * cq;
-      tmem_ld16(tmem_addr(tm, 32 * q4, kTmW + col), d0);
-      tmem_ld16(tmem_addr(tm, 32 * q4, kTmW + col + 16), d1);
+      float d[16];
+      tmem_ld16(tmem_addr(tm, 32 * q4, dcol + 64 * blk + 16 * cq), d);
       tmem_ld_wait();
-      if (m64) {
-        if (blk == 0) {
-          const uint4* ug = reinterpret_cast<const uint4*>(st + L::kUt);
+      if (blk == 0) {
+        const uint4* ug = reinterpret_cast<const uint4*>(st + L::kUt);
+        float u0[8], u1[8];
+        unpack8(ug[ut_index(q4, cq, 0, lane)], u0);
+        unpack8(ug[ut_index(q4, cq, 1, lane)], u1);
 #pragma unroll
-          for (int pc = 0; pc < 2; ++pc) {
-            float u0[8], u1[8];
-            unpack8(ug[ut_index(q4, cq, pc, lane)], u0);
-            unpack8(ug[ut_index(q4, cq, pc + 2, lane)], u1);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              d0[8 * pc + e] = u0[e] - d0[8 * pc + e];
-              d1[8 * pc + e] = u1[e] - d1[8 * pc + e];
-            }
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) { d0[i] = -d0[i]; d1[i] = -d1[i]; }
+        for (int e = 0; e < 8; ++e) {
+          d[e] = u0[e] - d[e];
+          d[8 + e] = u1[e] - d[8 + e];
         }
-        st16(sm + L::kU, mnmaj(col, r64, SbL), d0);
-        st16(sm + L::kU, mnmaj(col + 8, r64, SbL), d0 + 8);
-        st16(sm + L::kU, mnmaj(col + 16, r64, SbL), d1);
-        st16(sm + L::kU, mnmaj(col + 24, r64, SbL), d1 + 8);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) d[e] = -d[e];
       }
+      st16(sm + L::kU, kmaj(128 * blk + srow, 16 * cq, 1024), d);
+      st16(sm + L::kU, kmaj(128 * blk + srow, 16 * cq + 8, 1024), d + 8);
     }
     sync_for_mma();
-    // ---- C2: [S | X] += K'^T U (M=128, K=64); D_Q += A_qk U (full pass)
+    // ---- C2: [S | X] += K'^T U (K' MN-major A, U K-major B); D_Q^T += U^T A_qk^T
     if (tid == 0) {
-      const uint64_t kd = smem_desc(smem_u32(st + L::kK), 2048, 128);  // K' MN-major
-      const uint64_t ud = smem_desc(smem_u32(sm + L::kU), SbL, 128);
-      constexpr uint32_t ids = instr_desc(kFmtBF16, 128, SbN, true, true);
+      const uint64_t kd = smem_desc(smem_u32(st + L::kK), 2048, 128);
+      const uint64_t ud = smem_desc(smem_u32(sm + L::kU), 128, 1024);
+      constexpr uint32_t ids = instr_desc(kFmtBF16, 128, SbN, true, false);
       const uint64_t a3 = smem_desc(smem_u32(st + L::kA3), 1024, 128);
-      constexpr uint32_t ido = instr_desc(kFmtBF16, 64, 128, true, true);
+      constexpr uint32_t ido = instr_desc(kFmtBF16, 128, 64, false, true);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        mma_bf16(tm + kTmS, kd + 256 * k, ud + (2 * SbL >> 4) * k, ids, 1);
-        if (!TRANS) mma_bf16(tm + tmq, a3 + 128 * k, ud + (2 * SbL >> 4) * k, ido, 1);
+        mma_bf16(tm + kTmS, kd + 256 * k, ud + 16 * k, ids, 1);
+        if (!TRANS) mma_bf16(tm + dcol + 64, ud + 16 * k, a3 + 128 * k, ido, 1);
       }
       mma_commit(&s_bar);
     }
-    // (read before the barrier below, which orders it before the stage's refill)
-    if (!TRANS && m64) iq_prev = reinterpret_cast<const float*>(st + L::kIq)[r64];
+    // the query row scales of this chunk (read before the barrier below, which
+    // orders them before the stage's refill)
+    if (!TRANS && tid < kC) iqs[tid] = reinterpret_cast<const float*>(st + L::kIq)[tid];
     if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
     // the stage is consumed (its reads ended before the barrier above): refill it
     if (c + 2 < c1) {
       inflight |= 1u << s;
       if (tid == 0) load_slot(c + 2);
     }
-    // ---- [S | X] -> bf16 operand of the next chunk
+    // ---- [S | X] -> bf16 copy for the next chunk
 #pragma unroll
     for (int blk = 0; blk < NB; ++blk) {
       float s0[16], s1[16];
@@ -1545,8 +1555,9 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
   }
   // o of the last chunk
   if (!TRANS && !s_abort && c1 > c0) {
-    fence_after_sync();
-    write_o(c1 - 1, ((c1 - 1 - c0) & 1) ? kTmQ2 : kTmQ, iq_prev);
+    stage_o(((c1 - 1 - c0) & 1) ? 128u : 0u);
+    __syncthreads();
+    write_o(c1 - 1);
   }
 
   fence_before_sync();
