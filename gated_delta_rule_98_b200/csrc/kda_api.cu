@@ -138,6 +138,35 @@ kda_status kda_forward_g(const void* q, const void* k, const void* v,
   return forward_common(a);
 }
 
+kda_status kda_forward_checkpoints(const void* q, const void* k, const void* v,
+                                   const void* z, const float* A, const void* beta,
+                                   const float* S0, const int32_t* cu_seqlens,
+                                   int32_t num_seqs, int32_t total_tokens,
+                                   int32_t max_seqlen, int32_t H, int32_t dk,
+                                   int32_t dv, kda_dtype dt, int32_t chunk, void* o,
+                                   float* S_final, float* S_ckpt, int32_t interval,
+                                   void* workspace, size_t workspace_bytes,
+                                   kda_stream_t stream) {
+  kda_status st = check_forward(q, k, v, z, beta, S0, cu_seqlens, num_seqs,
+                                total_tokens, max_seqlen, H, dk, dv, dt, chunk,
+                                o, S_final, workspace, workspace_bytes);
+  if (st != KDA_OK) return st;
+  if (total_tokens > 0 && (!A || !aligned16(A))) return KDA_ERR_INVALID_ARG;
+  if (interval <= 0 || interval % chunk != 0) return KDA_ERR_INVALID_ARG;
+  const int32_t count = max_seqlen / interval;
+  if (count > 0 && (!S_ckpt || !aligned16(S_ckpt))) return KDA_ERR_INVALID_ARG;
+  kda::ForwardArgs a{q, k, v, z, beta, A, nullptr, S0, cu_seqlens, o, S_final,
+                     num_seqs, total_tokens, max_seqlen, H, dk, dv, chunk,
+                     dt == KDA_BF16, workspace, workspace_bytes,
+                     (cudaStream_t)stream};
+  if (count > 0) {
+    a.S_ckpt = S_ckpt;
+    a.ckpt_every = interval / chunk;
+    a.ckpt_count = count;
+  }
+  return forward_common(a);
+}
+
 kda_status kda_decode_step(const void* q, const void* k, const void* v,
                            const void* z, const float* A, const void* beta,
                            float* S_inout, int32_t B, int32_t H, int32_t dk,

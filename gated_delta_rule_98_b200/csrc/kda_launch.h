@@ -31,6 +31,9 @@ struct ForwardArgs {
   void* ws;              // workspace base (header at offset 0)
   size_t ws_bytes;
   cudaStream_t stream;
+  float* S_ckpt = nullptr;  // [N, H, ckpt_count, dk, dv] states every ckpt_every chunks, or null
+  int ckpt_every = 0;       // chunks between checkpoints
+  int ckpt_count = 0;       // checkpoints per (sequence, head): max_len / interval
 };
 
 cudaError_t launch_decode(const DecodeArgs& a);

@@ -55,6 +55,8 @@ struct SimtParams {
   const int32_t* cu;
   void* o;
   float* S_final;
+  float* S_ckpt;  // checkpoints every ckpt_every chunks (ckpt_count per sequence and head)
+  int ckpt_every, ckpt_count;
   int N, T, max_len, H, max_cps;
   float *W, *Ut, *Qp, *Kp, *Aqk, *gam;
   WsHeader* hdr;
@@ -311,12 +313,17 @@ __global__ void __launch_bounds__(256) simt_state_kernel(SimtParams p) {
       og[((size_t)(tok0 + r) * H + h) * DV + c0 + c] = from_f<T>(acc);
     }
     __syncthreads();
-    // S = Diag(gamma) S + K'^T U
+    // S = Diag(gamma) S + K'^T U; a checkpoint after every ckpt_every full chunks
+    const bool ckpt = p.S_ckpt && (j + 1) % p.ckpt_every == 0 && (j + 1) * C <= b - a;
+    float* Sc = ckpt ? p.S_ckpt + (((size_t)n * H + h) * p.ckpt_count + (j + 1) / p.ckpt_every - 1) *
+                                      DK * DV
+                     : nullptr;
     for (int e = tid; e < DK * BV; e += NT) {
       const int i = e / BV, c = e % BV;
       float acc = gs[i] * S[e];
       for (int r = 0; r < len; ++r) acc += Ks[r * LK + i] * Us[r * BV + c];
       S[e] = acc;
+      if (ckpt) Sc[(size_t)i * DV + c0 + c] = acc;
     }
   }
   __syncthreads();
@@ -386,6 +393,7 @@ cudaError_t launch_forward_simt(const ForwardArgs& a) {
   SimtParams p;
   p.q = a.q; p.k = a.k; p.v = a.v; p.z = a.z; p.beta = a.beta;
   p.A = a.A; p.g = a.g; p.S0 = a.S0; p.cu = a.cu; p.o = a.o; p.S_final = a.S_final;
+  p.S_ckpt = a.S_ckpt; p.ckpt_every = a.ckpt_every; p.ckpt_count = a.ckpt_count;
   p.N = a.N; p.T = a.T; p.max_len = a.max_len; p.H = a.H;
   p.max_cps = (a.max_len + a.chunk - 1) / a.chunk;
   p.W = (float*)(base + L.W);

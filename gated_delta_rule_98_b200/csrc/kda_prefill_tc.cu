@@ -159,11 +159,20 @@ struct alignas(64) TcParams {
   const int32_t* cu;
   __nv_bfloat16* o;
   float* S_final;
+  float* S_ckpt;  // checkpoints every ckpt_every chunks (ckpt_count per sequence and head)
+  int ckpt_every, ckpt_count;
   int N, T, max_len, H, P;
   float* seg;  // per (n, h): transitions (M, N) of segments 0..P-2, incoming states of 0..P-1
   unsigned char* prep;  // per (chunk slot, h): chain operands left by the transition pass
   WsHeader* hdr;
 };
+
+// Checkpoint slot of the state after sequence-relative chunk c (n_tok tokens in
+// the sequence), or null when no checkpoint falls there.
+__device__ __forceinline__ float* ckpt_state(const TcParams& p, int n, int h, int c, int n_tok) {
+  if (!p.S_ckpt || (c + 1) % p.ckpt_every != 0 || (c + 1) * 64 > n_tok) return nullptr;
+  return p.S_ckpt + (((size_t)n * p.H + h) * p.ckpt_count + (c + 1) / p.ckpt_every - 1) * 128 * 128;
+}
 
 // Segment p of a sequence with nch chunks: chunks [c0, c1).
 __device__ __forceinline__ void segment_chunks(int nch, int P, int p, int& c0, int& c1) {
@@ -661,13 +670,22 @@ __global__ void __launch_bounds__(kNT, 1) fused_kernel(const __grid_constant__ T
       mma_commit(&s_bar);
     }
     if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
-    // ---- S -> bf16 operand for the next chunk; O -> global
+    // ---- S -> bf16 operand for the next chunk (and the fp32 checkpoint, if one
+    //      falls after this chunk); O -> global
     {
       float s0[16], s1[16];
       const int col = 32 * cq;
       tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + col), s0);
       tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + col + 16), s1);
       tmem_ld_wait();
+      if (float* ck = ckpt_state(p, n, h, c, b - a)) {
+        float4* d4 = reinterpret_cast<float4*>(ck + (size_t)srow * kD + col);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          d4[i] = make_float4(s0[4 * i], s0[4 * i + 1], s0[4 * i + 2], s0[4 * i + 3]);
+          d4[4 + i] = make_float4(s1[4 * i], s1[4 * i + 1], s1[4 * i + 2], s1[4 * i + 3]);
+        }
+      }
       st16(sm + L::kSb, mnmaj(col, srow, SbL), s0);
       st16(sm + L::kSb, mnmaj(col + 8, srow, SbL), s0 + 8);
       st16(sm + L::kSb, mnmaj(col + 16, srow, SbL), s1);
@@ -1539,7 +1557,9 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       inflight |= 1u << s;
       if (tid == 0) load_slot(c + 2);
     }
-    // ---- [S | X] -> bf16 copy for the next chunk
+    // ---- [S | X] -> bf16 copy for the next chunk (and the fp32 checkpoint, if one
+    //      falls after this chunk)
+    float* ck = TRANS ? nullptr : ckpt_state(p, n, h, c, b - a);
 #pragma unroll
     for (int blk = 0; blk < NB; ++blk) {
       float s0[16], s1[16];
@@ -1547,6 +1567,14 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + col), s0);
       tmem_ld16(tmem_addr(tm, 32 * q4, kTmS + col + 16), s1);
       tmem_ld_wait();
+      if (ck) {
+        float4* d4 = reinterpret_cast<float4*>(ck + (size_t)srow * kD + col);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          d4[i] = make_float4(s0[4 * i], s0[4 * i + 1], s0[4 * i + 2], s0[4 * i + 3]);
+          d4[4 + i] = make_float4(s1[4 * i], s1[4 * i + 1], s1[4 * i + 2], s1[4 * i + 3]);
+        }
+      }
       st16(sm + L::kSb, mnmaj(col, srow, SbL), s0);
       st16(sm + L::kSb, mnmaj(col + 8, srow, SbL), s0 + 8);
       st16(sm + L::kSb, mnmaj(col + 16, srow, SbL), s1);
@@ -1779,6 +1807,9 @@ cudaError_t launch_forward_tc(const ForwardArgs& a) {
   p.cu = a.cu;
   p.o = (__nv_bfloat16*)a.o;
   p.S_final = a.S_final;
+  p.S_ckpt = a.S_ckpt;
+  p.ckpt_every = a.ckpt_every;
+  p.ckpt_count = a.ckpt_count;
   p.N = a.N;
   p.T = a.T;
   p.max_len = a.max_len;

@@ -26,7 +26,8 @@ KDA_F32, KDA_BF16 = 0, 1
 # Every symbol include/kda.h declares.
 EXPORTS = ("kda_status_string", "kda_version", "kda_forward_workspace_size",
            "kda_forward_launches", "kda_forward",
-           "kda_forward_g", "kda_decode_step", "kda_forward_noalloc", "kda_check_device_error")
+           "kda_forward_g", "kda_decode_step", "kda_forward_noalloc", "kda_forward_checkpoints",
+           "kda_check_device_error")
 
 # Bytes of the library's fixed scratch array used by kda_forward_noalloc.
 KDA_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -66,6 +67,9 @@ def lib():
     L.kda_decode_step.restype = ctypes.c_int
     L.kda_forward_noalloc.argtypes = [vp] * 8 + [i32] * 6 + [ctypes.c_int, i32, vp, vp, vp]
     L.kda_forward_noalloc.restype = ctypes.c_int
+    L.kda_forward_checkpoints.argtypes = ([vp] * 8 + [i32] * 6 + [ctypes.c_int, i32, vp, vp, vp,
+                                          i32, vp, sz, vp])
+    L.kda_forward_checkpoints.restype = ctypes.c_int
     L.kda_check_device_error.argtypes = [vp, vp]
     L.kda_check_device_error.restype = ctypes.c_int
     _lib = L
@@ -112,6 +116,15 @@ def kda_forward_noalloc(q, k, v, z, A, beta, S0, cu_seqlens, num_seqs, total_tok
     return lib().kda_forward_noalloc(q, k, v, z, A, beta, S0, cu_seqlens, num_seqs,
                                      total_tokens, max_seqlen, H, dk, dv, dt, chunk, o, S_final,
                                      stream)
+
+
+def kda_forward_checkpoints(q, k, v, z, A, beta, S0, cu_seqlens, num_seqs, total_tokens,
+                            max_seqlen, H, dk, dv, dt, chunk, o, S_final, S_ckpt, interval,
+                            workspace, workspace_bytes, stream):
+    return lib().kda_forward_checkpoints(q, k, v, z, A, beta, S0, cu_seqlens, num_seqs,
+                                         total_tokens, max_seqlen, H, dk, dv, dt, chunk, o,
+                                         S_final, S_ckpt, interval, workspace, workspace_bytes,
+                                         stream)
 
 
 def kda_check_device_error(workspace, stream):
@@ -169,6 +182,9 @@ def workspace(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype, chunk, devic
     return torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
 
 
+_new_workspace = workspace
+
+
 def _forward(entry, q, k, v, gate_a, gate_b, beta, S0, cu_seqlens, num_seqs, max_seqlen, chunk,
              o, S_final, ws, stream, want_state):
     _check_cuda(q, k, v, gate_a, gate_b, beta, S0, cu_seqlens, o, S_final, ws)
@@ -199,6 +215,33 @@ def forward(q, k, v, z, A, beta, *, S0=None, cu_seqlens=None, num_seqs=None, max
     (then ``num_seqs`` equal sequences).  Returns (o, S_final)."""
     return _forward("z", q, k, v, z, A, beta, S0, cu_seqlens, num_seqs, max_seqlen, chunk, o,
                     S_final, workspace, stream, output_final_state)
+
+
+def forward_checkpoints(q, k, v, z, A, beta, interval, *, S0=None, cu_seqlens=None,
+                        num_seqs=None, max_seqlen=None, chunk=64, o=None, S_final=None,
+                        S_ckpt=None, workspace=None, stream=None):
+    """KDA prefill that also returns the state after every ``interval`` tokens of
+    each sequence: (o, S_final, S_ckpt) with S_ckpt [N, H, max_seqlen // interval,
+    dk, dv] fp32 (entries past a sequence's end are left as allocated: zeros
+    when the binding allocates them)."""
+    _check_cuda(q, k, v, z, A, beta, S0, cu_seqlens, o, S_final, S_ckpt, workspace)
+    T, H, dk, dv, N, max_len = _geometry(q, v, cu_seqlens, num_seqs, max_seqlen)
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
+    if S_final is None:
+        S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    if S_ckpt is None:
+        S_ckpt = torch.zeros((N, H, max_len // interval, dk, dv), dtype=torch.float32,
+                             device=q.device)
+    ws = workspace if workspace is not None else _new_workspace(N, T, max_len, H, dk, dv,
+                                                                q.dtype, chunk, device=q.device)
+    st = kda_forward_checkpoints(_p(q), _p(k), _p(v), _p(z), _p(A), _p(beta), _p(S0),
+                                 _p(cu_seqlens), N, T, max_len, H, dk, dv, _dt(q), chunk, _p(o),
+                                 _p(S_final), _p(S_ckpt), int(interval), _p(ws), ws.numel(),
+                                 _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_forward_checkpoints")
+    return o, S_final, S_ckpt
 
 
 def forward_g(q, k, v, g, beta, *, S0=None, cu_seqlens=None, num_seqs=None, max_seqlen=None,

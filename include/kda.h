@@ -145,6 +145,33 @@ kda_status kda_forward_g(const void* q, const void* k, const void* v,
                          size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * kda_forward that also writes sparse state checkpoints: the state after
+ * every `interval` tokens of each sequence.  This is the operator's side of a
+ * prefix cache that keeps KDA states at fixed token boundaries inside a paged
+ * pool (Kimi Linear summary, hybrid paged cache with sparse KDA checkpoints);
+ * the pages describe the cache, not a kernel for it.
+ *
+ *  interval : tokens between checkpoints, a positive multiple of `chunk`
+ *             (else KDA_ERR_INVALID_ARG).
+ *  S_ckpt   : [N, H, J, dk, dv] float32 with J = max_seqlen / interval
+ *             (rounded down).  Entry (n, h, j) receives the state after the
+ *             first (j+1)·interval tokens of sequence n when (j+1)·interval
+ *             is at most its length; the other entries are not written.
+ *             16-byte aligned; may be NULL only when J = 0; must not overlap
+ *             any other argument.
+ * Everything else, including the workspace size, is kda_forward's.
+ */
+kda_status kda_forward_checkpoints(const void* q, const void* k, const void* v,
+                                   const void* z, const float* A, const void* beta,
+                                   const float* S0, const int32_t* cu_seqlens,
+                                   int32_t num_seqs, int32_t total_tokens,
+                                   int32_t max_seqlen, int32_t H, int32_t dk,
+                                   int32_t dv, kda_dtype dt, int32_t chunk, void* o,
+                                   float* S_final, float* S_ckpt, int32_t interval,
+                                   void* workspace, size_t workspace_bytes,
+                                   kda_stream_t stream);
+
+/*
  * One recurrent KDA step for B independent sequences (one token each),
  * updating the float32 states in place (Kimi Linear summary §6.3: token
  * generation uses the recurrent update).

@@ -127,3 +127,18 @@ def test_binding_rejects_cpu_tensors(L):
     q = torch.zeros(4, 1, 32)
     with pytest.raises(ValueError):
         kda.decode_step(q, q, q, q, torch.zeros(1), torch.zeros(4, 1), torch.zeros(4, 1, 32, 32))
+
+
+def test_checkpoints_reject_bad_interval_and_buffer(L):
+    def ck(**over):
+        a = dict(interval=64, S_ckpt=FAKE, chunk=16)
+        a.update(over)
+        return kda.kda_forward_checkpoints(
+            FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 1, 128, 128, 2, 32, 32,
+            kda.KDA_F32, a["chunk"], FAKE, FAKE, a["S_ckpt"], a["interval"], FAKE, 1 << 40, None)
+    assert ck(interval=0) == kda.KDA_ERR_INVALID_ARG
+    assert ck(interval=-16) == kda.KDA_ERR_INVALID_ARG
+    assert ck(interval=24) == kda.KDA_ERR_INVALID_ARG          # not a multiple of the chunk
+    assert ck(S_ckpt=None) == kda.KDA_ERR_INVALID_ARG          # 2 checkpoints need a buffer
+    assert ck(S_ckpt=FAKE + 4) == kda.KDA_ERR_INVALID_ARG      # misaligned
+    assert ck(chunk=32) == kda.KDA_ERR_UNSUPPORTED

@@ -78,6 +78,23 @@ def test_brute_force_transition_products(seed):
     assert np.abs(Sf - Sb).max() < 1e-12
 
 
+def test_state_trace_matches_brute_force_prefixes():
+    """The state after token t (what intermediate-state checkpoints store) is the
+    final state of the sequence cut after t, here from the transition-product
+    view, for every t of two packed sequences."""
+    cu = np.array([0, 7, 16])
+    p = _rand_problem(3, 16, 2, 5, 4, N=2, cu=cu)
+    _, _, St = ref.forward(p["q"], p["k"], p["v"], p["beta"], z=p["z"], A=p["A"],
+                           S0=p["S0"], cu_seqlens=cu, trace=True)
+    for n in range(2):
+        for t in range(cu[n], cu[n + 1]):
+            sl = slice(cu[n], t + 1)
+            _, Sb = brute.forward(p["q"][sl], p["k"][sl], p["v"][sl], p["beta"][sl],
+                                  z=p["z"][sl], A=p["A"], S0=p["S0"][n:n + 1],
+                                  cu_seqlens=np.array([0, t + 1 - cu[n]]))
+            assert np.abs(St[t] - Sb[0]).max() < 1e-12
+
+
 def test_brute_force_attention_matrix_is_causal():
     p = _rand_problem(5, 12, 1, 4, 3)
     g = brute.lower_bounded_gate(p["z"], p["A"])
