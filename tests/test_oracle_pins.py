@@ -13,7 +13,7 @@ import os
 import numpy as np
 import pytest
 
-from oracle import brute, chunk_mirror, ref
+from oracle import brute, chunk_mirror, epilogue, ref
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -399,3 +399,65 @@ def test_planted_mistakes_are_caught(mistake):
     # and the unmodified recurrence passes the same checks
     o3, S3 = _planted(p["q"], p["k"], p["v"], p["beta"], gg, p["S0"], None)
     assert np.abs(o3 - ob).max() < 1e-12 and np.abs(S3 - Sb).max() < 1e-12
+
+
+# --------------------------------------------------------- output epilogue ---
+
+def _golden_epilogue():
+    with open(os.path.join(GOLDEN, "kda_output_norm_gate.json")) as f:
+        return json.load(f)
+
+
+def test_output_norm_gate_hand_worked():
+    d = _golden_epilogue()
+    o = np.array(d["o"])[None]           # [T=1, H=2, dv=4]
+    y = epilogue.norm_gate(o, np.array(d["r"])[None], np.array(d["w"]), eps=d["eps"])
+    assert np.abs(y[0] - np.array(d["expected_y"])).max() < d["tolerance_abs"]
+
+
+def test_output_norm_gate_invariants():
+    rng = np.random.default_rng(31)
+    o = rng.standard_normal((5, 3, 16)) * rng.uniform(0.1, 10, (5, 3, 1))
+    r = rng.standard_normal((5, 3, 16))
+    y = epilogue.norm_gate(o, r, eps=0.0)
+    # per-head scale invariance: each (token, head) row may carry its own scale
+    c = rng.uniform(0.01, 100, (5, 3, 1))
+    assert np.abs(epilogue.norm_gate(c * o, r, eps=0.0) - y).max() < 1e-12
+    # a gate wide open and unit gain leave rows of unit root mean square
+    y1 = epilogue.norm_gate(o, np.full_like(r, 60.0), eps=0.0)
+    assert np.abs(np.sqrt(np.mean(y1 * y1, axis=-1)) - 1.0).max() < 1e-12
+    # a closed gate zeroes the output; sigmoid(0) halves it
+    assert np.abs(epilogue.norm_gate(o, np.full_like(r, -60.0), eps=0.0)).max() < 1e-20
+    half = epilogue.norm_gate(o, np.zeros_like(r), eps=0.0)
+    assert np.abs(2 * half - y1).max() < 1e-12
+    # eps only matters against the row's mean square
+    tiny = 1e-4 * o[:1, :1]
+    assert np.abs(epilogue.norm_gate(tiny, r[:1, :1], eps=1.0) -
+                  tiny / np.sqrt(np.mean(tiny ** 2) + 1.0) * epilogue.sigmoid(r[:1, :1])).max() < 1e-15
+
+
+@pytest.mark.parametrize("mistake", ["sum", "no_sqrt", "swish", "both_heads", "no_gain",
+                                     "gate_first", "one_minus"])
+def test_output_epilogue_mistakes_are_caught(mistake):
+    """Plausible mistakes in the epilogue, each restated here on the CPU, fail
+    the hand-worked pin."""
+    d = _golden_epilogue()
+    o, r, w = np.array(d["o"]), np.array(d["r"]), np.array(d["w"])
+    sig = epilogue.sigmoid
+    ms = np.mean(o * o, axis=-1, keepdims=True)
+    if mistake == "sum":
+        y = o / np.sqrt(np.sum(o * o, axis=-1, keepdims=True)) * w * sig(r)
+    elif mistake == "no_sqrt":
+        y = o / ms * w * sig(r)
+    elif mistake == "swish":
+        y = o / np.sqrt(ms) * w * r * sig(r)
+    elif mistake == "both_heads":
+        y = o / np.sqrt(np.mean(o * o)) * w * sig(r)
+    elif mistake == "no_gain":
+        y = o / np.sqrt(ms) * sig(r)
+    elif mistake == "gate_first":
+        og = o * sig(r)
+        y = og / np.sqrt(np.mean(og * og, axis=-1, keepdims=True)) * w
+    else:
+        y = o / np.sqrt(ms) * w * (1 - sig(r))
+    assert np.abs(y - np.array(d["expected_y"])).max() > 1e-3
