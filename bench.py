@@ -244,7 +244,7 @@ def main():
     e1 = torch.cuda.Event(enable_timing=True)
     pk = peaks()
     out = {"ms": None, "value": None, "roofline": None, "e2e": None, "clocks": None,
-           "launches": 0, "decode": None}
+           "launches": 0, "decode": None, "variants": None}
 
     # ---------------------------------------------------------- prefill ---
     if args.only != "decode":
@@ -321,6 +321,47 @@ def main():
         ms_e2e = rank_max(e0.elapsed_time(e1) / n_e2e)
         out["e2e"] = {"value": weak_scaling_value(T, world, ms_e2e), "unit": "tokens/s",
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+        # ----------------------------------------------------- variants ---
+        # The same workload through the entry points that add the output
+        # epilogue and sparse state checkpoints; each is timed like the main
+        # step and reported beside it with the bytes it adds.
+        r_gate, w_gain = synth.out_gate_inputs(T, H, D, seed=5)
+        r_gate, w_gain = r_gate.to(dev), w_gain.to(dev)
+        interval = 4096
+        ck = torch.empty((B, H, L // interval, D, D), dtype=torch.float32, device=dev)
+
+        def fwd_norm_gate():
+            kda.forward_norm_gate(d["q"], d["k"], d["v"], d["z"], d["A"], d["beta"], r_gate,
+                                  norm_weight=w_gain, eps=1e-6, num_seqs=B, chunk=CHUNK, o=o,
+                                  S_final=Sf, workspace=ws, stream=stream)
+
+        def fwd_ckpt():
+            kda.forward_checkpoints(d["q"], d["k"], d["v"], d["z"], d["A"], d["beta"], interval,
+                                    num_seqs=B, chunk=CHUNK, o=o, S_final=Sf, S_ckpt=ck,
+                                    workspace=ws, stream=stream)
+
+        out["variants"] = {}
+        n_var = max(3, min(args.steps, 20))
+        for name, fn, extra in (
+                ("norm_gate", fwd_norm_gate, T * H * D * 2 + D * 4),
+                ("checkpoints_every_%d" % interval, fwd_ckpt, ck.numel() * 4)):
+            for _ in range(args.warmup):
+                fn()
+            torch.cuda.synchronize()
+            barrier()
+            e0.record(stream)
+            for _ in range(n_var):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms_v = e0.elapsed_time(e1) / n_var
+            assert kda.check_device_error(ws) == kda.KDA_OK
+            ms_v = rank_max(ms_v)
+            out["variants"][name] = {
+                "ms_per_step": ms_v, "value": weak_scaling_value(T, world, ms_v),
+                "unit": "tokens/s", "steps": n_var, "extra_alg_bytes": extra,
+                "achieved_gbs": (fwd_bytes + extra) / (ms_v / 1e3) / 1e9}
         del ws
         torch.cuda.empty_cache()
 
@@ -349,6 +390,27 @@ def main():
         torch.cuda.synchronize()
         ms_dec_local = e0.elapsed_time(e1) / args.decode_steps
         ms_dec = rank_max(ms_dec_local)
+        # the decode step with the output epilogue fused in
+        r_dec, w_dec = synth.out_gate_inputs(DEC_B, H, D, seed=6)
+        r_dec, w_dec = r_dec.to(dev), w_dec.to(dev)
+
+        def dec_ng(s):
+            tk = pool[s % len(pool)]
+            kda.decode_step_norm_gate(tk["q"], tk["k"], tk["v"], tk["z"], A_dec, tk["beta"],
+                                      S_dec, r_dec, norm_weight=w_dec, eps=1e-6, o=o_dec,
+                                      stream=stream)
+
+        n_ng = max(10, args.decode_steps // 5)
+        for s in range(10):
+            dec_ng(s)
+        torch.cuda.synchronize()
+        barrier()
+        e0.record(stream)
+        for s in range(n_ng):
+            dec_ng(s)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms_ng = rank_max(e0.elapsed_time(e1) / n_ng)
         dec_bytes = alg_bytes_decode()
         dec_ach = dec_bytes / (ms_dec_local / 1e3) / 1e9
         out["decode"] = {
@@ -357,6 +419,8 @@ def main():
             "config": {"B": DEC_B, "H": H, "dk": D, "dv": D, "dtype": "bf16",
                        "state": "fp32 in place (268 MB, exceeds L2)"},
             "gpu_launches": args.decode_steps,
+            "norm_gate": {"ms_per_step": ms_ng, "steps": n_ng,
+                          "extra_alg_bytes": DEC_B * H * D * 2 + D * 4},
             "roofline": {"bound": "hbm", "achieved": dec_ach, "peak": pk["hbm"],
                          "unit": "GB/s", "frac": dec_ach / pk["hbm"],
                          "traffic": recorded_traffic("decode"),
@@ -388,6 +452,7 @@ def main():
                    "parallelism": f"weak x{world} (independent problems per rank)"},
         "roofline": out["roofline"], "cpu_baseline": cpu, "e2e": out["e2e"],
         "gpu_launches": out["launches"], "clocks": out["clocks"], "decode": out["decode"],
+        "variants": out["variants"],
     }), flush=True)
 
 

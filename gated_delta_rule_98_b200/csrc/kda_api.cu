@@ -50,6 +50,36 @@ kda_status check_forward(const void* q, const void* k, const void* v,
   return KDA_OK;
 }
 
+// Output-epilogue arguments: the gate input is required when there is work,
+// the gain is optional; both 16-byte aligned; eps finite and not negative.
+bool epilogue_ok(bool work, const void* out_gate, const float* norm_weight, float eps) {
+  if (!(eps >= 0.f && eps <= 3.0e38f)) return false;  // rejects NaN and infinities
+  if (work && !out_gate) return false;
+  return opt_aligned16(out_gate) && opt_aligned16(norm_weight);
+}
+
+kda_status decode_common(const void* q, const void* k, const void* v, const void* z,
+                         const float* A, const void* beta, float* S_inout, int32_t B,
+                         int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
+                         const void* out_gate, const float* norm_weight, float eps, void* o,
+                         kda_stream_t stream) {
+  if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_UNSUPPORTED;
+  if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  if (B < 0 || H < 1) return KDA_ERR_INVALID_ARG;
+  if ((int64_t)B * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+  if (B == 0) return KDA_OK;
+  if (!q || !k || !v || !z || !A || !beta || !S_inout || !o) return KDA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(z) ||
+      !aligned16(A) || !aligned16(beta) || !aligned16(S_inout) || !aligned16(o))
+    return KDA_ERR_INVALID_ARG;
+  kda::DecodeArgs a{q, k, v, z, beta, A, S_inout, o, B, H, dk, dv,
+                    dt == KDA_BF16, (cudaStream_t)stream};
+  a.out_gate = out_gate;
+  a.norm_w = norm_weight;
+  a.norm_eps = eps;
+  return kda::launch_decode(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 kda_status forward_common(kda::ForwardArgs& a) {
   if (a.N == 0) {
     // nothing to launch: still leave a clean error word for this call
@@ -167,23 +197,49 @@ kda_status kda_forward_checkpoints(const void* q, const void* k, const void* v,
   return forward_common(a);
 }
 
+kda_status kda_forward_norm_gate(const void* q, const void* k, const void* v,
+                                 const void* z, const float* A, const void* beta,
+                                 const float* S0, const int32_t* cu_seqlens,
+                                 int32_t num_seqs, int32_t total_tokens,
+                                 int32_t max_seqlen, int32_t H, int32_t dk, int32_t dv,
+                                 kda_dtype dt, int32_t chunk, const void* out_gate,
+                                 const float* norm_weight, float eps, void* o,
+                                 float* S_final, void* workspace, size_t workspace_bytes,
+                                 kda_stream_t stream) {
+  kda_status st = check_forward(q, k, v, z, beta, S0, cu_seqlens, num_seqs,
+                                total_tokens, max_seqlen, H, dk, dv, dt, chunk,
+                                o, S_final, workspace, workspace_bytes);
+  if (st != KDA_OK) return st;
+  if (total_tokens > 0 && (!A || !aligned16(A))) return KDA_ERR_INVALID_ARG;
+  if (!epilogue_ok(total_tokens > 0, out_gate, norm_weight, eps)) return KDA_ERR_INVALID_ARG;
+  kda::ForwardArgs a{q, k, v, z, beta, A, nullptr, S0, cu_seqlens, o, S_final,
+                     num_seqs, total_tokens, max_seqlen, H, dk, dv, chunk,
+                     dt == KDA_BF16, workspace, workspace_bytes,
+                     (cudaStream_t)stream};
+  a.out_gate = out_gate;
+  a.norm_w = norm_weight;
+  a.norm_eps = eps;
+  return forward_common(a);
+}
+
 kda_status kda_decode_step(const void* q, const void* k, const void* v,
                            const void* z, const float* A, const void* beta,
                            float* S_inout, int32_t B, int32_t H, int32_t dk,
                            int32_t dv, kda_dtype dt, void* o,
                            kda_stream_t stream) {
-  if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_UNSUPPORTED;
-  if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
-  if (B < 0 || H < 1) return KDA_ERR_INVALID_ARG;
-  if ((int64_t)B * H > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
-  if (B == 0) return KDA_OK;
-  if (!q || !k || !v || !z || !A || !beta || !S_inout || !o) return KDA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(z) ||
-      !aligned16(A) || !aligned16(beta) || !aligned16(S_inout) || !aligned16(o))
-    return KDA_ERR_INVALID_ARG;
-  kda::DecodeArgs a{q, k, v, z, beta, A, S_inout, o, B, H, dk, dv,
-                    dt == KDA_BF16, (cudaStream_t)stream};
-  return kda::launch_decode(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+  return decode_common(q, k, v, z, A, beta, S_inout, B, H, dk, dv, dt, nullptr, nullptr, 0.f, o,
+                       stream);
+}
+
+kda_status kda_decode_step_norm_gate(const void* q, const void* k, const void* v,
+                                     const void* z, const float* A, const void* beta,
+                                     float* S_inout, int32_t B, int32_t H, int32_t dk,
+                                     int32_t dv, kda_dtype dt, const void* out_gate,
+                                     const float* norm_weight, float eps, void* o,
+                                     kda_stream_t stream) {
+  if (!epilogue_ok(B > 0, out_gate, norm_weight, eps)) return KDA_ERR_INVALID_ARG;
+  return decode_common(q, k, v, z, A, beta, S_inout, B, H, dk, dv, dt, out_gate, norm_weight,
+                       eps, o, stream);
 }
 
 kda_status kda_check_device_error(const void* workspace, kda_stream_t stream) {

@@ -34,6 +34,9 @@ __device__ __forceinline__ float gate_logdecay(float z, float expA) {
   return kGateMin / (1.0f + expf(-expA * z));
 }
 
+// Output gate of the epilogue: sigmoid(x) = 1 / (1 + e^{-x}) (0 for x -> -inf).
+__device__ __forceinline__ float out_sigmoid(float x) { return 1.0f / (1.0f + __expf(-x)); }
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);

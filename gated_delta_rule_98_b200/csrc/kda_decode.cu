@@ -21,7 +21,8 @@ __global__ void __launch_bounds__(256)
 decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k,
                    const T* __restrict__ v, const T* __restrict__ z,
                    const float* __restrict__ A, const T* __restrict__ beta,
-                   float* __restrict__ S, int H, T* __restrict__ o) {
+                   float* __restrict__ S, int H, T* __restrict__ o,
+                   const T* __restrict__ og, const float* __restrict__ ow, float oeps) {
   constexpr int NT = 256;
   constexpr int CG = DV / 4;   // float4 column groups per state row
   constexpr int RG = NT / CG;  // row groups
@@ -32,6 +33,7 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k,
   __shared__ __align__(16) float s_p[RG][DV + 4], s_r[RG][DV + 4];
   __shared__ __align__(16) float s_u[DV];
   __shared__ float s_scal[4];
+  __shared__ float s_ss[DV / 32];
 
   const int bh = blockIdx.x;
   const int h = bh % H;
@@ -87,17 +89,34 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k,
   *reinterpret_cast<float4*>(&s_r[rg][4 * cg]) = r;
   __syncthreads();
   const float b = to_f(beta[bh]);
-  for (int j = tid; j < DV; j += NT) {
+  static_assert(DV <= NT, "one output feature per thread");
+  float oj = 0.f;
+  if (tid < DV) {
     float pj = 0.f, rj = 0.f;
 #pragma unroll
     for (int g2 = 0; g2 < RG; ++g2) {
-      pj += s_p[g2][j];
-      rj += s_r[g2][j];
+      pj += s_p[g2][tid];
+      rj += s_r[g2][tid];
     }
-    const float u = b * (s_v[j] - pj);
-    s_u[j] = u;
-    o[(size_t)bh * DV + j] = from_f<T>(rj + kq * u);
+    const float u = b * (s_v[tid] - pj);
+    s_u[tid] = u;
+    oj = rj + kq * u;
   }
+  if (og) {
+    // output epilogue (Kimi Linear summary, §4): head-wise RMSNorm over the DV
+    // outputs, gain, sigmoid gate; the sum of squares is reduced over the DV / 32 warps
+    const float ss = warp_sum(oj * oj);  // zero beyond DV
+    if (tid < DV && (tid & 31) == 0) s_ss[tid >> 5] = ss;
+    __syncthreads();
+    if (tid < DV) {
+      float tot = 0.f;
+#pragma unroll
+      for (int w = 0; w < DV / 32; ++w) tot += s_ss[w];
+      const float wj = ow ? ow[tid] : 1.f;
+      oj = oj * rsqrtf(tot * (1.0f / DV) + oeps) * wj * out_sigmoid(to_f(og[(size_t)bh * DV + tid]));
+    }
+  }
+  if (tid < DV) o[(size_t)bh * DV + tid] = from_f<T>(oj);
   __syncthreads();
   const float4 u4 = *reinterpret_cast<const float4*>(&s_u[4 * cg]);
 #pragma unroll
@@ -114,7 +133,7 @@ template <int DK, int DV, typename T>
 static cudaError_t launch_decode_t(const DecodeArgs& a) {
   decode_step_kernel<DK, DV, T><<<a.B * a.H, 256, 0, a.stream>>>(
       (const T*)a.q, (const T*)a.k, (const T*)a.v, (const T*)a.z, a.A,
-      (const T*)a.beta, a.S, a.H, (T*)a.o);
+      (const T*)a.beta, a.S, a.H, (T*)a.o, (const T*)a.out_gate, a.norm_w, a.norm_eps);
   return cudaGetLastError();
 }
 

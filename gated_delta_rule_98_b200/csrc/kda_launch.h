@@ -16,6 +16,9 @@ struct DecodeArgs {
   int B, H, dk, dv;
   bool bf16;
   cudaStream_t stream;
+  const void* out_gate = nullptr;  // [B, H, dv] sigmoid output-gate input (input dtype), or null
+  const float* norm_w = nullptr;   // [dv] RMSNorm gain, or null (ones)
+  float norm_eps = 0.f;
 };
 
 struct ForwardArgs {
@@ -34,6 +37,10 @@ struct ForwardArgs {
   float* S_ckpt = nullptr;  // [N, H, ckpt_count, dk, dv] states every ckpt_every chunks, or null
   int ckpt_every = 0;       // chunks between checkpoints
   int ckpt_count = 0;       // checkpoints per (sequence, head): max_len / interval
+  // Output epilogue (head-wise RMSNorm over dv, gain, sigmoid gate) on o, when out_gate is set.
+  const void* out_gate = nullptr;  // [T, H, dv] gate input (input dtype)
+  const float* norm_w = nullptr;   // [dv] gain, or null (ones)
+  float norm_eps = 0.f;
 };
 
 cudaError_t launch_decode(const DecodeArgs& a);

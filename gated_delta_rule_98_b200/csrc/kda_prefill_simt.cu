@@ -57,6 +57,9 @@ struct SimtParams {
   float* S_final;
   float* S_ckpt;  // checkpoints every ckpt_every chunks (ckpt_count per sequence and head)
   int ckpt_every, ckpt_count;
+  const void* og;  // output epilogue: sigmoid gate input [T, H, DV] (input dtype), or null
+  const float* ow;  // RMSNorm gain [DV], or null (ones)
+  float oeps;
   int N, T, max_len, H, max_cps;
   float *W, *Ut, *Qp, *Kp, *Aqk, *gam;
   WsHeader* hdr;
@@ -334,6 +337,35 @@ __global__ void __launch_bounds__(256) simt_state_kernel(SimtParams p) {
     }
 }
 
+// Output epilogue (Kimi Linear summary, §4: head-wise RMSNorm of o, then a
+// data-dependent sigmoid gate), in place on o after the state pass.  The state
+// kernel splits a head's DV features over DV / 32 CTAs, so the row reduction
+// runs here: one warp per (token, head) row of DV features.
+template <int DV, typename T>
+__global__ void __launch_bounds__(256) simt_norm_gate_kernel(SimtParams p) {
+  constexpr int PER = DV / 32;
+  if (p.hdr->err != kErrNone) return;  // invalid cu_seqlens: o was not written
+  const int lane = threadIdx.x & 31;
+  const size_t row = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= (size_t)p.T * p.H) return;
+  T* o = (T*)p.o + row * DV;
+  const T* r = (const T*)p.og + row * DV;
+  float x[PER], ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    x[i] = to_f(o[lane + 32 * i]);
+    ss += x[i] * x[i];
+  }
+  ss = warp_sum(ss);
+  const float inv = rsqrtf(ss * (1.0f / DV) + p.oeps);
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int j = lane + 32 * i;
+    const float w = p.ow ? p.ow[j] : 1.f;
+    o[j] = from_f<T>(x[i] * inv * w * out_sigmoid(to_f(r[j])));
+  }
+}
+
 template <int DK, int DV, int C, typename T>
 cudaError_t launch_t(const ForwardArgs& a, const SimtParams& p) {
   cudaError_t err;
@@ -353,6 +385,11 @@ cudaError_t launch_t(const ForwardArgs& a, const SimtParams& p) {
     if (err != cudaSuccess) return err;
     dim3 grid(a.N, a.H, DV / kBV);
     simt_state_kernel<DK, DV, C, T><<<grid, 256, smem, a.stream>>>(p);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
+  if (p.og && a.T > 0) {
+    const unsigned rows = (unsigned)((size_t)a.T * a.H);
+    simt_norm_gate_kernel<DV, T><<<(rows + 7) / 8, 256, 0, a.stream>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
   return cudaSuccess;
@@ -394,6 +431,7 @@ cudaError_t launch_forward_simt(const ForwardArgs& a) {
   p.q = a.q; p.k = a.k; p.v = a.v; p.z = a.z; p.beta = a.beta;
   p.A = a.A; p.g = a.g; p.S0 = a.S0; p.cu = a.cu; p.o = a.o; p.S_final = a.S_final;
   p.S_ckpt = a.S_ckpt; p.ckpt_every = a.ckpt_every; p.ckpt_count = a.ckpt_count;
+  p.og = a.out_gate; p.ow = a.norm_w; p.oeps = a.norm_eps;
   p.N = a.N; p.T = a.T; p.max_len = a.max_len; p.H = a.H;
   p.max_cps = (a.max_len + a.chunk - 1) / a.chunk;
   p.W = (float*)(base + L.W);

@@ -126,6 +126,17 @@ __device__ __forceinline__ uint4 pack8(const float* v) {
   u.w = *reinterpret_cast<uint32_t*>(&d);
   return u;
 }
+// 8 bf16 (one 16-byte vector) -> fp32, exactly
+__device__ __forceinline__ void unpack8(const uint4 u, float* f) {
+  f[0] = __uint_as_float(u.x << 16); f[1] = __uint_as_float(u.x & 0xffff0000u);
+  f[2] = __uint_as_float(u.y << 16); f[3] = __uint_as_float(u.y & 0xffff0000u);
+  f[4] = __uint_as_float(u.z << 16); f[5] = __uint_as_float(u.z & 0xffff0000u);
+  f[6] = __uint_as_float(u.w << 16); f[7] = __uint_as_float(u.w & 0xffff0000u);
+}
+__device__ __forceinline__ void ld8f(const float* p, float* f) {  // 8 fp32, 16-byte aligned
+  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
 __device__ __forceinline__ void st16(unsigned char* base, uint32_t off, const float* v) {
   *reinterpret_cast<uint4*>(base + off) = pack8(v);
 }
@@ -161,6 +172,9 @@ struct alignas(64) TcParams {
   float* S_final;
   float* S_ckpt;  // checkpoints every ckpt_every chunks (ckpt_count per sequence and head)
   int ckpt_every, ckpt_count;
+  const __nv_bfloat16* og;  // output epilogue: sigmoid gate input [T, H, 128], or null (no epilogue)
+  const float* ow;          // RMSNorm gain [128], or null (ones)
+  float oeps;
   int N, T, max_len, H, P;
   float* seg;  // per (n, h): transitions (M, N) of segments 0..P-2, incoming states of 0..P-1
   unsigned char* prep;  // per (chunk slot, h): chain operands left by the transition pass
@@ -172,6 +186,29 @@ struct alignas(64) TcParams {
 __device__ __forceinline__ float* ckpt_state(const TcParams& p, int n, int h, int c, int n_tok) {
   if (!p.S_ckpt || (c + 1) % p.ckpt_every != 0 || (c + 1) * 64 > n_tok) return nullptr;
   return p.S_ckpt + (((size_t)n * p.H + h) * p.ckpt_count + (c + 1) / p.ckpt_every - 1) * 128 * 128;
+}
+
+// Output epilogue (Kimi Linear summary, §4: head-wise RMSNorm of o, then a
+// data-dependent sigmoid gate) on x[0..NX) of one token's 128 features, given
+// the sum of squares over all 128: x * rsqrt(mean + eps) * w * sigmoid(r).
+// r: the gate input at the same features (16-byte aligned); w: the gain or null.
+template <int NX>
+__device__ __forceinline__ void norm_gate(float* x, float sumsq, const __nv_bfloat16* r,
+                                          const float* w, float eps) {
+  const float inv = rsqrtf(sumsq * (1.0f / 128) + eps);
+#pragma unroll
+  for (int i = 0; i < NX; i += 8) {
+    float rv[8], wv[8];
+    unpack8(*reinterpret_cast<const uint4*>(r + i), rv);
+    if (w) {
+      ld8f(w + i, wv);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) wv[e] = 1.f;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[i + e] = x[i + e] * inv * wv[e] * out_sigmoid(rv[e]);
+  }
 }
 
 // Segment p of a sequence with nch chunks: chunks [c0, c1).
@@ -694,11 +731,30 @@ __global__ void __launch_bounds__(kNT, 1) fused_kernel(const __grid_constant__ T
       tmem_ld16(tmem_addr(tm, 32 * q4, kTmQ + col), o0);
       tmem_ld16(tmem_addr(tm, 32 * q4, kTmQ + col + 16), o1);
       tmem_ld_wait();
-      if (m64 && r64 < len) {
+      const size_t orow = ((size_t)(tok0 + r64) * H + h) * kD;
+      if (m64) {
         const float iq = vec[kVecIq + r64];
 #pragma unroll
         for (int i = 0; i < 16; ++i) { o0[i] *= iq; o1[i] *= iq; }
-        uint4* dst = reinterpret_cast<uint4*>(p.o + ((size_t)(tok0 + r64) * H + h) * kD + col);
+      }
+      if (p.og) {
+        // output epilogue: a token's 128 features lie in the four column quarters
+        float* red = vec + kVecY;  // [4 quarters][64 tokens] partial sums of squares
+        if (m64) {
+          float ss = 0.f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) ss += o0[i] * o0[i] + o1[i] * o1[i];
+          red[cq * 64 + r64] = ss;
+        }
+        __syncthreads();
+        if (m64 && r64 < len) {
+          const float ss = red[r64] + red[64 + r64] + red[128 + r64] + red[192 + r64];
+          norm_gate<16>(o0, ss, p.og + orow + col, p.ow ? p.ow + col : nullptr, p.oeps);
+          norm_gate<16>(o1, ss, p.og + orow + col + 16, p.ow ? p.ow + col + 16 : nullptr, p.oeps);
+        }
+      }
+      if (m64 && r64 < len) {
+        uint4* dst = reinterpret_cast<uint4*>(p.o + orow + col);
         dst[0] = pack8(o0);
         dst[1] = pack8(o0 + 8);
         dst[2] = pack8(o1);
@@ -808,17 +864,6 @@ __device__ __forceinline__ bool group_wait(uint64_t* bar, uint32_t& phase, WsHea
   return true;
 }
 
-// 8 bf16 (one 16-byte vector) -> fp32, exactly
-__device__ __forceinline__ void unpack8(const uint4 u, float* f) {
-  f[0] = __uint_as_float(u.x << 16); f[1] = __uint_as_float(u.x & 0xffff0000u);
-  f[2] = __uint_as_float(u.y << 16); f[3] = __uint_as_float(u.y & 0xffff0000u);
-  f[4] = __uint_as_float(u.z << 16); f[5] = __uint_as_float(u.z & 0xffff0000u);
-  f[6] = __uint_as_float(u.w << 16); f[7] = __uint_as_float(u.w & 0xffff0000u);
-}
-__device__ __forceinline__ void ld8f(const float* p, float* f) {  // 8 fp32, 16-byte aligned
-  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
-  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-}
 __device__ __forceinline__ void st8f(float* p, const float* f) {
   *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
   *reinterpret_cast<float4*>(p + 4) = make_float4(f[4], f[5], f[6], f[7]);
@@ -1448,11 +1493,24 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
   };
   auto write_o = [&](int cc) {  // staging -> o rows of chunk cc (after a barrier)
     const int t0c = a + cc * kC, lenc = min(kC, b - t0c);
-    for (int u = tid; u < kC * kD / 8; u += kNT) {
+    for (int u = tid; u < kC * kD / 8; u += kNT) {  // 16 lanes per token, 8 features each
       const int t = u >> 4, d8 = (u & 15) * 8;
-      if (t < lenc)
-        *reinterpret_cast<uint4*>(p.o + ((size_t)(t0c + t) * H + h) * kD + d8) =
-            *reinterpret_cast<const uint4*>(ost + t * kD + d8);
+      const size_t off = ((size_t)(t0c + t) * H + h) * kD + d8;
+      uint4 w8 = *reinterpret_cast<const uint4*>(ost + t * kD + d8);
+      if (p.og) {  // output epilogue (uniform branch: every lane takes part in the sums)
+        float x[8];
+        unpack8(w8, x);
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss += x[e] * x[e];
+#pragma unroll
+        for (int m = 8; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+        if (t < lenc) {
+          norm_gate<8>(x, ss, p.og + off, p.ow ? p.ow + d8 : nullptr, p.oeps);
+          w8 = pack8(x);
+        }
+      }
+      if (t < lenc) *reinterpret_cast<uint4*>(p.o + off) = w8;
     }
   };
 
@@ -1810,6 +1868,9 @@ cudaError_t launch_forward_tc(const ForwardArgs& a) {
   p.S_ckpt = a.S_ckpt;
   p.ckpt_every = a.ckpt_every;
   p.ckpt_count = a.ckpt_count;
+  p.og = (const __nv_bfloat16*)a.out_gate;
+  p.ow = a.norm_w;
+  p.oeps = a.norm_eps;
   p.N = a.N;
   p.T = a.T;
   p.max_len = a.max_len;

@@ -27,7 +27,7 @@ KDA_F32, KDA_BF16 = 0, 1
 EXPORTS = ("kda_status_string", "kda_version", "kda_forward_workspace_size",
            "kda_forward_launches", "kda_forward",
            "kda_forward_g", "kda_decode_step", "kda_forward_noalloc", "kda_forward_checkpoints",
-           "kda_check_device_error")
+           "kda_forward_norm_gate", "kda_decode_step_norm_gate", "kda_check_device_error")
 
 # Bytes of the library's fixed scratch array used by kda_forward_noalloc.
 KDA_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -70,6 +70,12 @@ def lib():
     L.kda_forward_checkpoints.argtypes = ([vp] * 8 + [i32] * 6 + [ctypes.c_int, i32, vp, vp, vp,
                                           i32, vp, sz, vp])
     L.kda_forward_checkpoints.restype = ctypes.c_int
+    L.kda_forward_norm_gate.argtypes = ([vp] * 8 + [i32] * 6 + [ctypes.c_int, i32, vp, vp,
+                                        ctypes.c_float, vp, vp, vp, sz, vp])
+    L.kda_forward_norm_gate.restype = ctypes.c_int
+    L.kda_decode_step_norm_gate.argtypes = ([vp] * 7 + [i32] * 4 + [ctypes.c_int, vp, vp,
+                                            ctypes.c_float, vp, vp])
+    L.kda_decode_step_norm_gate.restype = ctypes.c_int
     L.kda_check_device_error.argtypes = [vp, vp]
     L.kda_check_device_error.restype = ctypes.c_int
     _lib = L
@@ -125,6 +131,21 @@ def kda_forward_checkpoints(q, k, v, z, A, beta, S0, cu_seqlens, num_seqs, total
                                          total_tokens, max_seqlen, H, dk, dv, dt, chunk, o,
                                          S_final, S_ckpt, interval, workspace, workspace_bytes,
                                          stream)
+
+
+def kda_forward_norm_gate(q, k, v, z, A, beta, S0, cu_seqlens, num_seqs, total_tokens,
+                          max_seqlen, H, dk, dv, dt, chunk, out_gate, norm_weight, eps, o,
+                          S_final, workspace, workspace_bytes, stream):
+    return lib().kda_forward_norm_gate(q, k, v, z, A, beta, S0, cu_seqlens, num_seqs,
+                                       total_tokens, max_seqlen, H, dk, dv, dt, chunk, out_gate,
+                                       norm_weight, eps, o, S_final, workspace, workspace_bytes,
+                                       stream)
+
+
+def kda_decode_step_norm_gate(q, k, v, z, A, beta, S_inout, B, H, dk, dv, dt, out_gate,
+                              norm_weight, eps, o, stream):
+    return lib().kda_decode_step_norm_gate(q, k, v, z, A, beta, S_inout, B, H, dk, dv, dt,
+                                           out_gate, norm_weight, eps, o, stream)
 
 
 def kda_check_device_error(workspace, stream):
@@ -264,6 +285,47 @@ def decode_step(q, k, v, z, A, beta, S, *, o=None, stream=None):
                          _dt(q), _p(o), _stream(stream))
     if st != KDA_OK:
         raise KdaError(st, "kda_decode_step")
+    return o
+
+
+def forward_norm_gate(q, k, v, z, A, beta, out_gate, *, norm_weight=None, eps=1e-6, S0=None,
+                      cu_seqlens=None, num_seqs=None, max_seqlen=None, chunk=64, o=None,
+                      S_final=None, workspace=None, stream=None):
+    """KDA prefill followed by the output epilogue: o = RMSNorm(attention output
+    over dv) * norm_weight * sigmoid(out_gate), out_gate [T,H,dv] in q's dtype,
+    norm_weight [dv] fp32 or None.  Returns (o, S_final)."""
+    _check_cuda(q, k, v, z, A, beta, out_gate, norm_weight, S0, cu_seqlens, o, S_final,
+                workspace)
+    T, H, dk, dv, N, max_len = _geometry(q, v, cu_seqlens, num_seqs, max_seqlen)
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
+    if S_final is None:
+        S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    ws = workspace if workspace is not None else _new_workspace(N, T, max_len, H, dk, dv,
+                                                                q.dtype, chunk, device=q.device)
+    st = kda_forward_norm_gate(_p(q), _p(k), _p(v), _p(z), _p(A), _p(beta), _p(S0),
+                               _p(cu_seqlens), N, T, max_len, H, dk, dv, _dt(q), chunk,
+                               _p(out_gate), _p(norm_weight), float(eps), _p(o), _p(S_final),
+                               _p(ws), ws.numel(), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_forward_norm_gate")
+    return o, S_final
+
+
+def decode_step_norm_gate(q, k, v, z, A, beta, S, out_gate, *, norm_weight=None, eps=1e-6,
+                          o=None, stream=None):
+    """decode_step followed by the output epilogue (see forward_norm_gate);
+    out_gate [B,H,dv].  S is updated in place.  Returns o [B,H,dv]."""
+    _check_cuda(q, k, v, z, A, beta, S, out_gate, norm_weight, o)
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    st = kda_decode_step_norm_gate(_p(q), _p(k), _p(v), _p(z), _p(A), _p(beta), _p(S), B, H, dk,
+                                   dv, _dt(q), _p(out_gate), _p(norm_weight), float(eps), _p(o),
+                                   _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_decode_step_norm_gate")
     return o
 
 

@@ -15,6 +15,10 @@ Recipe (numpy ``default_rng(seed)``, PCG64, draws in float64 in this order):
   S0 ~ N(0, s0_std^2) [N,H,dk,dv]     (kept fp32; omitted when s0_std is None)
 q, k, v, z, beta are then rounded to the compute dtype (round-to-nearest-even).
 
+Output epilogue inputs (``out_gate_inputs``, numpy ``default_rng(seed)``):
+  r ~ N(0,1) [T,H,dv]                 (gate logits; rounded to the compute dtype)
+  w ~ U(0.5, 1.5) [dv]                (RMSNorm gain, fp32)
+
 Workloads (sizes follow the operator's published benchmark settings):
   tiny      B=1 H=2  L=64    d=32  fp32 chunk 16  S0=0           seed 0
   bf16      B=1 H=16 L=4096  d=128 bf16 chunk 64  S0=0           seed 1
@@ -67,6 +71,15 @@ def draw(T, H, dk, dv, *, seed, dtype="bf16", num_seqs=1, s0_std=None, rng=None)
     else:
         out["S0"] = None
     return out
+
+
+def out_gate_inputs(T, H, dv, *, seed, dtype="bf16"):
+    """Gate input r [T,H,dv] (compute dtype) and gain w [dv] (fp32) for the
+    output epilogue, drawn in that order."""
+    rng = np.random.default_rng(seed)
+    r = _cast(rng.standard_normal((T, H, dv)), torch_dtype(dtype))
+    w = torch.from_numpy(rng.uniform(0.5, 1.5, dv)).float()
+    return r, w
 
 
 def varlen_lengths(total=32768, lo=512, hi=8192, seed=3):

@@ -172,6 +172,41 @@ kda_status kda_forward_checkpoints(const void* q, const void* k, const void* v,
                                    kda_stream_t stream);
 
 /*
+ * kda_forward followed by the layer's output epilogue, fused into the kernels
+ * that write o (Kimi Linear summary, §4 "The Kimi Linear Model Architecture":
+ * head-wise RMSNorm of the output, then a data-dependent sigmoid gate; §5.2:
+ * the gate is a sigmoid, not Swish).  For every token t and head h, over the
+ * head's dv features j:
+ *
+ *   o[t,h,j] = a[t,h,j] / sqrt(mean_j' a[t,h,j']^2 + eps) * w[j] * sigmoid(r[t,h,j])
+ *
+ * where a is the attention output kda_forward would write.  The output
+ * projection that follows in the layer is not part of this call.
+ *
+ *  out_gate    : r, [T, H, dv] in `dt`, the gate input (the layer's low-rank
+ *                projection of its input, computed by the caller).  Required
+ *                when total_tokens > 0; must not overlap o.
+ *  norm_weight : w, [dv] float32, the RMSNorm gain shared by the heads, or
+ *                NULL for ones.  The pages name no gain; this one is optional.
+ *  eps         : added to the mean square, finite and >= 0 (else
+ *                KDA_ERR_INVALID_ARG); the pages give no value.
+ * On the tensor-core path the epilogue runs in the kernels that write o, from
+ * the fp32 (fused unsegmented kernel) or bf16-staged (segmented full pass)
+ * attention output; on the CUDA-core path it is one extra launch after the
+ * state pass (kda_forward_launches + 1), since that pass splits a head's dv
+ * features over several blocks.  Everything else is kda_forward's.
+ */
+kda_status kda_forward_norm_gate(const void* q, const void* k, const void* v,
+                                 const void* z, const float* A, const void* beta,
+                                 const float* S0, const int32_t* cu_seqlens,
+                                 int32_t num_seqs, int32_t total_tokens,
+                                 int32_t max_seqlen, int32_t H, int32_t dk, int32_t dv,
+                                 kda_dtype dt, int32_t chunk, const void* out_gate,
+                                 const float* norm_weight, float eps, void* o,
+                                 float* S_final, void* workspace, size_t workspace_bytes,
+                                 kda_stream_t stream);
+
+/*
  * One recurrent KDA step for B independent sequences (one token each),
  * updating the float32 states in place (Kimi Linear summary §6.3: token
  * generation uses the recurrent update).
@@ -187,6 +222,22 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v,
                            float* S_inout, int32_t B, int32_t H, int32_t dk,
                            int32_t dv, kda_dtype dt, void* o,
                            kda_stream_t stream);
+
+/*
+ * kda_decode_step with the output epilogue of kda_forward_norm_gate fused
+ * into the step: o[b,h,:] is the RMS-normalised attention output times the
+ * gain times sigmoid(out_gate[b,h,:]).
+ *
+ *  out_gate    : [B, H, dv] in `dt`; required when B > 0.
+ *  norm_weight : [dv] float32 or NULL (ones).   eps : finite, >= 0.
+ * Everything else is kda_decode_step's.
+ */
+kda_status kda_decode_step_norm_gate(const void* q, const void* k, const void* v,
+                                     const void* z, const float* A, const void* beta,
+                                     float* S_inout, int32_t B, int32_t H, int32_t dk,
+                                     int32_t dv, kda_dtype dt, const void* out_gate,
+                                     const float* norm_weight, float eps, void* o,
+                                     kda_stream_t stream);
 
 /*
  * kda_forward without a caller-provided workspace, for callers that cannot

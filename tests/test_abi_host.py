@@ -142,3 +142,24 @@ def test_checkpoints_reject_bad_interval_and_buffer(L):
     assert ck(S_ckpt=None) == kda.KDA_ERR_INVALID_ARG          # 2 checkpoints need a buffer
     assert ck(S_ckpt=FAKE + 4) == kda.KDA_ERR_INVALID_ARG      # misaligned
     assert ck(chunk=32) == kda.KDA_ERR_UNSUPPORTED
+
+
+def test_norm_gate_rejects_bad_epilogue_arguments(L):
+    def fw(gate=FAKE, w=None, eps=1e-6, T=128):
+        return kda.kda_forward_norm_gate(
+            FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 1, T, T, 2, 32, 32,
+            kda.KDA_F32, 16, gate, w, eps, FAKE, FAKE, FAKE, 1 << 40, None)
+    assert fw(gate=None) == kda.KDA_ERR_INVALID_ARG             # gate input required
+    assert fw(gate=FAKE + 8) == kda.KDA_ERR_INVALID_ARG         # misaligned
+    assert fw(w=FAKE + 4) == kda.KDA_ERR_INVALID_ARG
+    assert fw(eps=-1e-6) == kda.KDA_ERR_INVALID_ARG
+    assert fw(eps=float("nan")) == kda.KDA_ERR_INVALID_ARG
+    assert fw(eps=float("inf")) == kda.KDA_ERR_INVALID_ARG
+
+    def dec(gate=FAKE, eps=1e-6, B=4, dk=32):
+        return kda.kda_decode_step_norm_gate(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, B, 2, dk,
+                                             32, kda.KDA_F32, gate, None, eps, FAKE, None)
+    assert dec(gate=None) == kda.KDA_ERR_INVALID_ARG
+    assert dec(eps=float("nan")) == kda.KDA_ERR_INVALID_ARG
+    assert dec(dk=48) == kda.KDA_ERR_UNSUPPORTED
+    assert dec(gate=None, B=0) == kda.KDA_OK                    # nothing to do
