@@ -168,6 +168,25 @@ kda_status kda_forward_g(const void* q, const void* k, const void* v,
   return forward_common(a);
 }
 
+kda_status kda_forward_scalar_gate(const void* q, const void* k, const void* v,
+                                   const float* g_head, const void* beta, const float* S0,
+                                   const int32_t* cu_seqlens, int32_t num_seqs,
+                                   int32_t total_tokens, int32_t max_seqlen, int32_t H,
+                                   int32_t dk, int32_t dv, kda_dtype dt, int32_t chunk,
+                                   void* o, float* S_final, void* workspace,
+                                   size_t workspace_bytes, kda_stream_t stream) {
+  kda_status st = check_forward(q, k, v, g_head, beta, S0, cu_seqlens, num_seqs,
+                                total_tokens, max_seqlen, H, dk, dv, dt, chunk,
+                                o, S_final, workspace, workspace_bytes);
+  if (st != KDA_OK) return st;
+  kda::ForwardArgs a{q, k, v, nullptr, beta, nullptr, nullptr, S0, cu_seqlens, o,
+                     S_final, num_seqs, total_tokens, max_seqlen, H, dk, dv,
+                     chunk, dt == KDA_BF16, workspace, workspace_bytes,
+                     (cudaStream_t)stream};
+  a.g_head = g_head;
+  return forward_common(a);
+}
+
 kda_status kda_forward_checkpoints(const void* q, const void* k, const void* v,
                                    const void* z, const float* A, const void* beta,
                                    const float* S0, const int32_t* cu_seqlens,

@@ -41,6 +41,9 @@ struct ForwardArgs {
   const void* out_gate = nullptr;  // [T, H, dv] gate input (input dtype)
   const float* norm_w = nullptr;   // [dv] gain, or null (ones)
   float norm_eps = 0.f;
+  // Scalar gate (Gated DeltaNet): [T, H] fp32 log-decay shared by a head's dk
+  // channels, instead of z, A and g.
+  const float* g_head = nullptr;
 };
 
 cudaError_t launch_decode(const DecodeArgs& a);

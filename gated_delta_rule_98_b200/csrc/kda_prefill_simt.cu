@@ -52,6 +52,7 @@ SimtLayout simt_layout(int N, int T, int H, int dk, int dv, int C) {
 struct SimtParams {
   const void *q, *k, *v, *z, *beta;
   const float *A, *g, *S0;
+  const float* gs;  // scalar log-decay [T, H] (one per token and head), or null
   const int32_t* cu;
   void* o;
   float* S_final;
@@ -106,7 +107,7 @@ __global__ void __launch_bounds__(256) simt_prep_kernel(SimtParams p) {
   const T* vg = (const T*)p.v;
   const T* zg = (const T*)p.z;
   const T* bg = (const T*)p.beta;
-  const float expA = p.g ? 0.f : expf(p.A[h]);
+  const float expA = p.z ? expf(p.A[h]) : 0.f;
 
   // ---- load (rows past the chunk end are zero: q = k = v = 0, g = 0, beta = 0)
   for (int e = tid; e < C * DK; e += NT) {
@@ -116,7 +117,9 @@ __global__ void __launch_bounds__(256) simt_prep_kernel(SimtParams p) {
       const size_t idx = ((size_t)(tok0 + r) * H + h) * DK + c;
       qv = to_f(qg[idx]);
       kv = to_f(kg[idx]);
-      gv = p.g ? p.g[idx] : gate_logdecay(to_f(zg[idx]), expA);
+      gv = p.g    ? p.g[idx]
+           : p.gs ? p.gs[(size_t)(tok0 + r) * H + h]
+                  : gate_logdecay(to_f(zg[idx]), expA);
     }
     qh[r * LK + c] = qv;
     kh[r * LK + c] = kv;
@@ -429,7 +432,7 @@ cudaError_t launch_forward_simt(const ForwardArgs& a) {
   char* base = (char*)a.ws;
   SimtParams p;
   p.q = a.q; p.k = a.k; p.v = a.v; p.z = a.z; p.beta = a.beta;
-  p.A = a.A; p.g = a.g; p.S0 = a.S0; p.cu = a.cu; p.o = a.o; p.S_final = a.S_final;
+  p.A = a.A; p.g = a.g; p.gs = a.g_head; p.S0 = a.S0; p.cu = a.cu; p.o = a.o; p.S_final = a.S_final;
   p.S_ckpt = a.S_ckpt; p.ckpt_every = a.ckpt_every; p.ckpt_count = a.ckpt_count;
   p.og = a.out_gate; p.ow = a.norm_w; p.oeps = a.norm_eps;
   p.N = a.N; p.T = a.T; p.max_len = a.max_len; p.H = a.H;

@@ -167,6 +167,7 @@ struct alignas(64) TcParams {
   CUtensorMap sq, sk, sz, sv;  // the same, box 64 tokens x 1 x 64 channels, 128-byte swizzle
   const __nv_bfloat16 *q, *k, *beta, *z, *v;
   const float *A, *g, *S0;
+  const float* gs;  // scalar log-decay [T, H] (one per token and head), or null
   const int32_t* cu;
   __nv_bfloat16* o;
   float* S_final;
@@ -247,13 +248,14 @@ __device__ __forceinline__ void tma_box_x(void* dst, const CUtensorMap* map, int
       : "memory");
 }
 
-// q, k, z, v rows of the chunk starting at tok0 (single thread).
+// q, k, z, v rows of the chunk starting at tok0 (single thread); z only when
+// the gate is computed from it.
 __device__ __forceinline__ void stage_chunk(const TcParams& p, unsigned char* raw, uint64_t* bar,
                                             int tok0, int h) {
-  mbar_arrive_expect_tx(bar, 4 * 16384);
+  mbar_arrive_expect_tx(bar, (p.z ? 4 : 3) * 16384);
   tma_box(raw + 0 * 16384, &p.tq, h, tok0, bar);
   tma_box(raw + 1 * 16384, &p.tk, h, tok0, bar);
-  tma_box(raw + 2 * 16384, &p.tz, h, tok0, bar);
+  if (p.z) tma_box(raw + 2 * 16384, &p.tz, h, tok0, bar);
   tma_box(raw + 3 * 16384, &p.tv, h, tok0, bar);
 }
 
@@ -360,7 +362,7 @@ __global__ void __launch_bounds__(kNT, 1) fused_kernel(const __grid_constant__ T
     tmem_st_wait();
   }
 
-  const float expA = p.g ? 0.f : expf(p.A[h]);
+  const float expA = p.z ? expf(p.A[h]) : 0.f;
   // prep ownership: channel j, row sub-tile qq (rows 16qq .. 16qq+15)
   const int j = tid & 127, qq = tid >> 7;
   // C_b window of row sub-tile b starts at row 8 b (b + 1) of C: 0, 16, 48, 96
@@ -414,6 +416,12 @@ __global__ void __launch_bounds__(kNT, 1) fused_kernel(const __grid_constant__ T
         for (int i = 0; i < 16; ++i) {
           const int r = 16 * qq + i;
           E[i] = r < len ? p.g[((size_t)(tok0 + r) * H + h) * kD + j] : 0.f;
+        }
+      } else if (p.gs) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int r = 16 * qq + i;
+          E[i] = r < len ? p.gs[(size_t)(tok0 + r) * H + h] : 0.f;
         }
       } else {
 #pragma unroll
@@ -946,13 +954,15 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
   };
   // q, k, z, v rows of an item -> the staging tile (two 64-channel boxes each)
   auto stage = [&](int tok, int hh) {
-    mbar_arrive_expect_tx(bar_raw, 4 * 16384);
+    mbar_arrive_expect_tx(bar_raw, (p.z ? 4 : 3) * 16384);
     tma_box_x(sm + L::kRaw, &p.sq, 0, hh, tok, bar_raw);
     tma_box_x(sm + L::kRaw + 8192, &p.sq, 64, hh, tok, bar_raw);
     tma_box_x(sm + L::kRaw + 16384, &p.sk, 0, hh, tok, bar_raw);
     tma_box_x(sm + L::kRaw + 24576, &p.sk, 64, hh, tok, bar_raw);
-    tma_box_x(sm + L::kRaw + 32768, &p.sz, 0, hh, tok, bar_raw);
-    tma_box_x(sm + L::kRaw + 40960, &p.sz, 64, hh, tok, bar_raw);
+    if (p.z) {  // z only when the gate is computed from it
+      tma_box_x(sm + L::kRaw + 32768, &p.sz, 0, hh, tok, bar_raw);
+      tma_box_x(sm + L::kRaw + 40960, &p.sz, 64, hh, tok, bar_raw);
+    }
     tma_box_x(sm + L::kRaw + 49152, &p.sv, 0, hh, tok, bar_raw);
     tma_box_x(sm + L::kRaw + 57344, &p.sv, 64, hh, tok, bar_raw);
   };
@@ -1021,6 +1031,11 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
 #pragma unroll
         for (int i = 0; i < 8; ++i) E[8 + i] = 0.f;
       }
+    } else if (p.gs) {  // one log-decay per token and head, shared by the channels
+      const float* g0 = p.gs + (size_t)(tok0 + t0) * H + hc;
+      const float ga = in0 ? g0[0] : 0.f, gb = in1 ? g0[H] : 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { E[i] = ga; E[8 + i] = gb; }
     } else {
       const float expA = expf(p.A[hc]);
       const uint4 z1 = rawv(2, t0 + sw), z2 = rawv(2, t0 + 1 - sw);
@@ -1860,6 +1875,7 @@ cudaError_t launch_forward_tc(const ForwardArgs& a) {
   p.z = (const __nv_bfloat16*)a.z;
   p.v = (const __nv_bfloat16*)a.v;
   p.A = a.A;
+  p.gs = a.g_head;
   p.g = a.g;
   p.S0 = a.S0;
   p.cu = a.cu;

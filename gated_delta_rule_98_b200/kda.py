@@ -27,7 +27,8 @@ KDA_F32, KDA_BF16 = 0, 1
 EXPORTS = ("kda_status_string", "kda_version", "kda_forward_workspace_size",
            "kda_forward_launches", "kda_forward",
            "kda_forward_g", "kda_decode_step", "kda_forward_noalloc", "kda_forward_checkpoints",
-           "kda_forward_norm_gate", "kda_decode_step_norm_gate", "kda_check_device_error")
+           "kda_forward_norm_gate", "kda_decode_step_norm_gate", "kda_forward_scalar_gate",
+           "kda_check_device_error")
 
 # Bytes of the library's fixed scratch array used by kda_forward_noalloc.
 KDA_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -76,6 +77,9 @@ def lib():
     L.kda_decode_step_norm_gate.argtypes = ([vp] * 7 + [i32] * 4 + [ctypes.c_int, vp, vp,
                                             ctypes.c_float, vp, vp])
     L.kda_decode_step_norm_gate.restype = ctypes.c_int
+    L.kda_forward_scalar_gate.argtypes = [vp] * 7 + [i32] * 6 + [ctypes.c_int, i32, vp, vp, vp,
+                                                                sz, vp]
+    L.kda_forward_scalar_gate.restype = ctypes.c_int
     L.kda_check_device_error.argtypes = [vp, vp]
     L.kda_check_device_error.restype = ctypes.c_int
     _lib = L
@@ -146,6 +150,14 @@ def kda_decode_step_norm_gate(q, k, v, z, A, beta, S_inout, B, H, dk, dv, dt, ou
                               norm_weight, eps, o, stream):
     return lib().kda_decode_step_norm_gate(q, k, v, z, A, beta, S_inout, B, H, dk, dv, dt,
                                            out_gate, norm_weight, eps, o, stream)
+
+
+def kda_forward_scalar_gate(q, k, v, g_head, beta, S0, cu_seqlens, num_seqs, total_tokens,
+                            max_seqlen, H, dk, dv, dt, chunk, o, S_final, workspace,
+                            workspace_bytes, stream):
+    return lib().kda_forward_scalar_gate(q, k, v, g_head, beta, S0, cu_seqlens, num_seqs,
+                                         total_tokens, max_seqlen, H, dk, dv, dt, chunk, o,
+                                         S_final, workspace, workspace_bytes, stream)
 
 
 def kda_check_device_error(workspace, stream):
@@ -222,7 +234,7 @@ def _forward(entry, q, k, v, gate_a, gate_b, beta, S0, cu_seqlens, num_seqs, max
         args.append(_p(gate_b))
     args += [_p(beta), _p(S0), _p(cu_seqlens), N, T, max_len, H, dk, dv, dt, chunk, _p(o),
              _p(S_final), _p(ws), ws.numel(), _stream(stream)]
-    fn = kda_forward if entry == "z" else kda_forward_g
+    fn = {"z": kda_forward, "g": kda_forward_g, "gs": kda_forward_scalar_gate}[entry]
     st = fn(*args)
     if st != KDA_OK:
         raise KdaError(st, fn.__name__)
@@ -271,6 +283,15 @@ def forward_g(q, k, v, g, beta, *, S0=None, cu_seqlens=None, num_seqs=None, max_
     """KDA prefill with the fp32 log-decay g [T,H,dk] given directly (g in [-5, 0])."""
     return _forward("g", q, k, v, g, None, beta, S0, cu_seqlens, num_seqs, max_seqlen, chunk, o,
                     S_final, workspace, stream, output_final_state)
+
+
+def forward_scalar_gate(q, k, v, g_head, beta, *, S0=None, cu_seqlens=None, num_seqs=None,
+                        max_seqlen=None, chunk=64, o=None, S_final=None, workspace=None,
+                        stream=None, output_final_state=True):
+    """Gated DeltaNet special case: one fp32 log-decay per token and head,
+    g_head [T,H] in [-5, 0], shared by the dk channels."""
+    return _forward("gs", q, k, v, g_head, None, beta, S0, cu_seqlens, num_seqs, max_seqlen,
+                    chunk, o, S_final, workspace, stream, output_final_state)
 
 
 def decode_step(q, k, v, z, A, beta, S, *, o=None, stream=None):

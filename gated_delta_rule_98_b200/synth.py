@@ -18,6 +18,8 @@ q, k, v, z, beta are then rounded to the compute dtype (round-to-nearest-even).
 Output epilogue inputs (``out_gate_inputs``, numpy ``default_rng(seed)``):
   r ~ N(0,1) [T,H,dv]                 (gate logits; rounded to the compute dtype)
   w ~ U(0.5, 1.5) [dv]                (RMSNorm gain, fp32)
+Scalar (per token and head) log-decay (``scalar_gate``, ``default_rng(seed)``):
+  g = -5 * logistic(2 N(0,1) - 3) [T,H] fp32, in (-5, 0), mostly near 0
 
 Workloads (sizes follow the operator's published benchmark settings):
   tiny      B=1 H=2  L=64    d=32  fp32 chunk 16  S0=0           seed 0
@@ -80,6 +82,13 @@ def out_gate_inputs(T, H, dv, *, seed, dtype="bf16"):
     r = _cast(rng.standard_normal((T, H, dv)), torch_dtype(dtype))
     w = torch.from_numpy(rng.uniform(0.5, 1.5, dv)).float()
     return r, w
+
+
+def scalar_gate(T, H, *, seed):
+    """One log-decay per token and head (Gated DeltaNet form), fp32 [T,H]."""
+    rng = np.random.default_rng(seed)
+    x = 2.0 * rng.standard_normal((T, H)) - 3.0
+    return torch.from_numpy(-5.0 / (1.0 + np.exp(-x))).float()
 
 
 def varlen_lengths(total=32768, lo=512, hi=8192, seed=3):

@@ -145,6 +145,27 @@ kda_status kda_forward_g(const void* q, const void* k, const void* v,
                          size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * The Gated DeltaNet special case (Kimi Linear summary, §2.2 "Linear Attention
+ * and the Gated Delta Rule": one scalar forget gate per head): the decay of
+ * token t in head h is one value shared by all dk channels,
+ * alpha_t = exp(g_head[t, h]).  Same algorithm and kernels as kda_forward with
+ * the gate broadcast over the channels; z is not read, so the call moves
+ * 2·dk bytes (bf16) less per token and head.
+ *
+ *  g_head : [T, H] float32 log-decay, in [-5, 0] (the range the lower-bounded
+ *           KDA gate guarantees and the 16-token sub-tile bound relies on;
+ *           values outside it give undefined results: not checked).
+ * Everything else, including the workspace size, is kda_forward's.
+ */
+kda_status kda_forward_scalar_gate(const void* q, const void* k, const void* v,
+                                   const float* g_head, const void* beta, const float* S0,
+                                   const int32_t* cu_seqlens, int32_t num_seqs,
+                                   int32_t total_tokens, int32_t max_seqlen, int32_t H,
+                                   int32_t dk, int32_t dv, kda_dtype dt, int32_t chunk,
+                                   void* o, float* S_final, void* workspace,
+                                   size_t workspace_bytes, kda_stream_t stream);
+
+/*
  * kda_forward that also writes sparse state checkpoints: the state after
  * every `interval` tokens of each sequence.  This is the operator's side of a
  * prefix cache that keeps KDA states at fixed token boundaries inside a paged

@@ -163,3 +163,12 @@ def test_norm_gate_rejects_bad_epilogue_arguments(L):
     assert dec(eps=float("nan")) == kda.KDA_ERR_INVALID_ARG
     assert dec(dk=48) == kda.KDA_ERR_UNSUPPORTED
     assert dec(gate=None, B=0) == kda.KDA_OK                    # nothing to do
+
+
+def test_scalar_gate_requires_the_gate(L):
+    st = kda.kda_forward_scalar_gate(FAKE, FAKE, FAKE, None, FAKE, None, None, 1, 64, 64, 2, 32,
+                                     32, kda.KDA_F32, 16, FAKE, FAKE, FAKE, 1 << 40, None)
+    assert st == kda.KDA_ERR_INVALID_ARG
+    st = kda.kda_forward_scalar_gate(FAKE, FAKE, FAKE, FAKE + 4, FAKE, None, None, 1, 64, 64, 2,
+                                     32, 32, kda.KDA_F32, 16, FAKE, FAKE, FAKE, 1 << 40, None)
+    assert st == kda.KDA_ERR_INVALID_ARG
