@@ -12,6 +12,8 @@ ref           ctypes wrapper around ``kda_ref.c``, the plain sequential float64
               recurrence (the oracle proper).
 brute         numpy float64 brute force: materialised products of per-token
               transition matrices (position-interaction view), tiny sizes only.
+prologue      numpy float64 input prologue (causal short convolution per
+              channel, then Swish).
 epilogue      numpy float64 output epilogue (head-wise RMSNorm, then the
               sigmoid output gate).
 chunk_mirror  numpy float64 restatement of the chunkwise (WY/UT) algorithm the

@@ -13,7 +13,7 @@ import os
 import numpy as np
 import pytest
 
-from oracle import brute, chunk_mirror, epilogue, ref
+from oracle import brute, chunk_mirror, epilogue, prologue, ref
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -460,4 +460,78 @@ def test_output_epilogue_mistakes_are_caught(mistake):
         y = og / np.sqrt(np.mean(og * og, axis=-1, keepdims=True)) * w
     else:
         y = o / np.sqrt(ms) * w * (1 - sig(r))
+    assert np.abs(y - np.array(d["expected_y"])).max() > 1e-3
+
+
+# ---------------------------------------------------------- input prologue ---
+
+def _golden_prologue():
+    with open(os.path.join(GOLDEN, "kda_short_conv_swish.json")) as f:
+        return json.load(f)
+
+
+def test_short_conv_swish_hand_worked():
+    d = _golden_prologue()
+    x, w, cu = np.array(d["x"]), np.array(d["w"]), np.array(d["cu_seqlens"])
+    u = prologue.causal_conv(x, w, cu_seqlens=cu)
+    assert np.abs(u - np.array(d["expected_u"])).max() < d["tolerance_abs"]
+    y = prologue.short_conv_swish(x, w, cu_seqlens=cu)
+    assert np.abs(y - np.array(d["expected_y"])).max() < d["tolerance_abs"]
+
+
+def test_short_conv_matches_numpy_convolve():
+    """Per sequence and channel the convolution is numpy's full convolution with
+    the taps reversed, cut to the sequence length (a library routine)."""
+    rng = np.random.default_rng(33)
+    lens = [7, 0, 1, 3, 12]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    x = rng.standard_normal((cu[-1], 2, 5))
+    w = rng.standard_normal((10, 4))
+    u = prologue.causal_conv(x, w, cu_seqlens=cu).reshape(cu[-1], 10)
+    xf = x.reshape(cu[-1], 10)
+    for n in range(len(lens)):
+        a, b = cu[n], cu[n + 1]
+        if a == b:
+            continue
+        for c in range(10):
+            want = np.convolve(xf[a:b, c], w[c, ::-1])[:b - a]
+            assert np.abs(u[a:b, c] - want).max() < 1e-12
+
+
+def test_short_conv_identity_filter_and_swish_values():
+    rng = np.random.default_rng(34)
+    x = rng.standard_normal((9, 3))
+    w = np.zeros((3, 4))
+    w[:, 3] = 1.0                      # only the current token
+    y = prologue.short_conv_swish(x, w, num_seqs=1)
+    assert np.abs(y - x / (1 + np.exp(-x))).max() < 1e-15
+    assert prologue.swish(np.array([0.0]))[0] == 0.0
+    assert abs(prologue.swish(np.array([40.0]))[0] - 40.0) < 1e-12
+    assert abs(prologue.swish(np.array([-40.0]))[0]) < 1e-15
+
+
+@pytest.mark.parametrize("mistake", ["flipped", "crosses_boundary", "anti_causal", "sigmoid",
+                                     "no_swish"])
+def test_short_conv_mistakes_are_caught(mistake):
+    """Plausible mistakes in the prologue, restated here on the CPU, fail the
+    hand-worked pin."""
+    d = _golden_prologue()
+    x, w, cu = np.array(d["x"]), np.array(d["w"]), np.array(d["cu_seqlens"])
+    T, W = x.shape[0], w.shape[1]
+    if mistake == "flipped":
+        y = prologue.short_conv_swish(x, w[:, ::-1], cu_seqlens=cu)
+    elif mistake == "crosses_boundary":
+        y = prologue.short_conv_swish(x, w, num_seqs=1)
+    elif mistake == "anti_causal":
+        u = np.zeros_like(x)
+        for t in range(T):
+            for i in range(W):
+                s = t + i
+                if s < T:
+                    u[t] += w[:, i] * x[s]
+        y = prologue.swish(u)
+    elif mistake == "sigmoid":
+        y = 1 / (1 + np.exp(-prologue.causal_conv(x, w, cu_seqlens=cu)))
+    else:
+        y = prologue.causal_conv(x, w, cu_seqlens=cu)
     assert np.abs(y - np.array(d["expected_y"])).max() > 1e-3
