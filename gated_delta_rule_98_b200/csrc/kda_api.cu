@@ -80,6 +80,22 @@ kda_status decode_common(const void* q, const void* k, const void* v, const void
   return kda::launch_decode(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+// Byte offsets, in a kda_forward_conv workspace, of the prologue's q, k, v
+// outputs and the end: after the forward's own fw bytes, 256-byte aligned.
+struct Offsets4 {
+  size_t v[4];
+  size_t operator[](int i) const { return v[i]; }
+};
+Offsets4 conv_offsets(size_t fw, size_t tok, int32_t dk, int32_t dv, size_t elt) {
+  auto up = [](size_t b) { return (b + 255) & ~(size_t)255; };
+  Offsets4 o;
+  o.v[0] = up(fw);
+  o.v[1] = up(o.v[0] + tok * dk * elt);
+  o.v[2] = up(o.v[1] + tok * dk * elt);
+  o.v[3] = up(o.v[2] + tok * dv * elt);
+  return o;
+}
+
 kda_status forward_common(kda::ForwardArgs& a) {
   if (a.N == 0) {
     // nothing to launch: still leave a clean error word for this call
@@ -259,6 +275,84 @@ kda_status kda_decode_step_norm_gate(const void* q, const void* k, const void* v
   if (!epilogue_ok(B > 0, out_gate, norm_weight, eps)) return KDA_ERR_INVALID_ARG;
   return decode_common(q, k, v, z, A, beta, S_inout, B, H, dk, dv, dt, out_gate, norm_weight,
                        eps, o, stream);
+}
+
+kda_status kda_short_conv_swish(const void* x, const float* w, const int32_t* cu_seqlens,
+                                int32_t num_seqs, int32_t total_tokens, int32_t max_seqlen,
+                                int32_t channels, int32_t width, kda_dtype dt, void* y,
+                                kda_stream_t stream) {
+  if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_UNSUPPORTED;
+  if (width < 1 || width > 4) return KDA_ERR_UNSUPPORTED;
+  if (channels < 8 || channels % 8 != 0) return KDA_ERR_UNSUPPORTED;
+  if (num_seqs < 0 || total_tokens < 0 || max_seqlen < 0) return KDA_ERR_INVALID_ARG;
+  if (!cu_seqlens && (int64_t)num_seqs * max_seqlen != total_tokens) return KDA_ERR_INVALID_ARG;
+  if (total_tokens == 0) return KDA_OK;
+  if (num_seqs == 0) return KDA_ERR_INVALID_ARG;
+  if (!x || !w || !y || !aligned16(x) || !aligned16(y)) return KDA_ERR_INVALID_ARG;
+  if (cu_seqlens && ((uintptr_t)cu_seqlens & 3u)) return KDA_ERR_INVALID_ARG;
+  if (((uintptr_t)w & 3u)) return KDA_ERR_INVALID_ARG;
+  kda::ConvArgs a{};
+  a.t[0] = {x, w, y, channels};
+  a.ntensors = 1;
+  a.cu = cu_seqlens;
+  a.N = num_seqs; a.T = total_tokens; a.L = max_seqlen; a.width = width;
+  a.bf16 = dt == KDA_BF16;
+  a.stream = (cudaStream_t)stream;
+  return kda::launch_conv_swish(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+size_t kda_forward_conv_workspace_size(int32_t num_seqs, int32_t total_tokens,
+                                       int32_t max_seqlen, int32_t H, int32_t dk, int32_t dv,
+                                       kda_dtype dt, int32_t chunk) {
+  const size_t fw = kda_forward_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv,
+                                               dt, chunk);
+  if (fw == 0) return 0;
+  const size_t elt = dt == KDA_BF16 ? 2 : 4, tok = (size_t)total_tokens * H;
+  return conv_offsets(fw, tok, dk, dv, elt)[3];
+}
+
+kda_status kda_forward_conv(const void* x_q, const void* x_k, const void* x_v,
+                            const float* w_q, const float* w_k, const float* w_v,
+                            int32_t conv_width, const void* z, const float* A, const void* beta,
+                            const float* S0, const int32_t* cu_seqlens, int32_t num_seqs,
+                            int32_t total_tokens, int32_t max_seqlen, int32_t H, int32_t dk,
+                            int32_t dv, kda_dtype dt, int32_t chunk, void* o, float* S_final,
+                            void* workspace, size_t workspace_bytes, kda_stream_t stream) {
+  const size_t fw = kda_forward_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv,
+                                               dt, chunk);
+  const size_t need = kda_forward_conv_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk,
+                                                      dv, dt, chunk);
+  // the forward's own checks, on its part of the workspace
+  kda_status st = check_forward(x_q, x_k, x_v, z, beta, S0, cu_seqlens, num_seqs,
+                                total_tokens, max_seqlen, H, dk, dv, dt, chunk, o, S_final,
+                                workspace, fw);
+  if (st != KDA_OK) return st;
+  if (total_tokens > 0 && (!A || !aligned16(A))) return KDA_ERR_INVALID_ARG;
+  if (conv_width < 1 || conv_width > 4) return KDA_ERR_UNSUPPORTED;
+  if (workspace_bytes < need) return KDA_ERR_INVALID_ARG;
+  if (total_tokens > 0 && (!w_q || !w_k || !w_v || ((uintptr_t)w_q & 3u) ||
+                           ((uintptr_t)w_k & 3u) || ((uintptr_t)w_v & 3u)))
+    return KDA_ERR_INVALID_ARG;
+  const size_t elt = dt == KDA_BF16 ? 2 : 4, tok = (size_t)total_tokens * H;
+  const auto off = conv_offsets(fw, tok, dk, dv, elt);
+  char* ws = (char*)workspace;
+  void *q = ws + off[0], *k = ws + off[1], *v = ws + off[2];
+  if (total_tokens > 0 && num_seqs > 0) {
+    kda::ConvArgs c{};
+    c.t[0] = {x_q, w_q, q, H * dk};
+    c.t[1] = {x_k, w_k, k, H * dk};
+    c.t[2] = {x_v, w_v, v, H * dv};
+    c.ntensors = 3;
+    c.cu = cu_seqlens;
+    c.N = num_seqs; c.T = total_tokens; c.L = max_seqlen; c.width = conv_width;
+    c.bf16 = dt == KDA_BF16;
+    c.stream = (cudaStream_t)stream;
+    if (kda::launch_conv_swish(c) != cudaSuccess) return KDA_ERR_CUDA;
+  }
+  kda::ForwardArgs a{q, k, v, z, beta, A, nullptr, S0, cu_seqlens, o, S_final,
+                     num_seqs, total_tokens, max_seqlen, H, dk, dv, chunk,
+                     dt == KDA_BF16, workspace, fw, (cudaStream_t)stream};
+  return forward_common(a);
 }
 
 kda_status kda_check_device_error(const void* workspace, kda_stream_t stream) {

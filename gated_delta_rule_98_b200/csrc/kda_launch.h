@@ -46,6 +46,23 @@ struct ForwardArgs {
   const float* g_head = nullptr;
 };
 
+// Input prologue: causal depthwise short convolution per sequence + Swish.
+struct ConvTensor {
+  const void* x;   // [T, channels] input (dtype of the call)
+  const float* w;  // [channels, width] taps, w[c][width-1] on the current token
+  void* y;         // [T, channels] output
+  int channels;    // a multiple of 8
+};
+struct ConvArgs {
+  ConvTensor t[3];
+  int ntensors;
+  const int32_t* cu;  // nullptr = N equal sequences of L tokens
+  int N, T, L, width;
+  bool bf16;
+  cudaStream_t stream;
+};
+cudaError_t launch_conv_swish(const ConvArgs& a);
+
 cudaError_t launch_decode(const DecodeArgs& a);
 
 // SIMT (CUDA-core, fp32) chunkwise path: any supported size and dtype.

@@ -15,6 +15,7 @@ from __future__ import annotations
 import ctypes
 import os
 
+import numpy as np
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -28,6 +29,7 @@ EXPORTS = ("kda_status_string", "kda_version", "kda_forward_workspace_size",
            "kda_forward_launches", "kda_forward",
            "kda_forward_g", "kda_decode_step", "kda_forward_noalloc", "kda_forward_checkpoints",
            "kda_forward_norm_gate", "kda_decode_step_norm_gate", "kda_forward_scalar_gate",
+           "kda_short_conv_swish", "kda_forward_conv_workspace_size", "kda_forward_conv",
            "kda_check_device_error")
 
 # Bytes of the library's fixed scratch array used by kda_forward_noalloc.
@@ -80,6 +82,13 @@ def lib():
     L.kda_forward_scalar_gate.argtypes = [vp] * 7 + [i32] * 6 + [ctypes.c_int, i32, vp, vp, vp,
                                                                 sz, vp]
     L.kda_forward_scalar_gate.restype = ctypes.c_int
+    L.kda_short_conv_swish.argtypes = [vp, vp, vp] + [i32] * 5 + [ctypes.c_int, vp, vp]
+    L.kda_short_conv_swish.restype = ctypes.c_int
+    L.kda_forward_conv_workspace_size.argtypes = [i32] * 6 + [ctypes.c_int, i32]
+    L.kda_forward_conv_workspace_size.restype = sz
+    L.kda_forward_conv.argtypes = ([vp] * 6 + [i32] + [vp] * 5 + [i32] * 6 +
+                                   [ctypes.c_int, i32, vp, vp, vp, sz, vp])
+    L.kda_forward_conv.restype = ctypes.c_int
     L.kda_check_device_error.argtypes = [vp, vp]
     L.kda_check_device_error.restype = ctypes.c_int
     _lib = L
@@ -158,6 +167,25 @@ def kda_forward_scalar_gate(q, k, v, g_head, beta, S0, cu_seqlens, num_seqs, tot
     return lib().kda_forward_scalar_gate(q, k, v, g_head, beta, S0, cu_seqlens, num_seqs,
                                          total_tokens, max_seqlen, H, dk, dv, dt, chunk, o,
                                          S_final, workspace, workspace_bytes, stream)
+
+
+def kda_short_conv_swish(x, w, cu_seqlens, num_seqs, total_tokens, max_seqlen, channels, width,
+                         dt, y, stream):
+    return lib().kda_short_conv_swish(x, w, cu_seqlens, num_seqs, total_tokens, max_seqlen,
+                                      channels, width, dt, y, stream)
+
+
+def kda_forward_conv_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv, dt, chunk):
+    return lib().kda_forward_conv_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv,
+                                                 dt, chunk)
+
+
+def kda_forward_conv(x_q, x_k, x_v, w_q, w_k, w_v, conv_width, z, A, beta, S0, cu_seqlens,
+                     num_seqs, total_tokens, max_seqlen, H, dk, dv, dt, chunk, o, S_final,
+                     workspace, workspace_bytes, stream):
+    return lib().kda_forward_conv(x_q, x_k, x_v, w_q, w_k, w_v, conv_width, z, A, beta, S0,
+                                  cu_seqlens, num_seqs, total_tokens, max_seqlen, H, dk, dv, dt,
+                                  chunk, o, S_final, workspace, workspace_bytes, stream)
 
 
 def kda_check_device_error(workspace, stream):
@@ -348,6 +376,57 @@ def decode_step_norm_gate(q, k, v, z, A, beta, S, out_gate, *, norm_weight=None,
     if st != KDA_OK:
         raise KdaError(st, "kda_decode_step_norm_gate")
     return o
+
+
+def short_conv_swish(x, w, *, cu_seqlens=None, num_seqs=None, max_seqlen=None, y=None,
+                     stream=None):
+    """Input prologue on one tensor x [T, ...] (trailing axes = channels):
+    y = Swish(causal depthwise convolution with taps w [channels, width])."""
+    _check_cuda(x, w, cu_seqlens, y)
+    T = x.shape[0]
+    C = x.numel() // T if T else int(np.prod(x.shape[1:]))
+    if cu_seqlens is None:
+        N = 1 if num_seqs is None else int(num_seqs)
+        L = T // N if N else 0
+    else:
+        N = cu_seqlens.numel() - 1
+        if max_seqlen is None:
+            raise ValueError("max_seqlen is required with cu_seqlens")
+        L = int(max_seqlen)
+    if y is None:
+        y = torch.empty_like(x)
+    st = kda_short_conv_swish(_p(x), _p(w), _p(cu_seqlens), N, T, L, C, w.shape[-1], _dt(x),
+                              _p(y), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_short_conv_swish")
+    return y
+
+
+def forward_conv(x_q, x_k, x_v, w_q, w_k, w_v, z, A, beta, *, S0=None, cu_seqlens=None,
+                 num_seqs=None, max_seqlen=None, chunk=64, o=None, S_final=None, workspace=None,
+                 stream=None):
+    """KDA prefill on the input prologue's outputs: q, k, v = Swish(short causal
+    convolution of x_q, x_k, x_v) with taps w_* [H*d, width] fp32.  Returns
+    (o, S_final)."""
+    _check_cuda(x_q, x_k, x_v, w_q, w_k, w_v, z, A, beta, S0, cu_seqlens, o, S_final, workspace)
+    T, H, dk, dv, N, max_len = _geometry(x_q, x_v, cu_seqlens, num_seqs, max_seqlen)
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=x_q.dtype, device=x_q.device)
+    if S_final is None:
+        S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=x_q.device)
+    dt = _dt(x_q)
+    if workspace is None:
+        nbytes = kda_forward_conv_workspace_size(N, T, max_len, H, dk, dv, dt, chunk)
+        if nbytes == 0:
+            raise KdaError(KDA_ERR_UNSUPPORTED, "kda_forward_conv_workspace_size")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=x_q.device)
+    st = kda_forward_conv(_p(x_q), _p(x_k), _p(x_v), _p(w_q), _p(w_k), _p(w_v), w_q.shape[-1],
+                          _p(z), _p(A), _p(beta), _p(S0), _p(cu_seqlens), N, T, max_len, H, dk,
+                          dv, dt, chunk, _p(o), _p(S_final), _p(workspace), workspace.numel(),
+                          _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_forward_conv")
+    return o, S_final
 
 
 def check_device_error(ws, stream=None):

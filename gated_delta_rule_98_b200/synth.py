@@ -18,6 +18,9 @@ q, k, v, z, beta are then rounded to the compute dtype (round-to-nearest-even).
 Output epilogue inputs (``out_gate_inputs``, numpy ``default_rng(seed)``):
   r ~ N(0,1) [T,H,dv]                 (gate logits; rounded to the compute dtype)
   w ~ U(0.5, 1.5) [dv]                (RMSNorm gain, fp32)
+Input prologue (``conv_inputs``, ``default_rng(seed)``, in this order):
+  x_q, x_k ~ N(0,1) [T,H,dk], x_v ~ N(0,1) [T,H,dv]   (rounded to the compute dtype)
+  w_q, w_k ~ N(0,1/width) [H*dk,width], w_v ~ N(0,1/width) [H*dv,width]   (fp32)
 Scalar (per token and head) log-decay (``scalar_gate``, ``default_rng(seed)``):
   g = -5 * logistic(2 N(0,1) - 3) [T,H] fp32, in (-5, 0), mostly near 0
 
@@ -82,6 +85,21 @@ def out_gate_inputs(T, H, dv, *, seed, dtype="bf16"):
     r = _cast(rng.standard_normal((T, H, dv)), torch_dtype(dtype))
     w = torch.from_numpy(rng.uniform(0.5, 1.5, dv)).float()
     return r, w
+
+
+def conv_inputs(T, H, dk, dv, width, *, seed, dtype="bf16"):
+    """Pre-convolution q, k, v and the depthwise taps of the input prologue."""
+    rng = np.random.default_rng(seed)
+    dt = torch_dtype(dtype)
+    out = {}
+    out["x_q"] = _cast(rng.standard_normal((T, H, dk)), dt)
+    out["x_k"] = _cast(rng.standard_normal((T, H, dk)), dt)
+    out["x_v"] = _cast(rng.standard_normal((T, H, dv)), dt)
+    s = 1.0 / np.sqrt(width)
+    out["w_q"] = torch.from_numpy(rng.standard_normal((H * dk, width)) * s).float()
+    out["w_k"] = torch.from_numpy(rng.standard_normal((H * dk, width)) * s).float()
+    out["w_v"] = torch.from_numpy(rng.standard_normal((H * dv, width)) * s).float()
+    return out
 
 
 def scalar_gate(T, H, *, seed):

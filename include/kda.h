@@ -299,6 +299,64 @@ kda_status kda_forward_noalloc(const void* q, const void* k, const void* v,
                                void* o, float* S_final, kda_stream_t stream);
 
 /*
+ * The layer's input prologue on one tensor (Kimi Linear summary, §4 "The Kimi
+ * Linear Model Architecture": a short convolution captures dependencies
+ * between neighbouring tokens, and a Swish nonlinearity is applied to the
+ * queries, keys and values).  The pages give neither the width nor the form
+ * of the convolution; this is a causal depthwise convolution along the tokens
+ * of each sequence, no bias, never reaching across a sequence boundary:
+ *
+ *   u[t,c] = sum_{i<width} w[c,i] * x[t-(width-1)+i, c]   (x = 0 before the
+ *            first token of t's sequence)
+ *   y[t,c] = u[t,c] * sigmoid(u[t,c])
+ *
+ *  x, y      : [T, channels] in `dt` (channels = H * d for a [T, H, d]
+ *              tensor), 16-byte aligned; y must not overlap x.
+ *  w         : [channels, width] float32 (4-byte aligned); w[c, width-1]
+ *              weighs the current token.
+ *  cu_seqlens, num_seqs, total_tokens, max_seqlen : as in kda_forward
+ *              (cu_seqlens is not validated here: a malformed one gives
+ *              undefined values, never an out-of-range access).
+ *  channels  : a positive multiple of 8;  width : 1..4 (else
+ *              KDA_ERR_UNSUPPORTED).
+ * One launch; no workspace.
+ */
+kda_status kda_short_conv_swish(const void* x, const float* w, const int32_t* cu_seqlens,
+                                int32_t num_seqs, int32_t total_tokens, int32_t max_seqlen,
+                                int32_t channels, int32_t width, kda_dtype dt, void* y,
+                                kda_stream_t stream);
+
+/* Workspace bytes for kda_forward_conv: kda_forward's, plus room for the
+ * prologue's q, k and v (0 for unsupported arguments). */
+size_t kda_forward_conv_workspace_size(int32_t num_seqs, int32_t total_tokens,
+                                       int32_t max_seqlen, int32_t H, int32_t dk, int32_t dv,
+                                       kda_dtype dt, int32_t chunk);
+
+/*
+ * kda_forward on the prologue's outputs: q = Swish(conv(x_q)), k = Swish(
+ * conv(x_k)), v = Swish(conv(x_v)) as in kda_short_conv_swish (one launch for
+ * the three tensors, written into the workspace), then the operator, which
+ * normalises q and k to unit length itself.  z (the forget-gate input) and
+ * beta are used as given.
+ *
+ *  x_q, x_k : [T, H, dk]; x_v : [T, H, dv], in `dt`.
+ *  w_q, w_k : [H*dk, conv_width]; w_v : [H*dv, conv_width] float32.
+ *  conv_width : 1..4.
+ *  workspace_bytes >= kda_forward_conv_workspace_size(...).
+ * Everything else is kda_forward's.  One launch more than kda_forward.  The
+ * prologue runs as its own HBM-bound pass (one read and one write of q, k,
+ * v); kda_forward's first kernel is bound by instruction issue, so the same
+ * arithmetic inside it would cost about as much time as the extra pass.
+ */
+kda_status kda_forward_conv(const void* x_q, const void* x_k, const void* x_v,
+                            const float* w_q, const float* w_k, const float* w_v,
+                            int32_t conv_width, const void* z, const float* A, const void* beta,
+                            const float* S0, const int32_t* cu_seqlens, int32_t num_seqs,
+                            int32_t total_tokens, int32_t max_seqlen, int32_t H, int32_t dk,
+                            int32_t dv, kda_dtype dt, int32_t chunk, void* o, float* S_final,
+                            void* workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
  * Reads the workspace's error word of the most recent kda_forward /
  * kda_forward_g call on that workspace (synchronises `stream`).  Returns
  * KDA_OK, KDA_ERR_INVALID_ARG (bad cu_seqlens seen on the device),

@@ -172,3 +172,33 @@ def test_scalar_gate_requires_the_gate(L):
     st = kda.kda_forward_scalar_gate(FAKE, FAKE, FAKE, FAKE + 4, FAKE, None, None, 1, 64, 64, 2,
                                      32, 32, kda.KDA_F32, 16, FAKE, FAKE, FAKE, 1 << 40, None)
     assert st == kda.KDA_ERR_INVALID_ARG
+
+
+def test_short_conv_swish_rejects_bad_arguments(L):
+    def sc(x=FAKE, w=FAKE, channels=64, width=4, T=32, N=1, Lm=32):
+        return kda.kda_short_conv_swish(x, w, None, N, T, Lm, channels, width, kda.KDA_BF16, FAKE,
+                                        None)
+    assert sc(width=0) == kda.KDA_ERR_UNSUPPORTED
+    assert sc(width=5) == kda.KDA_ERR_UNSUPPORTED
+    assert sc(channels=12) == kda.KDA_ERR_UNSUPPORTED
+    assert sc(x=FAKE + 8) == kda.KDA_ERR_INVALID_ARG
+    assert sc(w=None) == kda.KDA_ERR_INVALID_ARG
+    assert sc(T=33) == kda.KDA_ERR_INVALID_ARG                  # N * max_seqlen != T
+    assert sc(T=0, Lm=0) == kda.KDA_OK
+
+
+def test_forward_conv_workspace_and_arguments(L):
+    args = (2, 256, 128, 4, 128, 128, kda.KDA_BF16, 64)
+    fw = kda.kda_forward_workspace_size(*args)
+    cw = kda.kda_forward_conv_workspace_size(*args)
+    # the prologue's q, k, v (bf16) follow the forward's workspace
+    assert cw >= fw + 3 * 256 * 4 * 128 * 2
+    assert kda.kda_forward_conv_workspace_size(2, 256, 128, 4, 48, 128, kda.KDA_BF16, 64) == 0
+
+    def fc(ws_bytes=cw, width=4, wq=FAKE):
+        return kda.kda_forward_conv(FAKE, FAKE, FAKE, wq, FAKE, FAKE, width, FAKE, FAKE, FAKE,
+                                    None, None, 2, 256, 128, 4, 128, 128, kda.KDA_BF16, 64, FAKE,
+                                    FAKE, FAKE, ws_bytes, None)
+    assert fc(ws_bytes=cw - 1) == kda.KDA_ERR_INVALID_ARG
+    assert fc(width=0) == kda.KDA_ERR_UNSUPPORTED
+    assert fc(wq=None) == kda.KDA_ERR_INVALID_ARG
