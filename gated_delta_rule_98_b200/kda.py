@@ -219,6 +219,30 @@ def _check_cuda(*ts):
             raise ValueError("KDA tensors must be contiguous")
 
 
+_F32_ROLES = ("A", "g", "g_head", "S0", "S_final", "S", "norm_weight", "S_ckpt")
+
+
+def _shapes(T, H, dk, dv, N, dtype, **ts):
+    """Raise ValueError unless every tensor given has the shape and dtype of its
+    role (the C ABI takes raw pointers and cannot see either)."""
+    want = {"q": (T, H, dk), "k": (T, H, dk), "z": (T, H, dk), "g": (T, H, dk),
+            "v": (T, H, dv), "o": (T, H, dv), "out_gate": (T, H, dv), "beta": (T, H),
+            "g_head": (T, H), "A": (H,), "S0": (N, H, dk, dv), "S_final": (N, H, dk, dv),
+            "S": (N, H, dk, dv), "norm_weight": (dv,), "cu_seqlens": (N + 1,)}
+    for name, t in ts.items():
+        if t is None:
+            continue
+        if name in want and tuple(t.shape) != want[name]:
+            raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {want[name]}")
+        if name == "S_ckpt" and (t.dim() != 5 or tuple(t.shape[:2]) != (N, H) or
+                                 tuple(t.shape[3:]) != (dk, dv)):
+            raise ValueError(f"S_ckpt: shape {tuple(t.shape)}, expected ({N}, {H}, J, {dk}, {dv})")
+        need = (torch.float32 if name in _F32_ROLES else
+                torch.int32 if name == "cu_seqlens" else dtype)
+        if t.dtype != need:
+            raise ValueError(f"{name}: dtype {t.dtype}, expected {need}")
+
+
 def _geometry(q, v, cu_seqlens, num_seqs, max_seqlen):
     T, H, dk = q.shape
     dv = v.shape[-1]
@@ -250,6 +274,10 @@ def _forward(entry, q, k, v, gate_a, gate_b, beta, S0, cu_seqlens, num_seqs, max
              o, S_final, ws, stream, want_state):
     _check_cuda(q, k, v, gate_a, gate_b, beta, S0, cu_seqlens, o, S_final, ws)
     T, H, dk, dv, N, max_len = _geometry(q, v, cu_seqlens, num_seqs, max_seqlen)
+    gate_roles = {"z": dict(z=gate_a, A=gate_b), "g": dict(g=gate_a),
+                  "gs": dict(g_head=gate_a)}[entry]
+    _shapes(T, H, dk, dv, N, q.dtype, q=q, k=k, v=v, beta=beta, S0=S0, cu_seqlens=cu_seqlens,
+            o=o, S_final=S_final, **gate_roles)
     dt = _dt(q)
     if o is None:
         o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
@@ -287,6 +315,11 @@ def forward_checkpoints(q, k, v, z, A, beta, interval, *, S0=None, cu_seqlens=No
     when the binding allocates them)."""
     _check_cuda(q, k, v, z, A, beta, S0, cu_seqlens, o, S_final, S_ckpt, workspace)
     T, H, dk, dv, N, max_len = _geometry(q, v, cu_seqlens, num_seqs, max_seqlen)
+    _shapes(T, H, dk, dv, N, q.dtype, q=q, k=k, v=v, z=z, A=A, beta=beta, S0=S0,
+            cu_seqlens=cu_seqlens, o=o, S_final=S_final, S_ckpt=S_ckpt)
+    if S_ckpt is not None and S_ckpt.shape[2] != max_len // int(interval):
+        raise ValueError(f"S_ckpt: {S_ckpt.shape[2]} checkpoints, expected "
+                         f"{max_len // int(interval)}")
     if o is None:
         o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
     if S_final is None:
@@ -328,6 +361,7 @@ def decode_step(q, k, v, z, A, beta, S, *, o=None, stream=None):
     _check_cuda(q, k, v, z, A, beta, S, o)
     B, H, dk = q.shape
     dv = v.shape[-1]
+    _shapes(B, H, dk, dv, B, q.dtype, q=q, k=k, v=v, z=z, A=A, beta=beta, S=S, o=o)
     if o is None:
         o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
     st = kda_decode_step(_p(q), _p(k), _p(v), _p(z), _p(A), _p(beta), _p(S), B, H, dk, dv,
@@ -346,6 +380,8 @@ def forward_norm_gate(q, k, v, z, A, beta, out_gate, *, norm_weight=None, eps=1e
     _check_cuda(q, k, v, z, A, beta, out_gate, norm_weight, S0, cu_seqlens, o, S_final,
                 workspace)
     T, H, dk, dv, N, max_len = _geometry(q, v, cu_seqlens, num_seqs, max_seqlen)
+    _shapes(T, H, dk, dv, N, q.dtype, q=q, k=k, v=v, z=z, A=A, beta=beta, out_gate=out_gate,
+            norm_weight=norm_weight, S0=S0, cu_seqlens=cu_seqlens, o=o, S_final=S_final)
     if o is None:
         o = torch.empty((T, H, dv), dtype=q.dtype, device=q.device)
     if S_final is None:
@@ -368,6 +404,8 @@ def decode_step_norm_gate(q, k, v, z, A, beta, S, out_gate, *, norm_weight=None,
     _check_cuda(q, k, v, z, A, beta, S, out_gate, norm_weight, o)
     B, H, dk = q.shape
     dv = v.shape[-1]
+    _shapes(B, H, dk, dv, B, q.dtype, q=q, k=k, v=v, z=z, A=A, beta=beta, S=S, o=o,
+            out_gate=out_gate, norm_weight=norm_weight)
     if o is None:
         o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
     st = kda_decode_step_norm_gate(_p(q), _p(k), _p(v), _p(z), _p(A), _p(beta), _p(S), B, H, dk,
@@ -393,6 +431,13 @@ def short_conv_swish(x, w, *, cu_seqlens=None, num_seqs=None, max_seqlen=None, y
         if max_seqlen is None:
             raise ValueError("max_seqlen is required with cu_seqlens")
         L = int(max_seqlen)
+    if cu_seqlens is not None and (cu_seqlens.dtype != torch.int32 or
+                                   cu_seqlens.numel() != N + 1):
+        raise ValueError("cu_seqlens: int32 [N+1] expected")
+    if w.dtype != torch.float32 or w.dim() != 2 or w.shape[0] != C:
+        raise ValueError(f"w: {tuple(w.shape)} {w.dtype}, expected ({C}, width) float32")
+    if y is not None and (y.shape != x.shape or y.dtype != x.dtype):
+        raise ValueError("y: must match x in shape and dtype")
     if y is None:
         y = torch.empty_like(x)
     st = kda_short_conv_swish(_p(x), _p(w), _p(cu_seqlens), N, T, L, C, w.shape[-1], _dt(x),
@@ -410,6 +455,13 @@ def forward_conv(x_q, x_k, x_v, w_q, w_k, w_v, z, A, beta, *, S0=None, cu_seqlen
     (o, S_final)."""
     _check_cuda(x_q, x_k, x_v, w_q, w_k, w_v, z, A, beta, S0, cu_seqlens, o, S_final, workspace)
     T, H, dk, dv, N, max_len = _geometry(x_q, x_v, cu_seqlens, num_seqs, max_seqlen)
+    _shapes(T, H, dk, dv, N, x_q.dtype, q=x_q, k=x_k, v=x_v, z=z, A=A, beta=beta, S0=S0,
+            cu_seqlens=cu_seqlens, o=o, S_final=S_final)
+    width = w_q.shape[-1]
+    for name, w, rows in (("w_q", w_q, H * dk), ("w_k", w_k, H * dk), ("w_v", w_v, H * dv)):
+        if tuple(w.shape) != (rows, width) or w.dtype != torch.float32:
+            raise ValueError(f"{name}: {tuple(w.shape)} {w.dtype}, expected ({rows}, {width}) "
+                             "float32")
     if o is None:
         o = torch.empty((T, H, dv), dtype=x_q.dtype, device=x_q.device)
     if S_final is None:

@@ -202,3 +202,24 @@ def test_forward_conv_workspace_and_arguments(L):
     assert fc(ws_bytes=cw - 1) == kda.KDA_ERR_INVALID_ARG
     assert fc(width=0) == kda.KDA_ERR_UNSUPPORTED
     assert fc(wq=None) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_binding_rejects_mismatched_shapes_before_any_launch():
+    """The binding checks every tensor's shape and dtype against its role (the
+    C ABI only sees pointers); the checks run before the CUDA check would."""
+    import torch
+    from gated_delta_rule_98_b200.kda import _shapes
+    T, H, dk, dv, N = 10, 2, 32, 32, 3
+    ok = dict(q=torch.empty(T, H, dk), v=torch.empty(T, H, dv), beta=torch.empty(T, H),
+              S0=torch.empty(N, H, dk, dv), cu_seqlens=torch.zeros(N + 1, dtype=torch.int32))
+    _shapes(T, H, dk, dv, N, torch.float32, **ok)
+    bad = [dict(S0=torch.empty(1, H, dk, dv)),                  # one state for three sequences
+           dict(beta=torch.empty(T, H, 1)),
+           dict(cu_seqlens=torch.zeros(N + 1, dtype=torch.int64)),
+           dict(A=torch.empty(H, dtype=torch.float64)),
+           dict(k=torch.empty(T, H, dk, dtype=torch.bfloat16)),
+           dict(out_gate=torch.empty(T, H, dk + 1)),
+           dict(S_ckpt=torch.empty(N, H, 2, dk, dv + 1))]
+    for b in bad:
+        with pytest.raises(ValueError):
+            _shapes(T, H, dk, dv, N, torch.float32, **b)

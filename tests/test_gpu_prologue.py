@@ -43,10 +43,11 @@ def test_short_conv_swish(dtype, width, lens):
 
 def _forward_conv(T, H, d, width, dtype, chunk, lens=None, num_seqs=1, seed=0):
     from oracle import prologue, ref
-    inp = synth.draw(T, H, d, d, seed=seed, dtype=dtype, num_seqs=num_seqs, s0_std=0.02)
+    n_seq = len(lens) if lens else num_seqs
+    inp = synth.draw(T, H, d, d, seed=seed, dtype=dtype, num_seqs=n_seq, s0_std=0.02)
     ci = synth.conv_inputs(T, H, d, d, width, seed=seed + 1, dtype=dtype)
     cu = _cu(lens) if lens else None
-    inp["cu_seqlens"], inp["num_seqs"] = cu, (len(lens) if lens else num_seqs)
+    inp["cu_seqlens"], inp["num_seqs"] = cu, n_seq
     d_in, d_ci = to_cuda(inp), to_cuda(ci)
     o, S = kda.forward_conv(d_ci["x_q"], d_ci["x_k"], d_ci["x_v"], d_ci["w_q"], d_ci["w_k"],
                             d_ci["w_v"], d_in["z"], d_in["A"], d_in["beta"], S0=d_in["S0"],
