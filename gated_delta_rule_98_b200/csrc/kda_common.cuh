@@ -34,8 +34,11 @@ __device__ __forceinline__ float gate_logdecay(float z, float expA) {
   return kGateMin / (1.0f + expf(-expA * z));
 }
 
-// Output gate of the epilogue: sigmoid(x) = 1 / (1 + e^{-x}) (0 for x -> -inf).
-__device__ __forceinline__ float out_sigmoid(float x) { return 1.0f / (1.0f + __expf(-x)); }
+// Output gate of the epilogue: sigmoid(x) = 1 / (1 + e^{-x}), with the fast
+// exponential and division (a few ulp; 0 once e^{-x} overflows).
+__device__ __forceinline__ float out_sigmoid(float x) {
+  return __fdividef(1.0f, 1.0f + __expf(-x));
+}
 
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll

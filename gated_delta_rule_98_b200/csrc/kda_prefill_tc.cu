@@ -166,8 +166,9 @@ struct alignas(64) TcParams {
   CUtensorMap tq, tk, tz, tv;  // [T, H, 128] bf16, box 64 tokens x 1 x 128 channels
   CUtensorMap sq, sk, sz, sv;  // the same, box 64 tokens x 1 x 64 channels, 128-byte swizzle
   const __nv_bfloat16 *q, *k, *beta, *z, *v;
+  // g: the log-decay given directly, [T, H, 128], or the scalar gate's [T, H]
+  // (one value per token and head); null when it is computed from z and A.
   const float *A, *g, *S0;
-  const float* gs;  // scalar log-decay [T, H] (one per token and head), or null
   const int32_t* cu;
   __nv_bfloat16* o;
   float* S_final;
@@ -193,23 +194,25 @@ __device__ __forceinline__ float* ckpt_state(const TcParams& p, int n, int h, in
 // data-dependent sigmoid gate) on x[0..NX) of one token's 128 features, given
 // the sum of squares over all 128: x * rsqrt(mean + eps) * w * sigmoid(r).
 // r: the gate input at the same features (16-byte aligned); w: the gain or null.
+__device__ __forceinline__ void norm_gate8(float* x, float inv, uint4 r8, const float* w) {
+  float rv[8], wv[8];
+  unpack8(r8, rv);
+  if (w) {
+    ld8f(w, wv);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) wv[e] = 1.f;
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) x[e] = x[e] * inv * wv[e] * out_sigmoid(rv[e]);
+}
 template <int NX>
 __device__ __forceinline__ void norm_gate(float* x, float sumsq, const __nv_bfloat16* r,
                                           const float* w, float eps) {
   const float inv = rsqrtf(sumsq * (1.0f / 128) + eps);
 #pragma unroll
-  for (int i = 0; i < NX; i += 8) {
-    float rv[8], wv[8];
-    unpack8(*reinterpret_cast<const uint4*>(r + i), rv);
-    if (w) {
-      ld8f(w + i, wv);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) wv[e] = 1.f;
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) x[i + e] = x[i + e] * inv * wv[e] * out_sigmoid(rv[e]);
-  }
+  for (int i = 0; i < NX; i += 8)
+    norm_gate8(x + i, inv, *reinterpret_cast<const uint4*>(r + i), w ? w + i : nullptr);
 }
 
 // Segment p of a sequence with nch chunks: chunks [c0, c1).
@@ -248,14 +251,21 @@ __device__ __forceinline__ void tma_box_x(void* dst, const CUtensorMap* map, int
       : "memory");
 }
 
+// Where the log-decay comes from (a template parameter of the kernels that
+// compute it, so each variant carries only its own code): the KDA gate from z
+// and A; given per channel (g [T, H, 128]); given once per token and head
+// (g [T, H], the scalar gate of Gated DeltaNet, broadcast over the channels).
+enum GateSrc : int { kGateZ = 0, kGateChannel = 1, kGateHead = 2 };
+
 // q, k, z, v rows of the chunk starting at tok0 (single thread); z only when
 // the gate is computed from it.
+template <int GS>
 __device__ __forceinline__ void stage_chunk(const TcParams& p, unsigned char* raw, uint64_t* bar,
                                             int tok0, int h) {
-  mbar_arrive_expect_tx(bar, (p.z ? 4 : 3) * 16384);
+  mbar_arrive_expect_tx(bar, (GS == kGateZ ? 4 : 3) * 16384);
   tma_box(raw + 0 * 16384, &p.tq, h, tok0, bar);
   tma_box(raw + 1 * 16384, &p.tk, h, tok0, bar);
-  if (p.z) tma_box(raw + 2 * 16384, &p.tz, h, tok0, bar);
+  if (GS == kGateZ) tma_box(raw + 2 * 16384, &p.tz, h, tok0, bar);
   tma_box(raw + 3 * 16384, &p.tv, h, tok0, bar);
 }
 
@@ -287,6 +297,7 @@ __device__ __forceinline__ void sync_for_mma() {
 // Fused pass for sequences that are not split into segments: one CTA per
 // (sequence, head) prepares each chunk and advances the state through it,
 // chunk after chunk (incoming state S0 or S_in of its segment); o, S_final.
+template <int GS>
 __global__ void __launch_bounds__(kNT, 1) fused_kernel(const __grid_constant__ TcParams p) {
   using L = FusedSmem;
   extern __shared__ __align__(1024) unsigned char sm[];
@@ -327,7 +338,7 @@ __global__ void __launch_bounds__(kNT, 1) fused_kernel(const __grid_constant__ T
   const uint32_t tm = s_tmem;
   uint32_t phase = 0, phase_raw = 0;
   bool raw_pending = c0 < c1;  // a TMA load into the staging area is in flight
-  if (tid == 0 && c0 < c1) stage_chunk(p, raw, &s_bar_raw, a + c0 * kC, h);
+  if (tid == 0 && c0 < c1) stage_chunk<GS>(p, raw, &s_bar_raw, a + c0 * kC, h);
 
   constexpr int SbN = 128;                    // N extent of the bf16 state operand
   constexpr int SbL = SbN * 16;               // its K-group stride (LBO)
@@ -362,7 +373,7 @@ __global__ void __launch_bounds__(kNT, 1) fused_kernel(const __grid_constant__ T
     tmem_st_wait();
   }
 
-  const float expA = p.z ? expf(p.A[h]) : 0.f;
+  const float expA = GS == kGateZ ? expf(p.A[h]) : 0.f;
   // prep ownership: channel j, row sub-tile qq (rows 16qq .. 16qq+15)
   const int j = tid & 127, qq = tid >> 7;
   // C_b window of row sub-tile b starts at row 8 b (b + 1) of C: 0, 16, 48, 96
@@ -411,17 +422,17 @@ __global__ void __launch_bounds__(kNT, 1) fused_kernel(const __grid_constant__ T
     //      depends only on this sub-tile's own partial sums
     float E[16], Ei[16];
     {
-      if (p.g) {
+      if constexpr (GS == kGateChannel) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int r = 16 * qq + i;
           E[i] = r < len ? p.g[((size_t)(tok0 + r) * H + h) * kD + j] : 0.f;
         }
-      } else if (p.gs) {
+      } else if constexpr (GS == kGateHead) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int r = 16 * qq + i;
-          E[i] = r < len ? p.gs[(size_t)(tok0 + r) * H + h] : 0.f;
+          E[i] = r < len ? p.g[(size_t)(tok0 + r) * H + h] : 0.f;
         }
       } else {
 #pragma unroll
@@ -624,7 +635,7 @@ __global__ void __launch_bounds__(kNT, 1) fused_kernel(const __grid_constant__ T
     // the staged rows are consumed: prefetch the next chunk
     if (c + 1 < c1) {
       raw_pending = true;
-      if (tid == 0) stage_chunk(p, raw, &s_bar_raw, a + (c + 1) * kC, h);
+      if (tid == 0) stage_chunk<GS>(p, raw, &s_bar_raw, a + (c + 1) * kC, h);
     }
     // ---- M2: [W | U~] = T [X_K | X_V]  (M=64, N=256, K=64)
     if (tid == 0) {
@@ -877,6 +888,7 @@ __device__ __forceinline__ void st8f(float* p, const float* f) {
   *reinterpret_cast<float4*>(p + 4) = make_float4(f[4], f[5], f[6], f[7]);
 }
 
+template <int GS>
 __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_constant__ TcParams p) {
   using L = PrepSmem;
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -954,12 +966,12 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
   };
   // q, k, z, v rows of an item -> the staging tile (two 64-channel boxes each)
   auto stage = [&](int tok, int hh) {
-    mbar_arrive_expect_tx(bar_raw, (p.z ? 4 : 3) * 16384);
+    mbar_arrive_expect_tx(bar_raw, (GS == kGateZ ? 4 : 3) * 16384);
     tma_box_x(sm + L::kRaw, &p.sq, 0, hh, tok, bar_raw);
     tma_box_x(sm + L::kRaw + 8192, &p.sq, 64, hh, tok, bar_raw);
     tma_box_x(sm + L::kRaw + 16384, &p.sk, 0, hh, tok, bar_raw);
     tma_box_x(sm + L::kRaw + 24576, &p.sk, 64, hh, tok, bar_raw);
-    if (p.z) {  // z only when the gate is computed from it
+    if (GS == kGateZ) {  // z only when the gate is computed from it
       tma_box_x(sm + L::kRaw + 32768, &p.sz, 0, hh, tok, bar_raw);
       tma_box_x(sm + L::kRaw + 40960, &p.sz, 64, hh, tok, bar_raw);
     }
@@ -1021,7 +1033,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
 
     // ---- log-decay gate g of the 16 elements; E[8 s + i]: token t0 + s, channel c0 + i
     float E[16];
-    if (p.g) {
+    if constexpr (GS == kGateChannel) {
       const float* g0 = p.g + row0;
       if (in0) { ld8f(g0, E); } else {
 #pragma unroll
@@ -1031,8 +1043,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
 #pragma unroll
         for (int i = 0; i < 8; ++i) E[8 + i] = 0.f;
       }
-    } else if (p.gs) {  // one log-decay per token and head, shared by the channels
-      const float* g0 = p.gs + (size_t)(tok0 + t0) * H + hc;
+    } else if constexpr (GS == kGateHead) {  // one log-decay per token and head
+      const float* g0 = p.g + (size_t)(tok0 + t0) * H + hc;
       const float ga = in0 ? g0[0] : 0.f, gb = in1 ? g0[H] : 0.f;
 #pragma unroll
       for (int i = 0; i < 8; ++i) { E[i] = ga; E[8 + i] = gb; }
@@ -1506,10 +1518,24 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       ost[t * kD + srow] = __float2bfloat16_rn(v[i] * iqs[t]);
     }
   };
+  // o rows of a chunk: 16 lanes per token, 8 features each, kC * kD / 8 / kNT = 2 per thread
+  static_assert(kC * kD / 8 == 2 * kNT, "two o vectors per thread");
+  uint4 rg[2];  // output-epilogue gate inputs of the rows write_o stores next
+  auto load_gate = [&](int cc) {  // issued early; used by write_o(cc)
+    if (!p.og) return;
+    const int t0c = a + cc * kC, lenc = min(kC, b - t0c);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int u = tid + k * kNT, t = u >> 4, d8 = (u & 15) * 8;
+      rg[k] = t < lenc ? *reinterpret_cast<const uint4*>(p.og + ((size_t)(t0c + t) * H + h) * kD + d8)
+                       : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
   auto write_o = [&](int cc) {  // staging -> o rows of chunk cc (after a barrier)
     const int t0c = a + cc * kC, lenc = min(kC, b - t0c);
-    for (int u = tid; u < kC * kD / 8; u += kNT) {  // 16 lanes per token, 8 features each
-      const int t = u >> 4, d8 = (u & 15) * 8;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int u = tid + k * kNT, t = u >> 4, d8 = (u & 15) * 8;
       const size_t off = ((size_t)(t0c + t) * H + h) * kD + d8;
       uint4 w8 = *reinterpret_cast<const uint4*>(ost + t * kD + d8);
       if (p.og) {  // output epilogue (uniform branch: every lane takes part in the sums)
@@ -1520,10 +1546,8 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
         for (int e = 0; e < 8; ++e) ss += x[e] * x[e];
 #pragma unroll
         for (int m = 8; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-        if (t < lenc) {
-          norm_gate<8>(x, ss, p.og + off, p.ow ? p.ow + d8 : nullptr, p.oeps);
-          w8 = pack8(x);
-        }
+        norm_gate8(x, rsqrtf(ss * (1.0f / kD) + p.oeps), rg[k], p.ow ? p.ow + d8 : nullptr);
+        w8 = pack8(x);
       }
       if (t < lenc) *reinterpret_cast<uint4*>(p.o + off) = w8;
     }
@@ -1533,6 +1557,7 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
     const int s = (c - c0) & 1;
     const uint32_t dcol = (!TRANS && s) ? 128u : 0u;  // this chunk's products (two buffers)
     unsigned char* st = sm + L::kStage + s * L::kStageBytes;
+    if (!TRANS && c > c0) load_gate(c - 1);  // in flight until write_o(c - 1) below
     sync_for_mma();
     {
       const bool got = mbar_wait_cycles(&s_ld[s], (ph_ld >> s) & 1, kWaitCycles);
@@ -1582,7 +1607,6 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
     }
     if (!TRANS && c > c0) stage_o(dcol ^ 128u);
     if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
-    if (!TRANS && c > c0) write_o(c - 1);
     // ---- U^T = U~^T - D_W^T (transition: [U~^T - D_S^T ; -D_X^T]) -> K-major
 #pragma unroll
     for (int blk = 0; blk < NB; ++blk) {
@@ -1621,6 +1645,8 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       }
       mma_commit(&s_bar);
     }
+    // the previous chunk's o rows (staged before the last barrier) go out while C2 runs
+    if (!TRANS && c > c0) write_o(c - 1);
     // the query row scales of this chunk (read before the barrier below, which
     // orders them before the stage's refill)
     if (!TRANS && tid < kC) iqs[tid] = reinterpret_cast<const float*>(st + L::kIq)[tid];
@@ -1656,6 +1682,7 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
   }
   // o of the last chunk
   if (!TRANS && !s_abort && c1 > c0) {
+    load_gate(c1 - 1);
     stage_o(((c1 - 1 - c0) & 1) ? 128u : 0u);
     __syncthreads();
     write_o(c1 - 1);
@@ -1875,8 +1902,8 @@ cudaError_t launch_forward_tc(const ForwardArgs& a) {
   p.z = (const __nv_bfloat16*)a.z;
   p.v = (const __nv_bfloat16*)a.v;
   p.A = a.A;
-  p.gs = a.g_head;
-  p.g = a.g;
+  p.g = a.g_head ? a.g_head : a.g;
+  const int gs = a.g_head ? kGateHead : a.g ? kGateChannel : kGateZ;
   p.S0 = a.S0;
   p.cu = a.cu;
   p.o = (__nv_bfloat16*)a.o;
@@ -1898,14 +1925,16 @@ cudaError_t launch_forward_tc(const ForwardArgs& a) {
   if (p.P > 1) {
     // chunk preparation -> segment transitions -> incoming states -> chain pass
     p.prep = (unsigned char*)a.ws + prep_offset(a.N, a.H, p.P);
-    err = cudaFuncSetAttribute(prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    auto prep = gs == kGateHead ? prep_kernel<kGateHead>
+              : gs == kGateChannel ? prep_kernel<kGateChannel> : prep_kernel<kGateZ>;
+    err = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                PrepSmem::kBytes);
     if (err != cudaSuccess) return err;
     int sms = 0, dev = 0;
     if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
     if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
       return err;
-    prep_kernel<<<sms, kPrepThreads, PrepSmem::kBytes, a.stream>>>(p);
+    prep<<<sms, kPrepThreads, PrepSmem::kBytes, a.stream>>>(p);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     err = cudaFuncSetAttribute(chain_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                ChainSmem<true>::kBytes);
@@ -1923,10 +1952,12 @@ cudaError_t launch_forward_tc(const ForwardArgs& a) {
     chain_kernel<false><<<dim3(a.N, a.H, p.P), kNT, ChainSmem<false>::kBytes, a.stream>>>(p);
     return cudaGetLastError();
   }
-  err = cudaFuncSetAttribute(fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto fused = gs == kGateHead ? fused_kernel<kGateHead>
+               : gs == kGateChannel ? fused_kernel<kGateChannel> : fused_kernel<kGateZ>;
+  err = cudaFuncSetAttribute(fused, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              FusedSmem::kBytes);
   if (err != cudaSuccess) return err;
-  fused_kernel<<<dim3(a.N, a.H, p.P), kNT, FusedSmem::kBytes, a.stream>>>(p);
+  fused<<<dim3(a.N, a.H, p.P), kNT, FusedSmem::kBytes, a.stream>>>(p);
   return cudaGetLastError();
 }
 
