@@ -355,6 +355,76 @@ kda_status kda_forward_conv(const void* x_q, const void* x_k, const void* x_v,
   return forward_common(a);
 }
 
+size_t kda_cp_workspace_size(int32_t num_seqs, int32_t total_tokens, int32_t max_seqlen,
+                             int32_t H, int32_t dk, int32_t dv, kda_dtype dt, int32_t chunk) {
+  if (!use_tc(dt, dk, dv, chunk)) return 0;
+  if (num_seqs < 0 || total_tokens < 0 || max_seqlen < 0 || H < 1) return 0;
+  return kda::tc_cp_workspace_bytes(num_seqs, total_tokens, H, max_seqlen);
+}
+
+kda_status kda_cp_local(const void* q, const void* k, const void* v, const void* z,
+                        const float* A, const void* beta, const int32_t* cu_seqlens,
+                        int32_t num_seqs, int32_t total_tokens, int32_t max_seqlen, int32_t H,
+                        int32_t dk, int32_t dv, kda_dtype dt, int32_t chunk, float* M_out,
+                        float* N_out, void* workspace, size_t workspace_bytes,
+                        kda_stream_t stream) {
+  if (!use_tc(dt, dk, dv, chunk)) return KDA_ERR_UNSUPPORTED;
+  // the forward's geometry and input checks, with M_out standing in for o (its
+  // workspace size is at most the one this call needs, checked next)
+  kda_status st = check_forward(q, k, v, z, beta, nullptr, cu_seqlens, num_seqs, total_tokens,
+                                max_seqlen, H, dk, dv, dt, chunk, M_out, nullptr, workspace,
+                                workspace_bytes);
+  if (st != KDA_OK) return st;
+  if (workspace_bytes < kda_cp_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv, dt,
+                                              chunk))
+    return KDA_ERR_INVALID_ARG;
+  if (num_seqs > 0 && (!M_out || !N_out || !aligned16(M_out) || !aligned16(N_out)))
+    return KDA_ERR_INVALID_ARG;
+  if (total_tokens > 0 && (!A || !aligned16(A))) return KDA_ERR_INVALID_ARG;
+  kda::ForwardArgs a{q, k, v, z, beta, A, nullptr, nullptr, cu_seqlens, nullptr, nullptr,
+                     num_seqs, total_tokens, max_seqlen, H, dk, dv, chunk,
+                     true, workspace, workspace_bytes, (cudaStream_t)stream};
+  if (num_seqs == 0)
+    return cudaMemsetAsync(workspace, 0, sizeof(uint32_t), (cudaStream_t)stream) == cudaSuccess
+               ? KDA_OK : KDA_ERR_CUDA;
+  return kda::launch_cp_local_tc(a, M_out, N_out) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_cp_finish(const float* S_in, const int32_t* cu_seqlens, int32_t num_seqs,
+                         int32_t total_tokens, int32_t max_seqlen, int32_t H, int32_t dk,
+                         int32_t dv, kda_dtype dt, int32_t chunk, void* o, float* S_final,
+                         void* workspace, size_t workspace_bytes, kda_stream_t stream) {
+  if (!use_tc(dt, dk, dv, chunk)) return KDA_ERR_UNSUPPORTED;
+  if (num_seqs < 0 || total_tokens < 0 || max_seqlen < 0 || H < 1) return KDA_ERR_INVALID_ARG;
+  if (!cu_seqlens && (int64_t)num_seqs * max_seqlen != total_tokens) return KDA_ERR_INVALID_ARG;
+  if (cu_seqlens && ((uintptr_t)cu_seqlens & 3u)) return KDA_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace) ||
+      workspace_bytes < kda_cp_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv, dt,
+                                              chunk))
+    return KDA_ERR_INVALID_ARG;
+  if (total_tokens > 0 && (!o || !aligned16(o))) return KDA_ERR_INVALID_ARG;
+  if (!opt_aligned16(S_in) || !opt_aligned16(S_final)) return KDA_ERR_INVALID_ARG;
+  if (num_seqs == 0) return KDA_OK;
+  kda::ForwardArgs a{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, S_in,
+                     cu_seqlens, o, S_final, num_seqs, total_tokens, max_seqlen, H, dk, dv,
+                     chunk, true, workspace, workspace_bytes, (cudaStream_t)stream};
+  return kda::launch_cp_finish_tc(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+kda_status kda_state_compose(const float* M, const float* N, const float* S_in, float* S_out,
+                             int32_t count, int32_t dk, int32_t dv, kda_stream_t stream) {
+  if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+  if (count < 0) return KDA_ERR_INVALID_ARG;
+  if (count == 0) return KDA_OK;
+  if (!M || !N || !S_out || !aligned16(M) || !aligned16(N) || !aligned16(S_out) ||
+      !opt_aligned16(S_in))
+    return KDA_ERR_INVALID_ARG;
+  return kda::launch_state_compose(M, N, S_in, S_out, count, dk, dv, (cudaStream_t)stream) ==
+                 cudaSuccess
+             ? KDA_OK
+             : KDA_ERR_CUDA;
+}
+
 kda_status kda_check_device_error(const void* workspace, kda_stream_t stream) {
   if (!workspace || !aligned16(workspace)) return KDA_ERR_INVALID_ARG;
   uint32_t err = 0;

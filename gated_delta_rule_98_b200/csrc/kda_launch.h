@@ -77,4 +77,18 @@ size_t tc_workspace_bytes(int N, int T, int H, int max_len);
 int tc_launches(int N, int H, int max_len);
 cudaError_t launch_forward_tc(const ForwardArgs& a);
 
+// Context parallelism on the tensor-core path: the local pass (chunk
+// preparation, the transitions of all local segments, their fold into one
+// transition (M, N) per sequence and head) and the finishing pass (incoming
+// states of the local segments from S_in = a.S0, then the full chain pass).
+size_t tc_cp_workspace_bytes(int N, int T, int H, int max_len);
+int tc_cp_local_launches();
+int tc_cp_finish_launches(int N, int H, int max_len);
+cudaError_t launch_cp_local_tc(const ForwardArgs& a, float* M_out, float* N_out);
+cudaError_t launch_cp_finish_tc(const ForwardArgs& a);
+
+// S_out[i] = M[i] S_in[i] + Nt[i] for count (dk x dk, dk x dv) pairs, fp32.
+cudaError_t launch_state_compose(const float* M, const float* Nt, const float* S_in, float* S_out,
+                                 int count, int dk, int dv, cudaStream_t stream);
+
 }  // namespace kda

@@ -181,6 +181,11 @@ struct alignas(64) TcParams {
   float* seg;  // per (n, h): transitions (M, N) of segments 0..P-2, incoming states of 0..P-1
   unsigned char* prep;  // per (chunk slot, h): chain operands left by the transition pass
   WsHeader* hdr;
+  // Context parallelism: the segment buffers are laid out for Pseg segments
+  // (P, or P + 1 so that all P transitions fit); M_out, N_out receive the
+  // folded transition of each (sequence, head) when set.
+  int Pseg;
+  float *M_out, *N_out;
 };
 
 // Checkpoint slot of the state after sequence-relative chunk c (n_tok tokens in
@@ -349,7 +354,7 @@ __global__ void __launch_bounds__(kNT, 1) fused_kernel(const __grid_constant__ T
 
   // ---- initial state: S0 (or the composed incoming state)
   {
-    const float* S0 = seg > 0 ? seg_sin(p.seg, n, h, H, p.P, seg)
+    const float* S0 = seg > 0 ? seg_sin(p.seg, n, h, H, p.Pseg, seg)
                               : (p.S0 ? p.S0 + ((size_t)n * H + h) * kD * kD : nullptr);
 #pragma unroll
     for (int c16 = 0; c16 < 32; c16 += 16) {
@@ -1479,7 +1484,7 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
   {
     const float* S0 = nullptr;
     if (!TRANS)
-      S0 = seg > 0 ? seg_sin(p.seg, n, h, H, p.P, seg)
+      S0 = seg > 0 ? seg_sin(p.seg, n, h, H, p.Pseg, seg)
                    : (p.S0 ? p.S0 + ((size_t)n * H + h) * kD * kD : nullptr);
 #pragma unroll
     for (int blk = 0; blk < NB; ++blk)
@@ -1694,7 +1699,7 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
   if (!s_abort) {
     float* dst0 = nullptr;
     if (TRANS)
-      dst0 = seg_trans(p.seg, n, h, H, p.P, seg);  // M_p, then N_p
+      dst0 = seg_trans(p.seg, n, h, H, p.Pseg, seg);  // M_p, then N_p
     else if (p.S_final && seg == p.P - 1)
       dst0 = p.S_final + ((size_t)n * H + h) * kD * kD;
     if (dst0) {
@@ -1735,6 +1740,12 @@ struct ComposeSmem {
   static constexpr int kBytes = kBar + 16;
 };
 
+// FOLD = false: incoming states S_in(p + 1) = M_p S_in(p) + N_p of segments
+// 1 .. P-1 from S_in(0) = S0 (16 state columns per CTA).
+// FOLD = true: the transition of the whole sequence, [N | M] = fold over all
+// P segments of [N | M] <- M_p [N | M] + [N_p | 0] from [0 | I], written to
+// N_out and M_out (16 of the 256 columns of [N | M] per CTA).
+template <bool FOLD>
 __global__ void __launch_bounds__(kComposeThreads) compose_kernel(const __grid_constant__ TcParams p) {
   using L = ComposeSmem;
   extern __shared__ __align__(1024) unsigned char sm[];
@@ -1743,10 +1754,11 @@ __global__ void __launch_bounds__(kComposeThreads) compose_kernel(const __grid_c
   if (!seqlens_valid(p.cu, p.N, p.T, p.max_len)) return;
   float* Sct = reinterpret_cast<float*>(sm + L::kS);  // Sct[cc][r] = S[r][cb + cc]
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kBar);
-  const int steps = p.P - 1;
+  const int steps = FOLD ? p.P : p.P - 1;
+  const bool addn = !FOLD || cb < kD;  // columns of N take N_p; columns of M do not
   auto load_m = [&](int sg) {  // single thread
     mbar_arrive_expect_tx(&bar[sg & 1], kD * kD * 4);
-    bulk_g2s(sm + L::kM + (sg & 1) * kD * kD * 4, seg_trans(p.seg, n, h, H, p.P, sg), kD * kD * 4,
+    bulk_g2s(sm + L::kM + (sg & 1) * kD * kD * 4, seg_trans(p.seg, n, h, H, p.Pseg, sg), kD * kD * 4,
              &bar[sg & 1]);
   };
   if (tid == 0) {
@@ -1758,7 +1770,10 @@ __global__ void __launch_bounds__(kComposeThreads) compose_kernel(const __grid_c
   if (tid == 0 && steps > 0) load_m(0);
   for (int e = tid; e < kD * 16; e += kComposeThreads) {
     const int r = e >> 4, cc = e & 15;
-    Sct[cc * kSct + r] = p.S0 ? p.S0[((size_t)n * H + h) * kD * kD + (size_t)r * kD + cb + cc] : 0.f;
+    if (FOLD)
+      Sct[cc * kSct + r] = (cb >= kD && r == cb - kD + cc) ? 1.f : 0.f;
+    else
+      Sct[cc * kSct + r] = p.S0 ? p.S0[((size_t)n * H + h) * kD * kD + (size_t)r * kD + cb + cc] : 0.f;
   }
   const int c = tid & 15, r0 = tid >> 4;  // column c, rows r0 + 16 m
   uint32_t inflight = steps > 0 ? 1u : 0u;  // buffers being filled
@@ -1766,9 +1781,9 @@ __global__ void __launch_bounds__(kComposeThreads) compose_kernel(const __grid_c
   bool ok = true;
   // N_p columns, loaded one step ahead
   auto load_n = [&](int sg, float (&v)[8]) {
-    const float* Nt = seg_trans(p.seg, n, h, H, p.P, sg) + kD * kD;
+    const float* Nt = seg_trans(p.seg, n, h, H, p.Pseg, sg) + kD * kD;
 #pragma unroll
-    for (int m = 0; m < 8; ++m) v[m] = Nt[(size_t)(r0 + 16 * m) * kD + cb + c];
+    for (int m = 0; m < 8; ++m) v[m] = addn ? Nt[(size_t)(r0 + 16 * m) * kD + cb + c] : 0.f;
   };
   float nxt[8];
   if (steps > 0) load_n(0, nxt);
@@ -1805,10 +1820,19 @@ __global__ void __launch_bounds__(kComposeThreads) compose_kernel(const __grid_c
 #pragma unroll
     for (int m = 0; m < 8; ++m) Sct[c * kSct + r0 + 16 * m] = acc[m];
     __syncthreads();
-    float* Sin = seg_sin(p.seg, n, h, H, p.P, sg + 1);
+    if (!FOLD) {
+      float* Sin = seg_sin(p.seg, n, h, H, p.Pseg, sg + 1);
+      for (int e = tid; e < kD * 16; e += kComposeThreads) {
+        const int r = e >> 4, cc = e & 15;
+        Sin[(size_t)r * kD + cb + cc] = Sct[cc * kSct + r];
+      }
+    }
+  }
+  if (FOLD && ok) {
+    float* dst = (cb < kD ? p.N_out + cb : p.M_out + (cb - kD)) + ((size_t)n * H + h) * kD * kD;
     for (int e = tid; e < kD * 16; e += kComposeThreads) {
       const int r = e >> 4, cc = e & 15;
-      Sin[(size_t)r * kD + cb + cc] = Sct[cc * kSct + r];
+      dst[(size_t)r * kD + cc] = Sct[cc * kSct + r];
     }
   }
   if (!ok && tid == 0) {
@@ -1885,10 +1909,12 @@ int tc_launches(int N, int H, int max_len) {
   return tc_segments(N, H, max_len) > 1 ? 4 : 1;
 }
 
-cudaError_t launch_forward_tc(const ForwardArgs& a) {
-  TcParams p;
+namespace {
+
+// Kernel parameters of a call; tensor maps only when the call stages inputs.
+cudaError_t fill_params(const ForwardArgs& a, TcParams& p, bool maps) {
   memset(&p, 0, sizeof(p));
-  if (a.T > 0) {
+  if (maps && a.T > 0) {
     const void* zz = a.z ? a.z : a.k;
     if (!make_map(&p.tq, a.q, a.T, a.H) || !make_map(&p.tk, a.k, a.T, a.H) ||
         !make_map(&p.tz, zz, a.T, a.H) || !make_map(&p.tv, a.v, a.T, a.H) ||
@@ -1903,7 +1929,6 @@ cudaError_t launch_forward_tc(const ForwardArgs& a) {
   p.v = (const __nv_bfloat16*)a.v;
   p.A = a.A;
   p.g = a.g_head ? a.g_head : a.g;
-  const int gs = a.g_head ? kGateHead : a.g ? kGateChannel : kGateZ;
   p.S0 = a.S0;
   p.cu = a.cu;
   p.o = (__nv_bfloat16*)a.o;
@@ -1919,38 +1944,65 @@ cudaError_t launch_forward_tc(const ForwardArgs& a) {
   p.max_len = a.max_len;
   p.H = a.H;
   p.P = tc_segments(a.N, a.H, a.max_len);
+  p.Pseg = p.P;
   p.hdr = (WsHeader*)a.ws;
   p.seg = (float*)((char*)a.ws + sizeof(WsHeader));
-  cudaError_t err;
+  return cudaSuccess;
+}
+
+int gate_src(const ForwardArgs& a) {
+  return a.g_head ? kGateHead : a.g ? kGateChannel : kGateZ;
+}
+
+cudaError_t launch_prep(const TcParams& p, int gs, cudaStream_t st) {
+  auto prep = gs == kGateHead ? prep_kernel<kGateHead>
+            : gs == kGateChannel ? prep_kernel<kGateChannel> : prep_kernel<kGateZ>;
+  cudaError_t err = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         PrepSmem::kBytes);
+  if (err != cudaSuccess) return err;
+  int sms = 0, dev = 0;
+  if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+  if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return err;
+  prep<<<sms, kPrepThreads, PrepSmem::kBytes, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <bool TRANS>
+cudaError_t launch_chain(const TcParams& p, int segments, cudaStream_t st) {
+  cudaError_t err = cudaFuncSetAttribute(chain_kernel<TRANS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         ChainSmem<TRANS>::kBytes);
+  if (err != cudaSuccess) return err;
+  chain_kernel<TRANS><<<dim3(p.N, p.H, segments), kNT, ChainSmem<TRANS>::kBytes, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <bool FOLD>
+cudaError_t launch_compose(const TcParams& p, cudaStream_t st) {
+  cudaError_t err = cudaFuncSetAttribute(compose_kernel<FOLD>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         ComposeSmem::kBytes);
+  if (err != cudaSuccess) return err;
+  const int blocks = (FOLD ? 2 * kD : kD) / 16;
+  compose_kernel<FOLD><<<dim3(p.N, p.H, blocks), kComposeThreads, ComposeSmem::kBytes, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_forward_tc(const ForwardArgs& a) {
+  TcParams p;
+  cudaError_t err = fill_params(a, p, true);
+  if (err != cudaSuccess) return err;
+  const int gs = gate_src(a);
   if (p.P > 1) {
     // chunk preparation -> segment transitions -> incoming states -> chain pass
-    p.prep = (unsigned char*)a.ws + prep_offset(a.N, a.H, p.P);
-    auto prep = gs == kGateHead ? prep_kernel<kGateHead>
-              : gs == kGateChannel ? prep_kernel<kGateChannel> : prep_kernel<kGateZ>;
-    err = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               PrepSmem::kBytes);
-    if (err != cudaSuccess) return err;
-    int sms = 0, dev = 0;
-    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
-    if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-      return err;
-    prep<<<sms, kPrepThreads, PrepSmem::kBytes, a.stream>>>(p);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    err = cudaFuncSetAttribute(chain_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               ChainSmem<true>::kBytes);
-    if (err != cudaSuccess) return err;
-    chain_kernel<true><<<dim3(a.N, a.H, p.P - 1), kNT, ChainSmem<true>::kBytes, a.stream>>>(p);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    err = cudaFuncSetAttribute(compose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               ComposeSmem::kBytes);
-    if (err != cudaSuccess) return err;
-    compose_kernel<<<dim3(a.N, a.H, kD / 16), kComposeThreads, ComposeSmem::kBytes, a.stream>>>(p);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    err = cudaFuncSetAttribute(chain_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               ChainSmem<false>::kBytes);
-    if (err != cudaSuccess) return err;
-    chain_kernel<false><<<dim3(a.N, a.H, p.P), kNT, ChainSmem<false>::kBytes, a.stream>>>(p);
-    return cudaGetLastError();
+    p.prep = (unsigned char*)a.ws + prep_offset(a.N, a.H, p.Pseg);
+    if ((err = launch_prep(p, gs, a.stream)) != cudaSuccess) return err;
+    if ((err = launch_chain<true>(p, p.P - 1, a.stream)) != cudaSuccess) return err;
+    if ((err = launch_compose<false>(p, a.stream)) != cudaSuccess) return err;
+    return launch_chain<false>(p, p.P, a.stream);
   }
   auto fused = gs == kGateHead ? fused_kernel<kGateHead>
                : gs == kGateChannel ? fused_kernel<kGateChannel> : fused_kernel<kGateZ>;
@@ -1959,6 +2011,43 @@ cudaError_t launch_forward_tc(const ForwardArgs& a) {
   if (err != cudaSuccess) return err;
   fused<<<dim3(a.N, a.H, p.P), kNT, FusedSmem::kBytes, a.stream>>>(p);
   return cudaGetLastError();
+}
+
+// Context parallelism.  The workspace holds the segment buffers for P + 1
+// segments (room for all P transitions) and the chunk slots, and it carries
+// the slots and transitions from the local pass to the finishing pass.
+size_t tc_cp_workspace_bytes(int N, int T, int H, int max_len) {
+  const int P = tc_segments(N, H, max_len);
+  const size_t slots = (size_t)T / kC + (size_t)N;
+  return prep_offset(N, H, P + 1) + slots * H * kSlotBytes;
+}
+
+int tc_cp_local_launches() { return 3; }
+int tc_cp_finish_launches(int N, int H, int max_len) {
+  return tc_segments(N, H, max_len) > 1 ? 2 : 1;
+}
+
+cudaError_t launch_cp_local_tc(const ForwardArgs& a, float* M_out, float* N_out) {
+  TcParams p;
+  cudaError_t err = fill_params(a, p, true);
+  if (err != cudaSuccess) return err;
+  p.Pseg = p.P + 1;
+  p.prep = (unsigned char*)a.ws + prep_offset(a.N, a.H, p.Pseg);
+  p.M_out = M_out;
+  p.N_out = N_out;
+  if ((err = launch_prep(p, gate_src(a), a.stream)) != cudaSuccess) return err;
+  if ((err = launch_chain<true>(p, p.P, a.stream)) != cudaSuccess) return err;
+  return launch_compose<true>(p, a.stream);
+}
+
+cudaError_t launch_cp_finish_tc(const ForwardArgs& a) {
+  TcParams p;
+  cudaError_t err = fill_params(a, p, false);
+  if (err != cudaSuccess) return err;
+  p.Pseg = p.P + 1;
+  p.prep = (unsigned char*)a.ws + prep_offset(a.N, a.H, p.Pseg);
+  if (p.P > 1 && (err = launch_compose<false>(p, a.stream)) != cudaSuccess) return err;
+  return launch_chain<false>(p, p.P, a.stream);
 }
 
 }  // namespace kda

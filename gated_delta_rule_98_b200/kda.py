@@ -30,6 +30,7 @@ EXPORTS = ("kda_status_string", "kda_version", "kda_forward_workspace_size",
            "kda_forward_g", "kda_decode_step", "kda_forward_noalloc", "kda_forward_checkpoints",
            "kda_forward_norm_gate", "kda_decode_step_norm_gate", "kda_forward_scalar_gate",
            "kda_short_conv_swish", "kda_forward_conv_workspace_size", "kda_forward_conv",
+           "kda_cp_workspace_size", "kda_cp_local", "kda_cp_finish", "kda_state_compose",
            "kda_check_device_error")
 
 # Bytes of the library's fixed scratch array used by kda_forward_noalloc.
@@ -89,6 +90,14 @@ def lib():
     L.kda_forward_conv.argtypes = ([vp] * 6 + [i32] + [vp] * 5 + [i32] * 6 +
                                    [ctypes.c_int, i32, vp, vp, vp, sz, vp])
     L.kda_forward_conv.restype = ctypes.c_int
+    L.kda_cp_workspace_size.argtypes = [i32] * 6 + [ctypes.c_int, i32]
+    L.kda_cp_workspace_size.restype = sz
+    L.kda_cp_local.argtypes = [vp] * 7 + [i32] * 6 + [ctypes.c_int, i32, vp, vp, vp, sz, vp]
+    L.kda_cp_local.restype = ctypes.c_int
+    L.kda_cp_finish.argtypes = [vp, vp] + [i32] * 6 + [ctypes.c_int, i32, vp, vp, vp, sz, vp]
+    L.kda_cp_finish.restype = ctypes.c_int
+    L.kda_state_compose.argtypes = [vp] * 4 + [i32] * 3 + [vp]
+    L.kda_state_compose.restype = ctypes.c_int
     L.kda_check_device_error.argtypes = [vp, vp]
     L.kda_check_device_error.restype = ctypes.c_int
     _lib = L
@@ -186,6 +195,27 @@ def kda_forward_conv(x_q, x_k, x_v, w_q, w_k, w_v, conv_width, z, A, beta, S0, c
     return lib().kda_forward_conv(x_q, x_k, x_v, w_q, w_k, w_v, conv_width, z, A, beta, S0,
                                   cu_seqlens, num_seqs, total_tokens, max_seqlen, H, dk, dv, dt,
                                   chunk, o, S_final, workspace, workspace_bytes, stream)
+
+
+def kda_cp_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv, dt, chunk):
+    return lib().kda_cp_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv, dt, chunk)
+
+
+def kda_cp_local(q, k, v, z, A, beta, cu_seqlens, num_seqs, total_tokens, max_seqlen, H, dk, dv,
+                 dt, chunk, M_out, N_out, workspace, workspace_bytes, stream):
+    return lib().kda_cp_local(q, k, v, z, A, beta, cu_seqlens, num_seqs, total_tokens,
+                              max_seqlen, H, dk, dv, dt, chunk, M_out, N_out, workspace,
+                              workspace_bytes, stream)
+
+
+def kda_cp_finish(S_in, cu_seqlens, num_seqs, total_tokens, max_seqlen, H, dk, dv, dt, chunk, o,
+                  S_final, workspace, workspace_bytes, stream):
+    return lib().kda_cp_finish(S_in, cu_seqlens, num_seqs, total_tokens, max_seqlen, H, dk, dv,
+                               dt, chunk, o, S_final, workspace, workspace_bytes, stream)
+
+
+def kda_state_compose(M, N, S_in, S_out, count, dk, dv, stream):
+    return lib().kda_state_compose(M, N, S_in, S_out, count, dk, dv, stream)
 
 
 def kda_check_device_error(workspace, stream):
@@ -479,6 +509,76 @@ def forward_conv(x_q, x_k, x_v, w_q, w_k, w_v, z, A, beta, *, S0=None, cu_seqlen
     if st != KDA_OK:
         raise KdaError(st, "kda_forward_conv")
     return o, S_final
+
+
+class CpShard:
+    """A shard's context-parallel state between cp_local and cp_finish: its
+    geometry and the workspace that holds its chunk preparation."""
+
+    def __init__(self, geometry, dtype, cu_seqlens, workspace, chunk):
+        self.geometry, self.dtype, self.cu_seqlens = geometry, dtype, cu_seqlens
+        self.workspace, self.chunk = workspace, chunk
+
+
+def cp_local(q, k, v, z, A, beta, *, cu_seqlens=None, num_seqs=None, max_seqlen=None, chunk=64,
+             workspace=None, stream=None):
+    """Context parallelism, step 1 on this rank's shard: returns (M [N,H,dk,dk],
+    N [N,H,dk,dv], shard) with S_after = M S_before + N for each sequence and
+    head; ``shard`` carries the workspace to cp_finish."""
+    _check_cuda(q, k, v, z, A, beta, cu_seqlens, workspace)
+    T, H, dk, dv, N, max_len = _geometry(q, v, cu_seqlens, num_seqs, max_seqlen)
+    _shapes(T, H, dk, dv, N, q.dtype, q=q, k=k, v=v, z=z, A=A, beta=beta, cu_seqlens=cu_seqlens)
+    dt = _dt(q)
+    if workspace is None:
+        nbytes = kda_cp_workspace_size(N, T, max_len, H, dk, dv, dt, chunk)
+        if nbytes == 0:
+            raise KdaError(KDA_ERR_UNSUPPORTED, "kda_cp_workspace_size")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    M = torch.empty((N, H, dk, dk), dtype=torch.float32, device=q.device)
+    Nt = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    st = kda_cp_local(_p(q), _p(k), _p(v), _p(z), _p(A), _p(beta), _p(cu_seqlens), N, T, max_len,
+                      H, dk, dv, dt, chunk, _p(M), _p(Nt), _p(workspace), workspace.numel(),
+                      _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_cp_local")
+    return M, Nt, CpShard((T, H, dk, dv, N, max_len), q.dtype, cu_seqlens, workspace, chunk)
+
+
+def cp_finish(shard, S_in=None, *, o=None, S_final=None, stream=None):
+    """Context parallelism, step 4: o of the shard and the state after it, from
+    the state entering it (None: zeros) and the workspace cp_local filled."""
+    T, H, dk, dv, N, max_len = shard.geometry
+    _check_cuda(S_in, o, S_final)
+    _shapes(T, H, dk, dv, N, shard.dtype, S0=S_in, o=o, S_final=S_final)
+    if o is None:
+        o = torch.empty((T, H, dv), dtype=shard.dtype, device=shard.workspace.device)
+    if S_final is None:
+        S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=shard.workspace.device)
+    st = kda_cp_finish(_p(S_in), _p(shard.cu_seqlens), N, T, max_len, H, dk, dv,
+                       _dt(torch.empty(0, dtype=shard.dtype)), shard.chunk, _p(o), _p(S_final),
+                       _p(shard.workspace), shard.workspace.numel(), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_cp_finish")
+    return o, S_final
+
+
+def state_compose(M, N, S_in=None, *, S_out=None, stream=None):
+    """S_out = M S_in + N over leading batch axes (fp32; S_in None reads as 0)."""
+    _check_cuda(M, N, S_in, S_out)
+    dk, dv = N.shape[-2], N.shape[-1]
+    count = N.numel() // (dk * dv)
+    for name, t, shape in (("M", M, N.shape[:-2] + (dk, dk)), ("S_in", S_in, N.shape),
+                           ("S_out", S_out, N.shape)):
+        if t is not None and (tuple(t.shape) != tuple(shape) or t.dtype != torch.float32):
+            raise ValueError(f"{name}: {tuple(t.shape)} {t.dtype}, expected {tuple(shape)} float32")
+    if N.dtype != torch.float32:
+        raise ValueError("N: float32 expected")
+    if S_out is None:
+        S_out = torch.empty_like(N)
+    st = kda_state_compose(_p(M), _p(N), _p(S_in), _p(S_out), count, dk, dv, _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_state_compose")
+    return S_out
 
 
 def check_device_error(ws, stream=None):

@@ -357,6 +357,64 @@ kda_status kda_forward_conv(const void* x_q, const void* x_k, const void* x_v,
                             void* workspace, size_t workspace_bytes, kda_stream_t stream);
 
 /*
+ * Context parallelism: one long sequence split over ranks (Kimi K3
+ * architecture summary, infrastructure section: KDA context parallelism
+ * computes the local state updates on each rank and merges them with a prefix
+ * scan over a fixed-size all-gather).  The recurrence is affine in the state,
+ * so a shard of tokens acts on the state entering it as
+ *
+ *   S_after = M S_before + N     (M: dk x dk, N: dk x dv, per sequence and head)
+ *
+ * with M the product of the shard's per-token transitions
+ * (I - beta k k^T) Diag(alpha) and N the state the shard leaves from S = 0.
+ * Protocol, for the shards 0 .. R-1 of a sequence in token order, shard r on
+ * rank r:
+ *   1. kda_cp_local(shard r) -> (M_r, N_r); the workspace keeps the shard's
+ *      chunk preparation and segment transitions for step 4;
+ *   2. the caller all-gathers (M_j, N_j) of every rank (a fixed size: 2 x 64 KB
+ *      per head at d = 128), e.g. with one NCCL all-gather;
+ *   3. S_in(r) = fold of kda_state_compose over j = 0 .. r-1, starting from
+ *      the sequence's initial state: S_in(j+1) = M_j S_in(j) + N_j;
+ *   4. kda_cp_finish(S_in(r)) on the same workspace -> o of shard r and the
+ *      state after it (on the last rank, the sequence's final state).
+ * Several sequences may be processed together (num_seqs > 1 with their own
+ * cu_seqlens); each (sequence, head) has its own M and N.  The tensor-core
+ * configuration only (bf16, dk = dv = 128, chunk 64); others return
+ * KDA_ERR_UNSUPPORTED.  Step 1 is kda_forward's preparation and transition
+ * passes plus the last segment's transition and a fold; step 4 is its
+ * composition and full passes: the two together cost one kda_forward call plus
+ * one segment transition, with no preparation redone.
+ */
+size_t kda_cp_workspace_size(int32_t num_seqs, int32_t total_tokens, int32_t max_seqlen,
+                             int32_t H, int32_t dk, int32_t dv, kda_dtype dt, int32_t chunk);
+
+/*  q, k, v, z, A, beta, cu_seqlens, sizes: the shard, as in kda_forward.
+ *  M_out : [N, H, dk, dk] float32;  N_out : [N, H, dk, dv] float32.
+ *  workspace : kda_cp_workspace_size bytes, kept unchanged until the matching
+ *  kda_cp_finish.  Three launches. */
+kda_status kda_cp_local(const void* q, const void* k, const void* v, const void* z,
+                        const float* A, const void* beta, const int32_t* cu_seqlens,
+                        int32_t num_seqs, int32_t total_tokens, int32_t max_seqlen, int32_t H,
+                        int32_t dk, int32_t dv, kda_dtype dt, int32_t chunk, float* M_out,
+                        float* N_out, void* workspace, size_t workspace_bytes,
+                        kda_stream_t stream);
+
+/*  S_in : [N, H, dk, dv] float32, the state entering the shard (NULL: zeros).
+ *  o : [T, H, dv] bf16;  S_final : [N, H, dk, dv] float32 or NULL.
+ *  The sizes and cu_seqlens must be those of the kda_cp_local call that
+ *  filled the workspace.  One or two launches. */
+kda_status kda_cp_finish(const float* S_in, const int32_t* cu_seqlens, int32_t num_seqs,
+                         int32_t total_tokens, int32_t max_seqlen, int32_t H, int32_t dk,
+                         int32_t dv, kda_dtype dt, int32_t chunk, void* o, float* S_final,
+                         void* workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*  S_out[i] = M[i] S_in[i] + N[i] for i < count (fp32; M [count, dk, dk],
+ *  N, S_in, S_out [count, dk, dv]; S_in NULL reads as zeros; S_out may be
+ *  S_in but not M or N).  dk, dv in {32, 64, 128}.  One launch. */
+kda_status kda_state_compose(const float* M, const float* N, const float* S_in, float* S_out,
+                             int32_t count, int32_t dk, int32_t dv, kda_stream_t stream);
+
+/*
  * Reads the workspace's error word of the most recent kda_forward /
  * kda_forward_g call on that workspace (synchronises `stream`).  Returns
  * KDA_OK, KDA_ERR_INVALID_ARG (bad cu_seqlens seen on the device),

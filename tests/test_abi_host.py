@@ -223,3 +223,29 @@ def test_binding_rejects_mismatched_shapes_before_any_launch():
     for b in bad:
         with pytest.raises(ValueError):
             _shapes(T, H, dk, dv, N, torch.float32, **b)
+
+
+def test_cp_entry_points_reject_bad_arguments(L):
+    args = (1, 512, 512, 4, 128, 128, kda.KDA_BF16, 64)
+    cw = kda.kda_cp_workspace_size(*args)
+    assert cw > kda.kda_forward_workspace_size(*args)
+    assert kda.kda_cp_workspace_size(1, 512, 512, 4, 64, 64, kda.KDA_BF16, 64) == 0
+    assert kda.kda_cp_workspace_size(1, 512, 512, 4, 128, 128, kda.KDA_F32, 64) == 0
+
+    def loc(ws_bytes=cw, M=FAKE, dt=kda.KDA_BF16):
+        return kda.kda_cp_local(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 512, 512, 4, 128,
+                                128, dt, 64, M, FAKE, FAKE, ws_bytes, None)
+    assert loc(ws_bytes=cw - 1) == kda.KDA_ERR_INVALID_ARG
+    assert loc(M=None) == kda.KDA_ERR_INVALID_ARG
+    assert loc(dt=kda.KDA_F32) == kda.KDA_ERR_UNSUPPORTED
+
+    def fin(ws_bytes=cw, o=FAKE):
+        return kda.kda_cp_finish(None, None, 1, 512, 512, 4, 128, 128, kda.KDA_BF16, 64, o, None,
+                                 FAKE, ws_bytes, None)
+    assert fin(ws_bytes=cw - 1) == kda.KDA_ERR_INVALID_ARG
+    assert fin(o=None) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_state_compose(FAKE, FAKE, None, FAKE, 2, 128, 48, None) == \
+        kda.KDA_ERR_UNSUPPORTED
+    assert kda.kda_state_compose(FAKE, None, None, FAKE, 2, 128, 128, None) == \
+        kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_state_compose(None, None, None, None, 0, 128, 128, None) == kda.KDA_OK

@@ -1,0 +1,112 @@
+"""Context parallelism on one GPU with virtual ranks: each shard of a sequence
+goes through kda.cp_local, the incoming states are folded with
+kda.state_compose in shard order, and each shard finishes with kda.cp_finish
+(the steps a rank runs, minus the all-gather, whose logic the CPU tests drive
+with gloo ranks).  The concatenated o and the last shard's state are compared
+with the float64 oracle on the whole sequence; shard transitions (M, N) with
+the oracle's products of per-token transitions."""
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_98_b200 import kda, synth
+from kda_testutil import assert_close, f64, oracle_forward, to_cuda
+
+pytestmark = pytest.mark.gpu
+
+
+def _slice(inp, idx):
+    return {key: (val[idx] if key in ("q", "k", "v", "z", "beta") else val)
+            for key, val in inp.items()}
+
+
+def _run_shards(inp, shards, check_mn=False):
+    """shards: per virtual rank, (token index array, cu_seqlens or None)."""
+    from oracle import cp as ocp
+    S = inp["S0"].cuda() if inp.get("S0") is not None else None
+    N_seq = inp["num_seqs"]
+    Ms, outs, S_last = [], [], None
+    local = []
+    for idx, cu in shards:
+        s = to_cuda(_slice(inp, idx))
+        cu_d = None if cu is None else cu.cuda()
+        lens = np.diff(cu.numpy()) if cu is not None else [len(idx)]
+        M, Nt, shard = kda.cp_local(s["q"], s["k"], s["v"], s["z"], s["A"], s["beta"],
+                                    cu_seqlens=cu_d, num_seqs=1 if cu is None else None,
+                                    max_seqlen=int(max(lens)))
+        local.append((M, Nt, shard, s))
+    S_in = [S]
+    for M, Nt, _, _ in local[:-1]:
+        S_in.append(kda.state_compose(M, Nt, S_in[-1]))
+    for r, (M, Nt, shard, s) in enumerate(local):
+        o, S_last = kda.cp_finish(shard, S_in[r])
+        outs.append((shards[r][0], o))
+    torch.cuda.synchronize()
+    if check_mn:
+        for (M, Nt, shard, s), (idx, cu) in zip(local, shards):
+            sc = _slice(inp, idx)
+            M_ref, N_ref = ocp.shard_transition(sc["q"], sc["k"], sc["v"], sc["beta"], sc["z"],
+                                                sc["A"])
+            assert_close(M[0], M_ref, torch.bfloat16, "M")
+            assert_close(Nt[0], N_ref, torch.bfloat16, "N")
+    T = inp["q"].shape[0]
+    o_all = torch.empty((T,) + tuple(outs[0][1].shape[1:]), dtype=outs[0][1].dtype)
+    for idx, o in outs:
+        o_all[torch.from_numpy(np.asarray(idx))] = o.cpu()
+    o_ref, S_ref = oracle_forward(inp)
+    assert_close(o_all, o_ref, torch.bfloat16, "o")
+    assert_close(S_last, S_ref, torch.bfloat16, "S_final")
+
+
+def _one_sequence(T, H, seed):
+    inp = synth.draw(T, H, 128, 128, seed=seed, dtype="bf16", num_seqs=1, s0_std=0.02)
+    inp["cu_seqlens"], inp["num_seqs"] = None, 1
+    return inp
+
+
+def test_cp_four_shards_with_local_segments():
+    inp = _one_sequence(2048, 4, 91)
+    cuts = [0, 512, 1024, 1536, 2048]
+    _run_shards(inp, [(np.arange(a, b), None) for a, b in zip(cuts[:-1], cuts[1:])])
+
+
+def test_cp_single_chunk_shards_and_transitions():
+    inp = _one_sequence(192, 2, 92)
+    cuts = [0, 64, 128, 192]
+    _run_shards(inp, [(np.arange(a, b), None) for a, b in zip(cuts[:-1], cuts[1:])],
+                check_mn=True)
+
+
+def test_cp_ragged_shards():
+    inp = _one_sequence(777, 4, 93)
+    cuts = [0, 300, 301, 777]
+    _run_shards(inp, [(np.arange(a, b), None) for a, b in zip(cuts[:-1], cuts[1:])])
+
+
+def test_cp_two_sequences_per_shard():
+    """Two packed sequences (400 and 250 tokens), each split over two ranks:
+    rank 0 holds [0, 200) of the first and [0, 70) of the second."""
+    lens = [400, 250]
+    inp = synth.draw(sum(lens), 4, 128, 128, seed=94, dtype="bf16", num_seqs=2, s0_std=0.02)
+    inp["cu_seqlens"], inp["num_seqs"] = synth.cu_from_lengths(lens), 2
+    r0 = np.concatenate([np.arange(0, 200), 400 + np.arange(0, 70)])
+    r1 = np.concatenate([np.arange(200, 400), 400 + np.arange(70, 250)])
+    _run_shards(inp, [(r0, synth.cu_from_lengths([200, 70])),
+                      (r1, synth.cu_from_lengths([200, 180]))])
+
+
+@pytest.mark.parametrize("dk,dv", [(128, 128), (64, 32), (32, 128)])
+def test_state_compose(dk, dv):
+    rng = np.random.default_rng(dk + dv)
+    M = torch.from_numpy(rng.standard_normal((3, 2, dk, dk)) / np.sqrt(dk)).float()
+    N = torch.from_numpy(rng.standard_normal((3, 2, dk, dv))).float()
+    S = torch.from_numpy(rng.standard_normal((3, 2, dk, dv))).float()
+    want = f64(M) @ f64(S) + f64(N)
+    got = kda.state_compose(M.cuda(), N.cuda(), S.cuda())
+    Sd = S.cuda()
+    inplace = kda.state_compose(M.cuda(), N.cuda(), Sd, S_out=Sd)     # S_out aliasing S_in
+    zero = kda.state_compose(M.cuda(), N.cuda(), None)
+    torch.cuda.synchronize()
+    assert np.abs(f64(got) - want).max() < 1e-4
+    assert torch.equal(inplace, got)
+    assert torch.equal(zero.cpu(), N)
