@@ -160,6 +160,19 @@ def test_strongest_decay_everywhere():
     assert_close(S, S_ref, torch.bfloat16, "S")
 
 
+def test_weak_decay_long_memory_segmented():
+    """z shifted down so most channels barely decay (alpha^4096 mostly above
+    1e-3): the segment transitions M_p stay far from zero and every segment's
+    incoming state depends on them.  H = 4, L = 4096: 16 segments per head."""
+    inp = synth.draw(4096, 4, 128, 128, seed=131, dtype="bf16", num_seqs=1, s0_std=0.02)
+    inp["z"] = (inp["z"].float() - 8.0).to(torch.bfloat16)
+    inp["cu_seqlens"], inp["num_seqs"] = None, 1
+    o, S = gpu_forward(inp)
+    o_ref, S_ref = oracle_forward(inp)
+    assert_close(o, o_ref, torch.bfloat16, "o")
+    assert_close(S, S_ref, torch.bfloat16, "S_final")
+
+
 def test_beta_zero_gives_pure_decay():
     inp = synth.draw(130, 2, 64, 64, seed=14, dtype="f32", s0_std=0.5)
     inp["beta"] = torch.zeros_like(inp["beta"])
