@@ -83,6 +83,13 @@ def test_cp_single_chunk_shards_and_transitions():
                 check_mn=True)
 
 
+def test_cp_transitions_of_multi_segment_shards():
+    inp = _one_sequence(1024, 2, 95, z_shift=-8.0)
+    cuts = [0, 384, 1024]          # 6 and 10 chunks: several local segments each
+    _run_shards(inp, [(np.arange(a, b), None) for a, b in zip(cuts[:-1], cuts[1:])],
+                check_mn=True)
+
+
 def test_cp_ragged_shards():
     inp = _one_sequence(777, 4, 93)
     cuts = [0, 300, 301, 777]
