@@ -341,11 +341,20 @@ def main():
                                     num_seqs=B, chunk=CHUNK, o=o, S_final=Sf, S_ckpt=ck,
                                     workspace=ws, stream=stream)
 
+        cp_ws = torch.empty(kda.kda_cp_workspace_size(B, T, L, H, D, D, kda.KDA_BF16, CHUNK),
+                            dtype=torch.uint8, device=dev)
+
+        def fwd_cp():  # a context-parallel rank's two passes on one shard (the whole sequence)
+            _, _, shard = kda.cp_local(d["q"], d["k"], d["v"], d["z"], d["A"], d["beta"],
+                                       num_seqs=B, chunk=CHUNK, workspace=cp_ws, stream=stream)
+            kda.cp_finish(shard, None, o=o, S_final=Sf, stream=stream)
+
         out["variants"] = {}
         n_var = max(3, min(args.steps, 20))
         for name, fn, extra in (
                 ("norm_gate", fwd_norm_gate, T * H * D * 2 + D * 4),
-                ("checkpoints_every_%d" % interval, fwd_ckpt, ck.numel() * 4)):
+                ("checkpoints_every_%d" % interval, fwd_ckpt, ck.numel() * 4),
+                ("cp_local_and_finish", fwd_cp, 0)):
             for _ in range(args.warmup):
                 fn()
             torch.cuda.synchronize()
@@ -356,13 +365,13 @@ def main():
             e1.record(stream)
             torch.cuda.synchronize()
             ms_v = e0.elapsed_time(e1) / n_var
-            assert kda.check_device_error(ws) == kda.KDA_OK
+            assert kda.check_device_error(cp_ws if fn is fwd_cp else ws) == kda.KDA_OK
             ms_v = rank_max(ms_v)
             out["variants"][name] = {
                 "ms_per_step": ms_v, "value": weak_scaling_value(T, world, ms_v),
                 "unit": "tokens/s", "steps": n_var, "extra_alg_bytes": extra,
                 "achieved_gbs": (fwd_bytes + extra) / (ms_v / 1e3) / 1e9}
-        del ws
+        del ws, cp_ws
         torch.cuda.empty_cache()
 
     # ----------------------------------------------------------- decode ---
