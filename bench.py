@@ -349,12 +349,30 @@ def main():
                                        num_seqs=B, chunk=CHUNK, workspace=cp_ws, stream=stream)
             kda.cp_finish(shard, None, o=o, S_final=Sf, stream=stream)
 
+        g_head = synth.scalar_gate(T, H, seed=7).to(dev)
+
+        def fwd_scalar():  # the Gated DeltaNet case: one log-decay per token and head, no z
+            kda.forward_scalar_gate(d["q"], d["k"], d["v"], g_head, d["beta"], num_seqs=B,
+                                    chunk=CHUNK, o=o, S_final=Sf, workspace=ws, stream=stream)
+
+        ci = {k_: t.to(dev) for k_, t in synth.conv_inputs(T, H, D, D, 4, seed=8).items()}
+        conv_ws = torch.empty(kda.kda_forward_conv_workspace_size(B, T, L, H, D, D, kda.KDA_BF16,
+                                                                  CHUNK),
+                              dtype=torch.uint8, device=dev)
+
+        def fwd_conv():  # input prologue (width-4 short convolution + Swish), then the operator
+            kda.forward_conv(ci["x_q"], ci["x_k"], ci["x_v"], ci["w_q"], ci["w_k"], ci["w_v"],
+                             d["z"], d["A"], d["beta"], num_seqs=B, chunk=CHUNK, o=o,
+                             S_final=Sf, workspace=conv_ws, stream=stream)
+
         out["variants"] = {}
         n_var = max(3, min(args.steps, 20))
         for name, fn, extra in (
                 ("norm_gate", fwd_norm_gate, T * H * D * 2 + D * 4),
                 ("checkpoints_every_%d" % interval, fwd_ckpt, ck.numel() * 4),
-                ("cp_local_and_finish", fwd_cp, 0)):
+                ("cp_local_and_finish", fwd_cp, 0),
+                ("scalar_gate", fwd_scalar, T * H * 4 - T * H * D * 2),
+                ("conv_prologue_width4", fwd_conv, 4 * 3 * T * H * D)):
             for _ in range(args.warmup):
                 fn()
             torch.cuda.synchronize()
@@ -365,13 +383,14 @@ def main():
             e1.record(stream)
             torch.cuda.synchronize()
             ms_v = e0.elapsed_time(e1) / n_var
-            assert kda.check_device_error(cp_ws if fn is fwd_cp else ws) == kda.KDA_OK
+            wsv = cp_ws if fn is fwd_cp else conv_ws if fn is fwd_conv else ws
+            assert kda.check_device_error(wsv) == kda.KDA_OK
             ms_v = rank_max(ms_v)
             out["variants"][name] = {
                 "ms_per_step": ms_v, "value": weak_scaling_value(T, world, ms_v),
                 "unit": "tokens/s", "steps": n_var, "extra_alg_bytes": extra,
                 "achieved_gbs": (fwd_bytes + extra) / (ms_v / 1e3) / 1e9}
-        del ws, cp_ws
+        del ws, cp_ws, conv_ws, ci
         torch.cuda.empty_cache()
 
     # ----------------------------------------------------------- decode ---
