@@ -94,6 +94,7 @@ class ClockSampler:
         self.index = index
         self.proc = None
         self.f = None
+        self.start = 0
 
     def __enter__(self):
         try:
@@ -104,7 +105,18 @@ class ClockSampler:
                 stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return self
+        # nvidia-smi takes a while to start: wait (at most 5 s) for its first
+        # sample so that the timed region is covered from its start
+        t_end = time.time() + 5.0
+        while time.time() < t_end and os.path.getsize(self.f.name) == 0:
+            time.sleep(0.01)
         return self
+
+    def mark(self):
+        """Only samples written after this call count (call it when the timed region starts)."""
+        if self.proc is not None:
+            self.start = os.path.getsize(self.f.name)
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -118,7 +130,9 @@ class ClockSampler:
         if self.proc is None:
             return None
         self.f.flush()
-        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        with open(self.f.name) as fh:
+            fh.seek(self.start)
+            rows = [r.split(",") for r in fh.read().strip().splitlines() if r.strip()]
         os.unlink(self.f.name)
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -266,6 +280,7 @@ def main():
         with ClockSampler(local) as clk:
             barrier()
             torch.cuda.synchronize()
+            clk.mark()
             e0.record(stream)
             for _ in range(args.steps):
                 fwd()
