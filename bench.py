@@ -63,10 +63,18 @@ def peaks():
     return dict(hbm=6650.0, bf16=1590.0, src="fallback")
 
 
-def kernel_source_hash():
+# The sources each recorded kernel's traffic depends on (a change elsewhere
+# leaves its record valid).
+_TRAFFIC_SOURCES = {
+    "forward": ("kda_prefill_tc.cu", "tc_sm100.cuh", "kda_common.cuh", "kda_launch.h"),
+    "decode": ("kda_decode.cu", "kda_common.cuh", "kda_launch.h"),
+}
+
+
+def kernel_source_hash(kind):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_98_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
+    for fn in sorted(_TRAFFIC_SOURCES[kind]):
         h.update(fn.encode())
         h.update(open(os.path.join(csrc, fn), "rb").read())
     return h.hexdigest()[:16]
@@ -79,7 +87,7 @@ def recorded_traffic(kind):
         return None
     d = json.load(open(p))
     e = d.get(kind)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kind):
         return None
     return e.get("dram_bytes_per_launch")
 
