@@ -85,6 +85,23 @@ __device__ __forceinline__ int next_boundary(const int32_t* cu, int N, int L, in
   return min(max(cu[lo], t + 1), T);
 }
 
+// Swish u * sigmoid(u).  For bf16 outputs as u * (1/2 + tanh(u/2)/2) with the
+// hardware tanh approximation (one MUFU operation instead of an exponential
+// and a division; its relative error, about 2^-11, is below bf16's 2^-9); for
+// fp32 outputs with the exponential and division.
+template <typename T>
+__device__ __forceinline__ float swish(float u);
+template <>
+__device__ __forceinline__ float swish<__nv_bfloat16>(float u) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * u));
+  return fmaf(0.5f * u, t, 0.5f * u);
+}
+template <>
+__device__ __forceinline__ float swish<float>(float u) {
+  return u * out_sigmoid(u);
+}
+
 template <typename T, int W>
 __global__ void __launch_bounds__(kThreads) conv_swish_kernel(ConvArgs a) {
   const ConvTensor& ct = a.t[blockIdx.z];
@@ -135,7 +152,7 @@ __global__ void __launch_bounds__(kThreads) conv_swish_kernel(ConvArgs a) {
       float acc = w[e][W - 1] * xc[e];
 #pragma unroll
       for (int j = 0; j < W - 1; ++j) acc = fmaf(w[e][j], win[j][e], acc);
-      u[e] = acc * out_sigmoid(acc);
+      u[e] = swish<T>(acc);
     }
     st8<T>(y + (size_t)t * C, u);
     // slide the window by one token
