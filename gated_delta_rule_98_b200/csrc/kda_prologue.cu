@@ -22,6 +22,7 @@ namespace kda {
 namespace {
 
 constexpr int kTokens = 64;  // tokens per thread run
+constexpr int kGroup = 4;    // token rows loaded together
 constexpr int kThreads = 256;
 
 template <typename T>
@@ -135,31 +136,46 @@ __global__ void __launch_bounds__(kThreads) conv_swish_kernel(ConvArgs a) {
   }
   int next = next_boundary(a.cu, a.N, a.L, a.T, start, t0);
 
-#pragma unroll 4
-  for (int t = t0; t < t1; ++t) {
-    if (t >= next) {  // a new sequence starts at t: the window restarts from zeros
+  // groups of kGroup tokens: their rows are loaded together (independent
+  // loads in flight) before the window slides over them
+  for (int tg = t0; tg < t1; tg += kGroup) {
+    float xr[kGroup][8];
 #pragma unroll
-      for (int j = 0; j < W - 1; ++j)
+    for (int j = 0; j < kGroup; ++j) {
+      if (tg + j < t1) {
+        ld8<T>(x + (size_t)(tg + j) * C, xr[j]);
+      } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) win[j][e] = 0.f;
-      start = seq_start(a.cu, a.N, a.L, t);
-      next = next_boundary(a.cu, a.N, a.L, a.T, start, t);
+        for (int e = 0; e < 8; ++e) xr[j][e] = 0.f;
+      }
     }
-    float xc[8], u[8];
-    ld8<T>(x + (size_t)t * C, xc);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      float acc = w[e][W - 1] * xc[e];
+    for (int j = 0; j < kGroup; ++j) {
+      const int t = tg + j;
+      if (t >= t1) break;
+      if (t >= next) {  // a new sequence starts at t: the window restarts from zeros
 #pragma unroll
-      for (int j = 0; j < W - 1; ++j) acc = fmaf(w[e][j], win[j][e], acc);
-      u[e] = swish<T>(acc);
+        for (int i = 0; i < W - 1; ++i)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) win[i][e] = 0.f;
+        start = seq_start(a.cu, a.N, a.L, t);
+        next = next_boundary(a.cu, a.N, a.L, a.T, start, t);
+      }
+      float u[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        float acc = w[e][W - 1] * xr[j][e];
+#pragma unroll
+        for (int i = 0; i < W - 1; ++i) acc = fmaf(w[e][i], win[i][e], acc);
+        u[e] = swish<T>(acc);
+      }
+      st8<T>(y + (size_t)t * C, u);
+      // slide the window by one token
+#pragma unroll
+      for (int i = 0; i < W - 1; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) win[i][e] = (i + 1 < W - 1) ? win[i + 1][e] : xr[j][e];
     }
-    st8<T>(y + (size_t)t * C, u);
-    // slide the window by one token
-#pragma unroll
-    for (int j = 0; j < W - 1; ++j)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) win[j][e] = (j + 1 < W - 1) ? win[j + 1][e] : xc[e];
   }
 }
 
