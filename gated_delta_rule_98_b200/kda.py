@@ -5,10 +5,14 @@ CUDA kernels.  torch is used for device memory (outputs, workspace) and for
 the current CUDA stream.  There is no CPU path: if ``libkda.so`` is missing
 the first call raises, and CPU tensors are rejected.
 
-Low-level functions keep the C names (``kda_forward``, ``kda_forward_g``,
-``kda_decode_step``, ``kda_forward_workspace_size``, ``kda_check_device_error``,
-``kda_status_string``) and take raw pointers/ints.  ``forward``,
-``forward_g``, ``decode_step`` and ``workspace`` are tensor-level helpers.
+Low-level functions keep the C names (every symbol in ``EXPORTS``) and take
+raw pointers and ints.  Tensor-level helpers allocate outputs and workspaces
+with torch, check every tensor's shape and dtype against its role, and pass
+the current stream: ``forward``, ``forward_g``, ``forward_scalar_gate``,
+``forward_checkpoints``, ``forward_norm_gate``, ``forward_conv``,
+``short_conv_swish``, ``decode_step``, ``decode_step_norm_gate``,
+``cp_local`` / ``cp_finish`` / ``state_compose`` (context parallelism; the
+collective lives in ``cp.py``), ``workspace`` and ``check_device_error``.
 """
 from __future__ import annotations
 
@@ -297,6 +301,7 @@ def workspace(num_seqs, total_tokens, max_seqlen, H, dk, dv, dtype, chunk, devic
     return torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
 
 
+# the helpers below take a ``workspace`` argument that shadows the function
 _new_workspace = workspace
 
 

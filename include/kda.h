@@ -90,7 +90,10 @@ size_t kda_forward_workspace_size(int32_t num_seqs, int32_t total_tokens,
 
 /*
  * Number of kernel launches one kda_forward / kda_forward_g call with these
- * arguments enqueues (0 when the arguments are invalid or unsupported).
+ * arguments enqueues (0 when the arguments are invalid or unsupported).  The
+ * same count holds for kda_forward_scalar_gate, kda_forward_checkpoints and,
+ * on the tensor-core path, kda_forward_norm_gate; kda_forward_norm_gate on
+ * the CUDA-core path and kda_forward_conv enqueue one launch more.
  */
 int32_t kda_forward_launches(int32_t num_seqs, int32_t total_tokens,
                              int32_t max_seqlen, int32_t H, int32_t dk,
