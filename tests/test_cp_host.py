@@ -15,12 +15,14 @@ from oracle import ref
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _problem(seed, T, H, dk, dv, s0=0.3):
+def _problem(seed, T, H, dk, dv, s0=0.3, z_shift=-6.0):
+    """z is shifted down so that the decay is weak (alpha near 1) and the shard
+    maps M stay far from zero: the fold order then matters."""
     rng = np.random.default_rng(seed)
     return dict(q=rng.standard_normal((T, H, dk)), k=rng.standard_normal((T, H, dk)),
                 v=rng.standard_normal((T, H, dv)),
                 beta=1 / (1 + np.exp(-rng.standard_normal((T, H)))),
-                z=rng.standard_normal((T, H, dk)), A=rng.standard_normal(H),
+                z=rng.standard_normal((T, H, dk)) + z_shift, A=rng.standard_normal(H),
                 S0=rng.standard_normal((1, H, dk, dv)) * s0)
 
 
@@ -62,6 +64,10 @@ def test_sharded_oracle_equals_one_pass(cuts):
         outs.append(o_r)
     assert np.abs(np.concatenate(outs) - o).max() < 1e-12
     assert np.abs(S_r - Sf).max() < 1e-12
+    # the maps matter here: folding them in the wrong order changes the result
+    if len(Ms) > 2 and all(b > a for a, b in zip(cuts[:-1], cuts[1:])):
+        wrong = ocp.prefix_states(Ms[::-1], Ns[::-1], p["S0"][0])[-1]
+        assert np.abs(wrong - S_ins[-1]).max() > 1e-3
 
 
 class _OracleOps:
@@ -99,12 +105,15 @@ def _worker(rank, world, port, cuts, out):
     dist.destroy_process_group()
 
 
-def test_context_parallel_forward_two_gloo_ranks():
-    cuts = [0, 13, 29]
+@pytest.mark.parametrize("cuts", [[0, 13, 29], [0, 1, 12, 20]])
+def test_context_parallel_forward_gloo_ranks(cuts):
+    """Two ranks, then three (one holding a single token): rank r folds the
+    maps of ranks 0 .. r-1 in order."""
+    world = len(cuts) - 1
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = 29600 + os.getpid() % 1000
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, cuts, q)) for r in range(2)]
+    port = 29600 + os.getpid() % 1000 + 7 * world
+    procs = [ctx.Process(target=_worker, args=(r, world, port, cuts, q)) for r in range(world)]
     for pr in procs:
         pr.start()
     res = sorted((q.get(timeout=180) for _ in procs), key=lambda x: x[0])
