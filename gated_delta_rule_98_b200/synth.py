@@ -22,7 +22,7 @@ Input prologue (``conv_inputs``, ``default_rng(seed)``, in this order):
   x_q, x_k ~ N(0,1) [T,H,dk], x_v ~ N(0,1) [T,H,dv]   (rounded to the compute dtype)
   w_q, w_k ~ N(0,1/width) [H*dk,width], w_v ~ N(0,1/width) [H*dv,width]   (fp32)
 Scalar (per token and head) log-decay (``scalar_gate``, ``default_rng(seed)``):
-  g = -5 * logistic(2 N(0,1) - 3) [T,H] fp32, in (-5, 0), mostly near 0
+  alpha ~ U(e^-5, 1) [T,H], g = ln(alpha) fp32, in [-5, 0)
 
 Workloads (sizes follow the operator's published benchmark settings):
   tiny      B=1 H=2  L=64    d=32  fp32 chunk 16  S0=0           seed 0
@@ -103,10 +103,11 @@ def conv_inputs(T, H, dk, dv, width, *, seed, dtype="bf16"):
 
 
 def scalar_gate(T, H, *, seed):
-    """One log-decay per token and head (Gated DeltaNet form), fp32 [T,H]."""
+    """One log-decay per token and head (Gated DeltaNet form), fp32 [T,H]:
+    the log of a decay drawn uniformly from [e^-5, 1)."""
     rng = np.random.default_rng(seed)
-    x = 2.0 * rng.standard_normal((T, H)) - 3.0
-    return torch.from_numpy(-5.0 / (1.0 + np.exp(-x))).float()
+    g = np.log(rng.uniform(np.exp(-5.0), 1.0, (T, H)))
+    return torch.from_numpy(np.maximum(g, -5.0)).float()
 
 
 def varlen_lengths(total=32768, lo=512, hi=8192, seed=3):
