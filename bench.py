@@ -493,11 +493,13 @@ def main():
     print(json.dumps({
         "metric": METRIC, "value": out["value"], "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": out["ms"],
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": f"KDA fwd long: B={B} H={H} L={L} dk=dv={D}, bf16 inputs, "
                                f"fp32 state, chunk {CHUNK}, S0=0", "B": B, "H": H, "L": L,
                    "dk": D, "dv": D, "chunk": CHUNK,
+                   "arithmetic": "bf16 tensor-core operands with fp32 accumulation; gate, "
+                                 "cumulative decay, norms, inverse and state in fp32",
                    "l2": "inputs exceed L2 (q,k,v,z,o = %.0f MB per step)" % (
                        T * H * D * 2 * 5 / 1e6),
                    "parallelism": f"weak x{world} (independent problems per rank)"},
