@@ -172,7 +172,9 @@ kda_status kda_forward_scalar_gate(const void* q, const void* k, const void* v,
  * kda_forward that also writes sparse state checkpoints: the state after
  * every `interval` tokens of each sequence.  This is the operator's side of a
  * prefix cache that keeps KDA states at fixed token boundaries inside a paged
- * pool (Kimi Linear summary, hybrid paged cache with sparse KDA checkpoints);
+ * pool (Kimi K3 review, romaanj.github.io, Significance: a KDA-aware prefix cache
+ * that keeps MLA blocks and sparse KDA checkpoint boundaries in one paged
+ * pool; Kimi K3 architecture summary, serving engine);
  * the pages describe the cache, not a kernel for it.
  *
  *  interval : tokens between checkpoints, a positive multiple of `chunk`
