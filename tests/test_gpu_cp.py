@@ -123,3 +123,22 @@ def test_state_compose(dk, dv):
     assert np.abs(f64(got) - want).max() < 1e-4
     assert torch.equal(inplace, got)
     assert torch.equal(zero.cpu(), N)
+
+
+def test_cp_passes_equal_forward_at_full_size():
+    """B=1, H=16, L=65536 (the long workload's launch configuration): a rank's
+    two passes on the whole sequence from a zero state run the same kernels
+    on the same operands as kda_forward (the extra last-segment transition and
+    fold only add outputs), so o and the final state agree bit for bit."""
+    inp = synth.workload("long")
+    d = to_cuda(inp)
+    o, S = kda.forward(d["q"], d["k"], d["v"], d["z"], d["A"], d["beta"], num_seqs=1)
+    M, Nt, shard = kda.cp_local(d["q"], d["k"], d["v"], d["z"], d["A"], d["beta"], num_seqs=1)
+    o_cp, S_cp = kda.cp_finish(shard, None)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_cp)
+    assert torch.equal(S, S_cp)
+    # N is the state the sequence leaves from zero, here through the fold of
+    # the segment maps instead of the chain: equal within the bf16 bar
+    assert_close(Nt, f64(S), torch.bfloat16, "N")
+    assert torch.isfinite(M).all()
