@@ -92,3 +92,26 @@ def test_checkpoints_fp32_cuda_core_path():
                      s0_std=0.1)
     inp["cu_seqlens"], inp["num_seqs"] = synth.cu_from_lengths(lens), len(lens)
     _check(inp, 32, 16)
+
+
+def test_checkpoints_long_workload_full_size():
+    """B=1, H=16, L=65536 (the long workload's launch configuration),
+    checkpoints every 16384 tokens: the last one is the call's final state
+    (the same fp32 values), and each earlier one matches the final state of a
+    kda_forward call on that prefix within the bf16 bar (a different
+    segmentation, so different bf16 rounding on the way)."""
+    inp = synth.workload("long")
+    d = to_cuda(inp)
+    T = inp["q"].shape[0]
+    o, S, ck = kda.forward_checkpoints(d["q"], d["k"], d["v"], d["z"], d["A"], d["beta"], 16384,
+                                       num_seqs=1, max_seqlen=T)
+    o_plain, S_plain = kda.forward(d["q"], d["k"], d["v"], d["z"], d["A"], d["beta"], num_seqs=1)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_plain) and torch.equal(S, S_plain)
+    assert torch.equal(ck[:, :, 3], S)
+    for j in range(3):
+        E = 16384 * (j + 1)
+        _, S_pre = kda.forward(d["q"][:E], d["k"][:E], d["v"][:E], d["z"][:E], d["A"],
+                               d["beta"][:E], num_seqs=1)
+        torch.cuda.synchronize()
+        assert_close(ck[:, :, j], f64(S_pre), torch.bfloat16, f"checkpoint {j}")

@@ -81,3 +81,20 @@ def test_forward_conv_varlen():
 def test_forward_conv_cuda_core_path(dtype, chunk, d, width):
     lens = [70, 33, 130]
     _forward_conv(sum(lens), 2, d, width, dtype, chunk, lens=lens, seed=84)
+
+
+def test_forward_conv_long_workload_full_size():
+    """B=1, H=16, L=65536: kda_forward_conv equals the prologue run on each
+    tensor followed by kda_forward, bit for bit, at the full size."""
+    inp = synth.workload("long")
+    d = to_cuda(inp)
+    T, H, dk = inp["q"].shape
+    ci = to_cuda(synth.conv_inputs(T, H, dk, dk, 4, seed=85))
+    o, S = kda.forward_conv(ci["x_q"], ci["x_k"], ci["x_v"], ci["w_q"], ci["w_k"], ci["w_v"],
+                            d["z"], d["A"], d["beta"], num_seqs=1)
+    q = kda.short_conv_swish(ci["x_q"], ci["w_q"], num_seqs=1)
+    k = kda.short_conv_swish(ci["x_k"], ci["w_k"], num_seqs=1)
+    v = kda.short_conv_swish(ci["x_v"], ci["w_v"], num_seqs=1)
+    o2, S2 = kda.forward(q, k, v, d["z"], d["A"], d["beta"], num_seqs=1)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(S, S2)

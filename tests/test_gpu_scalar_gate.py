@@ -56,3 +56,17 @@ def test_scalar_gate_cuda_core_path(dtype, chunk, d):
     inp = synth.draw(sum(lens), 2, d, d, seed=64, dtype=dtype, num_seqs=len(lens), s0_std=0.1)
     inp["cu_seqlens"], inp["num_seqs"] = synth.cu_from_lengths(lens), len(lens)
     _run(inp, chunk, 4)
+
+
+def test_scalar_gate_long_workload_full_size():
+    """B=1, H=16, L=65536: the scalar-gate call equals kda_forward_g given the
+    gate broadcast over the channels, bit for bit, at the full size."""
+    inp = synth.workload("long")
+    d = to_cuda(inp)
+    T, H, dk = inp["q"].shape
+    gs = synth.scalar_gate(T, H, seed=9).cuda()
+    o, S = kda.forward_scalar_gate(d["q"], d["k"], d["v"], gs, d["beta"], num_seqs=1)
+    og, Sg = kda.forward_g(d["q"], d["k"], d["v"], gs[:, :, None].expand(T, H, dk).contiguous(),
+                           d["beta"], num_seqs=1)
+    torch.cuda.synchronize()
+    assert torch.equal(o, og) and torch.equal(S, Sg)
