@@ -97,11 +97,11 @@ Offsets4 conv_offsets(size_t fw, size_t tok, int32_t dk, int32_t dv, size_t elt)
 }
 
 kda_status forward_common(kda::ForwardArgs& a) {
-  if (a.N == 0) {
-    // nothing to launch: still leave a clean error word for this call
-    return cudaMemsetAsync(a.ws, 0, sizeof(uint32_t), a.stream) == cudaSuccess ? KDA_OK
-                                                                               : KDA_ERR_CUDA;
-  }
+  // A clean error word for this call, stream-ordered before its first kernel:
+  // the kernels only OR errors into it, so no report of one CTA can be wiped
+  // by another CTA's reset.
+  if (cudaMemsetAsync(a.ws, 0, sizeof(uint32_t), a.stream) != cudaSuccess) return KDA_ERR_CUDA;
+  if (a.N == 0) return KDA_OK;  // nothing to launch
   cudaError_t err = use_tc(a.bf16 ? KDA_BF16 : KDA_F32, a.dk, a.dv, a.chunk)
                         ? kda::launch_forward_tc(a)
                         : kda::launch_forward_simt(a);
@@ -384,9 +384,9 @@ kda_status kda_cp_local(const void* q, const void* k, const void* v, const void*
   kda::ForwardArgs a{q, k, v, z, beta, A, nullptr, nullptr, cu_seqlens, nullptr, nullptr,
                      num_seqs, total_tokens, max_seqlen, H, dk, dv, chunk,
                      true, workspace, workspace_bytes, (cudaStream_t)stream};
-  if (num_seqs == 0)
-    return cudaMemsetAsync(workspace, 0, sizeof(uint32_t), (cudaStream_t)stream) == cudaSuccess
-               ? KDA_OK : KDA_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), (cudaStream_t)stream) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  if (num_seqs == 0) return KDA_OK;
   return kda::launch_cp_local_tc(a, M_out, N_out) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

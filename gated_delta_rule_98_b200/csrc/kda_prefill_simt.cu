@@ -82,7 +82,7 @@ __global__ void __launch_bounds__(256) simt_prep_kernel(SimtParams p) {
   const int H = p.H;
 
   const bool ok = seqlens_valid(p.cu, p.N, p.T, p.max_len);
-  if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) p.hdr->err = ok ? kErrNone : kErrBadSeqlens;
+  if (!ok && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) atomicOr(&p.hdr->err, kErrBadSeqlens);
   if (!ok) return;
   int a, b;
   seq_bounds(p.cu, n, p.max_len, a, b);
@@ -262,10 +262,10 @@ __global__ void __launch_bounds__(256) simt_state_kernel(SimtParams p) {
   const int n = blockIdx.x, h = blockIdx.y, c0 = blockIdx.z * BV;
   const int H = p.H;
   const bool ok = seqlens_valid(p.cu, p.N, p.T, p.max_len);
-  // Also written by the prep kernel; repeated here for calls where every
-  // sequence is empty and prep is not launched.
-  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && tid == 0)
-    p.hdr->err = ok ? kErrNone : kErrBadSeqlens;
+  // Also reported by the prep kernel; repeated here for calls where every
+  // sequence is empty and prep is not launched.  The host cleared the word.
+  if (!ok && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && tid == 0)
+    atomicOr(&p.hdr->err, kErrBadSeqlens);
   if (!ok) return;
   int a, b;
   seq_bounds(p.cu, n, p.max_len, a, b);

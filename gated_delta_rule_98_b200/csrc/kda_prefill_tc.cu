@@ -317,8 +317,7 @@ __global__ void __launch_bounds__(kNT, 1) fused_kernel(const __grid_constant__ T
   const int H = p.H;
 
   const bool ok = seqlens_valid(p.cu, p.N, p.T, p.max_len);
-  if (n == 0 && h == 0 && seg == 0 && tid == 0)
-    p.hdr->err = ok ? kErrNone : kErrBadSeqlens;
+  if (!ok && n == 0 && h == 0 && seg == 0 && tid == 0) atomicOr(&p.hdr->err, kErrBadSeqlens);
   if (!ok) return;
   int a, b;
   seq_bounds(p.cu, n, p.max_len, a, b);
@@ -911,10 +910,9 @@ __global__ void __launch_bounds__(kPrepThreads, 1) prep_kernel(const __grid_cons
   const int H = p.H;
 
   if (!seqlens_valid(p.cu, p.N, p.T, p.max_len)) {
-    if (blockIdx.x == 0 && tid == 0) p.hdr->err = kErrBadSeqlens;
+    if (blockIdx.x == 0 && tid == 0) atomicOr(&p.hdr->err, kErrBadSeqlens);
     return;
   }
-  if (blockIdx.x == 0 && tid == 0) p.hdr->err = kErrNone;
   // the 128-byte swizzle needs 1024-byte aligned destinations
   if (smem_u32(smem) & 1023u) {
     if (tid == 0) atomicOr(&p.hdr->err, kErrTimeout);
@@ -1880,8 +1878,9 @@ bool tc_supported(const ForwardArgs& a) {
 
 int tc_segments(int N, int H, int max_len) {
   // enough (sequence, head, segment) CTAs to fill the 148 SMs; long sequences only
-  const int pairs = N * H;
-  int P = pairs >= 128 ? 1 : 148 / pairs;
+  if (N <= 0 || H <= 0) return 1;
+  const long long pairs = (long long)N * H;
+  int P = pairs >= 128 ? 1 : (int)(148 / pairs);
   const int nch = (max_len + kC - 1) / kC;
   if (P > nch / 2) P = nch / 2;
   if (P < 1) P = 1;

@@ -277,15 +277,22 @@ kda_status kda_decode_step_norm_gate(const void* q, const void* k, const void* v
  *
  * Arguments and results are those of kda_forward, minus the workspace.  The
  * scratch comes from one fixed array of KDA_NOALLOC_SCRATCH_BYTES in device
- * memory that the library defines at file scope; it is held on every GPU
- * where the entry point is used, until the process exits.  The call itself
- * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ * memory that the library defines at file scope.  The array is reserved on a
+ * GPU when the library's device code is loaded there -- with CUDA's default
+ * lazy module loading at the first kernel of this library launched on that
+ * GPU (any entry point, decode included), with CUDA_MODULE_LOADING=EAGER when
+ * the context is created -- and stays reserved until the process exits.  The
+ * call itself allocates nothing (no cudaMalloc, cudaFree or allocating
+ * library routine).
  *  - Problems needing more scratch than KDA_NOALLOC_SCRATCH_BYTES (see
  *    kda_forward_workspace_size) are rejected with KDA_ERR_UNSUPPORTED before
  *    anything is enqueued; use kda_forward with your own workspace instead.
  *  - The first call on a device, made with that device current, looks up the
  *    array's device address (cudaGetSymbolAddress) and caches it; make that
- *    first call before any stream capture begins on that device.
+ *    first call before any stream capture begins on that device.  The cached
+ *    address belongs to that device's primary context: do not use this entry
+ *    point after cudaDeviceReset (or any teardown of the primary context) in
+ *    the same process, since the array may then live at another address.
  *  - Every call on a device shares the one array, and it keeps the previous
  *    call's contents (nothing in it needs to start at zero).  Calls whose GPU
  *    work may overlap -- different streams, or different host threads without
@@ -421,7 +428,9 @@ kda_status kda_state_compose(const float* M, const float* N, const float* S_in, 
 
 /*
  * Reads the workspace's error word of the most recent kda_forward /
- * kda_forward_g call on that workspace (synchronises `stream`).  Returns
+ * kda_forward_g call on that workspace (synchronises `stream`).  Each call
+ * clears the word (a 4-byte cudaMemsetAsync ordered before its first kernel)
+ * and its kernels only OR errors into it.  Returns
  * KDA_OK, KDA_ERR_INVALID_ARG (bad cu_seqlens seen on the device),
  * KDA_ERR_TIMEOUT (a bounded device wait gave up) or KDA_ERR_CUDA.
  */

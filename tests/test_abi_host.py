@@ -249,3 +249,15 @@ def test_cp_entry_points_reject_bad_arguments(L):
     assert kda.kda_state_compose(FAKE, None, None, FAKE, 2, 128, 128, None) == \
         kda.KDA_ERR_INVALID_ARG
     assert kda.kda_state_compose(None, None, None, None, 0, 128, 128, None) == kda.KDA_OK
+
+
+def test_empty_problem_sizes_on_the_tensor_core_path(L):
+    """num_seqs = 0 on the bf16 d=128 chunk-64 path: the sizing calls return
+    the header-only workspace and no launches instead of failing."""
+    bf = kda.KDA_BF16
+    assert kda.kda_forward_workspace_size(0, 0, 0, 16, 128, 128, bf, 64) > 0
+    assert kda.kda_forward_launches(0, 0, 0, 16, 128, 128, bf, 64) == 0
+    assert kda.kda_forward_conv_workspace_size(0, 0, 0, 16, 128, 128, bf, 64) > 0
+    assert kda.kda_cp_workspace_size(0, 0, 0, 16, 128, 128, bf, 64) > 0
+    # (sequence, head) counts whose product overflows 32 bits still size
+    assert kda.kda_forward_workspace_size(70000, 70000, 1, 70000, 128, 128, bf, 64) > 0
