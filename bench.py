@@ -93,7 +93,7 @@ def recorded_traffic(kind):
 
 
 class ClockSampler:
-    """nvidia-smi clocks/throttle reasons sampled every 20 ms while running."""
+    """nvidia-smi clocks/throttle reasons sampled every 10 ms while running."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -109,7 +109,7 @@ class ClockSampler:
             self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "20"],
+                 "--format=csv,noheader,nounits", "-lms", "10"],
                 stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -176,6 +176,68 @@ def weak_scaling_value(units_per_rank, world, ms_max):
     return world * units_per_rank / (ms_max / 1e3)
 
 
+def time_configs(dev, stream, pk, world, rank_max, barrier, warmup, log_fn):
+    """ms per kda_forward call, tokens/s and HBM roofline fraction of the other
+    prefill configurations: the bf16 L=4096 workload, the long workload's
+    length sweep and the packed varlen workload (H=32, nonzero S0)."""
+    import torch
+
+    from gated_delta_rule_98_b200 import kda, synth
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    res = {}
+    for name, wl, L in (("bf16_L4096", "bf16", None), ("long_L2048", "long", 2048),
+                        ("long_L8192", "long", 8192), ("long_L32768", "long", 32768),
+                        ("varlen_T32768_H32", "varlen", None)):
+        inp = synth.workload(wl, L=L)
+        T, Hh = inp["q"].shape[0], inp["q"].shape[1]
+        N = inp["num_seqs"]
+        cu = inp.get("cu_seqlens")
+        max_len = int((cu[1:] - cu[:-1]).max()) if cu is not None else T // N
+        d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+        o = torch.empty((T, Hh, D), dtype=torch.bfloat16, device=dev)
+        Sf = torch.empty((N, Hh, D, D), dtype=torch.float32, device=dev)
+        ws = kda.workspace(N, T, max_len, Hh, D, D, torch.bfloat16, CHUNK, device=dev)
+
+        def fwd():
+            kda.forward(d["q"], d["k"], d["v"], d["z"], d["A"], d["beta"], S0=d.get("S0"),
+                        cu_seqlens=d.get("cu_seqlens"), num_seqs=N, max_seqlen=max_len,
+                        chunk=CHUNK, o=o, S_final=Sf, workspace=ws, stream=stream)
+
+        for _ in range(warmup):
+            fwd()
+        torch.cuda.synchronize()
+        assert kda.check_device_error(ws) == kda.KDA_OK
+        # enough calls for about 0.1 s of device time
+        e0.record(stream)
+        fwd()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        n = int(min(2000, max(20, 100.0 / max(e0.elapsed_time(e1), 1e-3))))
+        barrier()
+        e0.record(stream)
+        for _ in range(n):
+            fwd()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms_local = e0.elapsed_time(e1) / n
+        ms = rank_max(ms_local)
+        nbytes = alg_bytes_prefill(T, N=N, heads=Hh, s0=cu is not None)
+        flops = alg_flops(T, heads=Hh)
+        ach = nbytes / (ms_local / 1e3) / 1e9
+        res[name] = {"ms_per_call": ms, "calls": n, "tokens_per_s": world * T / (ms / 1e3),
+                     "B_or_N": N, "H": Hh, "tokens": T, "alg_bytes": nbytes,
+                     "achieved_gbs": ach, "hbm_frac": ach / pk["hbm"],
+                     "roofline_time_us": max(nbytes / pk["hbm"] / 1e3, flops / pk["bf16"] / 1e6),
+                     "tensor_flops_frac": flops / (ms_local / 1e3) / 1e12 / pk["bf16"],
+                     "launches": kda.kda_forward_launches(N, T, max_len, Hh, D, D, kda.KDA_BF16,
+                                                          CHUNK)}
+        log_fn(f"config {name}: {ms:.4f} ms/call, {res[name]['hbm_frac']:.3f} of HBM")
+        del d, o, Sf, ws
+        torch.cuda.empty_cache()
+    return res
+
+
 def oracle_baseline(inp, n_tokens):
     """Float64 oracle on the first n_tokens of the workload (all heads)."""
     from oracle import ref
@@ -221,12 +283,14 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--L", type=int, default=L_DEFAULT, help="prefill length (sweep)")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other prefill configurations (profiling captures)")
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run one part (profiling captures); the other part is reported as null")
     args = ap.parse_args()
@@ -266,7 +330,7 @@ def main():
     e1 = torch.cuda.Event(enable_timing=True)
     pk = peaks()
     out = {"ms": None, "value": None, "roofline": None, "e2e": None, "clocks": None,
-           "launches": 0, "decode": None, "variants": None}
+           "launches": 0, "decode": None, "variants": None, "configs": None}
 
     # ---------------------------------------------------------- prefill ---
     if args.only != "decode":
@@ -336,14 +400,14 @@ def main():
         torch.cuda.synchronize()
         barrier()
         e0.record(stream)
-        n_e2e = max(3, min(args.steps, 10))
+        n_e2e = max(10, min(args.steps, 20))
         for _ in range(n_e2e):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
         ms_e2e = rank_max(e0.elapsed_time(e1) / n_e2e)
         out["e2e"] = {"value": weak_scaling_value(T, world, ms_e2e), "unit": "tokens/s",
-                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
 
         # ----------------------------------------------------- variants ---
         # The same workload through the entry points that add the output
@@ -415,6 +479,9 @@ def main():
                 "achieved_gbs": (fwd_bytes + extra) / (ms_v / 1e3) / 1e9}
         del ws, cp_ws, conv_ws, ci
         torch.cuda.empty_cache()
+        if not args.no_configs:
+            out["configs"] = time_configs(dev, stream, pk, world, rank_max, barrier, args.warmup,
+                                          log)
 
     # ----------------------------------------------------------- decode ---
     if args.only != "prefill":
@@ -505,7 +572,7 @@ def main():
                    "parallelism": f"weak x{world} (independent problems per rank)"},
         "roofline": out["roofline"], "cpu_baseline": cpu, "e2e": out["e2e"],
         "gpu_launches": out["launches"], "clocks": out["clocks"], "decode": out["decode"],
-        "variants": out["variants"],
+        "variants": out["variants"], "configs": out["configs"],
     }), flush=True)
 
 

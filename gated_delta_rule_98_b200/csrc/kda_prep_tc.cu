@@ -1,0 +1,626 @@
+// kda_prep_tc.cu -- chunk preparation of the tensor-core KDA prefill (sm_100a):
+// everything of one (chunk, head) that does not depend on the state, left in
+// the chunk's slot for the chain passes (kda_prefill_tc.cu).
+//
+// Kimi Linear summary §3.1 (chunkwise WY / UT form: per-chunk cumulative
+// log-decay, the lower-triangular inverse by forward substitution, W and U~),
+// §3.2 (16-token sub-chunks keep the channel-wise decay factors in range).
+// Per 64-token chunk, with alpha = e^g the per-token, per-channel decay and
+// Gam the chunk-local inclusive cumulative log-decay:
+//
+//   A_kk[r][i] = beta_r sum_j k^_rj k^_ij e^{Gam_rj - Gam_ij}   (i < r)
+//   A_qk[r][i] =        sum_j q_rj  k^_ij e^{Gam_rj - Gam_ij}   (i <= r)
+//   T   = (I + A_kk)^{-1}
+//   W   = T (Diag(beta) K^ e^{Gam})       U~ = T Diag(beta) V
+//   Q'  = q e^{Gam},  K' = k^ e^{Gam_last - Gam},  gamma = e^{Gam_last}
+//
+// (k^ = k / |k|; q stays unnormalised and 1/|q| scales the output rows.)
+// The products are formed per 16-token row sub-tile b with the reference
+// rho_b = Gam at the sub-tile's first token: the row operand carries
+// E = e^{Gam_r - rho_b} <= 1, the column operand ("window" b, every token up
+// to the end of sub-tile b) carries e^{rho_b - Gam_i} (<= e^75 on the diagonal
+// sub-tile, <= 1 before it).  The decay factors are cumulative products of
+// alpha inside a sub-tile (16 tokens x alpha >= e^-5 stays above e^-80).
+//
+// Thread layout of the elementwise phases: thread (channel j, sub-tile b),
+// 512 threads; the 16 tokens of a sub-tile are a serial product in registers
+// and every operand image unit (8 consecutive tokens of one channel) is one
+// 16-byte store.  Persistent: one CTA per SM walks (chunk, sequence, head)
+// items; the next item's q, k, z rows are requested as soon as this item has
+// read them and its v rows as soon as the WY product that reads v in place
+// has completed.
+#include "kda_tc_common.cuh"
+
+namespace kda {
+namespace tcp {
+namespace {
+
+constexpr int kLd = 68;  // row stride (floats) of the fp32 work matrices of the inverse
+
+struct PrepSmem {
+  // staged rows: two 64-channel boxes [64 tokens][64 channels] per tensor, 128-byte swizzle
+  static constexpr int kQ = 0, kK = 16384, kZ = 32768, kV = 49152;
+  static constexpr int kWin = 65536;        // windows: pair p (windows 2p, 2p+1) = 128-row image
+  static constexpr int kR = kWin + 65536;   // R: 128-row image (sub-tile b: k rows 32b.., q rows 32b+16..)
+  static constexpr int kXK = kR + 32768;    // X_K: 64-row f16 image, the A operand X_K^T of M2
+  // after M1 the window / R region holds the inverse's work and the T images
+  static constexpr int kAf = kWin;                // A_kk fp32 [64][kLd], row r, column i
+  static constexpr int kTf = kAf + 64 * kLd * 4;  // T fp32 [64][kLd]
+  static constexpr int kTT = kTf + 64 * kLd * 4;  // T^T fp32 [64][kLd]
+  static constexpr int kY = kTT + 64 * kLd * 4;   // merge products, transposed [64][kLd]
+  static constexpr int kTb = kWin + 69632;        // T, the B operand T^T of M2 (64-row f16 image)
+  static constexpr int kTbb = kTb + 8192;         // T Diag(beta), the same for U~ (bf16, with V)
+  static constexpr int kNrm = kXK + 16384;        // 1/|q| (64), 1/|k| (64)
+  static constexpr int kBeta = kNrm + 512;        // beta (64)
+  static constexpr int kEx = kBeta + 256;         // [4][128] alpha at each sub-tile's first token,
+                                                  // then [4][128] E at its last token
+  static constexpr int kBar = kEx + 4096;         // three mbarriers, then the TMEM base
+  static constexpr int kBytes = kBar + 64;
+};
+static_assert(PrepSmem::kY + 64 * kLd * 4 <= PrepSmem::kTb, "inverse work overlaps T images");
+static_assert(PrepSmem::kTbb + 8192 <= PrepSmem::kXK, "T images overlap X_K");
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Shared-memory matrix descriptor with the 128-byte swizzle (the layout TMA
+// writes with CU_TENSOR_MAP_SWIZZLE_128B into a 1024-byte aligned buffer).
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return smem_desc(saddr, lbo, sbo) | ((uint64_t)2u << 61);
+}
+
+// 16 fp32 values of 16 consecutive tokens -> two units of a bf16 operand image
+__device__ __forceinline__ void put16(unsigned char* base, uint32_t unit0, uint32_t unit1,
+                                      const float* v) {
+  *reinterpret_cast<uint4*>(base + unit0) = pack8(v);
+  *reinterpret_cast<uint4*>(base + unit1) = pack8(v + 8);
+}
+// the same for an f16 image (the chain operands)
+__device__ __forceinline__ void put16h(unsigned char* base, uint32_t unit0, uint32_t unit1,
+                                       const float* v) {
+  *reinterpret_cast<uint4*>(base + unit0) = pack8h(v);
+  *reinterpret_cast<uint4*>(base + unit1) = pack8h(v + 8);
+}
+
+template <int GS>
+__global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ TcParams p) {
+  using L = PrepSmem;
+  extern __shared__ __align__(1024) unsigned char sm[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  float* nrm = reinterpret_cast<float*>(sm + L::kNrm);
+  float* bvec = reinterpret_cast<float*>(sm + L::kBeta);
+  float* exf = reinterpret_cast<float*>(sm + L::kEx);
+  float* exl = exf + 512;
+  uint64_t* bar_qkz = reinterpret_cast<uint64_t*>(sm + L::kBar);
+  uint64_t* bar_v = bar_qkz + 1;
+  uint64_t* bar_mma = bar_qkz + 2;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_qkz + 3);
+  const int H = p.H;
+
+  if (!seqlens_valid(p.cu, p.N, p.T, p.max_len)) {
+    if (blockIdx.x == 0 && tid == 0) atomicOr(&p.hdr->err, kErrBadSeqlens);
+    return;
+  }
+  // the 128-byte swizzle needs 1024-byte aligned destinations
+  if (smem_u32(sm) & 1023u) {
+    if (tid == 0) atomicOr(&p.hdr->err, kErrTimeout);
+    return;
+  }
+  if (warp == 0) {
+    tmem_alloc(s_tmem, 128);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(bar_qkz, 1);
+    mbar_init(bar_v, 1);
+    mbar_init(bar_mma, 1);
+    fence_mbar_init();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tm = *s_tmem;
+  uint32_t ph_qkz = 0, ph_v = 0, ph_mma = 0;
+  bool ok = true, qkz_pending = false, v_pending = false;
+
+  // elementwise phases: channel j, sub-tile b (tokens 16 b .. 16 b + 15)
+  const int j = tid & 127, b = tid >> 7;
+  // TMEM phases: lane quarter q4, column group cq
+  const int q4 = warp & 3, cq = warp >> 2;
+  // byte offset of (token 16 b + i, channel j) in a staged swizzled tile: box
+  // j / 64, row t, 16-byte unit ((j % 64) / 8) ^ (t % 8), element j % 8
+  const uint32_t jbox = (uint32_t)(j >> 6) * 8192u + (uint32_t)(j & 7) * 2u;
+  const uint32_t junit = (uint32_t)((j & 63) >> 3);
+  auto raw_off = [&](int i) -> uint32_t {
+    return jbox + (uint32_t)(16 * b + i) * 128u + ((junit ^ (uint32_t)(i & 7)) << 4);
+  };
+  auto raw_f = [&](int base, int i) -> float {
+    const uint32_t u = *reinterpret_cast<const uint16_t*>(sm + base + raw_off(i));
+    return __uint_as_float(u << 16);
+  };
+
+  // items (chunk c, sequence n, head h), heads fastest; the CTA takes every
+  // gridDim.x-th one, stepping the mixed-radix index without divisions
+  const int maxch = (p.max_len + kC - 1) / kC;
+  const long long it0 = blockIdx.x, stride = gridDim.x;
+  int h = (int)(it0 % H), n = (int)((it0 / H) % p.N), c = (int)(it0 / ((long long)H * p.N));
+  const int sh = (int)(stride % H), sn = (int)((stride / H) % p.N);
+  const int sc = (int)(stride / ((long long)H * p.N));
+  int a = 0, e = 0;  // token range [a, e) of sequence n
+  auto next_item = [&]() -> bool {
+    for (; c < maxch;) {
+      seq_bounds(p.cu, n, p.max_len, a, e);
+      if (a + c * kC < e) return true;
+      h += sh;
+      if (h >= H) { h -= H; ++n; }
+      n += sn;
+      if (n >= p.N) { n -= p.N; ++c; }
+      c += sc;
+    }
+    return false;
+  };
+  auto stage_qkz = [&](int tok, int hh) {  // one thread
+    mbar_arrive_expect_tx(bar_qkz, (GS == kGateZ ? 3 : 2) * 16384);
+    tma_box_x(sm + L::kQ, &p.sq, 0, hh, tok, bar_qkz);
+    tma_box_x(sm + L::kQ + 8192, &p.sq, 64, hh, tok, bar_qkz);
+    tma_box_x(sm + L::kK, &p.sk, 0, hh, tok, bar_qkz);
+    tma_box_x(sm + L::kK + 8192, &p.sk, 64, hh, tok, bar_qkz);
+    if (GS == kGateZ) {
+      tma_box_x(sm + L::kZ, &p.sz, 0, hh, tok, bar_qkz);
+      tma_box_x(sm + L::kZ + 8192, &p.sz, 64, hh, tok, bar_qkz);
+    }
+  };
+  auto stage_v = [&](int tok, int hh) {  // one thread
+    mbar_arrive_expect_tx(bar_v, 16384);
+    tma_box_x(sm + L::kV, &p.sv, 0, hh, tok, bar_v);
+    tma_box_x(sm + L::kV + 8192, &p.sv, 64, hh, tok, bar_v);
+  };
+  auto load_beta = [&](int tok, int end, int hh) -> float {  // thread t < 64: token t
+    return (tid < kC && tok + tid < end) ? __bfloat162float(p.beta[(size_t)(tok + tid) * H + hh])
+                                         : 0.f;
+  };
+
+  bool have = next_item();
+  float beta_nx = 0.f;
+  // e^{A_h} log2(e) of the next item's head, loaded an item ahead
+  float expA_nx = (GS == kGateZ && have) ? expf(p.A[h]) * kLog2e : 0.f;
+  if (have) {
+    if (tid == 0) {
+      stage_qkz(a + c * kC, h);
+      stage_v(a + c * kC, h);
+    }
+    qkz_pending = v_pending = true;
+    beta_nx = load_beta(a + c * kC, e, h);
+  }
+  while (have) {
+    const int hc = h, nc = n, ac = a, ec = e, cc0 = c;
+    h += sh;
+    if (h >= H) { h -= H; ++n; }
+    n += sn;
+    if (n >= p.N) { n -= p.N; ++c; }
+    c += sc;
+    have = next_item();  // the item after this one
+    const int tok0 = ac + cc0 * kC;
+    const int len = min(kC, ec - tok0);
+    const int tokn = have ? a + c * kC : 0, hn = h;
+    unsigned char* slot = chunk_slot(p.prep, ac, nc, cc0, hc, H);
+    if (tid < kC) bvec[tid] = beta_nx;
+    if (have) beta_nx = load_beta(tokn, e, hn);
+
+    // per-channel gate input, issued before the wait
+    float al[16];  // alpha of tokens 16 b + i (then 1 / E)
+    if constexpr (GS == kGateChannel) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int t = 16 * b + i;
+        al[i] = t < len ? p.g[((size_t)(tok0 + t) * H + hc) * kD + j] : 0.f;
+      }
+    } else if constexpr (GS == kGateHead) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int t = 16 * b + i;
+        al[i] = t < len ? p.g[(size_t)(tok0 + t) * H + hc] : 0.f;
+      }
+    }
+    const float expA_l2 = expA_nx;
+    if (GS == kGateZ && have) expA_nx = expf(p.A[hn]) * kLog2e;
+
+    if (!block_wait(bar_qkz, ph_qkz, p.hdr)) { ok = false; break; }
+    qkz_pending = false;
+
+    // ---- A1: row norms (thread: row tid / 4 of [q ; k], 32 channels)
+    {
+      const int r = tid >> 2, qt = tid & 3, t = r & 63;
+      const unsigned char* rowp =
+          sm + (r < 64 ? L::kQ : L::kK) + (qt >> 1) * 8192 + t * 128;
+      float ss = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t un = (uint32_t)(4 * (qt & 1) + u) ^ (uint32_t)(t & 7);
+        float f[8];
+        unpack8(*reinterpret_cast<const uint4*>(rowp + (un << 4)), f);
+#pragma unroll
+        for (int x = 0; x < 8; ++x) ss = fmaf(f[x], f[x], ss);
+      }
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+      if (qt == 0) nrm[r] = t < len ? rsqrtf(ss + kNormEps) : 0.f;
+    }
+    // ---- A2: gate -> alpha; E = e^{Gam - rho_b} (E = 1 at the sub-tile's first token)
+    if constexpr (GS == kGateZ) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float zz = raw_f(L::kZ, i);
+        const float ez = ex2(-expA_l2 * zz);                 // e^{-e^A z}
+        const float sg = rcp(1.0f + ez);                     // sigmoid(e^A z)
+        al[i] = 16 * b + i < len ? ex2((kGateMin * kLog2e) * sg) : 1.0f;  // e^{-5 sigmoid}
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) al[i] = ex2(al[i] * kLog2e);  // masked tokens: g = 0
+    }
+    float E[16];
+    E[0] = 1.0f;
+#pragma unroll
+    for (int i = 1; i < 16; ++i) E[i] = E[i - 1] * al[i];
+    exf[b * 128 + j] = al[0];
+    exl[b * 128 + j] = E[15];
+    // q, k of the thread's tokens (zero past the sequence end)
+    float qv[16], kv[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const bool in = 16 * b + i < len;
+      qv[i] = in ? raw_f(L::kQ, i) : 0.f;
+      kv[i] = in ? raw_f(L::kK, i) : 0.f;
+    }
+    __syncthreads();
+    // the staged q, k, z rows are consumed: load the next item's
+    if (have && tid == 0) stage_qkz(tokn, hn);
+    qkz_pending = have;
+
+    // ---- B: decay factors of (channel j, sub-tile b)
+    float Pb, Lb, F1 = 0.f, F2 = 0.f, F3 = 0.f;  // e^{rho_b}, e^{Gam_last - rho_b}, e^{rho_{b+s} - rho_b}
+    {
+      float a0[4], e15[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        a0[x] = exf[x * 128 + j];
+        e15[x] = exl[x * 128 + j];
+      }
+      float u[3];  // e^{rho_{x+1} - rho_x}
+#pragma unroll
+      for (int x = 0; x < 3; ++x) u[x] = e15[x] * a0[x + 1];
+      Pb = a0[0];
+#pragma unroll
+      for (int x = 0; x < 3; ++x)
+        if (x < b) Pb *= u[x];
+      Lb = b == 0 ? e15[0] : b == 1 ? e15[1] : b == 2 ? e15[2] : e15[3];
+#pragma unroll
+      for (int x = 1; x < 4; ++x)
+        if (x > b) Lb *= a0[x] * e15[x];
+      // F_s = e^{rho_{b+s} - rho_b} = u[b] ... u[b+s-1]
+      const float ub0 = b == 0 ? u[0] : b == 1 ? u[1] : u[2];
+      const float ub1 = b == 0 ? u[1] : u[2];
+      F1 = ub0;
+      F2 = ub0 * ub1;
+      F3 = ub0 * ub1 * u[2];
+      if (b == 0) reinterpret_cast<float*>(slot + kSlotGam)[j] = Pb * Lb;  // gamma = e^{Gam_last}
+      if (tid < kC) reinterpret_cast<float*>(slot + kSlotIq)[tid] = nrm[tid];
+    }
+    // 1 / E by the reverse product: e^{rho_b - Gam_i} = (prod_{s > i} alpha_s) / E_15
+    {
+      float rv = rcp(E[15]);
+#pragma unroll
+      for (int i = 15; i >= 0; --i) {
+        const float ai = al[i];
+        al[i] = rv;
+        rv *= ai;
+      }
+    }
+    float* Ei = al;
+    // k / |k|
+#pragma unroll
+    for (int i = 0; i < 16; ++i) kv[i] *= nrm[64 + 16 * b + i];
+
+    // ---- C: M1 operands.  R rows (beta k^ E, then q E), windows (k^ / E times
+    //      e^{rho_c - rho_b} for the later row sub-tiles c)
+    {
+      float x[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) x[i] = bvec[16 * b + i] * kv[i] * E[i];
+      put16(sm + L::kR, img_unit(32 * b, j, 128), img_unit(32 * b + 8, j, 128), x);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) x[i] = qv[i] * E[i];
+      put16(sm + L::kR, img_unit(32 * b + 16, j, 128), img_unit(32 * b + 24, j, 128), x);
+      float cd[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) cd[i] = kv[i] * Ei[i];
+      {
+        unsigned char* w = sm + L::kWin + (b >> 1) * 32768;
+        const int r0 = 64 * (b & 1) + 16 * b;
+        put16(w, img_unit(r0, j, 128), img_unit(r0 + 8, j, 128), cd);
+      }
+#pragma unroll
+      for (int s = 1; s < 4; ++s) {
+        const int cw = b + s;  // window of row sub-tile cw
+        if (cw < 4) {
+          const float f = s == 1 ? F1 : s == 2 ? F2 : F3;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) x[i] = cd[i] * f;
+          unsigned char* w = sm + L::kWin + (cw >> 1) * 32768;
+          const int r0 = 64 * (cw & 1) + 16 * b;
+          put16(w, img_unit(r0, j, 128), img_unit(r0 + 8, j, 128), x);
+        }
+      }
+      sync_for_mma();
+      // M1: per K step (16 channels) two M=128 x N=64 MMAs: window pair pr
+      // against R rows 64 pr .. 64 pr + 63 (row sub-tiles 2 pr, 2 pr + 1)
+      if (tid == 0) {
+        constexpr uint32_t id = instr_desc(kFmtBF16, 128, 64, true, true);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+#pragma unroll
+          for (int pr = 0; pr < 2; ++pr) {
+            const uint64_t ad = smem_desc(smem_u32(sm + L::kWin + pr * 32768 + k * 4096), 2048, 128);
+            const uint64_t bd = smem_desc(smem_u32(sm + L::kR + pr * 1024 + k * 4096), 2048, 128);
+            mma_bf16(tm + 64 * pr, ad, bd, id, k > 0);
+          }
+        mma_commit(bar_mma);
+      }
+      // meanwhile: X_K = beta k^ e^{Gam} (M2 operand), Q' = q e^{Gam} and
+      // K' = k^ e^{Gam_last - Gam} (slot)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) x[i] = bvec[16 * b + i] * kv[i] * E[i] * Pb;
+      put16h(sm + L::kXK, img_unit(16 * b, j, 64), img_unit(16 * b + 8, j, 64), x);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) x[i] = qv[i] * E[i] * Pb;
+      put16h(slot + kSlotWQ, img_unit(64 + 16 * b, j, 128), img_unit(72 + 16 * b, j, 128), x);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) x[i] = cd[i] * Lb;
+      put16h(slot + kSlotK, img_unit(16 * b, j, 64), img_unit(16 * b + 8, j, 64), x);
+    }
+    if (!block_wait(bar_mma, ph_mma, p.hdr)) { ok = false; break; }
+
+    // ---- D: products -> A_kk (fp32, strictly lower) and A_qk (bf16 slot
+    //      image, lower with the diagonal).  Warp (q4, cq): accumulator pr = cq / 2,
+    //      window w = 2 pr + q4 / 2, key token i = 32 (q4 % 2) + lane, query rows
+    //      16 w .. 16 w + 15; cq % 2 selects A_kk or A_qk.
+    float* Af = reinterpret_cast<float*>(sm + L::kAf);
+    {
+      const int pr = cq >> 1, part = cq & 1, w = 2 * pr + (q4 >> 1), i = 32 * (q4 & 1) + lane;
+      float v[16];
+      tmem_ld16(tmem_addr(tm, 32 * q4, 64 * pr + 32 * (q4 >> 1) + 16 * part), v);
+      tmem_ld_wait();
+      if (part == 0) {
+#pragma unroll
+        for (int x = 0; x < 16; ++x) {
+          const int r = 16 * w + x;
+          Af[r * kLd + i] = i < r ? v[x] : 0.f;
+        }
+      } else {
+#pragma unroll
+        for (int x = 0; x < 16; ++x) v[x] = i <= 16 * w + x ? v[x] : 0.f;
+        put16h(slot + kSlotA, img_unit(16 * w, i, 64), img_unit(16 * w + 8, i, 64), v);
+      }
+    }
+    fence_before_sync();
+    __syncthreads();
+
+    // ---- E: T = (I + A_kk)^{-1} in fp32.  Diagonal 16x16 blocks by forward
+    //      substitution (one warp per block, lane = column), then the blocks below
+    //      them by merging, 16 -> 32 -> 64: [[P,0],[B,Q]]^{-1} has lower-left
+    //      block -Q^{-1} B P^{-1}.
+    float* Tf = reinterpret_cast<float*>(sm + L::kTf);
+    float* TT = reinterpret_cast<float*>(sm + L::kTT);
+    float* Yb = reinterpret_cast<float*>(sm + L::kY);
+    if (warp < 4) {
+      const int base = 16 * warp, cc = lane & 15;
+      float x[16];
+#pragma unroll
+      for (int rr = 0; rr < 16; ++rr) x[rr] = rr == cc ? 1.f : 0.f;
+#pragma unroll
+      for (int m = 0; m < 15; ++m)
+#pragma unroll
+        for (int rr = m + 1; rr < 16; ++rr)
+          x[rr] = fmaf(-Af[(base + rr) * kLd + base + m], x[m], x[rr]);
+      if (lane < 16) {
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) Tf[(base + rr) * kLd + base + cc] = x[rr];
+#pragma unroll
+        for (int rr = 0; rr < 16; rr += 4)
+          *reinterpret_cast<float4*>(TT + (base + cc) * kLd + base + rr) =
+              make_float4(x[rr], x[rr + 1], x[rr + 2], x[rr + 3]);
+      }
+    } else {
+      // zero the upper blocks T[0:16][16:32], T[32:48][48:64] (and in T^T)
+      for (int u = tid - 128; u < 512; u += 384) {
+        const int blk = u >> 8, rr = (u >> 4) & 15, c2 = u & 15;
+        const int r = 32 * blk + rr, col = 32 * blk + 16 + c2;
+        Tf[r * kLd + col] = 0.f;
+        TT[col * kLd + r] = 0.f;
+      }
+    }
+    __syncthreads();
+    // 16 -> 32 for the pairs (0, 1) and (2, 3): Y = A[hi][lo] T[lo][lo]
+    {
+      const int pr = tid >> 8, r = (tid >> 4) & 15, c2 = tid & 15;
+      const int lo = 32 * pr, hi = lo + 16;
+      const float* ar = Af + (hi + r) * kLd + lo;
+      const float* tr = TT + (lo + c2) * kLd + lo;
+      float y = 0.f;
+#pragma unroll
+      for (int m = 0; m < 16; m += 4) {
+        const float4 x4 = *reinterpret_cast<const float4*>(ar + m);
+        const float4 t4 = *reinterpret_cast<const float4*>(tr + m);
+        y = fmaf(x4.x, t4.x, fmaf(x4.y, t4.y, fmaf(x4.z, t4.z, fmaf(x4.w, t4.w, y))));
+      }
+      Yb[(lo + c2) * kLd + r] = y;  // Y^T
+    }
+    __syncthreads();
+    // T[hi][lo] = -T[hi][hi] Y
+    {
+      const int pr = tid >> 8, r = (tid >> 4) & 15, c2 = tid & 15;
+      const int lo = 32 * pr, hi = lo + 16;
+      const float* tr = Tf + (hi + r) * kLd + hi;
+      const float* yr = Yb + (lo + c2) * kLd;
+      float t = 0.f;
+#pragma unroll
+      for (int m = 0; m < 16; m += 4) {
+        const float4 x4 = *reinterpret_cast<const float4*>(tr + m);
+        const float4 y4 = *reinterpret_cast<const float4*>(yr + m);
+        t = fmaf(x4.x, y4.x, fmaf(x4.y, y4.y, fmaf(x4.z, y4.z, fmaf(x4.w, y4.w, t))));
+      }
+      Tf[(hi + r) * kLd + lo + c2] = -t;
+      TT[(lo + c2) * kLd + hi + r] = -t;
+    }
+    __syncthreads();
+    // T -> the M2 operands, 8 columns k0 .. k0+7 of row r per 16-byte unit (upper
+    // triangle zero): T (f16) and T Diag(beta) (bf16, with the bf16 v rows)
+    auto put_t = [&](int r, int k0) {
+      float t8[8], tb8[8];
+      ld8f(Tf + r * kLd + k0, t8);
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        t8[x] = k0 + x <= r ? t8[x] : 0.f;
+        tb8[x] = t8[x] * bvec[k0 + x];
+      }
+      *reinterpret_cast<uint4*>(sm + L::kTb + img_unit(k0, r, 64)) = pack8h(t8);
+      *reinterpret_cast<uint4*>(sm + L::kTbb + img_unit(k0, r, 64)) = pack8(tb8);
+    };
+    // 32 -> 64 on threads 0..255 (2 x 2 tiles: rows 2 rp, 2 rp + 1 and columns
+    // 2 cp, 2 cp + 1 of the lower-left 32 x 32 block); meanwhile threads 256..511
+    // convert the final blocks T[0:32][0:64] and T[32:64][32:64]
+    const int rp = ((tid >> 5) & 3) * 4 + (lane & 3), cp = (tid >> 7) * 8 + ((lane >> 2) & 7);
+    if (tid < 256) {
+      // Y = A[32:64][0:32] T[0:32][0:32]
+      const float* a0 = Af + (32 + 2 * rp) * kLd;
+      const float* a1 = a0 + kLd;
+      const float* t0 = TT + (2 * cp) * kLd;
+      const float* t1 = t0 + kLd;
+      float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+#pragma unroll
+      for (int m = 0; m < 32; m += 4) {
+        const float4 x0 = *reinterpret_cast<const float4*>(a0 + m);
+        const float4 x1 = *reinterpret_cast<const float4*>(a1 + m);
+        const float4 u0 = *reinterpret_cast<const float4*>(t0 + m);
+        const float4 u1 = *reinterpret_cast<const float4*>(t1 + m);
+        y00 = fmaf(x0.x, u0.x, fmaf(x0.y, u0.y, fmaf(x0.z, u0.z, fmaf(x0.w, u0.w, y00))));
+        y01 = fmaf(x0.x, u1.x, fmaf(x0.y, u1.y, fmaf(x0.z, u1.z, fmaf(x0.w, u1.w, y01))));
+        y10 = fmaf(x1.x, u0.x, fmaf(x1.y, u0.y, fmaf(x1.z, u0.z, fmaf(x1.w, u0.w, y10))));
+        y11 = fmaf(x1.x, u1.x, fmaf(x1.y, u1.y, fmaf(x1.z, u1.z, fmaf(x1.w, u1.w, y11))));
+      }
+      *reinterpret_cast<float2*>(Yb + (2 * cp) * kLd + 2 * rp) = make_float2(y00, y10);      // Y^T
+      *reinterpret_cast<float2*>(Yb + (2 * cp + 1) * kLd + 2 * rp) = make_float2(y01, y11);
+    } else {
+      for (int u = tid - 256; u < 384; u += 256) {
+        // units 0..255: rows 0..31, k0 = 0..56; units 256..383: rows 32..63, k0 = 32..56
+        const int r = u < 256 ? (u & 31) : 32 + (u & 31);
+        const int k0 = u < 256 ? (u >> 5) * 8 : 32 + ((u - 256) >> 5) * 8;
+        put_t(r, k0);
+      }
+    }
+    if (tid < 256) {
+      asm volatile("bar.sync 1, 256;" ::: "memory");  // threads 0..255 only: Y is complete
+      // T[32:64][0:32] = -T[32:64][32:64] Y
+      const float* r0 = Tf + (32 + 2 * rp) * kLd + 32;
+      const float* r1 = r0 + kLd;
+      const float* y0 = Yb + (2 * cp) * kLd;
+      const float* y1 = y0 + kLd;
+      float t00 = 0.f, t01 = 0.f, t10 = 0.f, t11 = 0.f;
+#pragma unroll
+      for (int m = 0; m < 32; m += 4) {
+        const float4 x0 = *reinterpret_cast<const float4*>(r0 + m);
+        const float4 x1 = *reinterpret_cast<const float4*>(r1 + m);
+        const float4 u0 = *reinterpret_cast<const float4*>(y0 + m);
+        const float4 u1 = *reinterpret_cast<const float4*>(y1 + m);
+        t00 = fmaf(x0.x, u0.x, fmaf(x0.y, u0.y, fmaf(x0.z, u0.z, fmaf(x0.w, u0.w, t00))));
+        t01 = fmaf(x0.x, u1.x, fmaf(x0.y, u1.y, fmaf(x0.z, u1.z, fmaf(x0.w, u1.w, t01))));
+        t10 = fmaf(x1.x, u0.x, fmaf(x1.y, u0.y, fmaf(x1.z, u0.z, fmaf(x1.w, u0.w, t10))));
+        t11 = fmaf(x1.x, u1.x, fmaf(x1.y, u1.y, fmaf(x1.z, u1.z, fmaf(x1.w, u1.w, t11))));
+      }
+      *reinterpret_cast<float2*>(Tf + (32 + 2 * rp) * kLd + 2 * cp) = make_float2(-t00, -t01);
+      *reinterpret_cast<float2*>(Tf + (33 + 2 * rp) * kLd + 2 * cp) = make_float2(-t10, -t11);
+    }
+    __syncthreads();
+    // the merged block T[32:64][0:32]
+    if (tid < 128) put_t(32 + (tid & 31), (tid >> 5) * 8);
+    // the v rows must have landed (a block-wide wait that also orders the T images)
+    fence_async_smem();
+    fence_before_sync();
+    if (!block_wait(bar_v, ph_v, p.hdr)) { ok = false; break; }
+    v_pending = false;
+    // ---- M2: W^T = X_K^T T^T -> TMEM columns 0-63 and U~^T = V^T (T Diag(beta))^T
+    //      -> 64-127 (M = 128 channels, N = 64 tokens; V read in place from its
+    //      swizzled tile as an MN-major operand)
+    if (tid == 0) {
+      constexpr uint32_t idw = instr_desc(kFmtF16, 128, 64, false, false);
+      constexpr uint32_t idu = instr_desc(kFmtBF16, 128, 64, true, false);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint64_t xd = smem_desc(smem_u32(sm + L::kXK + k * 256), 128, 1024);
+        const uint64_t tb = smem_desc(smem_u32(sm + L::kTb + k * 256), 128, 1024);
+        const uint64_t vd = smem_desc_sw128(smem_u32(sm + L::kV + k * 2048), 8192, 1024);
+        const uint64_t tbb = smem_desc(smem_u32(sm + L::kTbb + k * 256), 128, 1024);
+        mma_bf16(tm, xd, tb, idw, k > 0);
+        mma_bf16(tm + 64, vd, tbb, idu, k > 0);
+      }
+      mma_commit(bar_mma);
+    }
+    if (!block_wait(bar_mma, ph_mma, p.hdr)) { ok = false; break; }
+    // v is consumed: load the next item's
+    if (have && tid == 0) stage_v(tokn, hn);
+    v_pending = have;
+    // ---- F: W (into the [W ; Q'] image) and U~^T -> slot
+    {
+      const int ch = 32 * q4 + lane;
+      float w16[16], u16[16];
+      tmem_ld16(tmem_addr(tm, 32 * q4, 16 * cq), w16);
+      tmem_ld16(tmem_addr(tm, 32 * q4, 64 + 16 * cq), u16);
+      tmem_ld_wait();
+      put16h(slot + kSlotWQ, img_unit(16 * cq, ch, 128), img_unit(16 * cq + 8, ch, 128), w16);
+      uint4* ug = reinterpret_cast<uint4*>(slot + kSlotU);
+      ug[ut_index(q4, cq, 0, lane)] = pack8h(u16);
+      ug[ut_index(q4, cq, 1, lane)] = pack8h(u16 + 8);
+    }
+    fence_before_sync();
+  }
+  if (tid == 0) {
+    // a wait gave up: let the row loads still in flight land before leaving
+    if (qkz_pending) (void)mbar_wait_cycles(bar_qkz, ph_qkz, kWaitCycles);
+    if (v_pending) (void)mbar_wait_cycles(bar_v, ph_v, kWaitCycles);
+  }
+  (void)ok;
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tm, 128);
+}
+
+}  // namespace
+
+size_t prep_tc_smem_bytes() { return PrepSmem::kBytes; }
+
+cudaError_t launch_prep_tc(const TcParams& p, int gs, cudaStream_t st) {
+  auto prep = gs == kGateHead ? prep_kernel<kGateHead>
+            : gs == kGateChannel ? prep_kernel<kGateChannel> : prep_kernel<kGateZ>;
+  cudaError_t err = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         PrepSmem::kBytes);
+  if (err != cudaSuccess) return err;
+  int sms = 0, dev = 0;
+  if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+  if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return err;
+  prep<<<sms, kNT, PrepSmem::kBytes, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace tcp
+}  // namespace kda

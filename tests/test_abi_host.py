@@ -57,17 +57,16 @@ def test_workspace_size(L):
 
 
 def test_workspace_holds_one_chunk_slot_per_chunk_and_head(L):
-    """A segmented bf16 problem (one long sequence, few heads) stores one chunk
-    slot of 74,496 bytes per (chunk, head) for every chunk id cu[n]/64 + n + j
-    below T/64 + N; an unsegmented one (many sequences x heads) needs none."""
+    """The bf16 tensor-core path stores one chunk slot of 74,496 bytes per
+    (chunk, head) for every chunk id cu[n]/64 + n + j below T/64 + N, whether
+    the sequences are cut into segments (one long sequence, few heads) or not
+    (many sequences x heads); the segment maps add at most a few MB."""
     ws = kda.kda_forward_workspace_size
     slot = 74496
-    for T, H in ((4096, 16), (65536, 16), (8192, 4)):
-        size = ws(1, T, T, H, 128, 128, kda.KDA_BF16, 64)
-        need = (T // 64 + 1) * H * slot
-        assert need <= size <= need + 64 * 1024 * 1024, (T, H, size, need)
-    # 8 sequences x 16 heads = 128 (sequence, head) pairs fill the GPU: no segments
-    assert ws(8, 8 * 4096, 4096, 16, 128, 128, kda.KDA_BF16, 64) < 8 * 16 * slot
+    for N, T, H in ((1, 4096, 16), (1, 65536, 16), (1, 8192, 4), (8, 8 * 4096, 16)):
+        size = ws(N, T, T // N, H, 128, 128, kda.KDA_BF16, 64)
+        need = (T // 64 + N) * H * slot
+        assert need <= size <= need + 64 * 1024 * 1024, (N, T, H, size, need)
 
 
 FAKE = 0x10000  # aligned fake device address: never dereferenced by these calls
