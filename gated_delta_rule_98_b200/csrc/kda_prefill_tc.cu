@@ -51,11 +51,12 @@ __device__ __forceinline__ float* ckpt_state(const TcParams& p, int n, int h, in
 template <bool TRANS>
 struct ChainSmem {
   static constexpr int kStages = 3;
-  // stage layout: the slot (full pass), or W (64-row image) | K' | U~^T | gamma (transition)
-  static constexpr int kK = TRANS ? 16384 : kSlotK;
-  static constexpr int kUt = TRANS ? 32768 : kSlotU;
-  static constexpr int kGam = TRANS ? 32768 + 16384 : kSlotGam;
-  static constexpr int kStageBytes = TRANS ? 32768 + 16384 + 512 : kSlotBytes;
+  // stage layout: the slot (full pass), or [W ; Q'] | K' | U~^T | gamma (transition:
+  // the slot without A_qk and 1/|q|; one bulk copy per part)
+  static constexpr int kK = TRANS ? 32768 : kSlotK;
+  static constexpr int kUt = TRANS ? 49152 : kSlotU;
+  static constexpr int kGam = TRANS ? 49152 + 16384 : kSlotGam;
+  static constexpr int kStageBytes = TRANS ? 49152 + 16384 + 512 : kSlotBytes;
   static constexpr int kBytes = kStages * kStageBytes;
 };
 // TMEM columns (512 allocated): fp32 S^T, fp32 X^T (transition), the products D^T
@@ -113,9 +114,7 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
     const unsigned char* src = chunk_slot(p.prep, a, n, c, h, H);
     mbar_arrive_expect_tx(&s_ld[s], L::kStageBytes);
     if (TRANS) {
-      // W: the first 1024 bytes (tokens 0..63) of each 8-channel group of [W ; Q']
-#pragma unroll 1
-      for (int g = 0; g < 16; ++g) bulk_g2s(dst + g * 1024, src + kSlotWQ + g * 2048, 1024, &s_ld[s]);
+      bulk_g2s(dst, src + kSlotWQ, 32768, &s_ld[s]);                     // [W ; Q']
       bulk_g2s(dst + L::kK, src + kSlotK, 16384, &s_ld[s]);             // K'
       bulk_g2s(dst + L::kUt, src + kSlotU, 16384 + 512, &s_ld[s]);      // U~^T | gamma
     } else {
@@ -284,7 +283,7 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
         constexpr uint32_t id = instr_desc(kFmtF16, 128, 64, false, true);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const uint64_t bd = smem_desc(smem_u32(st + k * 2048), 1024, 128);
+          const uint64_t bd = smem_desc(smem_u32(st + k * 4096), 2048, 128);  // the W rows
           mma_f16_ts(tm + TM::kD0, tm + TM::kCp + 8 * k, bd, id, k > 0);
           mma_f16_ts(tm + TM::kD0 + 64, tm + TM::kCp + 64 + 8 * k, bd, id, k > 0);
         }
@@ -323,17 +322,17 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
     __syncthreads();
     fence_after_sync();
     // ---- C2: S^T (X^T) += U^T K' (B = K' K-major: N = key channel, K = token);
-    //      D_Q^T += U^T A_qk^T (B MN-major: N = query row, K = key row)
+    //      D_Q^T += U^T A_qk^T (B K-major: N = query row, K = key row)
     if (tid == 0) {
       constexpr uint32_t ids = instr_desc(kFmtF16, 128, 128, false, false);
-      constexpr uint32_t ido = instr_desc(kFmtF16, 128, 64, false, true);
+      constexpr uint32_t ido = instr_desc(kFmtF16, 128, 64, false, false);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const uint64_t kd = smem_desc(smem_u32(st + L::kK + k * 256), 128, 1024);
         mma_f16_ts(tm + TM::kS, tm + TM::kCp + 8 * k, kd, ids, 1);
         if (TRANS) mma_f16_ts(tm + TM::kX, tm + TM::kCp + 64 + 8 * k, kd, ids, 1);
         if (!TRANS) {
-          const uint64_t ad = smem_desc(smem_u32(st + kSlotA + k * 2048), 1024, 128);
+          const uint64_t ad = smem_desc(smem_u32(st + kSlotA + k * 256), 128, 1024);
           mma_f16_ts(tm + dcol + 64, tm + TM::kCp + 8 * k, ad, ido, 1);
         }
       }

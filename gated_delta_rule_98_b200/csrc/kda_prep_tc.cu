@@ -37,19 +37,25 @@ namespace {
 
 constexpr int kLd = 68;  // row stride (floats) of the fp32 work matrices of the inverse
 
+// Windows: window w (the column operand of row sub-tile w) holds the 16 (w + 1)
+// tokens of sub-tiles 0 .. w and starts at row 8 w (w + 1) of one 160-row image.
+__host__ __device__ constexpr int win_row0(int w) { return 8 * w * (w + 1); }
+constexpr int kWinRows = 160;
+
 struct PrepSmem {
   // staged rows: two 64-channel boxes [64 tokens][64 channels] per tensor, 128-byte swizzle
   static constexpr int kQ = 0, kK = 16384, kZ = 32768, kV = 49152;
-  static constexpr int kWin = 65536;        // windows: pair p (windows 2p, 2p+1) = 128-row image
-  static constexpr int kR = kWin + 65536;   // R: 128-row image (sub-tile b: k rows 32b.., q rows 32b+16..)
-  static constexpr int kXK = kR + 32768;    // X_K: 64-row f16 image, the A operand X_K^T of M2
+  static constexpr int kWB = 65536;               // windows, 160-row image: the B operand of M1
+  static constexpr int kR = kWB + kWinRows * 256; // R: 128-row image (sub-tile b: k rows 32b..,
+                                                  //   q rows 32b+16..), the A operand of M1
   // after M1 the window / R region holds the inverse's work and the T images
-  static constexpr int kAf = kWin;                // A_kk fp32 [64][kLd], row r, column i
-  static constexpr int kTf = kAf + 64 * kLd * 4;  // T fp32 [64][kLd]
+  static constexpr int kAf = kWB;                 // A_kk fp32 [64][kLd], row r, column i
+  static constexpr int kAT = kAf + 64 * kLd * 4;  // merge products, transposed [64][kLd]
+  static constexpr int kTf = kAT + 64 * kLd * 4;  // T fp32 [64][kLd]
   static constexpr int kTT = kTf + 64 * kLd * 4;  // T^T fp32 [64][kLd]
-  static constexpr int kY = kTT + 64 * kLd * 4;   // merge products, transposed [64][kLd]
-  static constexpr int kTb = kWin + 69632;        // T, the B operand T^T of M2 (64-row f16 image)
+  static constexpr int kTb = kTT + 64 * kLd * 4;  // T, the B operand T^T of M2 (64-row f16 image)
   static constexpr int kTbb = kTb + 8192;         // T Diag(beta), the same for U~ (bf16, with V)
+  static constexpr int kXK = kTbb + 8192;         // X_K: 64-row f16 image, the A operand X_K^T of M2
   static constexpr int kNrm = kXK + 16384;        // 1/|q| (64), 1/|k| (64)
   static constexpr int kBeta = kNrm + 512;        // beta (64)
   static constexpr int kEx = kBeta + 256;         // [4][128] alpha at each sub-tile's first token,
@@ -57,8 +63,7 @@ struct PrepSmem {
   static constexpr int kBar = kEx + 4096;         // three mbarriers, then the TMEM base
   static constexpr int kBytes = kBar + 64;
 };
-static_assert(PrepSmem::kY + 64 * kLd * 4 <= PrepSmem::kTb, "inverse work overlaps T images");
-static_assert(PrepSmem::kTbb + 8192 <= PrepSmem::kXK, "T images overlap X_K");
+static_assert(PrepSmem::kR + 32768 <= PrepSmem::kXK, "M1 operands overlap X_K");
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -116,7 +121,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     return;
   }
   if (warp == 0) {
-    tmem_alloc(s_tmem, 128);
+    tmem_alloc(s_tmem, 256);
     tmem_relinquish();
   }
   if (tid == 0) {
@@ -184,15 +189,18 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     tma_box_x(sm + L::kV, &p.sv, 0, hh, tok, bar_v);
     tma_box_x(sm + L::kV + 8192, &p.sv, 64, hh, tok, bar_v);
   };
-  auto load_beta = [&](int tok, int end, int hh) -> float {  // thread t < 64: token t
-    return (tid < kC && tok + tid < end) ? __bfloat162float(p.beta[(size_t)(tok + tid) * H + hh])
-                                         : 0.f;
+  // beta of an item's token t = tid < 64 as raw bf16 bits (converted when used, so
+  // the load is not waited for until the next item)
+  auto load_beta = [&](int tok, int end, int hh) -> uint32_t {
+    return (tid < kC && tok + tid < end)
+               ? (uint32_t)reinterpret_cast<const uint16_t*>(p.beta)[(size_t)(tok + tid) * H + hh]
+               : 0u;
   };
 
   bool have = next_item();
-  float beta_nx = 0.f;
-  // e^{A_h} log2(e) of the next item's head, loaded an item ahead
-  float expA_nx = (GS == kGateZ && have) ? expf(p.A[h]) * kLog2e : 0.f;
+  uint32_t beta_nx = 0u;
+  // A_h of the next item's head, loaded an item ahead
+  float a_nx = (GS == kGateZ && have) ? p.A[h] : 0.f;
   if (have) {
     if (tid == 0) {
       stage_qkz(a + c * kC, h);
@@ -213,7 +221,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     const int len = min(kC, ec - tok0);
     const int tokn = have ? a + c * kC : 0, hn = h;
     unsigned char* slot = chunk_slot(p.prep, ac, nc, cc0, hc, H);
-    if (tid < kC) bvec[tid] = beta_nx;
+    if (tid < kC) bvec[tid] = __uint_as_float(beta_nx << 16);
     if (have) beta_nx = load_beta(tokn, e, hn);
 
     // per-channel gate input, issued before the wait
@@ -231,8 +239,8 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
         al[i] = t < len ? p.g[(size_t)(tok0 + t) * H + hc] : 0.f;
       }
     }
-    const float expA_l2 = expA_nx;
-    if (GS == kGateZ && have) expA_nx = expf(p.A[hn]) * kLog2e;
+    const float expA_l2 = GS == kGateZ ? expf(a_nx) * kLog2e : 0.f;
+    if (GS == kGateZ && have) a_nx = p.A[hn];
 
     if (!block_wait(bar_qkz, ph_qkz, p.hdr)) { ok = false; break; }
     qkz_pending = false;
@@ -345,9 +353,8 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
 #pragma unroll
       for (int i = 0; i < 16; ++i) cd[i] = kv[i] * Ei[i];
       {
-        unsigned char* w = sm + L::kWin + (b >> 1) * 32768;
-        const int r0 = 64 * (b & 1) + 16 * b;
-        put16(w, img_unit(r0, j, 128), img_unit(r0 + 8, j, 128), cd);
+        const int r0 = win_row0(b) + 16 * b;
+        put16(sm + L::kWB, img_unit(r0, j, kWinRows), img_unit(r0 + 8, j, kWinRows), cd);
       }
 #pragma unroll
       for (int s = 1; s < 4; ++s) {
@@ -356,24 +363,21 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
           const float f = s == 1 ? F1 : s == 2 ? F2 : F3;
 #pragma unroll
           for (int i = 0; i < 16; ++i) x[i] = cd[i] * f;
-          unsigned char* w = sm + L::kWin + (cw >> 1) * 32768;
-          const int r0 = 64 * (cw & 1) + 16 * b;
-          put16(w, img_unit(r0, j, 128), img_unit(r0 + 8, j, 128), x);
+          const int r0 = win_row0(cw) + 16 * b;
+          put16(sm + L::kWB, img_unit(r0, j, kWinRows), img_unit(r0 + 8, j, kWinRows), x);
         }
       }
       sync_for_mma();
-      // M1: per K step (16 channels) two M=128 x N=64 MMAs: window pair pr
-      // against R rows 64 pr .. 64 pr + 63 (row sub-tiles 2 pr, 2 pr + 1)
+      // M1: D[R row][window row] = R W^T, per K step (16 channels) one M=128 x
+      // N=160 MMA (both operands MN-major: 8 tokens of a channel per 16 bytes)
       if (tid == 0) {
-        constexpr uint32_t id = instr_desc(kFmtBF16, 128, 64, true, true);
+        constexpr uint32_t id = instr_desc(kFmtBF16, 128, kWinRows, true, true);
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-#pragma unroll
-          for (int pr = 0; pr < 2; ++pr) {
-            const uint64_t ad = smem_desc(smem_u32(sm + L::kWin + pr * 32768 + k * 4096), 2048, 128);
-            const uint64_t bd = smem_desc(smem_u32(sm + L::kR + pr * 1024 + k * 4096), 2048, 128);
-            mma_bf16(tm + 64 * pr, ad, bd, id, k > 0);
-          }
+        for (int k = 0; k < 8; ++k) {
+          const uint64_t ad = smem_desc(smem_u32(sm + L::kR + k * 4096), 2048, 128);
+          const uint64_t bd = smem_desc(smem_u32(sm + L::kWB + k * 2 * kWinRows * 16), kWinRows * 16, 128);
+          mma_bf16(tm, ad, bd, id, k > 0);
+        }
         mma_commit(bar_mma);
       }
       // meanwhile: X_K = beta k^ e^{Gam} (M2 operand), Q' = q e^{Gam} and
@@ -390,26 +394,31 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     }
     if (!block_wait(bar_mma, ph_mma, p.hdr)) { ok = false; break; }
 
-    // ---- D: products -> A_kk (fp32, strictly lower) and A_qk (bf16 slot
-    //      image, lower with the diagonal).  Warp (q4, cq): accumulator pr = cq / 2,
-    //      window w = 2 pr + q4 / 2, key token i = 32 (q4 % 2) + lane, query rows
-    //      16 w .. 16 w + 15; cq % 2 selects A_kk or A_qk.
+    // ---- D: products -> A_kk (fp32, strictly lower) and A_qk (f16 slot image,
+    //      lower with the diagonal).  Warp (q4, cq): R rows 32 q4 + lane, i.e. row sub-tile q4 (lanes
+    //      0-15 its k rows, 16-31 its q rows); key tokens i = 16 cq .. 16 cq + 15 from
+    //      window q4 (cq <= q4).
     float* Af = reinterpret_cast<float*>(sm + L::kAf);
     {
-      const int pr = cq >> 1, part = cq & 1, w = 2 * pr + (q4 >> 1), i = 32 * (q4 & 1) + lane;
+      const bool krow = lane < 16;
+      const int r = 16 * q4 + (lane & 15), i0 = 16 * cq;
       float v[16];
-      tmem_ld16(tmem_addr(tm, 32 * q4, 64 * pr + 32 * (q4 >> 1) + 16 * part), v);
-      tmem_ld_wait();
-      if (part == 0) {
+      if (cq <= q4) {
+        tmem_ld16(tmem_addr(tm, 32 * q4, win_row0(q4) + i0), v);
+        tmem_ld_wait();
+      }
+      if (krow) {
+        if (cq <= q4) {
 #pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const int r = 16 * w + x;
-          Af[r * kLd + i] = i < r ? v[x] : 0.f;
+          for (int x = 0; x < 16; ++x) v[x] = i0 + x < r ? v[x] : 0.f;
+#pragma unroll
+          for (int x = 0; x < 16; x += 4)
+            *reinterpret_cast<float4*>(Af + r * kLd + i0 + x) = make_float4(v[x], v[x + 1], v[x + 2], v[x + 3]);
         }
       } else {
 #pragma unroll
-        for (int x = 0; x < 16; ++x) v[x] = i <= 16 * w + x ? v[x] : 0.f;
-        put16h(slot + kSlotA, img_unit(16 * w, i, 64), img_unit(16 * w + 8, i, 64), v);
+        for (int x = 0; x < 16; ++x) v[x] = (cq <= q4 && i0 + x <= r) ? v[x] : 0.f;
+        put16h(slot + kSlotA, img_unit(i0, r, 64), img_unit(i0 + 8, r, 64), v);
       }
     }
     fence_before_sync();
@@ -421,7 +430,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     //      block -Q^{-1} B P^{-1}.
     float* Tf = reinterpret_cast<float*>(sm + L::kTf);
     float* TT = reinterpret_cast<float*>(sm + L::kTT);
-    float* Yb = reinterpret_cast<float*>(sm + L::kY);
+    float* Yb = reinterpret_cast<float*>(sm + L::kAT);  // merge products, transposed
     if (warp < 4) {
       const int base = 16 * warp, cc = lane & 15;
       float x[16];
@@ -601,7 +610,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
   (void)ok;
   fence_before_sync();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tm, 128);
+  if (warp == 0) tmem_dealloc(tm, 256);
 }
 
 }  // namespace

@@ -53,9 +53,9 @@ __host__ __device__ constexpr uint32_t img_unit(int t0, int c, int rows) {
 //   WQ   [W ; Q'] as one 128-row image (W tokens 0..63, Q' tokens 64..127), the
 //        B operand of C1 (N = 128 tokens, K = dk), MN-major.
 //   K    K' (64-row image): the A operand K'^T of C2 (M = dk, K = token), K-major.
-//   A    A_qk with query row r as the "token" and key column i as the channel
+//   A    A_qk with key column i as the "token" and query row r as the channel
 //        (64 x 64): the B operand A_qk^T of the output update (N = r, K = i),
-//        MN-major.
+//        K-major.
 //   U    U~^T (bf16 [dv][token]) in the order the chain threads read it (ut_index).
 //   Gam  gamma = e^{Gam_last} per key channel (128 fp32); Iq 1/|q| per token (64 fp32).
 constexpr int kSlotWQ = 0, kSlotK = 32768, kSlotA = 49152, kSlotU = 57344, kSlotGam = 73728,
