@@ -238,6 +238,115 @@ def time_configs(dev, stream, pk, world, rank_max, barrier, warmup, log_fn):
     return res
 
 
+def strong_scaling_value(total_units, ms_max):
+    """Whole-job throughput when the ranks share one problem of total_units."""
+    return total_units / (ms_max / 1e3)
+
+
+def shard_bounds(T, world, rank):
+    """Contiguous token range [a, b) of rank `rank` out of `world` (chunk-aligned)."""
+    per = ((T + world - 1) // world + CHUNK - 1) // CHUNK * CHUNK
+    a = min(T, rank * per)
+    return a, min(T, a + per)
+
+
+def cp_parity(o_shard, o_ref_shard, S_after, S_ref, last, world, device=None):
+    """Agreement of a context-parallel run with the single-GPU call, reduced over
+    the ranks: (max-abs over sampled o rows, their relative L2, max-abs of the
+    final state held by the last rank)."""
+    import torch
+    rows = torch.arange(0, o_shard.shape[0], 97, device=o_shard.device)
+    g, w = o_shard[rows].double(), o_ref_shard[rows].double()
+    err = float((g - w).abs().max()) if rows.numel() else 0.0
+    num, den = float(((g - w) ** 2).sum()), float((w ** 2).sum())
+    serr = float((S_after.double() - S_ref.double()).abs().max()) if last else 0.0
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([err, serr], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        n = torch.tensor([num, den], dtype=torch.float64, device=device)
+        dist.all_reduce(n, op=dist.ReduceOp.SUM)
+        err, serr, num, den = float(t[0]), float(t[1]), float(n[0]), float(n[1])
+    return err, (num / den) ** 0.5 if den > 0 else 0.0, serr
+
+
+def run_cp(args):
+    """Context parallelism: one sequence of args.L tokens split into contiguous
+    shards, one per rank (strong scaling); a step is one
+    cp.context_parallel_forward (local pass, one all-gather of the shard maps,
+    prefix fold, finishing pass)."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from gated_delta_rule_98_b200 import cp, kda, synth
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    L = args.L
+    inp = synth.workload("long", L=L)
+    d = {k_: (v_.to(dev) if isinstance(v_, torch.Tensor) else v_) for k_, v_ in inp.items()}
+    a, b = shard_bounds(L, world, rank)
+    sh = {k_: d[k_][a:b].contiguous() for k_ in ("q", "k", "v", "z", "beta")}
+    # the single-GPU call on the whole sequence (untimed), for the parity check
+    o_ref, S_ref = kda.forward(d["q"], d["k"], d["v"], d["z"], d["A"], d["beta"], num_seqs=1,
+                               chunk=CHUNK)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def step(ev=None):
+        return cp.context_parallel_forward(sh["q"], sh["k"], sh["v"], sh["z"], d["A"], sh["beta"],
+                                           max_seqlen=b - a, chunk=CHUNK, events=ev)
+
+    for _ in range(args.warmup):
+        o_sh, S_after = step()
+    torch.cuda.synchronize()
+    err, rel, serr = cp_parity(o_sh, o_ref[a:b], S_after[0], S_ref[0], rank == world - 1, world,
+                               dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ag_ms = 0.0
+    e0.record(stream)
+    for _ in range(args.steps):
+        step((g0, g1))
+        g1.synchronize()
+        ag_ms += g0.elapsed_time(g1)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_local = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms_local, world, dev)
+    ag = max_over_ranks(ag_ms / args.steps, world, dev)
+    fl = kda.kda_forward_launches(1, b - a, b - a, H, D, D, kda.KDA_BF16, CHUNK)
+    launches = 3 + rank + (2 if fl == 4 else 1)  # local pass, folds, finishing pass
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": METRIC, "value": strong_scaling_value(L, ms), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "mode": "context_parallel",
+        "config": {"workload": f"KDA fwd long, one sequence split over the ranks: B=1 H={H} "
+                               f"L={L} dk=dv={D}, bf16 inputs, fp32 state, chunk {CHUNK}",
+                   "B": 1, "H": H, "L": L, "shard_tokens": b - a,
+                   "parallelism": f"context parallel x{world} (one all-gather of the shard maps)"},
+        "allgather_ms": ag, "allgather_share": ag / ms if ms > 0 else None,
+        "parity_vs_single_gpu": {"o_sampled_max_abs": err, "o_sampled_rel_l2": rel,
+                                 "S_final_max_abs": serr, "bar": "max-abs 2e-2, rel-L2 5e-3"},
+        "gpu_launches": launches * args.steps,
+    }), flush=True)
+
+
 def oracle_baseline(inp, n_tokens):
     """Float64 oracle on the first n_tokens of the workload (all heads)."""
     from oracle import ref
@@ -286,6 +395,9 @@ def main():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
+    ap.add_argument("--mode", choices=["weak", "cp"], default="weak",
+                    help="weak: one independent problem per rank (default); cp: one sequence "
+                         "split over the ranks (context parallelism, strong scaling)")
     ap.add_argument("--L", type=int, default=L_DEFAULT, help="prefill length (sweep)")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -298,6 +410,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.mode == "cp":
+        return run_cp(args)
 
     import torch
     import torch.distributed as dist

@@ -44,24 +44,33 @@ class _KdaOps:
 
 
 def context_parallel_forward(q, k, v, z, A, beta, *, S0=None, cu_seqlens=None, max_seqlen=None,
-                             chunk=64, group=None, ops=None):
+                             chunk=64, group=None, ops=None, events=None):
     """KDA prefill of this rank's shard of the sequences split over ``group``.
 
     q, k, z [T_r,H,dk], v [T_r,H,dv], beta [T_r,H]: this rank's tokens (the
     same sequences on every rank, each rank holding the next contiguous piece
     of each); S0 [N,H,dk,dv] the sequences' initial states (read on every rank,
-    used by rank 0's fold); cu_seqlens the shard's own offsets.  Returns
-    (o [T_r,H,dv], S_after [N,H,dk,dv]): on the last rank S_after is the
-    sequences' final state.
+    used by rank 0's fold); cu_seqlens the shard's own offsets.  ``events``,
+    a pair of CUDA events, if given, is recorded around the all-gather (its
+    share of the call).  Returns (o [T_r,H,dv], S_after [N,H,dk,dv]): on the
+    last rank S_after is the sequences' final state.
     """
     ops = ops or _KdaOps()
-    rank = dist.get_rank(group)
-    world = dist.get_world_size(group)
+    alone = not dist.is_initialized()  # one rank without a process group
+    rank = 0 if alone else dist.get_rank(group)
+    world = 1 if alone else dist.get_world_size(group)
     M, N, shard = ops.local(q, k, v, z, A, beta, cu_seqlens, max_seqlen, chunk)
     dk = M.shape[-1]
     packed = torch.cat([M, N], dim=-1).contiguous()          # [N,H,dk,dk+dv]
     gathered = [torch.empty_like(packed) for _ in range(world)]
-    dist.all_gather(gathered, packed, group=group)
+    if events is not None:
+        events[0].record()
+    if world > 1:
+        dist.all_gather(gathered, packed, group=group)
+    else:
+        gathered[0] = packed
+    if events is not None:
+        events[1].record()
     S = S0
     for j in range(rank):
         Mj = gathered[j][..., :dk].contiguous()

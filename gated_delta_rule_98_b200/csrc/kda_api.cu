@@ -425,6 +425,11 @@ kda_status kda_state_compose(const float* M, const float* N, const float* S_in, 
              : KDA_ERR_CUDA;
 }
 
+kda_status kda_debug_set_wait_limit(int64_t cycles) {
+  kda::tc_set_wait_limit((long long)cycles);
+  return KDA_OK;
+}
+
 kda_status kda_check_device_error(const void* workspace, kda_stream_t stream) {
   if (!workspace || !aligned16(workspace)) return KDA_ERR_INVALID_ARG;
   uint32_t err = 0;

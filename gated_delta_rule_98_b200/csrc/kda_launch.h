@@ -76,6 +76,9 @@ int tc_segments(int N, int H, int max_len);
 size_t tc_workspace_bytes(int N, int T, int H, int max_len);
 int tc_launches(int N, int H, int max_len);
 cudaError_t launch_forward_tc(const ForwardArgs& a);
+// Limit (SM cycles) of the tensor-core kernels' first-giving-up waits; <= 0
+// restores the default (about 2 s).  A test hook: the timeout path.
+void tc_set_wait_limit(long long cycles);
 
 // Context parallelism on the tensor-core path: the local pass (chunk
 // preparation, the transitions of all local segments, their fold into one

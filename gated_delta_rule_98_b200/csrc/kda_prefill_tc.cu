@@ -18,6 +18,8 @@
 // the outputs.  This is the single-GPU form of the prefix scan over
 // per-segment state updates (Kimi K3 architecture summary, KDA context
 // parallelism).
+#include <atomic>
+
 #include "kda_tc_common.cuh"
 
 namespace kda {
@@ -124,12 +126,13 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
   if (tid == 0)
     for (int c = c0; c < c1 && c < c0 + NS; ++c) load_slot(c);
   uint32_t phase = 0, ph_ld = 0;  // ph_ld bit s: parity of stage s's next completion
+  bool mma_pending = false;       // products committed and not yet awaited
   uint32_t inflight = 0;          // stages being filled
   for (int c = c0; c < c1 && c < c0 + NS; ++c) inflight |= 1u << stage_of(c);
   // Block-wide bounded wait for the stage of chunk c; false if it gave up.
   auto wait_stage = [&](int c) -> bool {
     const int s = stage_of(c);
-    const bool got = mbar_wait_cycles(&s_ld[s], (ph_ld >> s) & 1, kWaitCycles);
+    const bool got = mbar_wait_cycles(&s_ld[s], (ph_ld >> s) & 1, p.wait_limit);
     if (__syncthreads_or(!got)) {
       if (tid == 0) atomicOr(&p.hdr->err, kErrTimeout);
       return false;
@@ -290,11 +293,13 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       }
       mma_commit(&s_bar);
     }
+    mma_pending = true;
     // ---- meanwhile: the first chunk decays the incoming state by its gamma (later
     //      chunks get it with the previous chunk's copy); the previous o goes out
     if (c == c0) decay_state(reinterpret_cast<const float*>(st + L::kGam));
     if (!TRANS && c > c0) write_o(c - 1, dcol == TM::kD0 ? TM::kD1 : TM::kD0);
-    if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
+    if (!block_wait(&s_bar, phase, p.hdr, p.wait_limit)) { s_abort = 1; break; }
+    mma_pending = false;
     // ---- U^T = U~^T - D_W^T (transition: U_S^T = U~^T - D_S^T, U_X^T = -D_X^T),
     //      f16 into the copy's columns (C1 has read them)
     {
@@ -338,9 +343,11 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       }
       mma_commit(&s_bar);
     }
+    mma_pending = true;
     // the query row scales of this chunk, for its o (written during the next C1)
     if (!TRANS && tid < kC) s_iq[tid] = reinterpret_cast<const float*>(st + kSlotIq)[tid];
-    if (!block_wait(&s_bar, phase, p.hdr)) { s_abort = 1; break; }
+    if (!block_wait(&s_bar, phase, p.hdr, p.wait_limit)) { s_abort = 1; break; }
+    mma_pending = false;
     // the stage is consumed (its reads ended before the barrier above): refill it
     if (c + NS < c1) {
       inflight |= 1u << s;
@@ -405,9 +412,11 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       }
     }
   } else if (tid == 0) {
-    // a wait gave up: let the slot copies still in flight land before leaving
+    // a wait gave up: let the slot copies and products still in flight land
+    // before the CTA frees its Tensor Memory and leaves (at most ~2 s each)
     for (int s = 0; s < NS; ++s)
       if (inflight & (1u << s)) (void)mbar_wait_cycles(&s_ld[s], (ph_ld >> s) & 1, kWaitCycles);
+    if (mma_pending) (void)mbar_wait_cycles(&s_bar, phase, kWaitCycles);
   }
   fence_before_sync();
   __syncthreads();
@@ -485,7 +494,7 @@ __global__ void __launch_bounds__(kComposeThreads) compose_kernel(const __grid_c
 #pragma unroll
     for (int m = 0; m < 8; ++m) acc[m] = nxt[m];
     if (sg + 1 < steps) load_n(sg + 1, nxt);
-    const bool got = mbar_wait_cycles(&bar[buf], (ph >> buf) & 1, kWaitCycles);
+    const bool got = mbar_wait_cycles(&bar[buf], (ph >> buf) & 1, p.wait_limit);
     if (__syncthreads_or(!got)) {
       if (tid == 0) atomicOr(&p.hdr->err, kErrTimeout);
       ok = false;
@@ -599,6 +608,10 @@ int tc_launches(int N, int H, int max_len) {
 
 namespace {
 
+// Limit of the first-giving-up waits of the tensor-core kernels (SM cycles);
+// kda_debug_set_wait_limit lowers it to exercise the timeout path.
+std::atomic<long long> g_wait_limit{kWaitCycles};
+
 // Kernel parameters of a call; tensor maps only when the call stages inputs.
 cudaError_t fill_params(const ForwardArgs& a, TcParams& p, bool maps) {
   memset(&p, 0, sizeof(p));
@@ -633,6 +646,7 @@ cudaError_t fill_params(const ForwardArgs& a, TcParams& p, bool maps) {
   p.Pseg = p.P;
   p.hdr = (WsHeader*)a.ws;
   p.seg = (float*)((char*)a.ws + sizeof(WsHeader));
+  p.wait_limit = g_wait_limit.load();
   return cudaSuccess;
 }
 
@@ -676,6 +690,8 @@ cudaError_t launch_forward_tc(const ForwardArgs& a) {
   }
   return launch_chain<false>(p, p.P, a.stream);
 }
+
+void tc_set_wait_limit(long long cycles) { g_wait_limit.store(cycles > 0 ? cycles : kWaitCycles); }
 
 // Context parallelism.  The workspace holds the segment buffers for P + 1
 // segments (room for all P transitions) and the chunk slots, and it carries

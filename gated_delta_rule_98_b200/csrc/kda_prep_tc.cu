@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
   fence_after_sync();
   const uint32_t tm = *s_tmem;
   uint32_t ph_qkz = 0, ph_v = 0, ph_mma = 0;
-  bool ok = true, qkz_pending = false, v_pending = false;
+  bool ok = true, qkz_pending = false, v_pending = false, mma_pending = false;
 
   // elementwise phases: channel j, sub-tile b (tokens 16 b .. 16 b + 15)
   const int j = tid & 127, b = tid >> 7;
@@ -242,7 +242,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     const float expA_l2 = GS == kGateZ ? expf(a_nx) * kLog2e : 0.f;
     if (GS == kGateZ && have) a_nx = p.A[hn];
 
-    if (!block_wait(bar_qkz, ph_qkz, p.hdr)) { ok = false; break; }
+    if (!block_wait(bar_qkz, ph_qkz, p.hdr, p.wait_limit)) { ok = false; break; }
     qkz_pending = false;
 
     // ---- A1: row norms (thread: row tid / 4 of [q ; k], 32 channels)
@@ -380,6 +380,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
         }
         mma_commit(bar_mma);
       }
+      mma_pending = true;
       // meanwhile: X_K = beta k^ e^{Gam} (M2 operand), Q' = q e^{Gam} and
       // K' = k^ e^{Gam_last - Gam} (slot)
 #pragma unroll
@@ -392,7 +393,8 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
       for (int i = 0; i < 16; ++i) x[i] = cd[i] * Lb;
       put16h(slot + kSlotK, img_unit(16 * b, j, 64), img_unit(16 * b + 8, j, 64), x);
     }
-    if (!block_wait(bar_mma, ph_mma, p.hdr)) { ok = false; break; }
+    if (!block_wait(bar_mma, ph_mma, p.hdr, p.wait_limit)) { ok = false; break; }
+    mma_pending = false;
 
     // ---- D: products -> A_kk (fp32, strictly lower) and A_qk (f16 slot image,
     //      lower with the diagonal).  Warp (q4, cq): R rows 32 q4 + lane, i.e. row sub-tile q4 (lanes
@@ -565,7 +567,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     // the v rows must have landed (a block-wide wait that also orders the T images)
     fence_async_smem();
     fence_before_sync();
-    if (!block_wait(bar_v, ph_v, p.hdr)) { ok = false; break; }
+    if (!block_wait(bar_v, ph_v, p.hdr, p.wait_limit)) { ok = false; break; }
     v_pending = false;
     // ---- M2: W^T = X_K^T T^T -> TMEM columns 0-63 and U~^T = V^T (T Diag(beta))^T
     //      -> 64-127 (M = 128 channels, N = 64 tokens; V read in place from its
@@ -584,7 +586,9 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
       }
       mma_commit(bar_mma);
     }
-    if (!block_wait(bar_mma, ph_mma, p.hdr)) { ok = false; break; }
+    mma_pending = true;
+    if (!block_wait(bar_mma, ph_mma, p.hdr, p.wait_limit)) { ok = false; break; }
+    mma_pending = false;
     // v is consumed: load the next item's
     if (have && tid == 0) stage_v(tokn, hn);
     v_pending = have;
@@ -603,9 +607,11 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     fence_before_sync();
   }
   if (tid == 0) {
-    // a wait gave up: let the row loads still in flight land before leaving
+    // a wait gave up: let the row loads and the products still in flight land
+    // before the CTA frees its Tensor Memory and leaves (at most ~2 s each)
     if (qkz_pending) (void)mbar_wait_cycles(bar_qkz, ph_qkz, kWaitCycles);
     if (v_pending) (void)mbar_wait_cycles(bar_v, ph_v, kWaitCycles);
+    if (mma_pending) (void)mbar_wait_cycles(bar_mma, ph_mma, kWaitCycles);
   }
   (void)ok;
   fence_before_sync();

@@ -99,6 +99,9 @@ struct alignas(64) TcParams {
   // folded transition of each (sequence, head) when set.
   int Pseg;
   float *M_out, *N_out;
+  // Limit (SM cycles) of the waits that can give up first; the waits that let
+  // in-flight copies and MMAs land before a kernel leaves use kWaitCycles.
+  long long wait_limit;
 };
 
 // Where the log-decay comes from (a template parameter of the preparation, so
@@ -178,15 +181,17 @@ __device__ __forceinline__ void st16(unsigned char* base, uint32_t off, const fl
   *reinterpret_cast<uint4*>(base + off) = pack8(v);
 }
 
-// Block-wide bounded wait on an mbarrier phase; false if it timed out (the
-// error word then carries kErrTimeout).
-__device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t& phase, WsHeader* hdr) {
-  const bool got = mbar_wait_cycles(bar, phase, kWaitCycles);
-  phase ^= 1;
+// Block-wide bounded wait on an mbarrier phase (at most `limit` SM cycles); false
+// if it timed out (the error word then carries kErrTimeout and `phase` still
+// names the pending phase, for the drain before the kernel leaves).
+__device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t& phase, WsHeader* hdr,
+                                           long long limit) {
+  const bool got = mbar_wait_cycles(bar, phase, limit);
   if (__syncthreads_or(!got)) {
     if (threadIdx.x == 0) atomicOr(&hdr->err, kErrTimeout);
     return false;
   }
+  phase ^= 1;
   fence_after_sync();
   return true;
 }

@@ -45,10 +45,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   return false;
 }
 
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait measured in SM clock cycles (about max_cycles / 1.9e9 seconds).
+// try_wait may suspend the thread for a while inside one call, so a limit
+// below about a million cycles polls with test_wait instead, which keeps the
+// limit exact (a test can then make a wait run out).
 __device__ __forceinline__ bool mbar_wait_cycles(uint64_t* bar, uint32_t parity,
                                                  long long max_cycles) {
   const long long t0 = clock64();
+  if (max_cycles < (1LL << 20)) {
+    while (!mbar_test_wait(bar, parity))
+      if (clock64() - t0 > max_cycles) return false;
+    return true;
+  }
   while (!mbar_try_wait(bar, parity))
     if (clock64() - t0 > max_cycles) return false;
   return true;

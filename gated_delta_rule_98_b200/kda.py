@@ -35,7 +35,7 @@ EXPORTS = ("kda_status_string", "kda_version", "kda_forward_workspace_size",
            "kda_forward_norm_gate", "kda_decode_step_norm_gate", "kda_forward_scalar_gate",
            "kda_short_conv_swish", "kda_forward_conv_workspace_size", "kda_forward_conv",
            "kda_cp_workspace_size", "kda_cp_local", "kda_cp_finish", "kda_state_compose",
-           "kda_check_device_error")
+           "kda_check_device_error", "kda_debug_set_wait_limit")
 
 # Bytes of the library's fixed scratch array used by kda_forward_noalloc.
 KDA_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -104,6 +104,8 @@ def lib():
     L.kda_state_compose.restype = ctypes.c_int
     L.kda_check_device_error.argtypes = [vp, vp]
     L.kda_check_device_error.restype = ctypes.c_int
+    L.kda_debug_set_wait_limit.argtypes = [ctypes.c_int64]
+    L.kda_debug_set_wait_limit.restype = ctypes.c_int
     _lib = L
     return L
 
@@ -224,6 +226,10 @@ def kda_state_compose(M, N, S_in, S_out, count, dk, dv, stream):
 
 def kda_check_device_error(workspace, stream):
     return lib().kda_check_device_error(workspace, stream)
+
+
+def kda_debug_set_wait_limit(cycles):
+    return lib().kda_debug_set_wait_limit(cycles)
 
 
 # ------------------------------------------------------- tensor helpers ---

@@ -427,6 +427,21 @@ kda_status kda_state_compose(const float* M, const float* N, const float* S_in, 
                              int32_t count, int32_t dk, int32_t dv, kda_stream_t stream);
 
 /*
+ * Test hook for the failure path; no passage of the pages corresponds to it.
+ * Every device-side wait of the tensor-core prefill kernels (on a TMA or bulk
+ * copy, or on the completion of tensor-core products) is bounded: by default
+ * a wait that has not finished after about 2 s of SM clock gives up, records
+ * KDA_ERR_TIMEOUT in the workspace's error word, lets the copies and products
+ * it already issued land (each again bounded by about 2 s), frees its Tensor
+ * Memory and leaves; the kernels after it in the same call give up the same
+ * way.  This call sets the limit of the first, giving-up waits to `cycles` SM
+ * cycles for later calls in this process (cycles <= 0 restores the default),
+ * so that a test can make a wait run out without any fault.  Not for
+ * production use: a small limit fails every call.  Returns KDA_OK.
+ */
+kda_status kda_debug_set_wait_limit(int64_t cycles);
+
+/*
  * Reads the workspace's error word of the most recent kda_forward /
  * kda_forward_g call on that workspace (synchronises `stream`).  Each call
  * clears the word (a 4-byte cudaMemsetAsync ordered before its first kernel)

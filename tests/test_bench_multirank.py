@@ -70,3 +70,53 @@ def test_reference_arm_json_line(steps):
     d = json.loads(r.stdout.strip().splitlines()[-1])
     assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _cp_worker(rank, world, port, out):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import bench
+    from gated_delta_rule_98_b200 import cp
+    from oracle import ref
+    from test_cp_host import _OracleOps, _problem
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    T = 150
+    p = _problem(3, T, 2, 6, 4, s0=0.0)
+    a, b = bench.shard_bounds(T, world, rank)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x))
+    o_sh, S_after = cp.context_parallel_forward(t(p["q"][a:b]), t(p["k"][a:b]), t(p["v"][a:b]),
+                                                t(p["z"][a:b]), t(p["A"]), t(p["beta"][a:b]),
+                                                max_seqlen=b - a, ops=_OracleOps())
+    o_ref, S_ref = ref.forward(p["q"], p["k"], p["v"], p["beta"], z=p["z"], A=p["A"], num_seqs=1)
+    err, rel, serr = bench.cp_parity(o_sh, t(o_ref[a:b]), S_after[0], t(S_ref[0]),
+                                     rank == world - 1, world)
+    ms = bench.max_over_ranks(4.0 + rank, world)
+    out.put((rank, a, b, err, rel, serr, ms, bench.strong_scaling_value(T, ms)))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_context_parallel_mode_aggregation_with_gloo():
+    """bench.py --mode cp on CPU ranks: the shards tile the sequence in chunk
+    multiples, the parity reduction sees the sharded result equal to the
+    one-pass oracle on every rank, and the strong-scaling throughput divides
+    the whole sequence by the slowest rank's time."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29700 + os.getpid() % 1000
+    procs = [ctx.Process(target=_cp_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=300) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert res[0][1] == 0 and res[0][2] == res[1][1] and res[1][2] == 150
+    assert res[0][2] % 64 == 0
+    for rank, a, b, err, rel, serr, ms, value in res:
+        assert err < 1e-10 and rel < 1e-10 and serr < 1e-10
+        assert ms == 5.0 and value == pytest.approx(150 / 0.005)
