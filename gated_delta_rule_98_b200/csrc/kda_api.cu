@@ -62,7 +62,7 @@ kda_status decode_common(const void* q, const void* k, const void* v, const void
                          const float* A, const void* beta, float* S_inout, int32_t B,
                          int32_t H, int32_t dk, int32_t dv, kda_dtype dt,
                          const void* out_gate, const float* norm_weight, float eps, void* o,
-                         kda_stream_t stream) {
+                         kda_stream_t stream, const kda::DecodeArgs* conv = nullptr) {
   if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_UNSUPPORTED;
   if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
   if (B < 0 || H < 1) return KDA_ERR_INVALID_ARG;
@@ -77,6 +77,13 @@ kda_status decode_common(const void* q, const void* k, const void* v, const void
   a.out_gate = out_gate;
   a.norm_w = norm_weight;
   a.norm_eps = eps;
+  if (conv) {
+    a.conv_wq = conv->conv_wq;
+    a.conv_wk = conv->conv_wk;
+    a.conv_wv = conv->conv_wv;
+    a.conv_state = conv->conv_state;
+    a.conv_width = conv->conv_width;
+  }
   return kda::launch_decode(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -277,6 +284,29 @@ kda_status kda_decode_step_norm_gate(const void* q, const void* k, const void* v
                        eps, o, stream);
 }
 
+kda_status kda_decode_step_conv(const void* x_q, const void* x_k, const void* x_v,
+                                const float* w_q, const float* w_k, const float* w_v,
+                                int32_t conv_width, void* conv_state, const void* z,
+                                const float* A, const void* beta, float* S_inout, int32_t B,
+                                int32_t H, int32_t dk, int32_t dv, kda_dtype dt, void* o,
+                                kda_stream_t stream) {
+  if (conv_width < 1 || conv_width > 4) return KDA_ERR_UNSUPPORTED;
+  if (B > 0 && (!w_q || !w_k || !w_v || ((uintptr_t)w_q & 3u) || ((uintptr_t)w_k & 3u) ||
+                ((uintptr_t)w_v & 3u)))
+    return KDA_ERR_INVALID_ARG;
+  if (B > 0 && conv_width > 1 &&
+      (!conv_state || ((uintptr_t)conv_state & (dt == KDA_BF16 ? 1u : 3u))))
+    return KDA_ERR_INVALID_ARG;
+  kda::DecodeArgs c{};
+  c.conv_wq = w_q;
+  c.conv_wk = w_k;
+  c.conv_wv = w_v;
+  c.conv_state = conv_state;
+  c.conv_width = conv_width;
+  return decode_common(x_q, x_k, x_v, z, A, beta, S_inout, B, H, dk, dv, dt, nullptr, nullptr,
+                       0.f, o, stream, &c);
+}
+
 kda_status kda_short_conv_swish(const void* x, const float* w, const int32_t* cu_seqlens,
                                 int32_t num_seqs, int32_t total_tokens, int32_t max_seqlen,
                                 int32_t channels, int32_t width, kda_dtype dt, void* y,
@@ -307,6 +337,8 @@ size_t kda_forward_conv_workspace_size(int32_t num_seqs, int32_t total_tokens,
   const size_t fw = kda_forward_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv,
                                                dt, chunk);
   if (fw == 0) return 0;
+  // the tensor-core path runs the prologue inside its chunk preparation
+  if (use_tc(dt, dk, dv, chunk)) return fw;
   const size_t elt = dt == KDA_BF16 ? 2 : 4, tok = (size_t)total_tokens * H;
   return conv_offsets(fw, tok, dk, dv, elt)[3];
 }
@@ -333,6 +365,17 @@ kda_status kda_forward_conv(const void* x_q, const void* x_k, const void* x_v,
   if (total_tokens > 0 && (!w_q || !w_k || !w_v || ((uintptr_t)w_q & 3u) ||
                            ((uintptr_t)w_k & 3u) || ((uintptr_t)w_v & 3u)))
     return KDA_ERR_INVALID_ARG;
+  if (use_tc(dt, dk, dv, chunk)) {
+    // fused: the chunk preparation convolves the staged rows itself
+    kda::ForwardArgs a{x_q, x_k, x_v, z, beta, A, nullptr, S0, cu_seqlens, o, S_final,
+                       num_seqs, total_tokens, max_seqlen, H, dk, dv, chunk,
+                       dt == KDA_BF16, workspace, fw, (cudaStream_t)stream};
+    a.conv_wq = w_q;
+    a.conv_wk = w_k;
+    a.conv_wv = w_v;
+    a.conv_width = conv_width;
+    return forward_common(a);
+  }
   const size_t elt = dt == KDA_BF16 ? 2 : 4, tok = (size_t)total_tokens * H;
   const auto off = conv_offsets(fw, tok, dk, dv, elt);
   char* ws = (char*)workspace;

@@ -11,10 +11,33 @@
 // contiguous 512-byte rows; the state lives in registers between the load and
 // the store.  Column sums are reduced across row groups through shared memory
 // in a fixed order (deterministic, no atomics).
+//
+// With the input prologue (Kimi Linear summary §4: short convolution and Swish
+// on q, k, v) the step also carries each sequence's rolling window of the last
+// width - 1 inputs per channel: the convolution of this token reads the window
+// and the token's own input, and the window then shifts by one.
 #include "kda_common.cuh"
 #include "kda_launch.h"
 
 namespace kda {
+
+// Rolling input window of the decode-side prologue (width 0: none).
+struct DecodeConv {
+  const float *wq, *wk, *wv;  // taps [channels, width], w[c][width - 1] on the current token
+  void* state;                // [B, H * (2 dk + dv), width - 1], input dtype
+  int width;
+};
+
+// Swish(conv) of one channel (taps wc[0 .. W-1]) for this token's input x; the
+// window win[0 .. W-2] holds the earlier inputs, oldest first, and is shifted.
+template <typename T>
+__device__ __forceinline__ float conv_step(const float* wc, T* win, int W, float x) {
+  float u = wc[W - 1] * x;
+  for (int m = 0; m < W - 1; ++m) u = fmaf(wc[m], to_f(win[m]), u);
+  for (int m = 0; m + 1 < W - 1; ++m) win[m] = win[m + 1];
+  if (W > 1) win[W - 2] = from_f<T>(x);
+  return u / (1.0f + expf(-u));
+}
 
 template <int DK, int DV, typename T>
 __global__ void __launch_bounds__(256)
@@ -22,7 +45,8 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k,
                    const T* __restrict__ v, const T* __restrict__ z,
                    const float* __restrict__ A, const T* __restrict__ beta,
                    float* __restrict__ S, int H, T* __restrict__ o,
-                   const T* __restrict__ og, const float* __restrict__ ow, float oeps) {
+                   const T* __restrict__ og, const float* __restrict__ ow, float oeps,
+                   const DecodeConv cv) {
   constexpr int NT = 256;
   constexpr int CG = DV / 4;   // float4 column groups per state row
   constexpr int RG = NT / CG;  // row groups
@@ -47,12 +71,31 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k,
   for (int m = 0; m < RPT; ++m) s[m] = __ldcs(&Sp[(rg + m * RG) * CG + cg]);
 
   const float expA = expf(A[h]);
-  for (int i = tid; i < DK; i += NT) {
-    s_k[i] = to_f(k[(size_t)bh * DK + i]);
-    s_q[i] = to_f(q[(size_t)bh * DK + i]);
-    s_a[i] = expf(gate_logdecay(to_f(z[(size_t)bh * DK + i]), expA));
+  if (cv.width > 0) {
+    // prologue: the window's channels of (b, h) are q h*DK+i, k H*DK+h*DK+i, v 2*H*DK+h*DV+j
+    const int W = cv.width, b = bh / H;
+    T* win = reinterpret_cast<T*>(cv.state) + (size_t)b * H * (2 * DK + DV) * (W - 1);
+    for (int i = tid; i < DK; i += NT) {
+      const int cq = h * DK + i, ck = H * DK + h * DK + i;
+      s_q[i] = conv_step(cv.wq + (size_t)cq * W, win + (size_t)cq * (W - 1), W,
+                         to_f(q[(size_t)bh * DK + i]));
+      s_k[i] = conv_step(cv.wk + (size_t)cq * W, win + (size_t)ck * (W - 1), W,
+                         to_f(k[(size_t)bh * DK + i]));
+      s_a[i] = expf(gate_logdecay(to_f(z[(size_t)bh * DK + i]), expA));
+    }
+    for (int j = tid; j < DV; j += NT) {
+      const int cvh = h * DV + j, cvw = 2 * H * DK + h * DV + j;
+      s_v[j] = conv_step(cv.wv + (size_t)cvh * W, win + (size_t)cvw * (W - 1), W,
+                         to_f(v[(size_t)bh * DV + j]));
+    }
+  } else {
+    for (int i = tid; i < DK; i += NT) {
+      s_k[i] = to_f(k[(size_t)bh * DK + i]);
+      s_q[i] = to_f(q[(size_t)bh * DK + i]);
+      s_a[i] = expf(gate_logdecay(to_f(z[(size_t)bh * DK + i]), expA));
+    }
+    for (int j = tid; j < DV; j += NT) s_v[j] = to_f(v[(size_t)bh * DV + j]);
   }
-  for (int j = tid; j < DV; j += NT) s_v[j] = to_f(v[(size_t)bh * DV + j]);
   __syncthreads();
   if (tid < 32) {
     float kk = 0.f, qq = 0.f, kq = 0.f;
@@ -133,7 +176,8 @@ template <int DK, int DV, typename T>
 static cudaError_t launch_decode_t(const DecodeArgs& a) {
   decode_step_kernel<DK, DV, T><<<a.B * a.H, 256, 0, a.stream>>>(
       (const T*)a.q, (const T*)a.k, (const T*)a.v, (const T*)a.z, a.A,
-      (const T*)a.beta, a.S, a.H, (T*)a.o, (const T*)a.out_gate, a.norm_w, a.norm_eps);
+      (const T*)a.beta, a.S, a.H, (T*)a.o, (const T*)a.out_gate, a.norm_w, a.norm_eps,
+      DecodeConv{a.conv_wq, a.conv_wk, a.conv_wv, a.conv_state, a.conv_width});
   return cudaGetLastError();
 }
 

@@ -19,6 +19,13 @@ struct DecodeArgs {
   const void* out_gate = nullptr;  // [B, H, dv] sigmoid output-gate input (input dtype), or null
   const float* norm_w = nullptr;   // [dv] RMSNorm gain, or null (ones)
   float norm_eps = 0.f;
+  // Input prologue (conv_width > 0): q, k, v are the convolution's inputs of
+  // this token, conv_wq/wk/wv [channels, conv_width] its taps and conv_state
+  // [B, H * (2 dk + dv), conv_width - 1] (input dtype) the rolling window of
+  // earlier inputs, updated in place.
+  const float *conv_wq = nullptr, *conv_wk = nullptr, *conv_wv = nullptr;
+  void* conv_state = nullptr;
+  int conv_width = 0;
 };
 
 struct ForwardArgs {
@@ -44,6 +51,11 @@ struct ForwardArgs {
   // Scalar gate (Gated DeltaNet): [T, H] fp32 log-decay shared by a head's dk
   // channels, instead of z, A and g.
   const float* g_head = nullptr;
+  // Input prologue fused into the chunk preparation (tensor-core path, KDA
+  // gate): q, k, v are the short convolution's inputs and these its
+  // [channels, conv_width] fp32 taps.  conv_width 0: q, k, v as given.
+  const float *conv_wq = nullptr, *conv_wk = nullptr, *conv_wv = nullptr;
+  int conv_width = 0;
 };
 
 // Input prologue: causal depthwise short convolution per sequence + Swish.

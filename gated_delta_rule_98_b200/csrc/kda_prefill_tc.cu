@@ -552,14 +552,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [T, H, 128] bf16 tensor; box 64 tokens x 1 head x 64 channels with the
-// 128-byte swizzle; rows past T read as zero.
-bool make_map(CUtensorMap* map, const void* base, int T, int H) {
+// [T, H, 128] bf16 tensor; box `rows` tokens x 1 head x 64 channels with the
+// 128-byte swizzle; rows before 0 or past T read as zero.
+bool make_map(CUtensorMap* map, const void* base, int T, int H, int rows = kC) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)T};
   const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2};
-  const cuuint32_t box[3] = {(cuuint32_t)(kD / 2), 1, (cuuint32_t)kC};
+  const cuuint32_t box[3] = {(cuuint32_t)(kD / 2), 1, (cuuint32_t)rows};
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -617,8 +617,9 @@ cudaError_t fill_params(const ForwardArgs& a, TcParams& p, bool maps) {
   memset(&p, 0, sizeof(p));
   if (maps && a.T > 0) {
     const void* zz = a.z ? a.z : a.k;
-    if (!make_map(&p.sq, a.q, a.T, a.H) || !make_map(&p.sk, a.k, a.T, a.H) ||
-        !make_map(&p.sz, zz, a.T, a.H) || !make_map(&p.sv, a.v, a.T, a.H))
+    const int rows = a.conv_width > 0 ? kC + 8 : kC;  // with the convolution's history
+    if (!make_map(&p.sq, a.q, a.T, a.H, rows) || !make_map(&p.sk, a.k, a.T, a.H, rows) ||
+        !make_map(&p.sz, zz, a.T, a.H) || !make_map(&p.sv, a.v, a.T, a.H, rows))
       return cudaErrorInvalidValue;
   }
   p.beta = (const __nv_bfloat16*)a.beta;
@@ -647,6 +648,10 @@ cudaError_t fill_params(const ForwardArgs& a, TcParams& p, bool maps) {
   p.hdr = (WsHeader*)a.ws;
   p.seg = (float*)((char*)a.ws + sizeof(WsHeader));
   p.wait_limit = g_wait_limit.load();
+  p.cwq = a.conv_wq;
+  p.cwk = a.conv_wk;
+  p.cwv = a.conv_wv;
+  p.cw = a.conv_width;
   return cudaSuccess;
 }
 

@@ -42,10 +42,16 @@ constexpr int kLd = 68;  // row stride (floats) of the fp32 work matrices of the
 __host__ __device__ constexpr int win_row0(int w) { return 8 * w * (w + 1); }
 constexpr int kWinRows = 160;
 
+// CV: the input prologue runs here (q, k, v arrive before their short
+// convolution and Swish).  Their boxes then start 8 tokens before the chunk,
+// so box row 8 + t holds token t and rows 5 .. 7 the convolution's history.
+template <bool CV>
 struct PrepSmem {
-  // staged rows: two 64-channel boxes [64 tokens][64 channels] per tensor, 128-byte swizzle
-  static constexpr int kQ = 0, kK = 16384, kZ = 32768, kV = 49152;
-  static constexpr int kWB = 65536;               // windows, 160-row image: the B operand of M1
+  // staged rows: per tensor two 64-channel boxes of kRows tokens, 128-byte swizzle
+  static constexpr int kRows = CV ? kC + 8 : kC;
+  static constexpr int kBox = kRows * 128;
+  static constexpr int kQ = 0, kK = 2 * kBox, kZ = 4 * kBox, kV = kZ + 16384;
+  static constexpr int kWB = kV + 2 * kBox;        // windows, 160-row image: the B operand of M1
   static constexpr int kR = kWB + kWinRows * 256; // R: 128-row image (sub-tile b: k rows 32b..,
                                                   //   q rows 32b+16..), the A operand of M1
   // after M1 the window / R region holds the inverse's work and the T images
@@ -60,10 +66,22 @@ struct PrepSmem {
   static constexpr int kBeta = kNrm + 512;        // beta (64)
   static constexpr int kEx = kBeta + 256;         // [4][128] alpha at each sub-tile's first token,
                                                   // then [4][128] E at its last token
-  static constexpr int kBar = kEx + 4096;         // three mbarriers, then the TMEM base
+  // CV: the prologue's taps (x 1/2) of the item's head and of the next item's,
+  // [2][q, k, v][128 channels] float4 (right-aligned: the last on the current token)
+  static constexpr int kTaps = kEx + 4096;
+  // CV: a 16 x 16 bf16 block of ones, the B operand of the norm product
+  static constexpr int kOnes = kTaps + (CV ? 12288 : 0);
+  // CV: Swish(conv(v)) as a 64-row bf16 image, the A operand V^T of M2 (K-major)
+  static constexpr int kVc = kOnes + (CV ? 512 : 0);
+  static constexpr int kBar = kVc + (CV ? 16384 : 0);  // three mbarriers, then the TMEM base
   static constexpr int kBytes = kBar + 64;
+  // CV, before M1: squares of q, k (hi and lo bf16 parts), a 128-row image with
+  // 256 channels over the window / R region: the A operand of the norm product
+  static constexpr int kSq = kWB;
+  static_assert(kSq + 65536 <= kXK, "norm operand overlaps X_K");
+  static_assert(kR + 32768 <= kXK, "M1 operands overlap X_K");
+  static_assert(kBox % 1024 == 0 && kV % 1024 == 0, "swizzled boxes need 1024-byte alignment");
 };
-static_assert(PrepSmem::kR + 32768 <= PrepSmem::kXK, "M1 operands overlap X_K");
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -76,6 +94,16 @@ __device__ __forceinline__ float rcp(float x) {
   return y;
 }
 constexpr float kLog2e = 1.4426950408889634f;
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// Swish: u sigmoid(u) = h + h tanh(h) with h = u / 2 (sigmoid(u) = (1 + tanh(u / 2)) / 2)
+__device__ __forceinline__ float swish(float u) {
+  const float h = 0.5f * u;
+  return fmaf(h, tanh_approx(h), h);
+}
 
 // Shared-memory matrix descriptor with the 128-byte swizzle (the layout TMA
 // writes with CU_TENSOR_MAP_SWIZZLE_128B into a 1024-byte aligned buffer).
@@ -96,9 +124,9 @@ __device__ __forceinline__ void put16h(unsigned char* base, uint32_t unit0, uint
   *reinterpret_cast<uint4*>(base + unit1) = pack8h(v + 8);
 }
 
-template <int GS>
+template <int GS, bool CV>
 __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ TcParams p) {
-  using L = PrepSmem;
+  using L = PrepSmem<CV>;
   extern __shared__ __align__(1024) unsigned char sm[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   float* nrm = reinterpret_cast<float*>(sm + L::kNrm);
@@ -152,6 +180,75 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     const uint32_t u = *reinterpret_cast<const uint16_t*>(sm + base + raw_off(i));
     return __uint_as_float(u << 16);
   };
+  // CV: input prologue of channel j, tokens 16 b .. 16 b + 15 (box row 8 + t holds token t):
+  // y_i = Swish(sum_m w4[m] x[16 b + i - 3 + m]), the taps w4 right-aligned (w4[3] on
+  // the current token); history before the sequence's first token reads as zero
+  // (first: this chunk is its sequence's first), tokens from len on give zero
+  // Token pairs (16 b + 2 p, 16 b + 2 p + 1) go through packed fp32x2 arithmetic;
+  // the taps hw are halved, so the sum is u / 2 and Swish(u) = h + h tanh(h).
+  const uint32_t jboxc = (uint32_t)(j >> 6) * (uint32_t)L::kBox + (uint32_t)(j & 7) * 2u;
+  auto conv16 = [&](int base, const float4 hw, bool first, int len, float* y) {
+    float x[19];  // tokens 16 b - 3 .. 16 b + 15
+#pragma unroll
+    for (int i = 0; i < 19; ++i) {
+      const int r = 16 * b + 5 + i;
+      const uint32_t off = jboxc + (uint32_t)r * 128u + ((junit ^ (uint32_t)(r & 7)) << 4);
+      x[i] = __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t*>(sm + base + off) << 16);
+    }
+    if (first && b == 0) x[0] = x[1] = x[2] = 0.f;
+    const float2 w0 = make_float2(hw.x, hw.x), w1 = make_float2(hw.y, hw.y),
+                 w2 = make_float2(hw.z, hw.z), w3 = make_float2(hw.w, hw.w);
+#pragma unroll
+    for (int q2 = 0; q2 < 8; ++q2) {
+      const int i = 2 * q2;
+      float2 h = __fmul2_rn(w0, make_float2(x[i], x[i + 1]));
+      h = __ffma2_rn(w1, make_float2(x[i + 1], x[i + 2]), h);
+      h = __ffma2_rn(w2, make_float2(x[i + 2], x[i + 3]), h);
+      h = __ffma2_rn(w3, make_float2(x[i + 3], x[i + 4]), h);
+      const float2 s = __ffma2_rn(h, make_float2(tanh_approx(h.x), tanh_approx(h.y)), h);
+      y[i] = s.x;
+      y[i + 1] = s.y;
+    }
+    if (len < kC) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) y[i] = 16 * b + i < len ? y[i] : 0.f;
+    }
+  };
+  // CV: taps of head hh (x 1/2) for thread (j, b < 3): tensor b (q, k, v), channel j
+  float4* tapbuf = reinterpret_cast<float4*>(sm + L::kTaps);
+  auto load_taps = [&](int hh) -> float4 {
+    const float* wc = (b == 0 ? p.cwq : b == 1 ? p.cwk : p.cwv) + (size_t)(hh * kD + j) * p.cw;
+    float w[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) w[m] = m >= 4 - p.cw ? 0.5f * wc[m - (4 - p.cw)] : 0.f;
+    return make_float4(w[0], w[1], w[2], w[3]);
+  };
+  // CV: squares of y (16 tokens of channel j at rows r0 ..) as hi and lo bf16
+  // parts (hi = bf16(y^2), lo = bf16(y^2 - hi)) into the norm operand: hi at
+  // channel j, lo at channel 128 + j
+  auto put_squares = [&](const float* y, int r0) {
+    float s[16], lo[16];
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      const float2 q2 = __fmul2_rn(make_float2(y[i], y[i + 1]), make_float2(y[i], y[i + 1]));
+      s[i] = q2.x;
+      s[i + 1] = q2.y;
+    }
+    const uint4 h0 = pack8(s), h1 = pack8(s + 8);
+    float hf[16];
+    unpack8(h0, hf);
+    unpack8(h1, hf + 8);
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      const float2 d = __fadd2_rn(make_float2(s[i], s[i + 1]), make_float2(-hf[i], -hf[i + 1]));
+      lo[i] = d.x;
+      lo[i + 1] = d.y;
+    }
+    *reinterpret_cast<uint4*>(sm + L::kSq + img_unit(r0, j, 128)) = h0;
+    *reinterpret_cast<uint4*>(sm + L::kSq + img_unit(r0 + 8, j, 128)) = h1;
+    *reinterpret_cast<uint4*>(sm + L::kSq + img_unit(r0, 128 + j, 128)) = pack8(lo);
+    *reinterpret_cast<uint4*>(sm + L::kSq + img_unit(r0 + 8, 128 + j, 128)) = pack8(lo + 8);
+  };
 
   // items (chunk c, sequence n, head h), heads fastest; the CTA takes every
   // gridDim.x-th one, stepping the mixed-radix index without divisions
@@ -173,21 +270,22 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     }
     return false;
   };
+  constexpr int kHist = CV ? 8 : 0;  // box rows before the chunk
   auto stage_qkz = [&](int tok, int hh) {  // one thread
-    mbar_arrive_expect_tx(bar_qkz, (GS == kGateZ ? 3 : 2) * 16384);
-    tma_box_x(sm + L::kQ, &p.sq, 0, hh, tok, bar_qkz);
-    tma_box_x(sm + L::kQ + 8192, &p.sq, 64, hh, tok, bar_qkz);
-    tma_box_x(sm + L::kK, &p.sk, 0, hh, tok, bar_qkz);
-    tma_box_x(sm + L::kK + 8192, &p.sk, 64, hh, tok, bar_qkz);
+    mbar_arrive_expect_tx(bar_qkz, 4 * L::kBox + (GS == kGateZ ? 16384 : 0));
+    tma_box_x(sm + L::kQ, &p.sq, 0, hh, tok - kHist, bar_qkz);
+    tma_box_x(sm + L::kQ + L::kBox, &p.sq, 64, hh, tok - kHist, bar_qkz);
+    tma_box_x(sm + L::kK, &p.sk, 0, hh, tok - kHist, bar_qkz);
+    tma_box_x(sm + L::kK + L::kBox, &p.sk, 64, hh, tok - kHist, bar_qkz);
     if (GS == kGateZ) {
       tma_box_x(sm + L::kZ, &p.sz, 0, hh, tok, bar_qkz);
       tma_box_x(sm + L::kZ + 8192, &p.sz, 64, hh, tok, bar_qkz);
     }
   };
   auto stage_v = [&](int tok, int hh) {  // one thread
-    mbar_arrive_expect_tx(bar_v, 16384);
-    tma_box_x(sm + L::kV, &p.sv, 0, hh, tok, bar_v);
-    tma_box_x(sm + L::kV + 8192, &p.sv, 64, hh, tok, bar_v);
+    mbar_arrive_expect_tx(bar_v, 2 * L::kBox);
+    tma_box_x(sm + L::kV, &p.sv, 0, hh, tok - kHist, bar_v);
+    tma_box_x(sm + L::kV + L::kBox, &p.sv, 64, hh, tok - kHist, bar_v);
   };
   // beta of an item's token t = tid < 64 as raw bf16 bits (converted when used, so
   // the load is not waited for until the next item)
@@ -208,6 +306,13 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     }
     qkz_pending = v_pending = true;
     beta_nx = load_beta(a + c * kC, e, h);
+  }
+  int tbuf = 0;  // CV: the taps buffer of the current item
+  if constexpr (CV) {
+    // the ones block (bf16 1.0) and the first item's taps; published by the
+    // first item's first block-wide wait
+    if (tid < 128) reinterpret_cast<uint32_t*>(sm + L::kOnes)[tid] = 0x3F803F80u;
+    if (have && b < 3) tapbuf[b * 128 + j] = load_taps(h);
   }
   while (have) {
     const int hc = h, nc = n, ac = a, ec = e, cc0 = c;
@@ -245,8 +350,28 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     if (!block_wait(bar_qkz, ph_qkz, p.hdr, p.wait_limit)) { ok = false; break; }
     qkz_pending = false;
 
-    // ---- A1: row norms (thread: row tid / 4 of [q ; k], 32 channels)
-    {
+    float qv[16], kv[16];  // q, k of the thread's tokens (zero past the sequence end)
+    if constexpr (CV) {
+      // ---- A0: input prologue on q and k; their squares (hi + lo bf16 parts)
+      //      go to one product with a block of ones, D[row][.] = sum over the
+      //      channels (rows 0-63 q, 64-127 k), read after the gate
+      const float4* tq = tapbuf + tbuf * 384;
+      conv16(L::kQ, tq[j], cc0 == 0, len, qv);
+      put_squares(qv, 16 * b);
+      conv16(L::kK, tq[128 + j], cc0 == 0, len, kv);
+      put_squares(kv, 64 + 16 * b);
+      sync_for_mma();
+      if (tid == 0) {
+        constexpr uint32_t id = instr_desc(kFmtBF16, 128, 16, true, true);
+        const uint64_t bd = smem_desc(smem_u32(sm + L::kOnes), 256, 128);
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          mma_bf16(tm + 160, smem_desc(smem_u32(sm + L::kSq + k * 4096), 2048, 128), bd, id, k > 0);
+        mma_commit(bar_mma);
+      }
+      mma_pending = true;
+    } else {
+      // ---- A1: row norms (thread: row tid / 4 of [q ; k], 32 channels)
       const int r = tid >> 2, qt = tid & 3, t = r & 63;
       const unsigned char* rowp =
           sm + (r < 64 ? L::kQ : L::kK) + (qt >> 1) * 8192 + t * 128;
@@ -282,13 +407,22 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     for (int i = 1; i < 16; ++i) E[i] = E[i - 1] * al[i];
     exf[b * 128 + j] = al[0];
     exl[b * 128 + j] = E[15];
-    // q, k of the thread's tokens (zero past the sequence end)
-    float qv[16], kv[16];
+    if constexpr (CV) {
+      if (!block_wait(bar_mma, ph_mma, p.hdr, p.wait_limit)) { ok = false; break; }
+      mma_pending = false;
+      if (warp < 4) {  // row 32 warp + lane of the norm product
+        const float ss = tmem_ld1(tmem_addr(tm, 32 * warp, 160));
+        tmem_ld_wait();
+        const int r = 32 * warp + lane;
+        nrm[r] = (r & 63) < len ? rsqrtf(ss + kNormEps) : 0.f;
+      }
+    } else {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const bool in = 16 * b + i < len;
-      qv[i] = in ? raw_f(L::kQ, i) : 0.f;
-      kv[i] = in ? raw_f(L::kK, i) : 0.f;
+      for (int i = 0; i < 16; ++i) {
+        const bool in = 16 * b + i < len;
+        qv[i] = in ? raw_f(L::kQ, i) : 0.f;
+        kv[i] = in ? raw_f(L::kK, i) : 0.f;
+      }
     }
     __syncthreads();
     // the staged q, k, z rows are consumed: load the next item's
@@ -425,6 +559,9 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     }
     fence_before_sync();
     __syncthreads();
+    // CV: the next item's taps, loaded during the inverse and stored after it
+    float4 tnext = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (CV && have && b < 3) tnext = load_taps(hn);
 
     // ---- E: T = (I + A_kk)^{-1} in fp32.  Diagonal 16x16 blocks by forward
     //      substitution (one warp per block, lane = column), then the blocks below
@@ -564,22 +701,35 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     __syncthreads();
     // the merged block T[32:64][0:32]
     if (tid < 128) put_t(32 + (tid & 31), (tid >> 5) * 8);
+    if (CV && have && b < 3) tapbuf[(tbuf ^ 1) * 384 + b * 128 + j] = tnext;
     // the v rows must have landed (a block-wide wait that also orders the T images)
     fence_async_smem();
     fence_before_sync();
     if (!block_wait(bar_v, ph_v, p.hdr, p.wait_limit)) { ok = false; break; }
     v_pending = false;
+    if constexpr (CV) {
+      // input prologue on v -> the bf16 image V^T of M2; the raw rows are then
+      // consumed and the next item's are requested at once
+      float y[16];
+      conv16(L::kV, tapbuf[tbuf * 384 + 256 + j], cc0 == 0, len, y);
+      put16(sm + L::kVc, img_unit(16 * b, j, 64), img_unit(16 * b + 8, j, 64), y);
+      sync_for_mma();
+      if (have && tid == 0) stage_v(tokn, hn);
+      v_pending = have;
+    }
     // ---- M2: W^T = X_K^T T^T -> TMEM columns 0-63 and U~^T = V^T (T Diag(beta))^T
     //      -> 64-127 (M = 128 channels, N = 64 tokens; V read in place from its
     //      swizzled tile as an MN-major operand)
     if (tid == 0) {
       constexpr uint32_t idw = instr_desc(kFmtF16, 128, 64, false, false);
-      constexpr uint32_t idu = instr_desc(kFmtBF16, 128, 64, true, false);
+      // V^T: MN-major from the swizzled rows as staged, or K-major from the CV image
+      constexpr uint32_t idu = instr_desc(kFmtBF16, 128, 64, !CV, false);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const uint64_t xd = smem_desc(smem_u32(sm + L::kXK + k * 256), 128, 1024);
         const uint64_t tb = smem_desc(smem_u32(sm + L::kTb + k * 256), 128, 1024);
-        const uint64_t vd = smem_desc_sw128(smem_u32(sm + L::kV + k * 2048), 8192, 1024);
+        const uint64_t vd = CV ? smem_desc(smem_u32(sm + L::kVc + k * 256), 128, 1024)
+                               : smem_desc_sw128(smem_u32(sm + L::kV + k * 2048), 8192, 1024);
         const uint64_t tbb = smem_desc(smem_u32(sm + L::kTbb + k * 256), 128, 1024);
         mma_bf16(tm, xd, tb, idw, k > 0);
         mma_bf16(tm + 64, vd, tbb, idu, k > 0);
@@ -589,9 +739,11 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     mma_pending = true;
     if (!block_wait(bar_mma, ph_mma, p.hdr, p.wait_limit)) { ok = false; break; }
     mma_pending = false;
-    // v is consumed: load the next item's
-    if (have && tid == 0) stage_v(tokn, hn);
-    v_pending = have;
+    if constexpr (!CV) {
+      // v is consumed: load the next item's
+      if (have && tid == 0) stage_v(tokn, hn);
+      v_pending = have;
+    }
     // ---- F: W (into the [W ; Q'] image) and U~^T -> slot
     {
       const int ch = 32 * q4 + lane;
@@ -605,6 +757,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
       ug[ut_index(q4, cq, 1, lane)] = pack8h(u16 + 8);
     }
     fence_before_sync();
+    tbuf ^= 1;
   }
   if (tid == 0) {
     // a wait gave up: let the row loads and the products still in flight land
@@ -621,19 +774,22 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
 
 }  // namespace
 
-size_t prep_tc_smem_bytes() { return PrepSmem::kBytes; }
+size_t prep_tc_smem_bytes() { return PrepSmem<true>::kBytes; }
 
 cudaError_t launch_prep_tc(const TcParams& p, int gs, cudaStream_t st) {
-  auto prep = gs == kGateHead ? prep_kernel<kGateHead>
-            : gs == kGateChannel ? prep_kernel<kGateChannel> : prep_kernel<kGateZ>;
-  cudaError_t err = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         PrepSmem::kBytes);
+  // the input prologue comes with the KDA gate only
+  if (p.cw > 0 && gs != kGateZ) return cudaErrorInvalidValue;
+  auto prep = p.cw > 0 ? prep_kernel<kGateZ, true>
+            : gs == kGateHead ? prep_kernel<kGateHead, false>
+            : gs == kGateChannel ? prep_kernel<kGateChannel, false> : prep_kernel<kGateZ, false>;
+  const int bytes = p.cw > 0 ? PrepSmem<true>::kBytes : PrepSmem<false>::kBytes;
+  cudaError_t err = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (err != cudaSuccess) return err;
   int sms = 0, dev = 0;
   if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
   if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return err;
-  prep<<<sms, kNT, PrepSmem::kBytes, st>>>(p);
+  prep<<<sms, kNT, bytes, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -77,7 +77,9 @@ __device__ __forceinline__ unsigned char* chunk_slot(const unsigned char* prep_b
 }
 
 struct alignas(64) TcParams {
-  CUtensorMap sq, sk, sz, sv;  // [T, H, 128] bf16, box 64 tokens x 1 x 64 channels, 128-byte swizzle
+  // [T, H, 128] bf16, box 64 tokens x 1 x 64 channels, 128-byte swizzle (q, k,
+  // v: 72 tokens from 8 before the chunk when the input prologue runs in the preparation)
+  CUtensorMap sq, sk, sz, sv;
   const __nv_bfloat16 *q, *k, *beta, *z, *v;
   // g: the log-decay given directly, [T, H, 128], or the scalar gate's [T, H]
   // (one value per token and head); null when it is computed from z and A.
@@ -102,6 +104,10 @@ struct alignas(64) TcParams {
   // Limit (SM cycles) of the waits that can give up first; the waits that let
   // in-flight copies and MMAs land before a kernel leaves use kWaitCycles.
   long long wait_limit;
+  // Input prologue in the preparation (cw > 0): q, k, v are the inputs of the
+  // short convolution, cwq, cwk [H * 128, cw] and cwv [H * 128, cw] its taps.
+  const float *cwq, *cwk, *cwv;
+  int cw;
 };
 
 // Where the log-decay comes from (a template parameter of the preparation, so

@@ -35,7 +35,7 @@ EXPORTS = ("kda_status_string", "kda_version", "kda_forward_workspace_size",
            "kda_forward_norm_gate", "kda_decode_step_norm_gate", "kda_forward_scalar_gate",
            "kda_short_conv_swish", "kda_forward_conv_workspace_size", "kda_forward_conv",
            "kda_cp_workspace_size", "kda_cp_local", "kda_cp_finish", "kda_state_compose",
-           "kda_check_device_error", "kda_debug_set_wait_limit")
+           "kda_check_device_error", "kda_debug_set_wait_limit", "kda_decode_step_conv")
 
 # Bytes of the library's fixed scratch array used by kda_forward_noalloc.
 KDA_NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -87,6 +87,9 @@ def lib():
     L.kda_forward_scalar_gate.argtypes = [vp] * 7 + [i32] * 6 + [ctypes.c_int, i32, vp, vp, vp,
                                                                 sz, vp]
     L.kda_forward_scalar_gate.restype = ctypes.c_int
+    L.kda_decode_step_conv.argtypes = ([vp] * 6 + [i32, vp] + [vp] * 4 + [i32] * 4 +
+                                       [ctypes.c_int, vp, vp])
+    L.kda_decode_step_conv.restype = ctypes.c_int
     L.kda_short_conv_swish.argtypes = [vp, vp, vp] + [i32] * 5 + [ctypes.c_int, vp, vp]
     L.kda_short_conv_swish.restype = ctypes.c_int
     L.kda_forward_conv_workspace_size.argtypes = [i32] * 6 + [ctypes.c_int, i32]
@@ -182,6 +185,12 @@ def kda_forward_scalar_gate(q, k, v, g_head, beta, S0, cu_seqlens, num_seqs, tot
     return lib().kda_forward_scalar_gate(q, k, v, g_head, beta, S0, cu_seqlens, num_seqs,
                                          total_tokens, max_seqlen, H, dk, dv, dt, chunk, o,
                                          S_final, workspace, workspace_bytes, stream)
+
+
+def kda_decode_step_conv(x_q, x_k, x_v, w_q, w_k, w_v, conv_width, conv_state, z, A, beta,
+                         S_inout, B, H, dk, dv, dt, o, stream):
+    return lib().kda_decode_step_conv(x_q, x_k, x_v, w_q, w_k, w_v, conv_width, conv_state, z,
+                                      A, beta, S_inout, B, H, dk, dv, dt, o, stream)
 
 
 def kda_short_conv_swish(x, w, cu_seqlens, num_seqs, total_tokens, max_seqlen, channels, width,
@@ -409,6 +418,43 @@ def decode_step(q, k, v, z, A, beta, S, *, o=None, stream=None):
                          _dt(q), _p(o), _stream(stream))
     if st != KDA_OK:
         raise KdaError(st, "kda_decode_step")
+    return o
+
+
+def conv_state_zeros(B, H, dk, dv, width, dtype, device="cuda"):
+    """The rolling input window of decode_step_conv before a sequence's first
+    token: [B, H*(2*dk+dv), width-1] zeros."""
+    return torch.zeros((B, H * (2 * dk + dv), width - 1), dtype=dtype, device=device)
+
+
+def decode_step_conv(x_q, x_k, x_v, w_q, w_k, w_v, conv_state, z, A, beta, S, *, o=None,
+                     stream=None):
+    """One recurrent step with the input prologue carried across steps: x_q,
+    x_k [B,H,dk], x_v [B,H,dv] are this token's convolution inputs, w_* [H*d,
+    width] fp32 the taps, conv_state [B, H*(2dk+dv), width-1] (x's dtype) the
+    rolling window, S [B,H,dk,dv] fp32; conv_state and S are updated in place.
+    Returns o [B,H,dv]."""
+    _check_cuda(x_q, x_k, x_v, w_q, w_k, w_v, conv_state, z, A, beta, S, o)
+    B, H, dk = x_q.shape
+    dv = x_v.shape[-1]
+    _shapes(B, H, dk, dv, B, x_q.dtype, q=x_q, k=x_k, v=x_v, z=z, A=A, beta=beta, S=S, o=o)
+    width = w_q.shape[-1]
+    for name, w, rows in (("w_q", w_q, H * dk), ("w_k", w_k, H * dk), ("w_v", w_v, H * dv)):
+        if tuple(w.shape) != (rows, width) or w.dtype != torch.float32:
+            raise ValueError(f"{name}: {tuple(w.shape)} {w.dtype}, expected ({rows}, {width}) "
+                             "float32")
+    want = (B, H * (2 * dk + dv), width - 1)
+    if conv_state is None or tuple(conv_state.shape) != want or conv_state.dtype != x_q.dtype \
+            or not conv_state.is_contiguous():
+        got = None if conv_state is None else (tuple(conv_state.shape), conv_state.dtype)
+        raise ValueError(f"conv_state: {got}, expected contiguous {want} {x_q.dtype}")
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=x_q.dtype, device=x_q.device)
+    st = kda_decode_step_conv(_p(x_q), _p(x_k), _p(x_v), _p(w_q), _p(w_k), _p(w_v), width,
+                              _p(conv_state), _p(z), _p(A), _p(beta), _p(S), B, H, dk, dv,
+                              _dt(x_q), _p(o), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_decode_step_conv")
     return o
 
 

@@ -311,6 +311,32 @@ kda_status kda_forward_noalloc(const void* q, const void* k, const void* v,
                                void* o, float* S_final, kda_stream_t stream);
 
 /*
+ * kda_decode_step with the input prologue (Kimi Linear summary, §4: short
+ * convolution and Swish on q, k, v, as in kda_short_conv_swish) carried
+ * across steps: each sequence keeps a rolling window of its last
+ * conv_width - 1 inputs per channel, so that a run of steps equals
+ * kda_forward_conv over the same tokens.
+ *
+ *  x_q, x_k : [B, H, dk]; x_v : [B, H, dv]: this token's convolution inputs.
+ *  w_q, w_k : [H*dk, conv_width]; w_v : [H*dv, conv_width] float32
+ *             (4-byte aligned); conv_width : 1..4 (else KDA_ERR_UNSUPPORTED).
+ *  conv_state : [B, H*(2*dk + dv), conv_width - 1] in `dt`, channels in the
+ *             order q (h*dk + i), k (H*dk + h*dk + i), v (2*H*dk + h*dv + j);
+ *             element m holds the input of the token conv_width - 1 - m
+ *             steps back (m = 0 the oldest).  Read, then overwritten with the
+ *             window of the next step (zeros before a sequence's first token).
+ *             May be NULL when conv_width = 1.  Must not overlap any other
+ *             argument.
+ * Everything else is kda_decode_step's; the step is one launch.
+ */
+kda_status kda_decode_step_conv(const void* x_q, const void* x_k, const void* x_v,
+                                const float* w_q, const float* w_k, const float* w_v,
+                                int32_t conv_width, void* conv_state, const void* z,
+                                const float* A, const void* beta, float* S_inout, int32_t B,
+                                int32_t H, int32_t dk, int32_t dv, kda_dtype dt, void* o,
+                                kda_stream_t stream);
+
+/*
  * The layer's input prologue on one tensor (Kimi Linear summary, §4 "The Kimi
  * Linear Model Architecture": a short convolution captures dependencies
  * between neighbouring tokens, and a Swish nonlinearity is applied to the
@@ -338,27 +364,31 @@ kda_status kda_short_conv_swish(const void* x, const float* w, const int32_t* cu
                                 int32_t channels, int32_t width, kda_dtype dt, void* y,
                                 kda_stream_t stream);
 
-/* Workspace bytes for kda_forward_conv: kda_forward's, plus room for the
- * prologue's q, k and v (0 for unsupported arguments). */
+/* Workspace bytes for kda_forward_conv: kda_forward's on the tensor-core
+ * path (bf16, dk = dv = 128, chunk 64), where the prologue runs inside the
+ * chunk preparation; elsewhere kda_forward's plus room for the prologue's q,
+ * k and v (0 for unsupported arguments). */
 size_t kda_forward_conv_workspace_size(int32_t num_seqs, int32_t total_tokens,
                                        int32_t max_seqlen, int32_t H, int32_t dk, int32_t dv,
                                        kda_dtype dt, int32_t chunk);
 
 /*
  * kda_forward on the prologue's outputs: q = Swish(conv(x_q)), k = Swish(
- * conv(x_k)), v = Swish(conv(x_v)) as in kda_short_conv_swish (one launch for
- * the three tensors, written into the workspace), then the operator, which
- * normalises q and k to unit length itself.  z (the forget-gate input) and
- * beta are used as given.
+ * conv(x_k)), v = Swish(conv(x_v)) as in kda_short_conv_swish, then the
+ * operator, which normalises q and k to unit length itself.  z (the
+ * forget-gate input) and beta are used as given.
  *
  *  x_q, x_k : [T, H, dk]; x_v : [T, H, dv], in `dt`.
  *  w_q, w_k : [H*dk, conv_width]; w_v : [H*dv, conv_width] float32.
  *  conv_width : 1..4.
  *  workspace_bytes >= kda_forward_conv_workspace_size(...).
- * Everything else is kda_forward's.  One launch more than kda_forward.  The
- * prologue runs as its own HBM-bound pass (one read and one write of q, k,
- * v); kda_forward's first kernel is bound by instruction issue, so the same
- * arithmetic inside it would cost about as much time as the extra pass.
+ * Everything else is kda_forward's.  On the tensor-core path the prologue is
+ * fused into the chunk preparation: it stages each chunk's x rows with the
+ * three tokens before them, convolves and applies Swish in registers (q and
+ * k stay fp32 up to their norms; v is rounded to bf16 for the WY product), so
+ * the call reads x_q, x_k, x_v once and launches what kda_forward launches.
+ * On the CUDA-core path the prologue is one extra launch that writes q, k, v
+ * into the workspace.
  */
 kda_status kda_forward_conv(const void* x_q, const void* x_k, const void* x_v,
                             const float* w_q, const float* w_k, const float* w_v,

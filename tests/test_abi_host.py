@@ -164,6 +164,20 @@ def test_norm_gate_rejects_bad_epilogue_arguments(L):
     assert dec(gate=None, B=0) == kda.KDA_OK                    # nothing to do
 
 
+def test_decode_conv_rejects_bad_arguments(L):
+    def dec(width=4, wq=FAKE, state=FAKE, B=4, dk=32):
+        return kda.kda_decode_step_conv(FAKE, FAKE, FAKE, wq, FAKE, FAKE, width, state, FAKE,
+                                        FAKE, FAKE, FAKE, B, 2, dk, 32, kda.KDA_F32, FAKE, None)
+    assert dec(width=0) == kda.KDA_ERR_UNSUPPORTED
+    assert dec(width=5) == kda.KDA_ERR_UNSUPPORTED
+    assert dec(wq=None) == kda.KDA_ERR_INVALID_ARG
+    assert dec(wq=FAKE + 2) == kda.KDA_ERR_INVALID_ARG          # taps are 4-byte aligned
+    assert dec(state=None) == kda.KDA_ERR_INVALID_ARG           # width 4 carries a window
+    assert dec(state=FAKE + 2) == kda.KDA_ERR_INVALID_ARG       # fp32 window, misaligned
+    assert dec(dk=48) == kda.KDA_ERR_UNSUPPORTED
+    assert dec(state=None, wq=None, B=0) == kda.KDA_OK          # nothing to do
+
+
 def test_scalar_gate_requires_the_gate(L):
     st = kda.kda_forward_scalar_gate(FAKE, FAKE, FAKE, None, FAKE, None, None, 1, 64, 64, 2, 32,
                                      32, kda.KDA_F32, 16, FAKE, FAKE, FAKE, 1 << 40, None)
@@ -190,8 +204,12 @@ def test_forward_conv_workspace_and_arguments(L):
     args = (2, 256, 128, 4, 128, 128, kda.KDA_BF16, 64)
     fw = kda.kda_forward_workspace_size(*args)
     cw = kda.kda_forward_conv_workspace_size(*args)
-    # the prologue's q, k, v (bf16) follow the forward's workspace
-    assert cw >= fw + 3 * 256 * 4 * 128 * 2
+    # tensor-core path: the prologue runs inside the chunk preparation
+    assert cw == fw > 0
+    # CUDA-core path: the prologue's q, k, v (fp32) follow the forward's workspace
+    args32 = (2, 256, 128, 4, 64, 64, kda.KDA_F32, 16)
+    fw32 = kda.kda_forward_workspace_size(*args32)
+    assert kda.kda_forward_conv_workspace_size(*args32) >= fw32 + 3 * 256 * 4 * 64 * 4
     assert kda.kda_forward_conv_workspace_size(2, 256, 128, 4, 48, 128, kda.KDA_BF16, 64) == 0
 
     def fc(ws_bytes=cw, width=4, wq=FAKE):

@@ -84,12 +84,17 @@ def test_forward_conv_cuda_core_path(dtype, chunk, d, width):
 
 
 def test_forward_conv_long_workload_full_size():
-    """B=1, H=16, L=65536: kda_forward_conv equals the prologue run on each
-    tensor followed by kda_forward, bit for bit, at the full size."""
+    """B=1, H=16, L=65536 with the prologue fused into the chunk preparation:
+    o and S_final against the oracle prologue and recurrence on three sampled
+    heads, and, over all heads, agreement with the unfused route (the
+    prologue as its own pass, then kda_forward) within the bf16 bar."""
+    from oracle import prologue, ref
+    from kda_testutil import rel_l2, f64
     inp = synth.workload("long")
     d = to_cuda(inp)
     T, H, dk = inp["q"].shape
-    ci = to_cuda(synth.conv_inputs(T, H, dk, dk, 4, seed=85))
+    ci_h = synth.conv_inputs(T, H, dk, dk, 4, seed=85)
+    ci = to_cuda(ci_h)
     o, S = kda.forward_conv(ci["x_q"], ci["x_k"], ci["x_v"], ci["w_q"], ci["w_k"], ci["w_v"],
                             d["z"], d["A"], d["beta"], num_seqs=1)
     q = kda.short_conv_swish(ci["x_q"], ci["w_q"], num_seqs=1)
@@ -97,4 +102,14 @@ def test_forward_conv_long_workload_full_size():
     v = kda.short_conv_swish(ci["x_v"], ci["w_v"], num_seqs=1)
     o2, S2 = kda.forward(q, k, v, d["z"], d["A"], d["beta"], num_seqs=1)
     torch.cuda.synchronize()
-    assert torch.equal(o, o2) and torch.equal(S, S2)
+    assert rel_l2(f64(o), f64(o2)) <= 5e-3 and rel_l2(f64(S), f64(S2)) <= 5e-3
+    heads = [0, 7, 15]
+    rows = lambda w, d_: w.reshape(H, d_, -1)[heads].reshape(len(heads) * d_, -1)
+    xs = {key: ci_h[key][:, heads] for key in ("x_q", "x_k", "x_v")}
+    qh = prologue.short_conv_swish(xs["x_q"], rows(ci_h["w_q"], dk))
+    kh = prologue.short_conv_swish(xs["x_k"], rows(ci_h["w_k"], dk))
+    vh = prologue.short_conv_swish(xs["x_v"], rows(ci_h["w_v"], dk))
+    o_ref, S_ref = ref.forward(qh, kh, vh, inp["beta"][:, heads], z=inp["z"][:, heads],
+                               A=inp["A"][heads], num_seqs=1)
+    assert_close(o[:, heads], o_ref, torch.bfloat16, "o, sampled heads")
+    assert_close(S[:, heads], S_ref, torch.bfloat16, "S_final, sampled heads")
