@@ -49,16 +49,17 @@ __device__ __forceinline__ float* ckpt_state(const TcParams& p, int n, int h, in
 //   TRANS = false: full pass of segment p from its true incoming state; o, S_final.
 //   TRANS = true : transition of segments 0..P-2 on [S | X] from S = 0 (-> N_p)
 //                  and X = I (-> M_p), X^T a second 128-lane block; no Q', no o.
-// Slot parts are bulk-copied three chunks ahead into three stages.
+// Slot parts are bulk-copied ahead into a ring of stages (three chunks ahead in
+// the full pass, four in the transition pass, whose stages are smaller).
 template <bool TRANS>
 struct ChainSmem {
-  static constexpr int kStages = 3;
-  // stage layout: the slot (full pass), or [W ; Q'] | K' | U~^T | gamma (transition:
-  // the slot without A_qk and 1/|q|; one bulk copy per part)
-  static constexpr int kK = TRANS ? 32768 : kSlotK;
-  static constexpr int kUt = TRANS ? 49152 : kSlotU;
-  static constexpr int kGam = TRANS ? 49152 + 16384 : kSlotGam;
-  static constexpr int kStageBytes = TRANS ? 49152 + 16384 + 512 : kSlotBytes;
+  static constexpr int kStages = TRANS ? 4 : 3;
+  // stage layout: the slot (full pass), or W | K' | U~^T | gamma (transition: the
+  // W half of the [W ; Q'] image; no Q', A_qk or 1/|q|; one bulk copy per part)
+  static constexpr int kK = TRANS ? 16384 : kSlotK;
+  static constexpr int kUt = TRANS ? 32768 : kSlotU;
+  static constexpr int kGam = TRANS ? 32768 + 16384 : kSlotGam;
+  static constexpr int kStageBytes = TRANS ? 32768 + 16384 + 512 : kSlotBytes;
   static constexpr int kBytes = kStages * kStageBytes;
 };
 // TMEM columns (512 allocated): fp32 S^T, fp32 X^T (transition), the products D^T
@@ -116,7 +117,7 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
     const unsigned char* src = chunk_slot(p.prep, a, n, c, h, H);
     mbar_arrive_expect_tx(&s_ld[s], L::kStageBytes);
     if (TRANS) {
-      bulk_g2s(dst, src + kSlotWQ, 32768, &s_ld[s]);                     // [W ; Q']
+      bulk_g2s(dst, src + kSlotWQ, 16384, &s_ld[s]);                     // W
       bulk_g2s(dst + L::kK, src + kSlotK, 16384, &s_ld[s]);             // K'
       bulk_g2s(dst + L::kUt, src + kSlotU, 16384 + 512, &s_ld[s]);      // U~^T | gamma
     } else {
@@ -279,14 +280,14 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
         constexpr uint32_t id = instr_desc(kFmtF16, 128, 128, false, true);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const uint64_t bd = smem_desc(smem_u32(st + kSlotWQ + k * 4096), 2048, 128);
+          const uint64_t bd = smem_desc(smem_u32(st + kSlotWQ + k * 256), 128, 2048);
           mma_f16_ts(tm + dcol, tm + TM::kCp + 8 * k, bd, id, k > 0);
         }
       } else {
         constexpr uint32_t id = instr_desc(kFmtF16, 128, 64, false, true);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const uint64_t bd = smem_desc(smem_u32(st + k * 4096), 2048, 128);  // the W rows
+          const uint64_t bd = smem_desc(smem_u32(st + k * 256), 128, 2048);  // W
           mma_f16_ts(tm + TM::kD0, tm + TM::kCp + 8 * k, bd, id, k > 0);
           mma_f16_ts(tm + TM::kD0 + 64, tm + TM::kCp + 64 + 8 * k, bd, id, k > 0);
         }

@@ -99,16 +99,38 @@ __device__ __forceinline__ float tanh_approx(float x) {
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-// Swish: u sigmoid(u) = h + h tanh(h) with h = u / 2 (sigmoid(u) = (1 + tanh(u / 2)) / 2)
-__device__ __forceinline__ float swish(float u) {
-  const float h = 0.5f * u;
-  return fmaf(h, tanh_approx(h), h);
-}
 
 // Shared-memory matrix descriptor with the 128-byte swizzle (the layout TMA
 // writes with CU_TENSOR_MAP_SWIZZLE_128B into a 1024-byte aligned buffer).
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return smem_desc(saddr, lbo, sbo) | ((uint64_t)2u << 61);
+}
+
+// y = a * b and y = a * s over 16 values, in packed fp32x2 pairs
+__device__ __forceinline__ void mul16(float* y, const float* a, const float* b) {
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    const float2 r = __fmul2_rn(make_float2(a[i], a[i + 1]), make_float2(b[i], b[i + 1]));
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  }
+}
+__device__ __forceinline__ void scale16(float* y, const float* a, float s) {
+  const float2 s2 = make_float2(s, s);
+#pragma unroll
+  for (int i = 0; i < 16; i += 2) {
+    const float2 r = __fmul2_rn(make_float2(a[i], a[i + 1]), s2);
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  }
+}
+// 16 consecutive fp32 from shared memory (64-byte aligned)
+__device__ __forceinline__ void lds16(const float* p, float* y) {
+#pragma unroll
+  for (int i = 0; i < 16; i += 4) {
+    const float4 v = *reinterpret_cast<const float4*>(p + i);
+    y[i] = v.x; y[i + 1] = v.y; y[i + 2] = v.z; y[i + 3] = v.w;
+  }
 }
 
 // 16 fp32 values of 16 consecutive tokens -> two units of a bf16 operand image
@@ -185,7 +207,8 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
   // the current token); history before the sequence's first token reads as zero
   // (first: this chunk is its sequence's first), tokens from len on give zero
   // Token pairs (16 b + 2 p, 16 b + 2 p + 1) go through packed fp32x2 arithmetic;
-  // the taps hw are halved, so the sum is u / 2 and Swish(u) = h + h tanh(h).
+  // the taps hw are halved, so the sum is h = u / 2 and, with sigmoid(u) =
+  // (1 + tanh(u / 2)) / 2, Swish(u) = u sigmoid(u) = h + h tanh(h).
   const uint32_t jboxc = (uint32_t)(j >> 6) * (uint32_t)L::kBox + (uint32_t)(j & 7) * 2u;
   auto conv16 = [&](int base, const float4 hw, bool first, int len, float* y) {
     float x[19];  // tokens 16 b - 3 .. 16 b + 15
@@ -390,12 +413,19 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     }
     // ---- A2: gate -> alpha; E = e^{Gam - rho_b} (E = 1 at the sub-tile's first token)
     if constexpr (GS == kGateZ) {
+      const float2 nA = make_float2(-expA_l2, -expA_l2), one = make_float2(1.0f, 1.0f),
+                   c5 = make_float2(kGateMin * kLog2e, kGateMin * kLog2e);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float zz = raw_f(L::kZ, i);
-        const float ez = ex2(-expA_l2 * zz);                 // e^{-e^A z}
-        const float sg = rcp(1.0f + ez);                     // sigmoid(e^A z)
-        al[i] = 16 * b + i < len ? ex2((kGateMin * kLog2e) * sg) : 1.0f;  // e^{-5 sigmoid}
+      for (int i = 0; i < 16; i += 2) {
+        const float2 m = __fmul2_rn(make_float2(raw_f(L::kZ, i), raw_f(L::kZ, i + 1)), nA);
+        const float2 d = __fadd2_rn(make_float2(ex2(m.x), ex2(m.y)), one);  // 1 + e^{-e^A z}
+        const float2 s = __fmul2_rn(make_float2(rcp(d.x), rcp(d.y)), c5);   // -5 log2e sigmoid
+        al[i] = ex2(s.x);                                                   // e^{-5 sigmoid}
+        al[i + 1] = ex2(s.y);
+      }
+      if (len < kC) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) al[i] = 16 * b + i < len ? al[i] : 1.0f;
       }
     } else {
 #pragma unroll
@@ -470,22 +500,23 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     }
     float* Ei = al;
     // k / |k|
-#pragma unroll
-    for (int i = 0; i < 16; ++i) kv[i] *= nrm[64 + 16 * b + i];
+    {
+      float t[16];
+      lds16(nrm + 64 + 16 * b, t);
+      mul16(kv, kv, t);
+    }
 
     // ---- C: M1 operands.  R rows (beta k^ E, then q E), windows (k^ / E times
     //      e^{rho_c - rho_b} for the later row sub-tiles c)
     {
-      float x[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) x[i] = bvec[16 * b + i] * kv[i] * E[i];
-      put16(sm + L::kR, img_unit(32 * b, j, 128), img_unit(32 * b + 8, j, 128), x);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) x[i] = qv[i] * E[i];
-      put16(sm + L::kR, img_unit(32 * b + 16, j, 128), img_unit(32 * b + 24, j, 128), x);
-      float cd[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) cd[i] = kv[i] * Ei[i];
+      float x[16], bke[16], qe[16], cd[16];
+      lds16(bvec + 16 * b, x);
+      mul16(bke, kv, E);
+      mul16(bke, bke, x);   // beta k^ E
+      put16(sm + L::kR, img_unit(32 * b, j, 128), img_unit(32 * b + 8, j, 128), bke);
+      mul16(qe, qv, E);     // q E
+      put16(sm + L::kR, img_unit(32 * b + 16, j, 128), img_unit(32 * b + 24, j, 128), qe);
+      mul16(cd, kv, Ei);    // k^ / E
       {
         const int r0 = win_row0(b) + 16 * b;
         put16(sm + L::kWB, img_unit(r0, j, kWinRows), img_unit(r0 + 8, j, kWinRows), cd);
@@ -495,8 +526,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
         const int cw = b + s;  // window of row sub-tile cw
         if (cw < 4) {
           const float f = s == 1 ? F1 : s == 2 ? F2 : F3;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) x[i] = cd[i] * f;
+          scale16(x, cd, f);
           const int r0 = win_row0(cw) + 16 * b;
           put16(sm + L::kWB, img_unit(r0, j, kWinRows), img_unit(r0 + 8, j, kWinRows), x);
         }
@@ -517,14 +547,11 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
       mma_pending = true;
       // meanwhile: X_K = beta k^ e^{Gam} (M2 operand), Q' = q e^{Gam} and
       // K' = k^ e^{Gam_last - Gam} (slot)
-#pragma unroll
-      for (int i = 0; i < 16; ++i) x[i] = bvec[16 * b + i] * kv[i] * E[i] * Pb;
+      scale16(x, bke, Pb);
       put16h(sm + L::kXK, img_unit(16 * b, j, 64), img_unit(16 * b + 8, j, 64), x);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) x[i] = qv[i] * E[i] * Pb;
-      put16h(slot + kSlotWQ, img_unit(64 + 16 * b, j, 128), img_unit(72 + 16 * b, j, 128), x);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) x[i] = cd[i] * Lb;
+      scale16(x, qe, Pb);
+      put16h(slot + kSlotWQ, img_tg(64 + 16 * b, j), img_tg(72 + 16 * b, j), x);
+      scale16(x, cd, Lb);
       put16h(slot + kSlotK, img_unit(16 * b, j, 64), img_unit(16 * b + 8, j, 64), x);
     }
     if (!block_wait(bar_mma, ph_mma, p.hdr, p.wait_limit)) { ok = false; break; }
@@ -751,7 +778,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
       tmem_ld16(tmem_addr(tm, 32 * q4, 16 * cq), w16);
       tmem_ld16(tmem_addr(tm, 32 * q4, 64 + 16 * cq), u16);
       tmem_ld_wait();
-      put16h(slot + kSlotWQ, img_unit(16 * cq, ch, 128), img_unit(16 * cq + 8, ch, 128), w16);
+      put16h(slot + kSlotWQ, img_tg(16 * cq, ch), img_tg(16 * cq + 8, ch), w16);
       uint4* ug = reinterpret_cast<uint4*>(slot + kSlotU);
       ug[ut_index(q4, cq, 0, lane)] = pack8h(u16);
       ug[ut_index(q4, cq, 1, lane)] = pack8h(u16 + 8);

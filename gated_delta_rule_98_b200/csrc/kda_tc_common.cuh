@@ -43,6 +43,12 @@ __host__ __device__ constexpr uint32_t img(int t, int c, int rows) {
 __host__ __device__ constexpr uint32_t img_unit(int t0, int c, int rows) {
   return (uint32_t)((c >> 3) * (rows * 16) + (t0 >> 3) * 128 + (c & 7) * 16);
 }
+// The same units ordered token group first (a 128-channel image): group t0 / 8
+// of 8 tokens occupies 2 KB, so any run of token groups is contiguous; as an
+// MN-major operand with the tokens as N: LBO = 128 (channel groups), SBO = 2048.
+__host__ __device__ constexpr uint32_t img_tg(int t0, int c) {
+  return (uint32_t)((t0 >> 3) * 2048 + (c >> 3) * 128 + (c & 7) * 16);
+}
 
 // Chain operands of one (chunk, head), written by the preparation kernel and
 // read by the chain passes with bulk copies.  The images are f16 (10-bit
@@ -50,8 +56,9 @@ __host__ __device__ constexpr uint32_t img_unit(int t0, int c, int rows) {
 // and the state is non-expansive), so f16 holds them with 8x less rounding
 // than bf16; values below the f16 range flush towards zero (absolute error
 // under 1e-7) and out-of-range ones would saturate.
-//   WQ   [W ; Q'] as one 128-row image (W tokens 0..63, Q' tokens 64..127), the
-//        B operand of C1 (N = 128 tokens, K = dk), MN-major.
+//   WQ   [W ; Q'] as one 128-row token-group-first image (img_tg: W tokens
+//        0..63 in the first 16 KB, Q' tokens 64..127 in the next), the B operand
+//        of C1 (N = 128 tokens, K = dk; the transition pass reads the W half), MN-major.
 //   K    K' (64-row image): the A operand K'^T of C2 (M = dk, K = token), K-major.
 //   A    A_qk with key column i as the "token" and query row r as the channel
 //        (64 x 64): the B operand A_qk^T of the output update (N = r, K = i),
