@@ -47,10 +47,16 @@ constexpr int kWinRows = 160;
 // so box row 8 + t holds token t and rows 5 .. 7 the convolution's history.
 template <bool CV>
 struct PrepSmem {
-  // staged rows: per tensor two 64-channel boxes of kRows tokens, 128-byte swizzle
+  // staged rows: per tensor two 64-channel boxes of kRows tokens, 128-byte swizzle.
+  // q, k, z rows are double-buffered (kNQ buffers of kQKZ bytes: an item's rows
+  // are requested two items ahead) where shared memory allows, i.e. without the
+  // prologue; v rows have one buffer.
   static constexpr int kRows = CV ? kC + 8 : kC;
   static constexpr int kBox = kRows * 128;
-  static constexpr int kQ = 0, kK = 2 * kBox, kZ = 4 * kBox, kV = kZ + 16384;
+  static constexpr int kNQ = CV ? 1 : 2;
+  static constexpr int kQKZ = 4 * kBox + 16384;
+  static constexpr int kQ = 0, kK = 2 * kBox, kZ = 4 * kBox;  // in buffer 0 (+ kQKZ: buffer 1)
+  static constexpr int kV = kNQ * kQKZ;
   static constexpr int kWB = kV + 2 * kBox;        // windows, 160-row image: the B operand of M1
   static constexpr int kR = kWB + kWinRows * 256; // R: 128-row image (sub-tile b: k rows 32b..,
                                                   //   q rows 32b+16..), the A operand of M1
@@ -73,14 +79,16 @@ struct PrepSmem {
   static constexpr int kOnes = kTaps + (CV ? 12288 : 0);
   // CV: Swish(conv(v)) as a 64-row bf16 image, the A operand V^T of M2 (K-major)
   static constexpr int kVc = kOnes + (CV ? 512 : 0);
-  static constexpr int kBar = kVc + (CV ? 16384 : 0);  // three mbarriers, then the TMEM base
+  static constexpr int kBar = kVc + (CV ? 16384 : 0);  // four mbarriers, then the TMEM base
   static constexpr int kBytes = kBar + 64;
   // CV, before M1: squares of q, k (hi and lo bf16 parts), a 128-row image with
   // 256 channels over the window / R region: the A operand of the norm product
   static constexpr int kSq = kWB;
   static_assert(kSq + 65536 <= kXK, "norm operand overlaps X_K");
   static_assert(kR + 32768 <= kXK, "M1 operands overlap X_K");
-  static_assert(kBox % 1024 == 0 && kV % 1024 == 0, "swizzled boxes need 1024-byte alignment");
+  static_assert(kBox % 1024 == 0 && kQKZ % 1024 == 0 && kV % 1024 == 0,
+                "swizzled boxes need 1024-byte alignment");
+  static_assert(kBytes <= 232448, "shared memory per CTA");
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -155,10 +163,10 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
   float* bvec = reinterpret_cast<float*>(sm + L::kBeta);
   float* exf = reinterpret_cast<float*>(sm + L::kEx);
   float* exl = exf + 512;
-  uint64_t* bar_qkz = reinterpret_cast<uint64_t*>(sm + L::kBar);
-  uint64_t* bar_v = bar_qkz + 1;
-  uint64_t* bar_mma = bar_qkz + 2;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_qkz + 3);
+  uint64_t* bar_qkz = reinterpret_cast<uint64_t*>(sm + L::kBar);  // one per q, k, z buffer
+  uint64_t* bar_v = bar_qkz + 2;
+  uint64_t* bar_mma = bar_qkz + 3;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_qkz + 4);
   const int H = p.H;
 
   if (!seqlens_valid(p.cu, p.N, p.T, p.max_len)) {
@@ -176,6 +184,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
   }
   if (tid == 0) {
     mbar_init(bar_qkz, 1);
+    mbar_init(bar_qkz + 1, 1);
     mbar_init(bar_v, 1);
     mbar_init(bar_mma, 1);
     fence_mbar_init();
@@ -184,8 +193,9 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
   __syncthreads();
   fence_after_sync();
   const uint32_t tm = *s_tmem;
-  uint32_t ph_qkz = 0, ph_v = 0, ph_mma = 0;
-  bool ok = true, qkz_pending = false, v_pending = false, mma_pending = false;
+  uint32_t ph_qkz = 0, ph_v = 0, ph_mma = 0;  // ph_qkz bit s: parity of buffer s's next load
+  uint32_t qkz_pending = 0;                    // bit s: buffer s being filled
+  bool ok = true, v_pending = false, mma_pending = false;
 
   // elementwise phases: channel j, sub-tile b (tokens 16 b .. 16 b + 15)
   const int j = tid & 127, b = tid >> 7;
@@ -277,32 +287,35 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
   // gridDim.x-th one, stepping the mixed-radix index without divisions
   const int maxch = (p.max_len + kC - 1) / kC;
   const long long it0 = blockIdx.x, stride = gridDim.x;
-  int h = (int)(it0 % H), n = (int)((it0 / H) % p.N), c = (int)(it0 / ((long long)H * p.N));
   const int sh = (int)(stride % H), sn = (int)((stride / H) % p.N);
   const int sc = (int)(stride / ((long long)H * p.N));
-  int a = 0, e = 0;  // token range [a, e) of sequence n
-  auto next_item = [&]() -> bool {
-    for (; c < maxch;) {
-      seq_bounds(p.cu, n, p.max_len, a, e);
-      if (a + c * kC < e) return true;
-      h += sh;
-      if (h >= H) { h -= H; ++n; }
-      n += sn;
-      if (n >= p.N) { n -= p.N; ++c; }
-      c += sc;
+  struct Item { int h, n, c, a, e; };  // head, sequence, chunk; token range [a, e) of n
+  auto step = [&](Item& s) {
+    s.h += sh;
+    if (s.h >= H) { s.h -= H; ++s.n; }
+    s.n += sn;
+    if (s.n >= p.N) { s.n -= p.N; ++s.c; }
+    s.c += sc;
+  };
+  auto seek = [&](Item& s) -> bool {  // the first item from s on that holds tokens
+    for (; s.c < maxch;) {
+      seq_bounds(p.cu, s.n, p.max_len, s.a, s.e);
+      if (s.a + s.c * kC < s.e) return true;
+      step(s);
     }
     return false;
   };
   constexpr int kHist = CV ? 8 : 0;  // box rows before the chunk
-  auto stage_qkz = [&](int tok, int hh) {  // one thread
-    mbar_arrive_expect_tx(bar_qkz, 4 * L::kBox + (GS == kGateZ ? 16384 : 0));
-    tma_box_x(sm + L::kQ, &p.sq, 0, hh, tok - kHist, bar_qkz);
-    tma_box_x(sm + L::kQ + L::kBox, &p.sq, 64, hh, tok - kHist, bar_qkz);
-    tma_box_x(sm + L::kK, &p.sk, 0, hh, tok - kHist, bar_qkz);
-    tma_box_x(sm + L::kK + L::kBox, &p.sk, 64, hh, tok - kHist, bar_qkz);
+  auto stage_qkz = [&](int s, int tok, int hh) {  // one thread; buffer s
+    unsigned char* d = sm + s * L::kQKZ;
+    mbar_arrive_expect_tx(bar_qkz + s, 4 * L::kBox + (GS == kGateZ ? 16384 : 0));
+    tma_box_x(d + L::kQ, &p.sq, 0, hh, tok - kHist, bar_qkz + s);
+    tma_box_x(d + L::kQ + L::kBox, &p.sq, 64, hh, tok - kHist, bar_qkz + s);
+    tma_box_x(d + L::kK, &p.sk, 0, hh, tok - kHist, bar_qkz + s);
+    tma_box_x(d + L::kK + L::kBox, &p.sk, 64, hh, tok - kHist, bar_qkz + s);
     if (GS == kGateZ) {
-      tma_box_x(sm + L::kZ, &p.sz, 0, hh, tok, bar_qkz);
-      tma_box_x(sm + L::kZ + 8192, &p.sz, 64, hh, tok, bar_qkz);
+      tma_box_x(d + L::kZ, &p.sz, 0, hh, tok, bar_qkz + s);
+      tma_box_x(d + L::kZ + 8192, &p.sz, 64, hh, tok, bar_qkz + s);
     }
   };
   auto stage_v = [&](int tok, int hh) {  // one thread
@@ -318,39 +331,52 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
                : 0u;
   };
 
-  bool have = next_item();
+  // the current item, the next one and (two buffers) the one after
+  Item cur{(int)(it0 % H), (int)((it0 / H) % p.N), (int)(it0 / ((long long)H * p.N)), 0, 0};
+  bool have = seek(cur);
+  Item nx = cur;
+  bool have_nx = false;
+  if (have) {
+    step(nx);
+    have_nx = seek(nx);
+  }
   uint32_t beta_nx = 0u;
   // A_h of the next item's head, loaded an item ahead
-  float a_nx = (GS == kGateZ && have) ? p.A[h] : 0.f;
+  float a_nx = (GS == kGateZ && have) ? p.A[cur.h] : 0.f;
   if (have) {
     if (tid == 0) {
-      stage_qkz(a + c * kC, h);
-      stage_v(a + c * kC, h);
+      stage_qkz(0, cur.a + cur.c * kC, cur.h);
+      if (L::kNQ == 2 && have_nx) stage_qkz(1, nx.a + nx.c * kC, nx.h);
+      stage_v(cur.a + cur.c * kC, cur.h);
     }
-    qkz_pending = v_pending = true;
-    beta_nx = load_beta(a + c * kC, e, h);
+    qkz_pending = (L::kNQ == 2 && have_nx) ? 3u : 1u;
+    v_pending = true;
+    beta_nx = load_beta(cur.a + cur.c * kC, cur.e, cur.h);
   }
+  int qs = 0;  // the q, k, z buffer of the current item
   int tbuf = 0;  // CV: the taps buffer of the current item
   if constexpr (CV) {
     // the ones block (bf16 1.0) and the first item's taps; published by the
     // first item's first block-wide wait
     if (tid < 128) reinterpret_cast<uint32_t*>(sm + L::kOnes)[tid] = 0x3F803F80u;
-    if (have && b < 3) tapbuf[b * 128 + j] = load_taps(h);
+    if (have && b < 3) tapbuf[b * 128 + j] = load_taps(cur.h);
   }
   while (have) {
-    const int hc = h, nc = n, ac = a, ec = e, cc0 = c;
-    h += sh;
-    if (h >= H) { h -= H; ++n; }
-    n += sn;
-    if (n >= p.N) { n -= p.N; ++c; }
-    c += sc;
-    have = next_item();  // the item after this one
+    const int hc = cur.h, nc = cur.n, ac = cur.a, ec = cur.e, cc0 = cur.c;
+    // the item after the next: its q, k, z rows go to this item's buffer
+    Item nx2 = nx;
+    bool have_nx2 = false;
+    if (L::kNQ == 2 && have_nx) {
+      step(nx2);
+      have_nx2 = seek(nx2);
+    }
     const int tok0 = ac + cc0 * kC;
     const int len = min(kC, ec - tok0);
-    const int tokn = have ? a + c * kC : 0, hn = h;
+    const int tokn = have_nx ? nx.a + nx.c * kC : 0, hn = nx.h;
+    const int qb = qs * L::kQKZ;  // byte offset of this item's q, k, z buffer
     unsigned char* slot = chunk_slot(p.prep, ac, nc, cc0, hc, H);
     if (tid < kC) bvec[tid] = __uint_as_float(beta_nx << 16);
-    if (have) beta_nx = load_beta(tokn, e, hn);
+    if (have_nx) beta_nx = load_beta(tokn, nx.e, hn);
 
     // per-channel gate input, issued before the wait
     float al[16];  // alpha of tokens 16 b + i (then 1 / E)
@@ -368,10 +394,14 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
       }
     }
     const float expA_l2 = GS == kGateZ ? expf(a_nx) * kLog2e : 0.f;
-    if (GS == kGateZ && have) a_nx = p.A[hn];
+    if (GS == kGateZ && have_nx) a_nx = p.A[hn];
 
-    if (!block_wait(bar_qkz, ph_qkz, p.hdr, p.wait_limit)) { ok = false; break; }
-    qkz_pending = false;
+    {
+      uint32_t ph = (ph_qkz >> qs) & 1u;
+      if (!block_wait(bar_qkz + qs, ph, p.hdr, p.wait_limit)) { ok = false; break; }
+      ph_qkz ^= 1u << qs;
+      qkz_pending &= ~(1u << qs);
+    }
 
     float qv[16], kv[16];  // q, k of the thread's tokens (zero past the sequence end)
     if constexpr (CV) {
@@ -379,9 +409,9 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
       //      go to one product with a block of ones, D[row][.] = sum over the
       //      channels (rows 0-63 q, 64-127 k), read after the gate
       const float4* tq = tapbuf + tbuf * 384;
-      conv16(L::kQ, tq[j], cc0 == 0, len, qv);
+      conv16(L::kQ + qb, tq[j], cc0 == 0, len, qv);
       put_squares(qv, 16 * b);
-      conv16(L::kK, tq[128 + j], cc0 == 0, len, kv);
+      conv16(L::kK + qb, tq[128 + j], cc0 == 0, len, kv);
       put_squares(kv, 64 + 16 * b);
       sync_for_mma();
       if (tid == 0) {
@@ -397,7 +427,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
       // ---- A1: row norms (thread: row tid / 4 of [q ; k], 32 channels)
       const int r = tid >> 2, qt = tid & 3, t = r & 63;
       const unsigned char* rowp =
-          sm + (r < 64 ? L::kQ : L::kK) + (qt >> 1) * 8192 + t * 128;
+          sm + qb + (r < 64 ? L::kQ : L::kK) + (qt >> 1) * 8192 + t * 128;
       float ss = 0.f;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
@@ -417,7 +447,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
                    c5 = make_float2(kGateMin * kLog2e, kGateMin * kLog2e);
 #pragma unroll
       for (int i = 0; i < 16; i += 2) {
-        const float2 m = __fmul2_rn(make_float2(raw_f(L::kZ, i), raw_f(L::kZ, i + 1)), nA);
+        const float2 m = __fmul2_rn(make_float2(raw_f(L::kZ + qb, i), raw_f(L::kZ + qb, i + 1)), nA);
         const float2 d = __fadd2_rn(make_float2(ex2(m.x), ex2(m.y)), one);  // 1 + e^{-e^A z}
         const float2 s = __fmul2_rn(make_float2(rcp(d.x), rcp(d.y)), c5);   // -5 log2e sigmoid
         al[i] = ex2(s.x);                                                   // e^{-5 sigmoid}
@@ -450,14 +480,18 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const bool in = 16 * b + i < len;
-        qv[i] = in ? raw_f(L::kQ, i) : 0.f;
-        kv[i] = in ? raw_f(L::kK, i) : 0.f;
+        qv[i] = in ? raw_f(L::kQ + qb, i) : 0.f;
+        kv[i] = in ? raw_f(L::kK + qb, i) : 0.f;
       }
     }
     __syncthreads();
-    // the staged q, k, z rows are consumed: load the next item's
-    if (have && tid == 0) stage_qkz(tokn, hn);
-    qkz_pending = have;
+    // the staged q, k, z rows are consumed: load the rows of the item kNQ ahead
+    {
+      const bool more = L::kNQ == 2 ? have_nx2 : have_nx;
+      const Item& ld = L::kNQ == 2 ? nx2 : nx;
+      if (more && tid == 0) stage_qkz(qs, ld.a + ld.c * kC, ld.h);
+      if (more) qkz_pending |= 1u << qs;
+    }
 
     // ---- B: decay factors of (channel j, sub-tile b)
     float Pb, Lb, F1 = 0.f, F2 = 0.f, F3 = 0.f;  // e^{rho_b}, e^{Gam_last - rho_b}, e^{rho_{b+s} - rho_b}
@@ -588,7 +622,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     __syncthreads();
     // CV: the next item's taps, loaded during the inverse and stored after it
     float4 tnext = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (CV && have && b < 3) tnext = load_taps(hn);
+    if (CV && have_nx && b < 3) tnext = load_taps(hn);
 
     // ---- E: T = (I + A_kk)^{-1} in fp32.  Diagonal 16x16 blocks by forward
     //      substitution (one warp per block, lane = column), then the blocks below
@@ -728,7 +762,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     __syncthreads();
     // the merged block T[32:64][0:32]
     if (tid < 128) put_t(32 + (tid & 31), (tid >> 5) * 8);
-    if (CV && have && b < 3) tapbuf[(tbuf ^ 1) * 384 + b * 128 + j] = tnext;
+    if (CV && have_nx && b < 3) tapbuf[(tbuf ^ 1) * 384 + b * 128 + j] = tnext;
     // the v rows must have landed (a block-wide wait that also orders the T images)
     fence_async_smem();
     fence_before_sync();
@@ -741,8 +775,8 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
       conv16(L::kV, tapbuf[tbuf * 384 + 256 + j], cc0 == 0, len, y);
       put16(sm + L::kVc, img_unit(16 * b, j, 64), img_unit(16 * b + 8, j, 64), y);
       sync_for_mma();
-      if (have && tid == 0) stage_v(tokn, hn);
-      v_pending = have;
+      if (have_nx && tid == 0) stage_v(tokn, hn);
+      v_pending = have_nx;
     }
     // ---- M2: W^T = X_K^T T^T -> TMEM columns 0-63 and U~^T = V^T (T Diag(beta))^T
     //      -> 64-127 (M = 128 channels, N = 64 tokens; V read in place from its
@@ -768,8 +802,8 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     mma_pending = false;
     if constexpr (!CV) {
       // v is consumed: load the next item's
-      if (have && tid == 0) stage_v(tokn, hn);
-      v_pending = have;
+      if (have_nx && tid == 0) stage_v(tokn, hn);
+      v_pending = have_nx;
     }
     // ---- F: W (into the [W ; Q'] image) and U~^T -> slot
     {
@@ -785,11 +819,25 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     }
     fence_before_sync();
     tbuf ^= 1;
+    qs = L::kNQ == 2 ? qs ^ 1 : 0;
+    cur = nx;
+    have = have_nx;
+    if (L::kNQ == 2) {
+      nx = nx2;
+      have_nx = have_nx2;
+    } else if (have) {  // one buffer: the item after the new current one is found here
+      nx = cur;
+      step(nx);
+      have_nx = seek(nx);
+    } else {
+      have_nx = false;
+    }
   }
   if (tid == 0) {
     // a wait gave up: let the row loads and the products still in flight land
     // before the CTA frees its Tensor Memory and leaves (at most ~2 s each)
-    if (qkz_pending) (void)mbar_wait_cycles(bar_qkz, ph_qkz, kWaitCycles);
+    for (int q = 0; q < 2; ++q)
+      if (qkz_pending & (1u << q)) (void)mbar_wait_cycles(bar_qkz + q, (ph_qkz >> q) & 1u, kWaitCycles);
     if (v_pending) (void)mbar_wait_cycles(bar_v, ph_v, kWaitCycles);
     if (mma_pending) (void)mbar_wait_cycles(bar_mma, ph_mma, kWaitCycles);
   }
