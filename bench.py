@@ -66,7 +66,8 @@ def peaks():
 # The sources each recorded kernel's traffic depends on (a change elsewhere
 # leaves its record valid).
 _TRAFFIC_SOURCES = {
-    "forward": ("kda_prefill_tc.cu", "tc_sm100.cuh", "kda_common.cuh", "kda_launch.h"),
+    "forward": ("kda_prep_tc.cu", "kda_prefill_tc.cu", "kda_tc_common.cuh", "tc_sm100.cuh",
+                "kda_common.cuh", "kda_launch.h"),
     "decode": ("kda_decode.cu", "kda_common.cuh", "kda_launch.h"),
 }
 
@@ -561,7 +562,7 @@ def main():
                                                                   CHUNK),
                               dtype=torch.uint8, device=dev)
 
-        def fwd_conv():  # input prologue (width-4 short convolution + Swish), then the operator
+        def fwd_conv():  # input prologue (width-4 short convolution + Swish) fused into the operator
             kda.forward_conv(ci["x_q"], ci["x_k"], ci["x_v"], ci["w_q"], ci["w_k"], ci["w_v"],
                              d["z"], d["A"], d["beta"], num_seqs=B, chunk=CHUNK, o=o,
                              S_final=Sf, workspace=conv_ws, stream=stream)
@@ -573,7 +574,7 @@ def main():
                 ("checkpoints_every_%d" % interval, fwd_ckpt, ck.numel() * 4),
                 ("cp_local_and_finish", fwd_cp, 0),
                 ("scalar_gate", fwd_scalar, T * H * 4 - T * H * D * 2),
-                ("conv_prologue_width4", fwd_conv, 4 * 3 * T * H * D)):
+                ("conv_prologue_width4", fwd_conv, 3 * H * D * 4 * 4)):  # + the taps
             for _ in range(args.warmup):
                 fn()
             torch.cuda.synchronize()

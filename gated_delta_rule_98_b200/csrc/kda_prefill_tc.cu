@@ -84,6 +84,7 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
   __shared__ int s_abort;
   __shared__ float s_iq[64];        // 1/|q| of the chunk whose o is written next
   __shared__ float s_red[4][64];    // output epilogue: sum of squares per lane quarter and token
+  __shared__ float s_rs[64];        // output epilogue: 1 / RMS of each token's o row
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = blockIdx.x, h = blockIdx.y, seg = blockIdx.z;
@@ -180,17 +181,27 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
   // ---- o of a chunk from D_Q^T (columns dcol + 64 ..): lane v holds its column
   //      for tokens 16 cq .. 16 cq + 15; with the output epilogue the sums of
   //      squares over the 128 columns meet in shared memory.
-  uint32_t rg[8];  // output-epilogue gate inputs (f32 pairs as bf16x2) of the next write_o
+  // Output epilogue: the gate inputs of chunk cc (raw bf16 bits in rgr) are
+  // requested a chunk ahead, while the previous chunk's C2 product runs, and
+  // not touched until they are turned into sigmoids (sg) while cc's own C2
+  // runs, so their latency stays off the chain's critical path; write_o(cc)
+  // uses sg during the next chunk's C1.
+  uint32_t rgr[16];
+  float sg[16];
+  const float wv = (p.og && p.ow) ? p.ow[v] : 1.f;
   auto load_gate = [&](int cc) {
     if (!p.og) return;
     const int t0c = a + cc * kC, lenc = min(kC, b - t0c);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int t = 16 * cq + 2 * i;
-      const uint32_t x0 = t < lenc ? *reinterpret_cast<const uint16_t*>(p.og + ((size_t)(t0c + t) * H + h) * kD + v) : 0u;
-      const uint32_t x1 = t + 1 < lenc ? *reinterpret_cast<const uint16_t*>(p.og + ((size_t)(t0c + t + 1) * H + h) * kD + v) : 0u;
-      rg[i] = x0 | (x1 << 16);
+    for (int i = 0; i < 16; ++i) {
+      const int t = 16 * cq + i;
+      rgr[i] = t < lenc ? *reinterpret_cast<const uint16_t*>(p.og + ((size_t)(t0c + t) * H + h) * kD + v) : 0u;
     }
+  };
+  auto gate_sigmoids = [&]() {
+    if (!p.og) return;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) sg[i] = out_sigmoid(__uint_as_float(rgr[i] << 16));
   };
   auto write_o = [&](int cc, uint32_t dcol) {
     const int t0c = a + cc * kC, lenc = min(kC, b - t0c);
@@ -221,15 +232,13 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
       const int tl = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
       if ((lane & 1) == 0) s_red[q4][16 * cq + tl] = y[0];
       asm volatile("bar.sync %0, 128;" ::"r"(1 + cq) : "memory");  // the four warps of column quarter cq
-      const float w = p.ow ? p.ow[v] : 1.f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int t = 16 * cq + i;
-        const float ss = s_red[0][t] + s_red[1][t] + s_red[2][t] + s_red[3][t];
-        const uint32_t r2 = i & 1 ? rg[i >> 1] >> 16 : rg[i >> 1] & 0xffffu;
-        x[i] = x[i] * rsqrtf(ss * (1.0f / kD) + p.oeps) * w * out_sigmoid(__uint_as_float(r2 << 16));
+      if (q4 == 0 && lane < 16) {  // one reciprocal RMS per token
+        const int t = 16 * cq + lane;
+        s_rs[t] = rsqrtf((s_red[0][t] + s_red[1][t] + s_red[2][t] + s_red[3][t]) * (1.0f / kD) + p.oeps);
       }
-      asm volatile("bar.sync %0, 128;" ::"r"(1 + cq) : "memory");  // s_red is read
+      asm volatile("bar.sync %0, 128;" ::"r"(1 + cq) : "memory");  // s_rs is written
+#pragma unroll
+      for (int i = 0; i < 16; ++i) x[i] = x[i] * s_rs[16 * cq + i] * (wv * sg[i]);
     }
     // lanes v and v ^ 1 swap halves so that each stores bf16 pairs of adjacent columns
     const bool odd = lane & 1;
@@ -265,12 +274,12 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
   };
 
   // the first chunk's stage; later stages are awaited at the end of the chunk before
+  if (!TRANS && c0 < c1) load_gate(c0);
   if (c0 < c1 && !wait_stage(c0)) s_abort = 1;
   for (int c = c0; c < c1 && !s_abort; ++c) {
     const int s = stage_of(c);
     const uint32_t dcol = (!TRANS && ((c - c0) & 1)) ? TM::kD1 : TM::kD0;  // this chunk's products
     unsigned char* st = sm + s * L::kStageBytes;
-    if (!TRANS && c > c0) load_gate(c - 1);  // in flight until write_o(c - 1) below
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
@@ -347,6 +356,10 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
     mma_pending = true;
     // the query row scales of this chunk, for its o (written during the next C1)
     if (!TRANS && tid < kC) s_iq[tid] = reinterpret_cast<const float*>(st + kSlotIq)[tid];
+    if (!TRANS) {
+      gate_sigmoids();                  // this chunk's epilogue gates, while C2 runs
+      if (c + 1 < c1) load_gate(c + 1);  // and the next chunk's inputs
+    }
     if (!block_wait(&s_bar, phase, p.hdr, p.wait_limit)) { s_abort = 1; break; }
     mma_pending = false;
     // the stage is consumed (its reads ended before the barrier above): refill it
@@ -385,8 +398,7 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
   }
   // o of the last chunk
   if (!TRANS && !s_abort && c1 > c0) {
-    load_gate(c1 - 1);
-    __syncthreads();  // s_iq of the last chunk
+    __syncthreads();  // s_iq of the last chunk (its gate sigmoids are in sg)
     write_o(c1 - 1, ((c1 - 1 - c0) & 1) ? TM::kD1 : TM::kD0);
   }
 

@@ -70,7 +70,8 @@ struct PrepSmem {
   static constexpr int kXK = kTbb + 8192;         // X_K: 64-row f16 image, the A operand X_K^T of M2
   static constexpr int kNrm = kXK + 16384;        // 1/|q| (64), 1/|k| (64)
   static constexpr int kBeta = kNrm + 512;        // beta (64)
-  static constexpr int kEx = kBeta + 256;         // [4][128] alpha at each sub-tile's first token,
+  static constexpr int kGh = kBeta + 256;         // the scalar gate's log-decay of each token (64)
+  static constexpr int kEx = kGh + 256;           // [4][128] alpha at each sub-tile's first token,
                                                   // then [4][128] E at its last token
   // CV: the prologue's taps (x 1/2) of the item's head and of the next item's,
   // [2][q, k, v][128 channels] float4 (right-aligned: the last on the current token)
@@ -161,6 +162,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   float* nrm = reinterpret_cast<float*>(sm + L::kNrm);
   float* bvec = reinterpret_cast<float*>(sm + L::kBeta);
+  float* ghv = reinterpret_cast<float*>(sm + L::kGh);
   float* exf = reinterpret_cast<float*>(sm + L::kEx);
   float* exl = exf + 512;
   uint64_t* bar_qkz = reinterpret_cast<uint64_t*>(sm + L::kBar);  // one per q, k, z buffer
@@ -341,6 +343,11 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     have_nx = seek(nx);
   }
   uint32_t beta_nx = 0u;
+  // the scalar gate of an item's token tid < 64, loaded an item ahead like beta
+  auto load_gh = [&](int tok, int end, int hh) -> float {
+    return (GS == kGateHead && tid < kC && tok + tid < end) ? p.g[(size_t)(tok + tid) * H + hh] : 0.f;
+  };
+  float gh_nx = 0.f;
   // A_h of the next item's head, loaded an item ahead
   float a_nx = (GS == kGateZ && have) ? p.A[cur.h] : 0.f;
   if (have) {
@@ -352,6 +359,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     qkz_pending = (L::kNQ == 2 && have_nx) ? 3u : 1u;
     v_pending = true;
     beta_nx = load_beta(cur.a + cur.c * kC, cur.e, cur.h);
+    gh_nx = load_gh(cur.a + cur.c * kC, cur.e, cur.h);
   }
   int qs = 0;  // the q, k, z buffer of the current item
   int tbuf = 0;  // CV: the taps buffer of the current item
@@ -376,7 +384,11 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     const int qb = qs * L::kQKZ;  // byte offset of this item's q, k, z buffer
     unsigned char* slot = chunk_slot(p.prep, ac, nc, cc0, hc, H);
     if (tid < kC) bvec[tid] = __uint_as_float(beta_nx << 16);
-    if (have_nx) beta_nx = load_beta(tokn, nx.e, hn);
+    if (GS == kGateHead && tid < kC) ghv[tid] = gh_nx;
+    if (have_nx) {
+      beta_nx = load_beta(tokn, nx.e, hn);
+      gh_nx = load_gh(tokn, nx.e, hn);
+    }
 
     // per-channel gate input, issued before the wait
     float al[16];  // alpha of tokens 16 b + i (then 1 / E)
@@ -385,12 +397,6 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
       for (int i = 0; i < 16; ++i) {
         const int t = 16 * b + i;
         al[i] = t < len ? p.g[((size_t)(tok0 + t) * H + hc) * kD + j] : 0.f;
-      }
-    } else if constexpr (GS == kGateHead) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int t = 16 * b + i;
-        al[i] = t < len ? p.g[(size_t)(tok0 + t) * H + hc] : 0.f;
       }
     }
     const float expA_l2 = GS == kGateZ ? expf(a_nx) * kLog2e : 0.f;
@@ -458,6 +464,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
         for (int i = 0; i < 16; ++i) al[i] = 16 * b + i < len ? al[i] : 1.0f;
       }
     } else {
+      if constexpr (GS == kGateHead) lds16(ghv + 16 * b, al);  // zero past the sequence end
 #pragma unroll
       for (int i = 0; i < 16; ++i) al[i] = ex2(al[i] * kLog2e);  // masked tokens: g = 0
     }
