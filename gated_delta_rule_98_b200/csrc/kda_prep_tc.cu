@@ -249,14 +249,18 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
       for (int i = 0; i < 16; ++i) y[i] = 16 * b + i < len ? y[i] : 0.f;
     }
   };
-  // CV: taps of head hh (x 1/2) for thread (j, b < 3): tensor b (q, k, v), channel j
+  // CV: taps of head hh for thread (j, b < 3): tensor b (q, k, v), channel j; the
+  // loads are not waited for until the taps are stored, halved (store_taps)
   float4* tapbuf = reinterpret_cast<float4*>(sm + L::kTaps);
   auto load_taps = [&](int hh) -> float4 {
     const float* wc = (b == 0 ? p.cwq : b == 1 ? p.cwk : p.cwv) + (size_t)(hh * kD + j) * p.cw;
     float w[4];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) w[m] = m >= 4 - p.cw ? 0.5f * wc[m - (4 - p.cw)] : 0.f;
+    for (int m = 0; m < 4; ++m) w[m] = m >= 4 - p.cw ? wc[m - (4 - p.cw)] : 0.f;
     return make_float4(w[0], w[1], w[2], w[3]);
+  };
+  auto store_taps = [&](int buf, float4 w) {
+    tapbuf[buf * 384 + b * 128 + j] = make_float4(0.5f * w.x, 0.5f * w.y, 0.5f * w.z, 0.5f * w.w);
   };
   // CV: squares of y (16 tokens of channel j at rows r0 ..) as hi and lo bf16
   // parts (hi = bf16(y^2), lo = bf16(y^2 - hi)) into the norm operand: hi at
@@ -367,7 +371,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     // the ones block (bf16 1.0) and the first item's taps; published by the
     // first item's first block-wide wait
     if (tid < 128) reinterpret_cast<uint32_t*>(sm + L::kOnes)[tid] = 0x3F803F80u;
-    if (have && b < 3) tapbuf[b * 128 + j] = load_taps(cur.h);
+    if (have && b < 3) store_taps(0, load_taps(cur.h));
   }
   while (have) {
     const int hc = cur.h, nc = cur.n, ac = cur.a, ec = cur.e, cc0 = cur.c;
@@ -769,7 +773,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     __syncthreads();
     // the merged block T[32:64][0:32]
     if (tid < 128) put_t(32 + (tid & 31), (tid >> 5) * 8);
-    if (CV && have_nx && b < 3) tapbuf[(tbuf ^ 1) * 384 + b * 128 + j] = tnext;
+    if (CV && have_nx && b < 3) store_taps(tbuf ^ 1, tnext);
     // the v rows must have landed (a block-wide wait that also orders the T images)
     fence_async_smem();
     fence_before_sync();
