@@ -4,7 +4,7 @@
 // preparation leaves for the chain passes, bf16 operand-image addressing, TMA
 // box loads and bounded block-wide waits.  Internal; not part of the C ABI.
 //
-// Operand images.  Every bf16 MMA operand of the path is an "image" of 16-byte
+// Operand images.  Every MMA operand the kernels build is an "image" of 16-byte
 // units, each unit holding 8 consecutive tokens of one channel (or 8
 // consecutive query rows of one key column).  An image of R token rows and 128
 // channels places (token t, channel c) at
@@ -59,7 +59,8 @@ __host__ __device__ constexpr uint32_t img_tg(int t0, int c) {
 //   WQ   [W ; Q'] as one 128-row token-group-first image (img_tg: W tokens
 //        0..63 in the first 16 KB, Q' tokens 64..127 in the next), the B operand
 //        of C1 (N = 128 tokens, K = dk; the transition pass reads the W half), MN-major.
-//   K    K' (64-row image): the A operand K'^T of C2 (M = dk, K = token), K-major.
+//   K    K' (64-row image): the B operand of the state update in C2 (N = key
+//        channel, K = token), K-major.
 //   A    A_qk with key column i as the "token" and query row r as the channel
 //        (64 x 64): the B operand A_qk^T of the output update (N = r, K = i),
 //        K-major.
