@@ -63,12 +63,14 @@ struct ChainSmem {
   static constexpr int kBytes = kStages * kStageBytes;
 };
 // TMEM columns (512 allocated): fp32 S^T, fp32 X^T (transition), the products D^T
-// (full pass: two buffers of [D_W^T | D_Q^T]; transition: D_S^T | D_X^T), and
-// the f16 copies of S^T (and X^T), whose columns hold U^T while C2 runs.
+// (full pass: [D_Q^T | D_W^T] right after S^T, so that C2 accumulates into
+// [S^T | D_Q^T] with one N = 192 product per K step; transition: D_S^T | D_X^T),
+// and the f16 copies of S^T (and X^T), whose columns hold U^T while C2 runs.
 template <bool TRANS>
 struct ChainTmem {
   static constexpr uint32_t kS = 0, kX = 128;
-  static constexpr uint32_t kD0 = TRANS ? 256 : 128, kD1 = TRANS ? 256 : 256;
+  static constexpr uint32_t kD0 = TRANS ? 256 : 128;  // the products of C1
+  static constexpr uint32_t kDQ = 128, kDW = 192;     // full pass: D_Q^T, D_W^T
   static constexpr uint32_t kCp = 384;  // S^T copy (64 columns), then X^T copy
 };
 
@@ -118,7 +120,7 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
     const unsigned char* src = chunk_slot(p.prep, a, n, c, h, H);
     mbar_arrive_expect_tx(&s_ld[s], L::kStageBytes);
     if (TRANS) {
-      bulk_g2s(dst, src + kSlotWQ, 16384, &s_ld[s]);                     // W
+      bulk_g2s(dst, src + kSlotWQ + 16384, 16384, &s_ld[s]);             // W
       bulk_g2s(dst + L::kK, src + kSlotK, 16384, &s_ld[s]);             // K'
       bulk_g2s(dst + L::kUt, src + kSlotU, 16384 + 512, &s_ld[s]);      // U~^T | gamma
     } else {
@@ -178,8 +180,9 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
     tmem_st_wait();
   }
 
-  // ---- o of a chunk from D_Q^T (columns dcol + 64 ..): lane v holds its column
-  //      for tokens 16 cq .. 16 cq + 15; with the output epilogue the sums of
+  // ---- o of a chunk from D_Q^T: lane v holds its column for tokens 16 cq ..
+  //      16 cq + 15, loaded into x by load_o before the next chunk's C1
+  //      overwrites the product columns; with the output epilogue the sums of
   //      squares over the 128 columns meet in shared memory.
   // Output epilogue: the gate inputs of chunk cc (raw bf16 bits in rgr) are
   // requested a chunk ahead, while the previous chunk's C2 product runs, and
@@ -203,11 +206,12 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
 #pragma unroll
     for (int i = 0; i < 16; ++i) sg[i] = out_sigmoid(__uint_as_float(rgr[i] << 16));
   };
-  auto write_o = [&](int cc, uint32_t dcol) {
-    const int t0c = a + cc * kC, lenc = min(kC, b - t0c);
-    float x[16];
-    tmem_ld16(tm + lq + dcol + 64 + 16 * cq, x);
+  auto load_o = [&](float (&x)[16]) {
+    tmem_ld16(tm + lq + TM::kDQ + 16 * cq, x);
     tmem_ld_wait();
+  };
+  auto write_o = [&](int cc, float (&x)[16]) {
+    const int t0c = a + cc * kC, lenc = min(kC, b - t0c);
 #pragma unroll
     for (int i = 0; i < 16; ++i) x[i] *= s_iq[16 * cq + i];
     if (p.og) {
@@ -278,19 +282,21 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
   if (c0 < c1 && !wait_stage(c0)) s_abort = 1;
   for (int c = c0; c < c1 && !s_abort; ++c) {
     const int s = stage_of(c);
-    const uint32_t dcol = (!TRANS && ((c - c0) & 1)) ? TM::kD1 : TM::kD0;  // this chunk's products
     unsigned char* st = sm + s * L::kStageBytes;
+    // the previous chunk's D_Q^T leaves the product columns before C1 reuses them
+    float xo[16];
+    if (!TRANS && c > c0) load_o(xo);
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
-    // ---- C1: A = the f16 copy of S^T (X^T) in TMEM; B = [W ; Q'] or W, MN-major
+    // ---- C1: A = the f16 copy of S^T (X^T) in TMEM; B = [Q' ; W] or W, MN-major
     if (tid == 0) {
       if (!TRANS) {
         constexpr uint32_t id = instr_desc(kFmtF16, 128, 128, false, true);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint64_t bd = smem_desc(smem_u32(st + kSlotWQ + k * 256), 128, 2048);
-          mma_f16_ts(tm + dcol, tm + TM::kCp + 8 * k, bd, id, k > 0);
+          mma_f16_ts(tm + TM::kD0, tm + TM::kCp + 8 * k, bd, id, k > 0);
         }
       } else {
         constexpr uint32_t id = instr_desc(kFmtF16, 128, 64, false, true);
@@ -307,14 +313,14 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
     // ---- meanwhile: the first chunk decays the incoming state by its gamma (later
     //      chunks get it with the previous chunk's copy); the previous o goes out
     if (c == c0) decay_state(reinterpret_cast<const float*>(st + L::kGam));
-    if (!TRANS && c > c0) write_o(c - 1, dcol == TM::kD0 ? TM::kD1 : TM::kD0);
+    if (!TRANS && c > c0) write_o(c - 1, xo);
     if (!block_wait(&s_bar, phase, p.hdr, p.wait_limit)) { s_abort = 1; break; }
     mma_pending = false;
     // ---- U^T = U~^T - D_W^T (transition: U_S^T = U~^T - D_S^T, U_X^T = -D_X^T),
     //      f16 into the copy's columns (C1 has read them)
     {
       float d[16];
-      tmem_ld16(tm + lq + dcol + 16 * cq, d);
+      tmem_ld16(tm + lq + (TRANS ? TM::kD0 : TM::kDW) + 16 * cq, d);
       float dx[16];
       if (TRANS) tmem_ld16(tm + lq + TM::kD0 + 64 + 16 * cq, dx);
       const uint4* ug = reinterpret_cast<const uint4*>(st + L::kUt);
@@ -337,19 +343,15 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
     __syncthreads();
     fence_after_sync();
     // ---- C2: S^T (X^T) += U^T K' (B = K' K-major: N = key channel, K = token);
-    //      D_Q^T += U^T A_qk^T (B K-major: N = query row, K = key row)
+    //      full pass: with D_Q^T += U^T A_qk^T in the same product, B = [K' | A_qk^T]
+    //      (N = 128 key channels, then 64 query rows; K = key row)
     if (tid == 0) {
-      constexpr uint32_t ids = instr_desc(kFmtF16, 128, 128, false, false);
-      constexpr uint32_t ido = instr_desc(kFmtF16, 128, 64, false, false);
+      constexpr uint32_t id = instr_desc(kFmtF16, 128, TRANS ? 128 : 192, false, false);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const uint64_t kd = smem_desc(smem_u32(st + L::kK + k * 256), 128, 1024);
-        mma_f16_ts(tm + TM::kS, tm + TM::kCp + 8 * k, kd, ids, 1);
-        if (TRANS) mma_f16_ts(tm + TM::kX, tm + TM::kCp + 64 + 8 * k, kd, ids, 1);
-        if (!TRANS) {
-          const uint64_t ad = smem_desc(smem_u32(st + kSlotA + k * 256), 128, 1024);
-          mma_f16_ts(tm + dcol + 64, tm + TM::kCp + 8 * k, ad, ido, 1);
-        }
+        mma_f16_ts(tm + TM::kS, tm + TM::kCp + 8 * k, kd, id, 1);
+        if (TRANS) mma_f16_ts(tm + TM::kX, tm + TM::kCp + 64 + 8 * k, kd, id, 1);
       }
       mma_commit(&s_bar);
     }
@@ -399,7 +401,9 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
   // o of the last chunk
   if (!TRANS && !s_abort && c1 > c0) {
     __syncthreads();  // s_iq of the last chunk (its gate sigmoids are in sg)
-    write_o(c1 - 1, ((c1 - 1 - c0) & 1) ? TM::kD1 : TM::kD0);
+    float xo[16];
+    load_o(xo);
+    write_o(c1 - 1, xo);
   }
 
   fence_before_sync();

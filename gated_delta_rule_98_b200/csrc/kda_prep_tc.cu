@@ -595,7 +595,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
       scale16(x, bke, Pb);
       put16h(sm + L::kXK, img_unit(16 * b, j, 64), img_unit(16 * b + 8, j, 64), x);
       scale16(x, qe, Pb);
-      put16h(slot + kSlotWQ, img_tg(64 + 16 * b, j), img_tg(72 + 16 * b, j), x);
+      put16h(slot + kSlotWQ, img_tg(16 * b, j), img_tg(16 * b + 8, j), x);
       scale16(x, cd, Lb);
       put16h(slot + kSlotK, img_unit(16 * b, j, 64), img_unit(16 * b + 8, j, 64), x);
     }
@@ -823,7 +823,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
       tmem_ld16(tmem_addr(tm, 32 * q4, 16 * cq), w16);
       tmem_ld16(tmem_addr(tm, 32 * q4, 64 + 16 * cq), u16);
       tmem_ld_wait();
-      put16h(slot + kSlotWQ, img_tg(16 * cq, ch), img_tg(16 * cq + 8, ch), w16);
+      put16h(slot + kSlotWQ, img_tg(64 + 16 * cq, ch), img_tg(72 + 16 * cq, ch), w16);
       uint4* ug = reinterpret_cast<uint4*>(slot + kSlotU);
       ug[ut_index(q4, cq, 0, lane)] = pack8h(u16);
       ug[ut_index(q4, cq, 1, lane)] = pack8h(u16 + 8);

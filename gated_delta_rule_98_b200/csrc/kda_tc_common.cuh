@@ -56,11 +56,12 @@ __host__ __device__ constexpr uint32_t img_tg(int t0, int c) {
 // and the state is non-expansive), so f16 holds them with 8x less rounding
 // than bf16; values below the f16 range flush towards zero (absolute error
 // under 1e-7) and out-of-range ones would saturate.
-//   WQ   [W ; Q'] as one 128-row token-group-first image (img_tg: W tokens
-//        0..63 in the first 16 KB, Q' tokens 64..127 in the next), the B operand
+//   WQ   [Q' ; W] as one 128-row token-group-first image (img_tg: Q' tokens
+//        0..63 in the first 16 KB, W tokens 64..127 in the next), the B operand
 //        of C1 (N = 128 tokens, K = dk; the transition pass reads the W half), MN-major.
 //   K    K' (64-row image): the B operand of the state update in C2 (N = key
-//        channel, K = token), K-major.
+//        channel, K = token), K-major; directly followed by A, so that
+//        [K' | A_qk^T] is one B operand with N = 192.
 //   A    A_qk with key column i as the "token" and query row r as the channel
 //        (64 x 64): the B operand A_qk^T of the output update (N = r, K = i),
 //        K-major.
@@ -69,6 +70,7 @@ __host__ __device__ constexpr uint32_t img_tg(int t0, int c) {
 constexpr int kSlotWQ = 0, kSlotK = 32768, kSlotA = 49152, kSlotU = 57344, kSlotGam = 73728,
               kSlotIq = 74240, kSlotBytes = 74496;
 static_assert(kSlotU + 16384 == kSlotGam && kSlotGam + 512 == kSlotIq, "slot layout");
+static_assert(kSlotK + 16384 == kSlotA, "[K' | A_qk^T] is one operand");
 
 // 16-byte unit of U~^T (value column 32 q4 + l; tokens 16 cq + 8 half .. +7) in
 // a slot: warp (q4, cq) reads 512 consecutive bytes per vector.
