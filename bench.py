@@ -393,7 +393,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--steps", type=int, default=360)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--mode", choices=["weak", "cp"], default="weak",

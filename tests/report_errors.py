@@ -53,6 +53,18 @@ def epilogue():
         o_r, S_r = oracle_forward(inp)
         y_r = ep.norm_gate(o_r, f64(r), f64(w), eps=1e-6)
         line(f"kda_forward_norm_gate y T={T} H={H} N={ns}", y, y_r, S, S_r)
+        # per-row relative error of y (one row = one token and head, dv values),
+        # against the row's o norm relative to the median o row norm
+        yg = f64(y)
+        row_err = np.linalg.norm(yg - y_r, axis=-1) / np.maximum(np.linalg.norm(y_r, axis=-1), 1e-30)
+        o_norm = np.linalg.norm(o_r, axis=-1)
+        rel_norm = o_norm / np.median(o_norm)
+        shares = ", ".join(f">{t:g}: {100 * np.mean(row_err > t):.2f}%" for t in (1e-3, 5e-3, 1e-2, 5e-2, 1e-1))
+        low = row_err[rel_norm < 0.1]
+        print(f"    y row errors: median {np.median(row_err):.2e}, p99 {np.quantile(row_err, 0.99):.2e}, "
+              f"max {row_err.max():.2e}; rows {shares}; rows with |o| < 0.1 x median: "
+              f"{100 * np.mean(rel_norm < 0.1):.2f}% of rows, their median error "
+              f"{(np.median(low) if low.size else 0):.2e}", flush=True)
 
 
 def prologue():
