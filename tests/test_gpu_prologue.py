@@ -77,7 +77,15 @@ def test_forward_conv_varlen():
     _forward_conv(sum(lens), 4, 128, 4, "bf16", 64, lens=lens, seed=83)
 
 
-@pytest.mark.parametrize("dtype,chunk,d,width", [("f32", 16, 64, 4), ("f32", 64, 32, 2)])
+@pytest.mark.parametrize("width", [1, 2, 3])
+def test_forward_conv_tensor_core_path_short_filters(width):
+    # the fused prologue right-aligns taps shorter than 4 (the last on the current token)
+    lens = [130, 5, 70]
+    _forward_conv(sum(lens), 2, 128, width, "bf16", 64, lens=lens, seed=90 + width)
+
+
+@pytest.mark.parametrize("dtype,chunk,d,width", [("f32", 16, 64, 4), ("f32", 64, 32, 2),
+                                                 ("bf16", 64, 64, 3)])
 def test_forward_conv_cuda_core_path(dtype, chunk, d, width):
     lens = [70, 33, 130]
     _forward_conv(sum(lens), 2, d, width, dtype, chunk, lens=lens, seed=84)
