@@ -40,9 +40,10 @@ __device__ __forceinline__ float* ckpt_state(const TcParams& p, int n, int h, in
 // that both A operands of the chain, an f16 copy of S^T and U^T, are read by
 // the MMAs from Tensor Memory and only the slot's images come from shared
 // memory.  Per chunk:
-//   C1: [D_W^T | D_Q^T] = S^T [W ; Q']^T   (M=128 value columns, N=128 tokens);
+//   C1: [D_Q^T | D_W^T] = S^T [Q' ; W]^T   (M=128 value columns, N=128 tokens);
 //   U^T = U~^T - D_W^T  (f16, in Tensor Memory);
-//   C2: S^T += U^T K'  (M=128, N=128 key channels);  D_Q^T += U^T A_qk^T  (N=64);
+//   C2: S^T += U^T K'  (M=128, N=128 key channels) and D_Q^T += U^T A_qk^T
+//       (N=64), one N=192 product in the full pass;
 //   the new S^T is copied to f16 for the next C1 and, in place, scaled by the
 //   next chunk's gamma (per key channel) before that chunk's C2 accumulates
 //   into it; o = (D_Q^T)^T / |q| of a chunk is written during the next C1.
@@ -55,7 +56,7 @@ template <bool TRANS>
 struct ChainSmem {
   static constexpr int kStages = TRANS ? 4 : 3;
   // stage layout: the slot (full pass), or W | K' | U~^T | gamma (transition: the
-  // W half of the [W ; Q'] image; no Q', A_qk or 1/|q|; one bulk copy per part)
+  // W half of the [Q' ; W] image; no Q', A_qk or 1/|q|; one bulk copy per part)
   static constexpr int kK = TRANS ? 16384 : kSlotK;
   static constexpr int kUt = TRANS ? 32768 : kSlotU;
   static constexpr int kGam = TRANS ? 32768 + 16384 : kSlotGam;

@@ -26,9 +26,10 @@
 // 512 threads; the 16 tokens of a sub-tile are a serial product in registers
 // and every operand image unit (8 consecutive tokens of one channel) is one
 // 16-byte store.  Persistent: one CTA per SM walks (chunk, sequence, head)
-// items; the next item's q, k, z rows are requested as soon as this item has
-// read them and its v rows as soon as the WY product that reads v in place
-// has completed.
+// items.  q, k, z rows are double-buffered: an item's rows are requested two
+// items ahead, as soon as the buffer's previous item has read them (one item
+// ahead, single-buffered, with the input prologue); v rows are requested as
+// soon as the WY product that reads them has completed.
 #include "kda_tc_common.cuh"
 
 namespace kda {
@@ -816,7 +817,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
       if (have_nx && tid == 0) stage_v(tokn, hn);
       v_pending = have_nx;
     }
-    // ---- F: W (into the [W ; Q'] image) and U~^T -> slot
+    // ---- F: W (the second half of the [Q' ; W] image) and U~^T -> slot
     {
       const int ch = 32 * q4 + lane;
       float w16[16], u16[16];
