@@ -1,6 +1,7 @@
 // kda_api.cu -- the C ABI of include/kda.h: argument validation, workspace
 // sizing and kernel selection.  Every host-visible fault returns before any
 // work is enqueued.
+#include <nvtx3/nvToolsExt.h>
 #include <cuda_runtime.h>
 
 #include "../../include/kda.h"
@@ -117,6 +118,14 @@ kda_status forward_common(kda::ForwardArgs& a) {
 
 }  // namespace
 
+// NVTX range around each enqueueing entry point: marks the host call that
+// validates the arguments and enqueues the launches (a no-op unless a
+// profiler is attached; NVTX v3 is header-only).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+
 extern "C" {
 
 const char* kda_status_string(kda_status s) {
@@ -161,6 +170,7 @@ kda_status kda_forward(const void* q, const void* k, const void* v,
                        kda_dtype dt, int32_t chunk, void* o, float* S_final,
                        void* workspace, size_t workspace_bytes,
                        kda_stream_t stream) {
+  const NvtxRange nvtx_range_("kda_forward");
   kda_status st = check_forward(q, k, v, z, beta, S0, cu_seqlens, num_seqs,
                                 total_tokens, max_seqlen, H, dk, dv, dt, chunk,
                                 o, S_final, workspace, workspace_bytes);
@@ -180,6 +190,7 @@ kda_status kda_forward_g(const void* q, const void* k, const void* v,
                          int32_t dk, int32_t dv, kda_dtype dt, int32_t chunk,
                          void* o, float* S_final, void* workspace,
                          size_t workspace_bytes, kda_stream_t stream) {
+  const NvtxRange nvtx_range_("kda_forward_g");
   kda_status st = check_forward(q, k, v, g, beta, S0, cu_seqlens, num_seqs,
                                 total_tokens, max_seqlen, H, dk, dv, dt, chunk,
                                 o, S_final, workspace, workspace_bytes);
@@ -198,6 +209,7 @@ kda_status kda_forward_scalar_gate(const void* q, const void* k, const void* v,
                                    int32_t dk, int32_t dv, kda_dtype dt, int32_t chunk,
                                    void* o, float* S_final, void* workspace,
                                    size_t workspace_bytes, kda_stream_t stream) {
+  const NvtxRange nvtx_range_("kda_forward_scalar_gate");
   kda_status st = check_forward(q, k, v, g_head, beta, S0, cu_seqlens, num_seqs,
                                 total_tokens, max_seqlen, H, dk, dv, dt, chunk,
                                 o, S_final, workspace, workspace_bytes);
@@ -219,6 +231,7 @@ kda_status kda_forward_checkpoints(const void* q, const void* k, const void* v,
                                    float* S_final, float* S_ckpt, int32_t interval,
                                    void* workspace, size_t workspace_bytes,
                                    kda_stream_t stream) {
+  const NvtxRange nvtx_range_("kda_forward_checkpoints");
   kda_status st = check_forward(q, k, v, z, beta, S0, cu_seqlens, num_seqs,
                                 total_tokens, max_seqlen, H, dk, dv, dt, chunk,
                                 o, S_final, workspace, workspace_bytes);
@@ -248,6 +261,7 @@ kda_status kda_forward_norm_gate(const void* q, const void* k, const void* v,
                                  const float* norm_weight, float eps, void* o,
                                  float* S_final, void* workspace, size_t workspace_bytes,
                                  kda_stream_t stream) {
+  const NvtxRange nvtx_range_("kda_forward_norm_gate");
   kda_status st = check_forward(q, k, v, z, beta, S0, cu_seqlens, num_seqs,
                                 total_tokens, max_seqlen, H, dk, dv, dt, chunk,
                                 o, S_final, workspace, workspace_bytes);
@@ -269,6 +283,7 @@ kda_status kda_decode_step(const void* q, const void* k, const void* v,
                            float* S_inout, int32_t B, int32_t H, int32_t dk,
                            int32_t dv, kda_dtype dt, void* o,
                            kda_stream_t stream) {
+  const NvtxRange nvtx_range_("kda_decode_step");
   return decode_common(q, k, v, z, A, beta, S_inout, B, H, dk, dv, dt, nullptr, nullptr, 0.f, o,
                        stream);
 }
@@ -279,6 +294,7 @@ kda_status kda_decode_step_norm_gate(const void* q, const void* k, const void* v
                                      int32_t dv, kda_dtype dt, const void* out_gate,
                                      const float* norm_weight, float eps, void* o,
                                      kda_stream_t stream) {
+  const NvtxRange nvtx_range_("kda_decode_step_norm_gate");
   if (!epilogue_ok(B > 0, out_gate, norm_weight, eps)) return KDA_ERR_INVALID_ARG;
   return decode_common(q, k, v, z, A, beta, S_inout, B, H, dk, dv, dt, out_gate, norm_weight,
                        eps, o, stream);
@@ -290,6 +306,7 @@ kda_status kda_decode_step_conv(const void* x_q, const void* x_k, const void* x_
                                 const float* A, const void* beta, float* S_inout, int32_t B,
                                 int32_t H, int32_t dk, int32_t dv, kda_dtype dt, void* o,
                                 kda_stream_t stream) {
+  const NvtxRange nvtx_range_("kda_decode_step_conv");
   if (conv_width < 1 || conv_width > 4) return KDA_ERR_UNSUPPORTED;
   if (B > 0 && (!w_q || !w_k || !w_v || ((uintptr_t)w_q & 3u) || ((uintptr_t)w_k & 3u) ||
                 ((uintptr_t)w_v & 3u)))
@@ -311,6 +328,7 @@ kda_status kda_short_conv_swish(const void* x, const float* w, const int32_t* cu
                                 int32_t num_seqs, int32_t total_tokens, int32_t max_seqlen,
                                 int32_t channels, int32_t width, kda_dtype dt, void* y,
                                 kda_stream_t stream) {
+  const NvtxRange nvtx_range_("kda_short_conv_swish");
   if (dt != KDA_F32 && dt != KDA_BF16) return KDA_ERR_UNSUPPORTED;
   if (width < 1 || width > 4) return KDA_ERR_UNSUPPORTED;
   if (channels < 8 || channels % 8 != 0) return KDA_ERR_UNSUPPORTED;
@@ -350,6 +368,7 @@ kda_status kda_forward_conv(const void* x_q, const void* x_k, const void* x_v,
                             int32_t total_tokens, int32_t max_seqlen, int32_t H, int32_t dk,
                             int32_t dv, kda_dtype dt, int32_t chunk, void* o, float* S_final,
                             void* workspace, size_t workspace_bytes, kda_stream_t stream) {
+  const NvtxRange nvtx_range_("kda_forward_conv");
   const size_t fw = kda_forward_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk, dv,
                                                dt, chunk);
   const size_t need = kda_forward_conv_workspace_size(num_seqs, total_tokens, max_seqlen, H, dk,
@@ -411,6 +430,7 @@ kda_status kda_cp_local(const void* q, const void* k, const void* v, const void*
                         int32_t dk, int32_t dv, kda_dtype dt, int32_t chunk, float* M_out,
                         float* N_out, void* workspace, size_t workspace_bytes,
                         kda_stream_t stream) {
+  const NvtxRange nvtx_range_("kda_cp_local");
   if (!use_tc(dt, dk, dv, chunk)) return KDA_ERR_UNSUPPORTED;
   // the forward's geometry and input checks, with M_out standing in for o (its
   // workspace size is at most the one this call needs, checked next)
@@ -437,6 +457,7 @@ kda_status kda_cp_finish(const float* S_in, const int32_t* cu_seqlens, int32_t n
                          int32_t total_tokens, int32_t max_seqlen, int32_t H, int32_t dk,
                          int32_t dv, kda_dtype dt, int32_t chunk, void* o, float* S_final,
                          void* workspace, size_t workspace_bytes, kda_stream_t stream) {
+  const NvtxRange nvtx_range_("kda_cp_finish");
   if (!use_tc(dt, dk, dv, chunk)) return KDA_ERR_UNSUPPORTED;
   if (num_seqs < 0 || total_tokens < 0 || max_seqlen < 0 || H < 1) return KDA_ERR_INVALID_ARG;
   if (!cu_seqlens && (int64_t)num_seqs * max_seqlen != total_tokens) return KDA_ERR_INVALID_ARG;
@@ -456,6 +477,7 @@ kda_status kda_cp_finish(const float* S_in, const int32_t* cu_seqlens, int32_t n
 
 kda_status kda_state_compose(const float* M, const float* N, const float* S_in, float* S_out,
                              int32_t count, int32_t dk, int32_t dv, kda_stream_t stream) {
+  const NvtxRange nvtx_range_("kda_state_compose");
   if (!dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
   if (count < 0) return KDA_ERR_INVALID_ARG;
   if (count == 0) return KDA_OK;
