@@ -92,8 +92,9 @@ size_t kda_forward_workspace_size(int32_t num_seqs, int32_t total_tokens,
  * Number of kernel launches one kda_forward / kda_forward_g call with these
  * arguments enqueues (0 when the arguments are invalid or unsupported).  The
  * same count holds for kda_forward_scalar_gate, kda_forward_checkpoints and,
- * on the tensor-core path, kda_forward_norm_gate; kda_forward_norm_gate on
- * the CUDA-core path and kda_forward_conv enqueue one launch more.
+ * on the tensor-core path, kda_forward_norm_gate and kda_forward_conv; on the
+ * CUDA-core path kda_forward_norm_gate and kda_forward_conv enqueue one
+ * launch more.
  */
 int32_t kda_forward_launches(int32_t num_seqs, int32_t total_tokens,
                              int32_t max_seqlen, int32_t H, int32_t dk,
@@ -216,11 +217,11 @@ kda_status kda_forward_checkpoints(const void* q, const void* k, const void* v,
  *                NULL for ones.  The pages name no gain; this one is optional.
  *  eps         : added to the mean square, finite and >= 0 (else
  *                KDA_ERR_INVALID_ARG); the pages give no value.
- * On the tensor-core path the epilogue runs in the kernels that write o, from
- * the fp32 (fused unsegmented kernel) or bf16-staged (segmented full pass)
- * attention output; on the CUDA-core path it is one extra launch after the
- * state pass (kda_forward_launches + 1), since that pass splits a head's dv
- * features over several blocks.  Everything else is kda_forward's.
+ * On the tensor-core path the epilogue runs in the full chain pass, which
+ * writes o, from the fp32 attention output in Tensor Memory; on the
+ * CUDA-core path it is one extra launch after the state pass
+ * (kda_forward_launches + 1), since that pass splits a head's dv features
+ * over several blocks.  Everything else is kda_forward's.
  */
 kda_status kda_forward_norm_gate(const void* q, const void* k, const void* v,
                                  const void* z, const float* A, const void* beta,
