@@ -250,6 +250,30 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
       for (int i = 0; i < 16; ++i) y[i] = 16 * b + i < len ? y[i] : 0.f;
     }
   };
+  // CV: Swish(conv(v)) of channel j, tokens t0 .. t0 + N - 1 (t0 a multiple of 8)
+  // into the bf16 image V^T of M2, from the staged rows (history and tail as in
+  // conv16); run by the warps that the diagonal solve leaves idle, in three token
+  // groups of 24, 24 and 16
+  auto conv_v = [&](auto n_tokens, int t0, const float4 hw, bool first, int len) {
+    constexpr int N = decltype(n_tokens)::value;
+    float x[N + 3];
+#pragma unroll
+    for (int i = 0; i < N + 3; ++i) {
+      const int r = t0 + 5 + i;
+      const uint32_t off = jboxc + (uint32_t)r * 128u + ((junit ^ (uint32_t)(r & 7)) << 4);
+      x[i] = __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t*>(sm + L::kV + off) << 16);
+    }
+    if (first && t0 == 0) x[0] = x[1] = x[2] = 0.f;
+    float y[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      const float h = fmaf(hw.w, x[i + 3], fmaf(hw.z, x[i + 2], fmaf(hw.y, x[i + 1], hw.x * x[i])));
+      y[i] = t0 + i < len ? fmaf(h, tanh_approx(h), h) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < N / 8; ++u)
+      *reinterpret_cast<uint4*>(sm + L::kVc + img_unit(t0 + 8 * u, j, 64)) = pack8(y + 8 * u);
+  };
   // CV: taps of head hh for thread (j, b < 3): tensor b (q, k, v), channel j; the
   // loads are not waited for until the taps are stored, halved (store_taps)
   float4* tapbuf = reinterpret_cast<float4*>(sm + L::kTaps);
@@ -635,6 +659,7 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     // CV: the next item's taps, loaded during the inverse and stored after it
     float4 tnext = make_float4(0.f, 0.f, 0.f, 0.f);
     if (CV && have_nx && b < 3) tnext = load_taps(hn);
+    bool v_got = true;  // CV: this thread's wait for the v rows succeeded
 
     // ---- E: T = (I + A_kk)^{-1} in fp32.  Diagonal 16x16 blocks by forward
     //      substitution (one warp per block, lane = column), then the blocks below
@@ -669,7 +694,20 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
         Tf[r * kLd + col] = 0.f;
         TT[col * kLd + r] = 0.f;
       }
+      if constexpr (CV) {
+        // meanwhile the input prologue on v (its rows were requested an item ago)
+        v_got = mbar_wait_cycles(bar_v, ph_v, p.wait_limit);
+        if (v_got) {
+          const float4 hw = tapbuf[tbuf * 384 + 256 + j];
+          const int g = b - 1;  // token group: 0..23, 24..47, 48..63
+          if (g < 2) conv_v(std::integral_constant<int, 24>{}, 24 * g, hw, cc0 == 0, len);
+          else conv_v(std::integral_constant<int, 16>{}, 48, hw, cc0 == 0, len);
+          fence_async_smem();
+        }
+      }
     }
+    // (every thread reaches the barrier; a v wait that gave up is reported by the
+    // block-wide wait on the same rows below)
     __syncthreads();
     // 16 -> 32 for the pairs (0, 1) and (2, 3): Y = A[hi][lo] T[lo][lo]
     {
@@ -781,14 +819,16 @@ __global__ void __launch_bounds__(kNT, 1) prep_kernel(const __grid_constant__ Tc
     if (!block_wait(bar_v, ph_v, p.hdr, p.wait_limit)) { ok = false; break; }
     v_pending = false;
     if constexpr (CV) {
-      // input prologue on v -> the bf16 image V^T of M2; the raw rows are then
-      // consumed and the next item's are requested at once
-      float y[16];
-      conv16(L::kV, tapbuf[tbuf * 384 + 256 + j], cc0 == 0, len, y);
-      put16(sm + L::kVc, img_unit(16 * b, j, 64), img_unit(16 * b + 8, j, 64), y);
-      sync_for_mma();
-      if (have_nx && tid == 0) stage_v(tokn, hn);
-      v_pending = have_nx;
+      // the v image was made during the diagonal solve (and published by the
+      // barriers since): the raw rows are consumed, request the next item's
+      if (!__syncthreads_or(!v_got)) {
+        if (have_nx && tid == 0) stage_v(tokn, hn);
+        v_pending = have_nx;
+      } else {
+        if (tid == 0) atomicOr(&p.hdr->err, kErrTimeout);
+        ok = false;
+        break;
+      }
     }
     // ---- M2: W^T = X_K^T T^T -> TMEM columns 0-63 and U~^T = V^T (T Diag(beta))^T
     //      -> 64-127 (M = 128 channels, N = 64 tokens; V read in place from its
