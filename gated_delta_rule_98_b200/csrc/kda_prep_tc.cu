@@ -30,6 +30,8 @@
 // items ahead, as soon as the buffer's previous item has read them (one item
 // ahead, single-buffered, with the input prologue); v rows are requested as
 // soon as the WY product that reads them has completed.
+#include <type_traits>
+
 #include "kda_tc_common.cuh"
 
 namespace kda {
