@@ -193,9 +193,6 @@ __device__ __forceinline__ void ld8f(const float* p, float* f) {  // 8 fp32, 16-
   const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
   f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
-__device__ __forceinline__ void st16(unsigned char* base, uint32_t off, const float* v) {
-  *reinterpret_cast<uint4*>(base + off) = pack8(v);
-}
 
 // Block-wide bounded wait on an mbarrier phase (at most `limit` SM cycles); false
 // if it timed out (the error word then carries kErrTimeout and `phase` still
