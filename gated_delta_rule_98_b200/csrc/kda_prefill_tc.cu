@@ -443,8 +443,13 @@ __global__ void __launch_bounds__(kNT, 1) chain_kernel(const __grid_constant__ T
 
 // Incoming state of every segment: S_in(0) = S0, S_in(p+1) = M_p S_in(p) + N_p.
 // One CTA per (n, h, 16-column block of the state); fp32 on CUDA cores.  Each
-// M_p (64 KB) is bulk-copied into shared memory one step ahead; the state
-// columns are kept transposed so both operands are read as float4.
+// M_p (64 KB) is bulk-copied into shared memory one step ahead.  The product
+// splits the contraction over lanes: warp (column group cg, row half rh) owns
+// columns 4 cg .. 4 cg + 3 and rows 64 rh .. 64 rh + 63; lane (row set rs, key
+// part kp) keeps the state at keys 4 kp + 32 j + e (j, e < 4) of its four
+// columns in registers, reads those keys of its 16 rows of M_p as float4 (one
+// 128-byte row segment per 8 lanes), and the 8 partial sums of each output
+// meet by shuffles.  The state columns are kept transposed in shared memory.
 constexpr int kComposeThreads = 256;
 constexpr int kSct = kD + 4;  // row stride (floats) of the transposed state columns
 struct ComposeSmem {
@@ -464,7 +469,7 @@ __global__ void __launch_bounds__(kComposeThreads) compose_kernel(const __grid_c
   using L = ComposeSmem;
   extern __shared__ __align__(1024) unsigned char sm[];
   const int n = blockIdx.x, h = blockIdx.y, cb = blockIdx.z * 16;
-  const int H = p.H, tid = threadIdx.x;
+  const int H = p.H, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (!seqlens_valid(p.cu, p.N, p.T, p.max_len)) return;
   float* Sct = reinterpret_cast<float*>(sm + L::kS);  // Sct[cc][r] = S[r][cb + cc]
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L::kBar);
@@ -489,18 +494,17 @@ __global__ void __launch_bounds__(kComposeThreads) compose_kernel(const __grid_c
     else
       Sct[cc * kSct + r] = p.S0 ? p.S0[((size_t)n * H + h) * kD * kD + (size_t)r * kD + cb + cc] : 0.f;
   }
-  const int c = tid & 15, r0 = tid >> 4;  // column c, rows r0 + 16 m
+  // this lane's part of the product
+  const int cg = warp & 3, rh = warp >> 2, kp = lane & 7, rs = lane >> 3;
+  const int b2 = (lane >> 2) & 1, b1 = (lane >> 1) & 1;
+  const int ci = 2 * b2 + b1;            // the column (of cg's four) this lane ends with
+  const int col = 4 * cg + ci;           // ... of the CTA's 16
+  const int rbase = 64 * rh + 16 * rs;   // its rows: rbase .. rbase + 15
+  const bool writer = (lane & 1) == 0;   // lanes 2m and 2m + 1 end with the same sum
   uint32_t inflight = steps > 0 ? 1u : 0u;  // buffers being filled
   uint32_t ph = 0;                            // bit b: parity of buffer b's next completion
   bool ok = true;
-  // N_p columns, loaded one step ahead
-  auto load_n = [&](int sg, float (&v)[8]) {
-    const float* Nt = seg_trans(p.seg, n, h, H, p.Pseg, sg) + kD * kD;
-#pragma unroll
-    for (int m = 0; m < 8; ++m) v[m] = addn ? Nt[(size_t)(r0 + 16 * m) * kD + cb + c] : 0.f;
-  };
-  float nxt[8];
-  if (steps > 0) load_n(0, nxt);
+  __syncthreads();
   for (int sg = 0; sg < steps; ++sg) {
     const int buf = sg & 1;
     // M_{sg+1} into the other buffer (its readers finished before the last barrier)
@@ -508,10 +512,25 @@ __global__ void __launch_bounds__(kComposeThreads) compose_kernel(const __grid_c
       if (tid == 0) load_m(sg + 1);
       inflight |= 1u << (buf ^ 1);
     }
-    float acc[8];
+    // N_p of this lane's outputs: issued now, added after the product
+    float nv[16];
+    {
+      const float* Nt = seg_trans(p.seg, n, h, H, p.Pseg, sg) + kD * kD;
 #pragma unroll
-    for (int m = 0; m < 8; ++m) acc[m] = nxt[m];
-    if (sg + 1 < steps) load_n(sg + 1, nxt);
+      for (int i = 0; i < 16; ++i) nv[i] = addn ? Nt[(size_t)(rbase + i) * kD + cb + col] : 0.f;
+    }
+    // the state at this lane's keys and columns
+    float sv[4][16];
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 x = *reinterpret_cast<const float4*>(Sct + (4 * cg + c4) * kSct + 4 * kp + 32 * j);
+        sv[c4][4 * j] = x.x;
+        sv[c4][4 * j + 1] = x.y;
+        sv[c4][4 * j + 2] = x.z;
+        sv[c4][4 * j + 3] = x.w;
+      }
     const bool got = mbar_wait_cycles(&bar[buf], (ph >> buf) & 1, p.wait_limit);
     if (__syncthreads_or(!got)) {
       if (tid == 0) atomicOr(&p.hdr->err, kErrTimeout);
@@ -521,18 +540,35 @@ __global__ void __launch_bounds__(kComposeThreads) compose_kernel(const __grid_c
     ph ^= 1u << buf;
     inflight &= ~(1u << buf);
     const float* Ms = reinterpret_cast<const float*>(sm + L::kM + buf * kD * kD * 4);
-#pragma unroll 4
-    for (int k = 0; k < kD; k += 4) {
-      const float4 sv = *reinterpret_cast<const float4*>(Sct + c * kSct + k);
+    float acc[16];
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const float4 mv = *reinterpret_cast<const float4*>(Ms + (r0 + 16 * m) * kD + k);
-        acc[m] += mv.x * sv.x + mv.y * sv.y + mv.z * sv.z + mv.w * sv.w;
+    for (int i = 0; i < 16; ++i) {
+      const float* mr = Ms + (rbase + i) * kD + 4 * kp;
+      float pc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 m4 = *reinterpret_cast<const float4*>(mr + 32 * j);
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4)
+          pc[c4] = fmaf(m4.x, sv[c4][4 * j],
+                        fmaf(m4.y, sv[c4][4 * j + 1],
+                             fmaf(m4.z, sv[c4][4 * j + 2], fmaf(m4.w, sv[c4][4 * j + 3], pc[c4]))));
       }
+      // the sums over the 8 key parts (lane bits 0..2): bit 2 splits the columns
+      // into pairs, bit 1 into single columns, bit 0 completes the sum
+      const float k0 = b2 ? pc[2] : pc[0], s0 = b2 ? pc[0] : pc[2];
+      const float k1 = b2 ? pc[3] : pc[1], s1 = b2 ? pc[1] : pc[3];
+      const float q0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 4);
+      const float q1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 4);
+      float r1 = (b1 ? q1 : q0) + __shfl_xor_sync(0xffffffffu, b1 ? q0 : q1, 2);
+      r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
+      acc[i] = r1;
     }
-    __syncthreads();
+    __syncthreads();  // every lane has read the state columns and this M_p
+    if (writer) {
 #pragma unroll
-    for (int m = 0; m < 8; ++m) Sct[c * kSct + r0 + 16 * m] = acc[m];
+      for (int i = 0; i < 16; ++i) Sct[col * kSct + rbase + i] = acc[i] + nv[i];
+    }
     __syncthreads();
     if (!FOLD) {
       float* Sin = seg_sin(p.seg, n, h, H, p.Pseg, sg + 1);
@@ -551,8 +587,8 @@ __global__ void __launch_bounds__(kComposeThreads) compose_kernel(const __grid_c
   }
   if (!ok && tid == 0) {
     // a wait gave up: let the copies still in flight land before leaving
-    for (int b2 = 0; b2 < 2; ++b2)
-      if (inflight & (1u << b2)) (void)mbar_wait_cycles(&bar[b2], (ph >> b2) & 1, kWaitCycles);
+    for (int b2w = 0; b2w < 2; ++b2w)
+      if (inflight & (1u << b2w)) (void)mbar_wait_cycles(&bar[b2w], (ph >> b2w) & 1, kWaitCycles);
   }
 }
 
