@@ -1,0 +1,154 @@
+"""Error budget of the tensor-core prefill on the CPU: where o's error against
+the float64 oracle comes from.
+
+The chunkwise algebra (Kimi Linear summary §3.1, with the 16-token sub-tiles
+of the Kimi K3 architecture summary) is evaluated in float32 with each
+operand rounding the tensor-core kernels apply switched on alone, all
+together, or all but one:
+
+  m1_kk     bf16 operands of A_kk (beta k E rows x key windows)
+  m1_qr     bf16 q E rows of A_qk
+  m1_qc     bf16 key windows of A_qk (off-diagonal 16 x 16 blocks)
+  m1_qd     bf16 operands of A_qk's four diagonal 16 x 16 blocks
+  slot_aqk  A_qk stored in f16
+  m2_t      f16 T and beta k e^Gamma in W = T Diag(beta) (K e^Gamma)
+  m2_v      bf16 T Diag(beta) and V in U~ = T Diag(beta) V
+  slot      W, U~, Q', K' stored in f16
+  chain_s   the f16 copy of S that multiplies [Q'; W]
+  chain_u   U = U~ - W S rounded to f16
+  out       o rounded to bf16
+
+Run from the repository root (CPU only, about a minute):
+
+    python tests/error_budget.py
+
+It measures four heads of the L=4096 bf16 workload.  The kernels' own
+figures for that workload come from ``tests/report_errors.py`` on a GPU."""
+import os
+import sys
+
+import numpy as np
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+
+from gated_delta_rule_98_b200 import synth  # noqa: E402
+from oracle import ref  # noqa: E402
+
+
+def bf16(x):
+    """Round to bfloat16 (nearest, ties to even), kept in float32."""
+    x = np.ascontiguousarray(x, np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32)
+
+
+def f16(x):
+    """Round to IEEE half (saturating at the largest finite value)."""
+    return np.clip(np.asarray(x, np.float32), -65504, 65504).astype(np.float16).astype(np.float32)
+
+
+def tf32(x):
+    """Round to 10 explicit mantissa bits with the float32 exponent."""
+    x = np.ascontiguousarray(x, np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    r = ((u + 0xFFF + ((u >> 13) & 1)) >> 13) << 13
+    return r.astype(np.uint32).view(np.float32)
+
+
+def hi_lo(x):
+    """A bf16 pair hi + lo (about 16 mantissa bits)."""
+    hi = bf16(x)
+    return hi + bf16(np.asarray(x, np.float32) - hi)
+
+
+def exact(x):
+    return np.asarray(x, np.float32)
+
+
+GROUPS = ("m1_kk", "m1_qr", "m1_qc", "m1_qd", "slot_aqk", "m2_t", "m2_v", "slot", "chain_s",
+          "chain_u", "out")
+KERNEL = dict(m1_kk=bf16, m1_qr=bf16, m1_qc=bf16, m1_qd=bf16, slot_aqk=f16, m2_t=f16, m2_v=bf16,
+              slot=f16, chain_s=f16, chain_u=f16, out=bf16)
+NONE = {g: exact for g in GROUPS}
+C, SUB = 64, 16
+
+
+def chunked(inp, heads, R):
+    """o [T, len(heads), dv] of the chunkwise form with the roundings R."""
+    q = inp["q"].float().numpy()
+    k = inp["k"].float().numpy()
+    v = inp["v"].float().numpy()
+    z = inp["z"].float().numpy()
+    beta = inp["beta"].float().numpy()
+    A = inp["A"].numpy()
+    T, _, D = q.shape
+    o = np.zeros((T, len(heads), v.shape[-1]), np.float32)
+    for hi, h in enumerate(heads):
+        S = np.zeros((D, v.shape[-1]), np.float32)
+        for c0 in range(0, T, C):
+            qc, kc, vc, bc = q[c0:c0 + C, h], k[c0:c0 + C, h], v[c0:c0 + C, h], beta[c0:c0 + C, h]
+            g = (-5.0 / (1.0 + np.exp(-np.exp(A[h]) * z[c0:c0 + C, h]))).astype(np.float32)
+            Gam = np.cumsum(g, axis=0, dtype=np.float32)
+            kn = kc / np.sqrt((kc * kc).sum(-1, keepdims=True) + 1e-6)
+            iq = 1.0 / np.sqrt((qc * qc).sum(-1, keepdims=True) + 1e-6)
+            Akk = np.zeros((C, C), np.float32)
+            Aqk = np.zeros((C, C), np.float32)
+            for b in range(C // SUB):
+                rb = slice(SUB * b, SUB * (b + 1))
+                rho = Gam[SUB * b - 1] if b > 0 else np.zeros(D, np.float32)
+                E = np.exp(Gam[rb] - rho)  # <= 1
+                for a in range(b + 1):
+                    ra = slice(SUB * a, SUB * (a + 1))
+                    col = kn[ra] * np.exp(rho - Gam[ra])  # <= 1 for a < b, up to e^80 for a = b
+                    Akk[rb, ra] = R["m1_kk"](bc[rb, None] * kn[rb] * E) @ R["m1_kk"](col).T
+                    if a == b:
+                        Aqk[rb, ra] = R["m1_qd"](qc[rb] * E) @ R["m1_qd"](col).T
+                    else:
+                        Aqk[rb, ra] = R["m1_qr"](qc[rb] * E) @ R["m1_qc"](col).T
+            Akk = np.tril(Akk, -1)
+            Aqk = R["slot_aqk"](np.tril(Aqk, 0))
+            Tm = np.tril(np.linalg.inv(np.eye(C, dtype=np.float32) + Akk).astype(np.float32))
+            W = R["slot"](R["m2_t"](Tm) @ R["m2_t"](bc[:, None] * kn * np.exp(Gam)))
+            Ut = R["slot"](R["m2_v"](Tm * bc[None, :]) @ R["m2_v"](vc))
+            Qp = R["slot"](qc * np.exp(Gam))
+            Kp = R["slot"](kn * np.exp(Gam[-1] - Gam))
+            Sc = R["chain_s"](S)
+            U = R["chain_u"](Ut - W @ Sc)
+            o[c0:c0 + C, hi] = R["out"]((Qp @ Sc + Aqk @ U) * iq)
+            S = np.exp(Gam[-1])[:, None] * S + Kp.T @ U
+    return o
+
+
+def main():
+    inp = synth.workload("bf16")
+    heads = [0, 5, 10, 15]
+    d = {n: inp[n].double().numpy()[:, heads] for n in ("q", "k", "v", "beta", "z")}
+    o_ref, _ = ref.forward(d["q"], d["k"], d["v"], d["beta"], z=d["z"],
+                           A=inp["A"].double().numpy()[heads])
+
+    def rel(R):
+        o = chunked(inp, heads, R)
+        return np.linalg.norm(o - o_ref) / np.linalg.norm(o_ref)
+
+    def show(name, R):
+        print(f"{name:58s} o rel-L2 {rel(R):.3e}", flush=True)
+
+    show("no rounding (float32 arithmetic)", NONE)
+    show("every rounding of the kernels", KERNEL)
+    for g in GROUPS:
+        show(f"only {g}", {**NONE, g: KERNEL[g]})
+    for g in GROUPS:
+        show(f"all but {g}", {**KERNEL, g: exact})
+    show("earlier kernel: slots and chain operands in bf16",
+         {**KERNEL, "slot": bf16, "slot_aqk": bf16, "chain_s": bf16, "chain_u": bf16, "m2_t": bf16})
+    show("only the S copy in bf16", {**NONE, "chain_s": bf16})
+    show("kernel, A_qk diagonal blocks as hi + lo bf16 pairs", {**KERNEL, "m1_qd": hi_lo})
+    show("kernel, A_qk diagonal blocks in tf32", {**KERNEL, "m1_qd": tf32})
+    show("kernel, A_qk diagonal blocks in float32", {**KERNEL, "m1_qd": exact})
+    show("kernel, A_qk diagonal blocks in float32, o in float32",
+         {**KERNEL, "m1_qd": exact, "out": exact})
+
+
+if __name__ == "__main__":
+    main()
