@@ -22,8 +22,11 @@ Run from the repository root (CPU only, about a minute):
 
     python tests/error_budget.py
 
-It measures four heads of the L=4096 bf16 workload.  The kernels' own
-figures for that workload come from ``tests/report_errors.py`` on a GPU."""
+It measures four heads of the L=4096 bf16 workload, then the output
+epilogue y = RMSNorm(o) * w * sigmoid(r) (Kimi Linear summary §4) on the
+T=1024, H=4 case with a nonzero initial state, where y is formed from the
+float32 o as the fused epilogue does.  The kernels' own figures for both
+come from ``tests/report_errors.py`` on a GPU."""
 import os
 import sys
 
@@ -32,7 +35,7 @@ import numpy as np
 sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
 
 from gated_delta_rule_98_b200 import synth  # noqa: E402
-from oracle import ref  # noqa: E402
+from oracle import epilogue, ref  # noqa: E402
 
 
 def bf16(x):
@@ -74,8 +77,9 @@ NONE = {g: exact for g in GROUPS}
 C, SUB = 64, 16
 
 
-def chunked(inp, heads, R):
-    """o [T, len(heads), dv] of the chunkwise form with the roundings R."""
+def chunked(inp, heads, R, S0=None):
+    """o [T, len(heads), dv] of the chunkwise form with the roundings R, from
+    the initial states S0 [1, H, dk, dv] (zero when None)."""
     q = inp["q"].float().numpy()
     k = inp["k"].float().numpy()
     v = inp["v"].float().numpy()
@@ -85,7 +89,8 @@ def chunked(inp, heads, R):
     T, _, D = q.shape
     o = np.zeros((T, len(heads), v.shape[-1]), np.float32)
     for hi, h in enumerate(heads):
-        S = np.zeros((D, v.shape[-1]), np.float32)
+        S = (np.zeros((D, v.shape[-1]), np.float32) if S0 is None
+             else np.array(S0[0, h], np.float32))
         for c0 in range(0, T, C):
             qc, kc, vc, bc = q[c0:c0 + C, h], k[c0:c0 + C, h], v[c0:c0 + C, h], beta[c0:c0 + C, h]
             g = (-5.0 / (1.0 + np.exp(-np.exp(A[h]) * z[c0:c0 + C, h]))).astype(np.float32)
@@ -148,6 +153,24 @@ def main():
     show("kernel, A_qk diagonal blocks in float32", {**KERNEL, "m1_qd": exact})
     show("kernel, A_qk diagonal blocks in float32, o in float32",
          {**KERNEL, "m1_qd": exact, "out": exact})
+
+    # the output epilogue, from the float32 o
+    T, H = 1024, 4
+    e_inp = synth.draw(T, H, 128, 128, seed=50 + H, dtype="bf16", num_seqs=1, s0_std=0.02)
+    r, w = synth.out_gate_inputs(T, H, 128, seed=51)
+    d = {n: e_inp[n].double().numpy() for n in ("q", "k", "v", "beta", "z")}
+    eo_ref, _ = ref.forward(d["q"], d["k"], d["v"], d["beta"], z=d["z"],
+                            A=e_inp["A"].double().numpy(), S0=e_inp["S0"].double().numpy())
+    y_ref = epilogue.norm_gate(eo_ref, r.double().numpy(), w.double().numpy(), eps=1e-6)
+    rn, wn = r.float().numpy(), w.numpy()
+    S0 = e_inp["S0"].numpy()
+    for name, R in (("kernel", KERNEL), ("kernel, A_qk diagonal blocks as hi + lo pairs",
+                                         {**KERNEL, "m1_qd": hi_lo})):
+        o32 = chunked(e_inp, list(range(H)), {**R, "out": exact}, S0)
+        y = bf16(o32 / np.sqrt(np.mean(o32 * o32, -1, keepdims=True) + 1e-6) * wn
+                 / (1.0 + np.exp(-rn)))
+        print(f"epilogue T={T} H={H}, {name:37s} y rel-L2 "
+              f"{np.linalg.norm(y - y_ref) / np.linalg.norm(y_ref):.3e}", flush=True)
 
 
 if __name__ == "__main__":
