@@ -18,6 +18,8 @@ together, or all but one:
   chain_u   U = U~ - W S rounded to f16
   out       o rounded to bf16
 
+and, once, with the chain products reassociated (see ``chunked``).
+
 Run from the repository root (CPU only, about a minute):
 
     python tests/error_budget.py
@@ -77,51 +79,74 @@ NONE = {g: exact for g in GROUPS}
 C, SUB = 64, 16
 
 
-def chunked(inp, heads, R, S0=None):
+def prepare(inp, h, R):
+    """The state-independent operands of every chunk of head h (what the
+    chunk preparation writes to the chunk slots), with the roundings R."""
+    q = inp["q"].float().numpy()[:, h]
+    k = inp["k"].float().numpy()[:, h]
+    v = inp["v"].float().numpy()[:, h]
+    z = inp["z"].float().numpy()[:, h]
+    beta = inp["beta"].float().numpy()[:, h]
+    a_h = float(inp["A"][h])
+    D = q.shape[-1]
+    chunks = []
+    for c0 in range(0, q.shape[0], C):
+        qc, kc, vc, bc = q[c0:c0 + C], k[c0:c0 + C], v[c0:c0 + C], beta[c0:c0 + C]
+        g = (-5.0 / (1.0 + np.exp(-np.exp(a_h) * z[c0:c0 + C]))).astype(np.float32)
+        Gam = np.cumsum(g, axis=0, dtype=np.float32)
+        kn = kc / np.sqrt((kc * kc).sum(-1, keepdims=True) + 1e-6)
+        Akk = np.zeros((C, C), np.float32)
+        Aqk = np.zeros((C, C), np.float32)
+        for b in range(C // SUB):
+            rb = slice(SUB * b, SUB * (b + 1))
+            rho = Gam[SUB * b - 1] if b > 0 else np.zeros(D, np.float32)
+            E = np.exp(Gam[rb] - rho)  # <= 1
+            for a in range(b + 1):
+                ra = slice(SUB * a, SUB * (a + 1))
+                col = kn[ra] * np.exp(rho - Gam[ra])  # <= 1 for a < b, up to e^80 for a = b
+                Akk[rb, ra] = R["m1_kk"](bc[rb, None] * kn[rb] * E) @ R["m1_kk"](col).T
+                if a == b:
+                    Aqk[rb, ra] = R["m1_qd"](qc[rb] * E) @ R["m1_qd"](col).T
+                else:
+                    Aqk[rb, ra] = R["m1_qr"](qc[rb] * E) @ R["m1_qc"](col).T
+        Akk = np.tril(Akk, -1)
+        Tm = np.tril(np.linalg.inv(np.eye(C, dtype=np.float32) + Akk).astype(np.float32))
+        W = R["slot"](R["m2_t"](Tm) @ R["m2_t"](bc[:, None] * kn * np.exp(Gam)))
+        chunks.append(dict(
+            Y=np.concatenate([R["slot"](qc * np.exp(Gam)), W]),     # [Q'; W]
+            Aqk=R["slot_aqk"](np.tril(Aqk, 0)),
+            Ut=R["slot"](R["m2_v"](Tm * bc[None, :]) @ R["m2_v"](vc)),
+            Kp=R["slot"](kn * np.exp(Gam[-1] - Gam)),              # K'
+            gam=np.exp(Gam[-1]),
+            iq=1.0 / np.sqrt((qc * qc).sum(-1, keepdims=True) + 1e-6)))
+    return chunks
+
+
+def chunked(inp, heads, R, S0=None, reassociated=False):
     """o [T, len(heads), dv] of the chunkwise form with the roundings R, from
-    the initial states S0 [1, H, dk, dv] (zero when None)."""
-    q = inp["q"].float().numpy()
-    k = inp["k"].float().numpy()
-    v = inp["v"].float().numpy()
-    z = inp["z"].float().numpy()
-    beta = inp["beta"].float().numpy()
-    A = inp["A"].numpy()
-    T, _, D = q.shape
-    o = np.zeros((T, len(heads), v.shape[-1]), np.float32)
+    the initial states S0 [1, H, dk, dv] (zero when None).
+
+    reassociated: each chunk's state product is formed from the state before
+    the previous chunk, Y_{c+1} S_c = (Y_{c+1} Diag(gamma_c)) S_{c-1} +
+    (Y_{c+1} K'_c^T) U_c, with both new factors rounded like the slot images
+    (a schedule with one dependent product per chunk instead of two)."""
+    dv = inp["v"].shape[-1]
+    o = np.zeros((inp["q"].shape[0], len(heads), dv), np.float32)
     for hi, h in enumerate(heads):
-        S = (np.zeros((D, v.shape[-1]), np.float32) if S0 is None
+        ch = prepare(inp, h, R)
+        S = (np.zeros((inp["q"].shape[-1], dv), np.float32) if S0 is None
              else np.array(S0[0, h], np.float32))
-        for c0 in range(0, T, C):
-            qc, kc, vc, bc = q[c0:c0 + C, h], k[c0:c0 + C, h], v[c0:c0 + C, h], beta[c0:c0 + C, h]
-            g = (-5.0 / (1.0 + np.exp(-np.exp(A[h]) * z[c0:c0 + C, h]))).astype(np.float32)
-            Gam = np.cumsum(g, axis=0, dtype=np.float32)
-            kn = kc / np.sqrt((kc * kc).sum(-1, keepdims=True) + 1e-6)
-            iq = 1.0 / np.sqrt((qc * qc).sum(-1, keepdims=True) + 1e-6)
-            Akk = np.zeros((C, C), np.float32)
-            Aqk = np.zeros((C, C), np.float32)
-            for b in range(C // SUB):
-                rb = slice(SUB * b, SUB * (b + 1))
-                rho = Gam[SUB * b - 1] if b > 0 else np.zeros(D, np.float32)
-                E = np.exp(Gam[rb] - rho)  # <= 1
-                for a in range(b + 1):
-                    ra = slice(SUB * a, SUB * (a + 1))
-                    col = kn[ra] * np.exp(rho - Gam[ra])  # <= 1 for a < b, up to e^80 for a = b
-                    Akk[rb, ra] = R["m1_kk"](bc[rb, None] * kn[rb] * E) @ R["m1_kk"](col).T
-                    if a == b:
-                        Aqk[rb, ra] = R["m1_qd"](qc[rb] * E) @ R["m1_qd"](col).T
-                    else:
-                        Aqk[rb, ra] = R["m1_qr"](qc[rb] * E) @ R["m1_qc"](col).T
-            Akk = np.tril(Akk, -1)
-            Aqk = R["slot_aqk"](np.tril(Aqk, 0))
-            Tm = np.tril(np.linalg.inv(np.eye(C, dtype=np.float32) + Akk).astype(np.float32))
-            W = R["slot"](R["m2_t"](Tm) @ R["m2_t"](bc[:, None] * kn * np.exp(Gam)))
-            Ut = R["slot"](R["m2_v"](Tm * bc[None, :]) @ R["m2_v"](vc))
-            Qp = R["slot"](qc * np.exp(Gam))
-            Kp = R["slot"](kn * np.exp(Gam[-1] - Gam))
-            Sc = R["chain_s"](S)
-            U = R["chain_u"](Ut - W @ Sc)
-            o[c0:c0 + C, hi] = R["out"]((Qp @ Sc + Aqk @ U) * iq)
-            S = np.exp(Gam[-1])[:, None] * S + Kp.T @ U
+        Dm = ch[0]["Y"] @ R["chain_s"](S)
+        for c, x in enumerate(ch):
+            if not reassociated:
+                Dm = x["Y"] @ R["chain_s"](S)
+            U = R["chain_u"](x["Ut"] - Dm[C:])
+            o[c * C:(c + 1) * C, hi] = R["out"]((Dm[:C] + x["Aqk"] @ U) * x["iq"])
+            if reassociated and c + 1 < len(ch):
+                y = ch[c + 1]["Y"]
+                Dm = (R["slot"](y * x["gam"][None, :]) @ R["chain_s"](S)
+                      + R["slot"](y @ x["Kp"].T) @ U)
+            S = x["gam"][:, None] * S + x["Kp"].T @ U
     return o
 
 
@@ -153,6 +178,9 @@ def main():
     show("kernel, A_qk diagonal blocks in float32", {**KERNEL, "m1_qd": exact})
     show("kernel, A_qk diagonal blocks in float32, o in float32",
          {**KERNEL, "m1_qd": exact, "out": exact})
+    o = chunked(inp, heads, KERNEL, reassociated=True)
+    print(f"{'kernel, reassociated chain schedule':58s} o rel-L2 "
+          f"{np.linalg.norm(o - o_ref) / np.linalg.norm(o_ref):.3e}", flush=True)
 
     # the output epilogue, from the float32 o
     T, H = 1024, 4
