@@ -69,6 +69,31 @@ def test_workspace_holds_one_chunk_slot_per_chunk_and_head(L):
         assert need <= size <= need + 64 * 1024 * 1024, (N, T, H, size, need)
 
 
+@pytest.mark.parametrize("N,H,L,P", [
+    (1, 16, 65536, 9),    # 148 // 16
+    (1, 4, 4096, 16),     # 148 // 4 = 37, at most 16
+    (1, 16, 256, 2),      # 4 chunks: at most half the chunk count
+    (1, 16, 64, 1),       # one chunk
+    (8, 16, 4096, 1),     # 128 (sequence, head) pairs fill the SMs without segments
+    (2, 32, 4096, 2),     # 64 pairs: 148 // 64
+    (1, 200, 4096, 1),
+])
+def test_segment_rule(L, N, H, P):
+    """Segments per sequence on the tensor-core path, P = 148 // (N H), at most
+    half the chunk count and at most 16 (1 when the pairs fill the SMs): the
+    workspace holds (3P - 2) 64 KB state maps per (sequence, head) before the
+    chunk slots, and the call makes 4 launches when P > 1, else 2."""
+    T = N * L
+    size = kda.kda_forward_workspace_size(N, T, L, H, 128, 128, kda.KDA_BF16, 64)
+    maps = size - (T // 64 + N) * H * 74496 - 256           # header, then the maps
+    assert maps >= 0 and maps // (N * H * 65536) == 3 * P - 2, (size, maps)
+    assert kda.kda_forward_launches(N, T, L, H, 128, 128, kda.KDA_BF16, 64) == (4 if P > 1 else 2)
+    # context parallelism keeps room for all P transitions (P + 1 segment buffers)
+    cw = kda.kda_cp_workspace_size(N, T, L, H, 128, 128, kda.KDA_BF16, 64)
+    cmaps = cw - (T // 64 + N) * H * 74496 - 256
+    assert cmaps // (N * H * 65536) == 3 * (P + 1) - 2
+
+
 FAKE = 0x10000  # aligned fake device address: never dereferenced by these calls
 
 
