@@ -18,7 +18,8 @@ together, or all but one:
   chain_u   U = U~ - W S rounded to f16
   out       o rounded to bf16
 
-and, once, with the chain products reassociated (see ``chunked``).
+and, once each, with the chain products reassociated (see ``chunked``) and
+with 128-token chunks.
 
 Run from the repository root (CPU only, about a minute):
 
@@ -79,9 +80,10 @@ NONE = {g: exact for g in GROUPS}
 C, SUB = 64, 16
 
 
-def prepare(inp, h, R):
-    """The state-independent operands of every chunk of head h (what the
-    chunk preparation writes to the chunk slots), with the roundings R."""
+def prepare(inp, h, R, C=C):
+    """The state-independent operands of every chunk (C tokens) of head h
+    (what the chunk preparation writes to the chunk slots), with the
+    roundings R."""
     q = inp["q"].float().numpy()[:, h]
     k = inp["k"].float().numpy()[:, h]
     v = inp["v"].float().numpy()[:, h]
@@ -122,7 +124,7 @@ def prepare(inp, h, R):
     return chunks
 
 
-def chunked(inp, heads, R, S0=None, reassociated=False):
+def chunked(inp, heads, R, S0=None, reassociated=False, C=C):
     """o [T, len(heads), dv] of the chunkwise form with the roundings R, from
     the initial states S0 [1, H, dk, dv] (zero when None).
 
@@ -133,7 +135,7 @@ def chunked(inp, heads, R, S0=None, reassociated=False):
     dv = inp["v"].shape[-1]
     o = np.zeros((inp["q"].shape[0], len(heads), dv), np.float32)
     for hi, h in enumerate(heads):
-        ch = prepare(inp, h, R)
+        ch = prepare(inp, h, R, C)
         S = (np.zeros((inp["q"].shape[-1], dv), np.float32) if S0 is None
              else np.array(S0[0, h], np.float32))
         Dm = ch[0]["Y"] @ R["chain_s"](S)
@@ -178,9 +180,11 @@ def main():
     show("kernel, A_qk diagonal blocks in float32", {**KERNEL, "m1_qd": exact})
     show("kernel, A_qk diagonal blocks in float32, o in float32",
          {**KERNEL, "m1_qd": exact, "out": exact})
-    o = chunked(inp, heads, KERNEL, reassociated=True)
-    print(f"{'kernel, reassociated chain schedule':58s} o rel-L2 "
-          f"{np.linalg.norm(o - o_ref) / np.linalg.norm(o_ref):.3e}", flush=True)
+    for name, kw in (("kernel, reassociated chain schedule", dict(reassociated=True)),
+                     ("kernel, 128-token chunks", dict(C=128))):
+        o = chunked(inp, heads, KERNEL, **kw)
+        print(f"{name:58s} o rel-L2 {np.linalg.norm(o - o_ref) / np.linalg.norm(o_ref):.3e}",
+              flush=True)
 
     # the output epilogue, from the float32 o
     T, H = 1024, 4
