@@ -1,6 +1,7 @@
-"""The rounding helpers of tests/error_budget.py against torch's own
-conversions (CPU): the error budget is only as good as its emulated bf16,
-f16 and tf32 roundings."""
+"""The error-budget script (tests/error_budget.py) pinned on the CPU: its
+bf16, f16 and tf32 roundings against torch's own conversions, and its
+chunkwise algebra, with every rounding off, against the float64 oracle.  The
+budget is only as good as these two."""
 import os
 import sys
 
@@ -46,3 +47,18 @@ def test_hi_lo_pair_is_near_float32():
     x = x[(np.abs(x) > 1e-30) & (np.abs(x) < 1e30)]
     y = eb.hi_lo(x)
     assert np.all(np.abs(y - x) <= np.abs(x) * 2.0 ** -16)
+
+
+def test_emulation_without_rounding_is_the_oracle():
+    """With every rounding off, the emulated chunkwise form (both chain
+    schedules, 64- and 128-token chunks) agrees with the float64 oracle to
+    float32 accuracy, so the budget measures roundings and nothing else."""
+    from gated_delta_rule_98_b200 import synth
+    from oracle import ref
+    inp = synth.draw(512, 2, 128, 128, seed=9, dtype="bf16")
+    d = {n: inp[n].double().numpy() for n in ("q", "k", "v", "beta", "z")}
+    o_ref, _ = ref.forward(d["q"], d["k"], d["v"], d["beta"], z=d["z"],
+                           A=inp["A"].double().numpy())
+    for kw in (dict(), dict(reassociated=True), dict(C=128)):
+        o = eb.chunked(inp, [0, 1], eb.NONE, **kw)
+        assert np.linalg.norm(o - o_ref) / np.linalg.norm(o_ref) < 1e-5, kw
